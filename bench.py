@@ -1,0 +1,582 @@
+"""Benchmark of the DBSA attention engine on B200 (one JSON line on stdout).
+
+One step = the whole hot path over one batch of the Llama-3.1-8B-shaped 90k
+workload: Stage 1 (dbsa_encode_blocks) for every layer, then Stage 2
+(dbsa_gather_rope_attend) for the query batch's prompt pass and every decode
+step, for every layer.  Inputs are seeded synthetic tensors, resident in HBM
+before the timed region; each layer's working set (Q/K/V/O ~2 GB) is far
+larger than L2, so no flush is needed between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (torchrun, one rank per GPU) every rank runs its own independent
+batch (weak scaling, no collective on the data path); value = work of all
+ranks / max-over-ranks time.  --impl reference times the CPU oracle, as it
+stands, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from many_shot_icl_b200 import inputs  # noqa: E402
+
+METRIC = "Stage-1 encode tok/s & Stage-2 query tok/s (L3.1-8B shape, 90k); % roofline"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p, "measured"
+    except OSError:
+        return dict(PEAKS_FALLBACK), "fallback"
+
+
+# ------------------------------------------------------------------ workload
+class Workload:
+    """Offsets, selections and per-layer tensors of one batch."""
+
+    def __init__(self, w: inputs.Workload, layers: int, device, rank: int = 0,
+                 append_room: int = 0):
+        import torch
+        self.w = w
+        self.layers = layers
+        self.offs = inputs_offsets(w)
+        self.nb = len(self.offs) - 1
+        self.T = int(self.offs[-1])
+        self.cap = self.T + append_room
+        self.sels = inputs.selections(w, seed_offset=rank)
+        from many_shot_icl_b200 import dbsa
+        self.sel_ptr, self.sel = dbsa.selection_csr(self.sels)
+        self.cfg = dbsa.DbsaConfig(w.n_q_heads, w.n_kv_heads, w.head_dim, w.dtype, w.rope_theta,
+                                   w.window_j)
+        Hq, Hkv, D, T = w.n_q_heads, w.n_kv_heads, w.head_dim, self.T
+        dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+        self.dt = dt
+        self.nq = w.n_queries
+        self.tail_cap = w.query_tokens + w.decode_steps
+        self.q, self.k, self.v, self.kc, self.vc, self.out = [], [], [], [], [], []
+        self.qp, self.qd, self.kt, self.vt = [], [], [], []
+        for l in range(layers):
+            s = lambda role, step=0: inputs.tensor_seed(w, l, role, step) + 7919 * rank
+            self.q.append(inputs.randn((T, Hq, D), s(0), w.dtype, device))
+            self.k.append(inputs.randn((T, Hkv, D), s(1), w.dtype, device))
+            self.v.append(inputs.randn((T, Hkv, D), s(2), w.dtype, device))
+            self.kc.append(torch.empty((Hkv, self.cap, D), dtype=dt, device=device))
+            self.vc.append(torch.empty((Hkv, self.cap, D), dtype=dt, device=device))
+            self.out.append(torch.empty((T, Hq, D), dtype=dt, device=device))
+            self.qp.append(inputs.randn((self.nq, w.query_tokens, Hq, D), s(3, 0), w.dtype, device))
+            self.qd.append(inputs.randn((self.nq, 1, Hq, D), s(3, 1), w.dtype, device))
+            self.kt.append(inputs.randn((self.nq, self.tail_cap, Hkv, D), s(3, 2), w.dtype, device))
+            self.vt.append(inputs.randn((self.nq, self.tail_cap, Hkv, D), s(3, 3), w.dtype, device))
+        self.out_p = torch.empty((self.nq, w.query_tokens, Hq, D), dtype=dt, device=device)
+        self.out_d = torch.empty((self.nq, 1, Hq, D), dtype=dt, device=device)
+        ws1 = dbsa.encode_workspace_size(self.cfg, T, self.nb)
+        ws2 = max(dbsa.gather_workspace_size(self.cfg, self.offs, self.sel_ptr, self.sel, n, t)
+                  for n, t in self.passes())
+        self.ws = torch.empty(max(ws1, ws2), dtype=torch.uint8, device=device)
+
+    def passes(self):
+        """(n_new, tail_len) of the prompt pass and each decode step."""
+        w = self.w
+        return [(w.query_tokens, w.query_tokens)] + [(1, w.query_tokens + i)
+                                                     for i in range(1, w.decode_steps + 1)]
+
+    def gathered(self):
+        return np.array([int(sum(self.offs[b + 1] - self.offs[b] for b in s)) for s in self.sels])
+
+
+def inputs_offsets(w):
+    from many_shot_icl_b200 import dbsa
+    return dbsa.group_blocks(inputs.demo_lengths(w), w.demos_per_block)
+
+
+def stage1_exact_pairs(offs, j):
+    """sum over rows of allowed keys: (t - offs[b] + 1) + lengths of the distinct
+    blocks {0} U {max(0, b-j) .. b-1} (bench accounting only)."""
+    lens = np.diff(offs).astype(np.int64)
+    total = 0
+    for b, L in enumerate(lens):
+        others = set(range(max(0, b - j), b)) | ({0} if b > 0 else set())
+        total += L * (L + 1) // 2 + L * int(sum(lens[x] for x in others))
+    return total
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", "dbsa_clocks_%d_%d.csv" % (os.getpid(), gpu_index))
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ our arm
+def run_step(wl: Workload, prof=None):
+    """One step; if prof is given, per-call kernel events are appended to it."""
+    import torch
+    from many_shot_icl_b200 import dbsa
+    for l in range(wl.layers):
+        if prof is not None:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            dbsa.set_profile_events(e0, e1)
+            prof["s1"].append((e0, e1))
+        dbsa.encode_blocks(wl.cfg, wl.q[l], wl.k[l], wl.v[l], wl.offs, wl.kc[l], wl.vc[l],
+                           wl.out[l], wl.ws)
+    for n_new, tail_len in wl.passes():
+        for l in range(wl.layers):
+            qn = wl.qp[l] if n_new > 1 else wl.qd[l]
+            out = wl.out_p if n_new > 1 else wl.out_d
+            if prof is not None:
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                dbsa.set_profile_events(e0, e1)
+                prof["s2p" if n_new > 1 else "s2d"].append((e0, e1))
+            dbsa.gather_rope_attend(wl.cfg, wl.kc[l], wl.vc[l], wl.offs, wl.sel_ptr, wl.sel, qn,
+                                    wl.kt[l], wl.vt[l], tail_len, out, wl.ws)
+
+
+def stage_times(wl: Workload):
+    """Device time of Stage 1 and Stage 2 of one step, measured separately."""
+    import torch
+    from many_shot_icl_b200 import dbsa
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    ev[0].record()
+    for l in range(wl.layers):
+        dbsa.encode_blocks(wl.cfg, wl.q[l], wl.k[l], wl.v[l], wl.offs, wl.kc[l], wl.vc[l],
+                           wl.out[l], wl.ws)
+    ev[1].record()
+    for n_new, tail_len in wl.passes():
+        for l in range(wl.layers):
+            qn, out = (wl.qp[l], wl.out_p) if n_new > 1 else (wl.qd[l], wl.out_d)
+            dbsa.gather_rope_attend(wl.cfg, wl.kc[l], wl.vc[l], wl.offs, wl.sel_ptr, wl.sel, qn,
+                                    wl.kt[l], wl.vt[l], tail_len, out, wl.ws)
+    ev[2].record()
+    torch.cuda.synchronize()
+    return ev[0].elapsed_time(ev[1]) / 1e3, ev[1].elapsed_time(ev[2]) / 1e3
+
+
+def e2e_step_time(wl: Workload, host, steps: int):
+    """Same step through the public API from pinned host buffers: per layer the
+    Q/K/V upload, the call and the output download are inside the timed region."""
+    import torch
+    from many_shot_icl_b200 import dbsa
+    dev_q, dev_k, dev_v, dev_o = wl.q[0], wl.k[0], wl.v[0], wl.out[0]
+    t1 = t2 = 0.0
+    for _ in range(steps):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        torch.cuda.synchronize()
+        ev[0].record()
+        for l in range(wl.layers):
+            dev_q.copy_(host["q"], non_blocking=True)
+            dev_k.copy_(host["k"], non_blocking=True)
+            dev_v.copy_(host["v"], non_blocking=True)
+            dbsa.encode_blocks(wl.cfg, dev_q, dev_k, dev_v, wl.offs, wl.kc[l], wl.vc[l], dev_o,
+                               wl.ws)
+            host["o"].copy_(dev_o, non_blocking=True)
+        ev[1].record()
+        for n_new, tail_len in wl.passes():
+            for l in range(wl.layers):
+                qn, out = (wl.qp[l], wl.out_p) if n_new > 1 else (wl.qd[l], wl.out_d)
+                hq, ho = (host["qp"], host["op"]) if n_new > 1 else (host["qd"], host["od"])
+                qn.copy_(hq, non_blocking=True)
+                # the pass's new tail tokens (K and V) arrive from the host too
+                wl.kt[l][:, tail_len - n_new:tail_len].copy_(host["kt"][:, :n_new], non_blocking=True)
+                wl.vt[l][:, tail_len - n_new:tail_len].copy_(host["vt"][:, :n_new], non_blocking=True)
+                dbsa.gather_rope_attend(wl.cfg, wl.kc[l], wl.vc[l], wl.offs, wl.sel_ptr, wl.sel,
+                                        qn, wl.kt[l], wl.vt[l], tail_len, out, wl.ws)
+                ho.copy_(out, non_blocking=True)
+        ev[2].record()
+        torch.cuda.synchronize()
+        t1 += ev[0].elapsed_time(ev[1]) / 1e3
+        t2 += ev[1].elapsed_time(ev[2]) / 1e3
+    return t1 / steps, t2 / steps
+
+
+def pinned_host_buffers(wl: Workload):
+    import torch
+    p = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t.cpu())
+    h = {"q": p(wl.q[0]), "k": p(wl.k[0]), "v": p(wl.v[0]),
+         "o": torch.empty(wl.out[0].shape, dtype=wl.dt, pin_memory=True),
+         "qp": p(wl.qp[0]), "qd": p(wl.qd[0]), "kt": p(wl.kt[0]), "vt": p(wl.vt[0]),
+         "op": torch.empty(wl.out_p.shape, dtype=wl.dt, pin_memory=True),
+         "od": torch.empty(wl.out_d.shape, dtype=wl.dt, pin_memory=True)}
+    return h
+
+
+def append_series(wl: Workload, n_appends: int):
+    """Stage-1 append of n_appends new 50-demo blocks after the encoded pool,
+    all layers each; returns per-append device ms and the flops of each."""
+    import torch
+    from many_shot_icl_b200 import dbsa
+    w = wl.w
+    lens = inputs.demo_lengths(w, n_blocks=w.n_blocks + n_appends)
+    all_offs = dbsa.group_blocks(lens, w.demos_per_block)
+    assert np.array_equal(all_offs[:wl.nb + 1], wl.offs)
+    Lmax = int(np.diff(all_offs[wl.nb:]).max())
+    Hq, Hkv, D = w.n_q_heads, w.n_kv_heads, w.head_dim
+    qa = inputs.randn((Lmax, Hq, D), 4242, w.dtype, "cuda")
+    ka = inputs.randn((Lmax, Hkv, D), 4243, w.dtype, "cuda")
+    va = inputs.randn((Lmax, Hkv, D), 4244, w.dtype, "cuda")
+    oa = torch.empty((Lmax, Hq, D), dtype=wl.dt, device="cuda")
+    ws = torch.empty(dbsa.append_workspace_size(wl.cfg, all_offs[:-1], Lmax) + (1 << 20),
+                     dtype=torch.uint8, device="cuda")
+    ms, flops = [], []
+    for a in range(n_appends):
+        nb = wl.nb + a
+        offs = all_offs[:nb + 1]
+        L = int(all_offs[nb + 1] - all_offs[nb])
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for l in range(wl.layers):
+            dbsa.append_block(wl.cfg, qa[:L], ka[:L], va[:L], offs, wl.kc[l], wl.vc[l], oa[:L], ws)
+        e1.record()
+        torch.cuda.synchronize()
+        ms.append(e0.elapsed_time(e1))
+        pairs = stage1_exact_pairs(all_offs[:nb + 2], w.window_j) - stage1_exact_pairs(offs, w.window_j)
+        flops.append(4.0 * D * Hq * pairs * wl.layers)
+    return ms, flops
+
+
+# ------------------------------------------------------------------ oracle timing
+def oracle_sample(w: inputs.Workload, budget_s: float, threads: int | None = None):
+    """Time the oracle on a bounded sample of the workload (layer 0 inputs):
+    Stage-1 rows and Stage-2 rows, each for about budget_s / 2 seconds.
+    Returns (stage-1 tok/s, stage-2 query tok/s, cores, sample description)."""
+    import torch
+    import oracle
+    offs = inputs_offsets(w)
+    T = int(offs[-1])
+    Hq, Hkv, D = w.n_q_heads, w.n_kv_heads, w.head_dim
+    q = inputs.randn((T, Hq, D), inputs.tensor_seed(w, 0, 0), w.dtype).float().numpy()
+    k = inputs.randn((T, Hkv, D), inputs.tensor_seed(w, 0, 1), w.dtype).float().numpy()
+    v = inputs.randn((T, Hkv, D), inputs.tensor_seed(w, 0, 2), w.dtype).float().numpy()
+    cores = threads or oracle.default_threads()
+    rng = np.random.default_rng(0)
+    # Stage 1: rows in batches until half the budget is spent
+    rows1, t1 = 0, 0.0
+    while t1 < budget_s / 2:
+        n = cores * 2
+        hh, tt = rng.integers(0, Hq, n), rng.integers(0, T, n)
+        t0 = time.perf_counter()
+        oracle.stage1_rows(q, k, v, offs, w.window_j, w.rope_theta, hh, tt, threads=cores)
+        t1 += time.perf_counter() - t0
+        rows1 += n
+    s1_tok_s = rows1 / t1 / (Hq * w.n_layers)          # a token = Hq rows in every layer
+    # Stage 2: rows of the prompt pass of query 0
+    sel = inputs.selections(w)[0]
+    kc = np.ascontiguousarray(k.transpose(1, 0, 2))
+    vc = np.ascontiguousarray(v.transpose(1, 0, 2))
+    n_new = max(w.query_tokens, 1)
+    qn = inputs.randn((n_new, Hq, D), 11, w.dtype).float().numpy()
+    kt = inputs.randn((n_new, Hkv, D), 12, w.dtype).float().numpy()
+    vt = inputs.randn((n_new, Hkv, D), 13, w.dtype).float().numpy()
+    rows2, t2 = 0, 0.0
+    while t2 < budget_s / 2:
+        n = cores * 2
+        hh, uu = rng.integers(0, Hq, n), rng.integers(0, n_new, n)
+        t0 = time.perf_counter()
+        oracle.stage2_rows(kc, vc, offs, sel, qn, kt, vt, w.rope_theta, hh, uu, threads=cores)
+        t2 += time.perf_counter() - t0
+        rows2 += n
+    passes = 1 + w.decode_steps
+    # a query token needs Hq rows per layer; the batch's token count over all passes:
+    s2_tok_s = rows2 / t2 / (Hq * w.n_layers)
+    desc = ("layer-0 inputs of %s: %d Stage-1 rows (random head, token) in %.1f s and %d Stage-2 "
+            "prompt-pass rows of query 0 in %.1f s, fp64 C oracle, %d threads; tok/s = rows/s / "
+            "(%d heads x %d layers)" % (w.name, rows1, t1, rows2, t2, cores, Hq, w.n_layers))
+    return s1_tok_s, s2_tok_s, cores, desc, passes
+
+
+# ------------------------------------------------------------------ main
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as tdist
+        torch.cuda.set_device(local)
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as tdist
+    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as tdist
+        tdist.barrier()
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    w = inputs.WORKLOADS[args.workload]
+    import oracle
+    oracle.build()
+    vals = []
+    for _ in range(args.warmup):
+        oracle_sample(w, args.ref_budget / max(args.steps, 1))
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        vals.append(oracle_sample(w, args.ref_budget / max(args.steps, 1)))
+    wall = time.perf_counter() - t0
+    s1 = float(np.mean([v[0] for v in vals]))
+    s2 = float(np.mean([v[1] for v in vals]))
+    cores, desc = vals[0][2], vals[0][3]
+    line = {"impl": "reference", "metric": METRIC, "value": s1, "unit": "tok/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": wall / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": w.name, "layers": w.n_layers,
+                                            "context_tokens": int(inputs_offsets(w)[-1])},
+            "stage2_query_tok_s": s2,
+            "cpu_baseline": {"value": s1, "unit": "tok/s", "cores": cores, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": s1, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=inputs.L31_8B_90K.name)
+    ap.add_argument("--layers", type=int, default=None, help="override the layer count")
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--appends", type=int, default=None)
+    ap.add_argument("--cpu-budget", type=float, default=16.0)
+    ap.add_argument("--ref-budget", type=float, default=60.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+    if args.warmup < 3:
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+
+    import torch
+    from many_shot_icl_b200 import build as lib_build
+    if rank == 0 and world == 1:
+        lib_build.build()
+    barrier(world)
+    from many_shot_icl_b200 import dbsa
+    dbsa.load()
+    torch.cuda.set_device(local)
+    peaks, peak_src = load_peaks()
+    w = inputs.WORKLOADS[args.workload]
+    layers = args.layers or w.n_layers
+    n_appends = inputs.L31_8B_APPEND.n_appends if args.appends is None else args.appends
+    room = (n_appends + 1) * w.demos_per_block * w.demo_len_hi if n_appends else 0
+    wl = Workload(w, layers, "cuda", rank=rank, append_room=room)
+    torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        run_step(wl)
+    torch.cuda.synchronize()
+    barrier(world)
+
+    gpu_idx = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]) \
+        if os.environ.get("CUDA_VISIBLE_DEVICES") else local
+    launches0 = dbsa.kernel_launches()
+    prof = {"s1": [], "s2p": [], "s2d": []}
+    with ClockSampler(gpu_idx) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        e_start, e_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e_start.record()
+        for _ in range(args.steps):
+            run_step(wl, prof)
+        e_stop.record()
+        torch.cuda.synchronize()
+        barrier(world)
+    launches = dbsa.kernel_launches() - launches0
+    step_s = e_start.elapsed_time(e_stop) / 1e3 / args.steps
+    step_s_max = max_over_ranks(step_s, world)
+    clocks = clk.summary()
+
+    # split of one step into its two stages (separate timed pass)
+    t_s1, t_s2 = stage_times(wl)
+    t_s1 = max_over_ranks(t_s1, world)
+    t_s2 = max_over_ranks(t_s2, world)
+
+    # algorithmic work
+    Hq, Hkv, D = w.n_q_heads, w.n_kv_heads, w.head_dim
+    tiles = dbsa.stage1_tile_count(wl.cfg, wl.offs)
+    tile_flop = 4.0 * 128 * 128 * D * tiles                      # per layer, unmasked tiles
+    exact_flop = 4.0 * D * Hq * stage1_exact_pairs(wl.offs, w.window_j)  # per layer
+    gath = wl.gathered()
+    bpe = 2 if w.dtype == "bf16" else 4
+
+    def s2_bytes(n_new, tail_len):
+        kv = float(gath.sum()) * Hkv * D * bpe * 2
+        tail = float(wl.nq) * tail_len * Hkv * D * bpe * 2
+        qo = float(wl.nq) * n_new * Hq * D * bpe * 2
+        return kv + tail + qo
+
+    def mean_ms(pairs):
+        return float(np.mean([a.elapsed_time(b) for a, b in pairs])) if pairs else float("nan")
+
+    s1_ms = mean_ms(prof["s1"])
+    s2p_ms = mean_ms(prof["s2p"])
+    s2d_ms = mean_ms(prof["s2d"])
+    s1_tflops = tile_flop / (s1_ms * 1e-3) / 1e12
+    s1_exact_tflops = exact_flop / (s1_ms * 1e-3) / 1e12
+    p_pass = wl.passes()
+    s2p_gbs = s2_bytes(*p_pass[0]) / (s2p_ms * 1e-3) / 1e9
+    s2d_bytes = float(np.mean([s2_bytes(n, t) for n, t in p_pass[1:]])) if len(p_pass) > 1 else 0.0
+    s2d_gbs = s2d_bytes / (s2d_ms * 1e-3) / 1e9 if len(p_pass) > 1 else float("nan")
+    s2_all_bytes = sum(s2_bytes(n, t) for n, t in p_pass)
+    s2_kernel_s = (s2p_ms + (len(p_pass) - 1) * (s2d_ms if len(p_pass) > 1 else 0)) * 1e-3
+    s2_gbs = s2_all_bytes / s2_kernel_s / 1e9
+
+    peak_tf = peaks.get("bf16_tflops_sustained", PEAKS_FALLBACK["bf16_tflops_sustained"])
+    peak_tf_burst = peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"])
+    peak_bw = peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
+    roof_s1 = {"kernel": "stage1_attn_kernel (tcgen05)", "bound": "tensor",
+               "achieved": round(s1_tflops, 1), "peak": peak_tf, "unit": "TFLOP/s",
+               "frac": round(s1_tflops / peak_tf, 4), "traffic": None,
+               "peak_kind": "sustained bf16, " + peak_src,
+               "frac_of_burst_peak": round(s1_tflops / peak_tf_burst, 4),
+               "exact_pair_tflops": round(s1_exact_tflops, 1),
+               "flop_per_launch": tile_flop, "launch_ms": round(s1_ms, 4)}
+    roof_s2 = {"kernel": "stage2_attn_kernel (split-KV gather/RoPE/attend)", "bound": "hbm",
+               "achieved": round(s2_gbs, 1), "peak": peak_bw, "unit": "GB/s",
+               "frac": round(s2_gbs / peak_bw, 4), "traffic": None, "peak_kind": "copy, " + peak_src,
+               "prompt_pass_gbs": round(s2p_gbs, 1), "decode_pass_gbs": round(s2d_gbs, 1),
+               "bytes_per_step_per_layer": s2_all_bytes,
+               "prompt_launch_ms": round(s2p_ms, 4), "decode_launch_ms": round(s2d_ms, 4)}
+    s1_share = s1_ms * layers
+    s2_share = s2_kernel_s * 1e3 * layers
+    roof, roof2 = (roof_s1, roof_s2) if s1_share >= s2_share else (roof_s2, roof_s1)
+
+    T = wl.T
+    q_tokens = wl.nq * (w.query_tokens + w.decode_steps)
+    s1_tok_s = T * world / t_s1
+    s2_tok_s = q_tokens * world / t_s2
+
+    # end to end from pinned host memory (rank-local)
+    host = pinned_host_buffers(wl)
+    e2e_t1, e2e_t2 = e2e_step_time(wl, host, args.e2e_steps)
+    e2e_t1 = max_over_ranks(e2e_t1, world)
+    e2e_t2 = max_over_ranks(e2e_t2, world)
+    elt = 2 if w.dtype == "bf16" else 4
+    h2d = layers * (T * (Hq + 2 * Hkv) * D * elt) + sum(
+        layers * wl.nq * (n * Hq * D + 2 * n * Hkv * D) * elt for n, _ in p_pass)
+    d2h = layers * T * Hq * D * elt + sum(layers * wl.nq * n * Hq * D * elt for n, _ in p_pass)
+
+    app = None
+    if n_appends and rank == 0:
+        ms, fl = append_series(wl, n_appends)
+        app = {"n_appends": n_appends, "layers": layers, "per_append_ms": [round(x, 3) for x in ms],
+               "tflops": [round(f / (m * 1e-3) / 1e12, 1) for f, m in zip(fl, ms)],
+               "slope_ms_per_append": round(float(np.polyfit(np.arange(len(ms)), ms, 1)[0]), 4)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        c1, c2, cores, desc, _ = oracle_sample(w, args.cpu_budget)
+        cpu = {"value": c1, "unit": "tok/s", "cores": cores, "kind": "oracle", "sample": desc,
+               "stage2_query_tok_s": c2}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(s1_tok_s, 1), "unit": "tok/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_s_max * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+            "data": "synthetic",
+            "config": {"workload": w.name, "layers": layers, "context_tokens": T,
+                       "blocks": wl.nb, "window_j": w.window_j, "q_heads": Hq, "kv_heads": Hkv,
+                       "head_dim": D, "queries": wl.nq, "query_tokens": w.query_tokens,
+                       "decode_steps": w.decode_steps,
+                       "retrieved_blocks_per_query": int(len(wl.sels[0]) - 1),
+                       "mean_gathered_tokens": float(gath.mean()),
+                       "parallelism": "dp%d (independent batch per GPU)" % world,
+                       "l2": "inputs larger than L2 (per-layer Q/K/V/O ~%.1f GB)" %
+                             ((wl.q[0].numel() * 2 + wl.k[0].numel() * 2 + wl.v[0].numel() * 2) * elt / 1e9)},
+            "value_definition": "context tokens encoded through all layers per second of Stage-1 time",
+            "stage1": {"tok_s": round(s1_tok_s, 1), "s_per_step": round(t_s1, 4)},
+            "stage2": {"query_tok_s": round(s2_tok_s, 1), "s_per_step": round(t_s2, 4),
+                       "query_tokens_per_step": q_tokens},
+            "roofline": roof, "roofline_secondary": roof2,
+            "e2e": {"value": round(T * world / e2e_t1, 1), "unit": "tok/s",
+                    "stage2_query_tok_s": round(q_tokens * world / e2e_t2, 1),
+                    "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+            "cpu_baseline": cpu,
+            "append": app,
+            "clocks": clocks,
+            "gpu_launches": int(launches / args.steps),
+            "gpu_launches_timed_region": int(launches),
+        }
+        print(json.dumps(line))
+    barrier(world)
+    if world > 1:
+        import torch.distributed as tdist
+        tdist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,753 @@
+// C-ABI entry points of the DBSA library: argument validation, host-side
+// planning (tile list, gather segments, split plan), workspace carving and
+// kernel launches.  All arithmetic of the method runs in the kernels.
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "dbsa_internal.h"
+
+using namespace dbsa;
+
+namespace {
+
+thread_local std::string g_err;
+thread_local cudaEvent_t g_prof_start = nullptr, g_prof_stop = nullptr;
+std::atomic<int64_t> g_launches{0};
+
+void count_launches(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+// Records the profiling events (if any) around the main kernel of a call.
+struct ProfileScope {
+  cudaStream_t st;
+  cudaEvent_t stop;
+  explicit ProfileScope(cudaStream_t s) : st(s), stop(g_prof_stop) {
+    if (g_prof_start) cudaEventRecord(g_prof_start, st);
+    g_prof_start = g_prof_stop = nullptr;
+  }
+  ~ProfileScope() {
+    if (stop) cudaEventRecord(stop, st);
+  }
+};
+
+dbsa_status fail(dbsa_status s, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return s;
+}
+
+dbsa_status cuda_fail(cudaError_t e, const char *where) {
+  return fail(DBSA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+constexpr size_t kAlign = 1024;
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Sequential sub-allocation of the caller's workspace.
+struct Carve {
+  size_t off = kStatusBytes;
+  size_t take(size_t bytes) {
+    const size_t o = align_up(off, kAlign);
+    off = o + bytes;
+    return o;
+  }
+  size_t total() const { return align_up(off, kAlign); }
+};
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+dbsa_status check_cfg(const dbsa_config *cfg) {
+  if (cfg == nullptr) return fail(DBSA_ERR_INVALID_ARG, "cfg is NULL");
+  if (cfg->n_q_heads <= 0 || cfg->n_kv_heads <= 0)
+    return fail(DBSA_ERR_INVALID_ARG, "head counts must be positive");
+  if (cfg->n_q_heads % cfg->n_kv_heads != 0)
+    return fail(DBSA_ERR_UNSUPPORTED, "n_q_heads must be a multiple of n_kv_heads");
+  if (cfg->n_q_heads / cfg->n_kv_heads > 64)
+    return fail(DBSA_ERR_UNSUPPORTED, "more than 64 query heads per KV head");
+  if (cfg->head_dim != 64 && cfg->head_dim != 128)
+    return fail(DBSA_ERR_UNSUPPORTED, "head_dim must be 64 or 128 (got %d)", cfg->head_dim);
+  if (cfg->dtype != DBSA_BF16 && cfg->dtype != DBSA_F32)
+    return fail(DBSA_ERR_UNSUPPORTED, "dtype must be DBSA_BF16 or DBSA_F32");
+  if (!(cfg->rope_theta > 1.0) || !std::isfinite(cfg->rope_theta))
+    return fail(DBSA_ERR_INVALID_ARG, "rope_theta must be a finite value > 1");
+  if (cfg->window_j < 0) return fail(DBSA_ERR_INVALID_ARG, "window_j must be >= 0");
+  if (cfg->pattern < 0 || cfg->pattern > 3) return fail(DBSA_ERR_INVALID_ARG, "unknown pattern");
+  if (cfg->reserved != 0) return fail(DBSA_ERR_INVALID_ARG, "reserved must be 0");
+  if (!std::isfinite(cfg->softmax_scale)) return fail(DBSA_ERR_INVALID_ARG, "bad softmax_scale");
+  return DBSA_OK;
+}
+
+dbsa_status check_offs(const int32_t *offs, int32_t nb) {
+  if (offs == nullptr) return fail(DBSA_ERR_INVALID_ARG, "offs is NULL");
+  if (nb < 1) return fail(DBSA_ERR_INVALID_ARG, "need at least one block (nb = %d)", nb);
+  if (offs[0] != 0) return fail(DBSA_ERR_INVALID_ARG, "offs[0] must be 0");
+  for (int32_t b = 0; b < nb; ++b)
+    if (offs[b + 1] <= offs[b])
+      return fail(DBSA_ERR_INVALID_ARG, "block %d is empty or offsets decrease", b);
+  if (offs[nb] > (1 << 30)) return fail(DBSA_ERR_INVALID_ARG, "context too long");
+  return DBSA_OK;
+}
+
+float scale_log2(const dbsa_config *cfg) {
+  const double s = cfg->softmax_scale > 0.f ? (double)cfg->softmax_scale
+                                            : 1.0 / std::sqrt((double)cfg->head_dim);
+  return (float)(s * 1.4426950408889634);  // * log2(e)
+}
+
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return 148;
+  return n;
+}
+
+// -------------------------------------------------------------- Stage-1 plan
+// Key ranges (positions [rs, re)) a block may attend to before the causal
+// clip, in processing order: the sink first, then the contiguous window that
+// ends with the block itself.  [DBSA notes] §Stage 1, item 2 and §Ablations.
+int key_ranges(int pattern, int j, const int32_t *offs, int b, int32_t rs[2], int32_t re[2]) {
+  const bool sink = pattern == DBSA_PATTERN_SINK_PREV_SELF || pattern == DBSA_PATTERN_SINK_SELF;
+  int w0;
+  if (pattern == DBSA_PATTERN_SINK_PREV_SELF) w0 = std::max(0, b - j);
+  else if (pattern == DBSA_PATTERN_FULL) w0 = 0;
+  else w0 = b;
+  if (!sink || w0 <= 1) {
+    rs[0] = offs[sink ? 0 : w0];
+    re[0] = offs[b + 1];
+    return 1;
+  }
+  rs[0] = offs[0];
+  re[0] = offs[1];
+  rs[1] = offs[w0];
+  re[1] = offs[b + 1];
+  return 2;
+}
+
+int64_t tiles_of(const dbsa_tile_item &it) {
+  int64_t n = 0;
+  for (int r = 0; r < it.n_ranges; ++r) n += (it.len[r] + kTileKeys - 1) / kTileKeys;
+  return n;
+}
+
+// Items of one block: one per (query head, 128-row tile).  Rows of the tile
+// at positions q_pos0.., stored at rows q_row0.. of q / out.  Key rows of
+// range r start at k_row_of[r] in the rotated-K buffer, v_row_of[r] in V.
+void block_items(const dbsa_config *cfg, const int32_t *offs, int b, int32_t q_row_shift,
+                 const int32_t k_row_of[2], const int32_t v_row_of[2], int nr, const int32_t rs[2],
+                 const int32_t re[2], std::vector<dbsa_tile_item> &items) {
+  const int Hq = cfg->n_q_heads, Hkv = cfg->n_kv_heads, g = Hq / Hkv;
+  const int L = offs[b + 1] - offs[b];
+  const int n_qt = (L + kTileRows - 1) / kTileRows;
+  for (int c = 0; c < Hkv; ++c)
+    for (int m = 0; m < n_qt; ++m)
+      for (int hl = 0; hl < g; ++hl) {
+        dbsa_tile_item it;
+        std::memset(&it, 0, sizeof it);
+        it.head = c * g + hl;
+        it.q_pos0 = offs[b] + m * kTileRows;
+        it.q_row0 = it.q_pos0 - q_row_shift;
+        it.n_rows = std::min(kTileRows, offs[b + 1] - it.q_pos0);
+        it.block = b;
+        const int32_t qend = it.q_pos0 + it.n_rows;
+        int n = 0;
+        for (int r = 0; r < nr; ++r) {
+          const int32_t e = std::min(re[r], qend);
+          if (e <= rs[r]) continue;
+          it.k_row0[n] = k_row_of[r];
+          it.v_row0[n] = v_row_of[r];
+          it.pos0[n] = rs[r];
+          it.len[n] = e - rs[r];
+          ++n;
+        }
+        it.n_ranges = n;
+        items.push_back(it);
+      }
+}
+
+// The encode tile list: blocks in decreasing order of work (the light blocks
+// at the start of the context go last), then KV head, query tile, query head
+// so that neighbouring CTAs share K/V tiles in L2.
+void encode_items(const dbsa_config *cfg, const int32_t *offs, int32_t nb,
+                  std::vector<dbsa_tile_item> &items) {
+  std::vector<std::pair<int64_t, int>> order;
+  for (int b = 0; b < nb; ++b) {
+    int32_t rs[2], re[2];
+    const int nr = key_ranges(cfg->pattern, cfg->window_j, offs, b, rs, re);
+    int64_t keys = 0;
+    for (int r = 0; r < nr; ++r) keys += re[r] - rs[r];
+    order.push_back({-keys * (offs[b + 1] - offs[b]), b});
+  }
+  std::stable_sort(order.begin(), order.end(),
+                   [](const auto &x, const auto &y) { return x.first < y.first; });
+  for (const auto &ob : order) {
+    const int b = ob.second;
+    int32_t rs[2], re[2];
+    const int nr = key_ranges(cfg->pattern, cfg->window_j, offs, b, rs, re);
+    block_items(cfg, offs, b, 0, rs, rs, nr, rs, re, items);
+  }
+}
+
+// Append plan: the new block nb (positions T0..T0+L-1) attends to ranges of
+// the extended offset table; the rotated keys of those ranges are packed
+// contiguously ("compact rows").
+struct AppendPlan {
+  std::vector<int32_t> offs;  // extended, nb + 2 entries
+  int nr;
+  int32_t rs[2], re[2], cs[2];
+  int32_t k_rows;             // compact rows
+  int32_t new_row;            // compact row of position T0
+};
+AppendPlan append_plan(const dbsa_config *cfg, const int32_t *offs, int32_t nb, int32_t L) {
+  AppendPlan p;
+  p.offs.assign(offs, offs + nb + 1);
+  p.offs.push_back(offs[nb] + L);
+  p.nr = key_ranges(cfg->pattern, cfg->window_j, p.offs.data(), nb, p.rs, p.re);
+  p.cs[0] = 0;
+  p.cs[1] = p.re[0] - p.rs[0];
+  p.k_rows = 0;
+  for (int r = 0; r < p.nr; ++r) p.k_rows += p.re[r] - p.rs[r];
+  const int rl = p.nr - 1;  // the last range holds the new block
+  p.new_row = p.cs[rl] + (offs[nb] - p.rs[rl]);
+  return p;
+}
+
+// -------------------------------------------------------------- Stage-2 plan
+struct GatherPlan {
+  std::vector<S2Query> queries;
+  std::vector<S2Segment> segs;
+  std::vector<S2Item> items;
+  int32_t max_pos;  // largest key / query position + 1
+};
+
+dbsa_status gather_plan(const dbsa_config *cfg, const int32_t *offs, int32_t nb, int32_t nq,
+                        const int32_t *sel_ptr, const int32_t *sel, int32_t n_new,
+                        int32_t tail_len, GatherPlan &gp) {
+  if (nq < 1) return fail(DBSA_ERR_INVALID_ARG, "nq must be >= 1");
+  if (sel_ptr == nullptr || sel == nullptr) return fail(DBSA_ERR_INVALID_ARG, "selection is NULL");
+  if (sel_ptr[0] != 0) return fail(DBSA_ERR_INVALID_ARG, "sel_ptr[0] must be 0");
+  if (n_new < 1 || tail_len < n_new)
+    return fail(DBSA_ERR_INVALID_ARG, "need 1 <= n_new <= tail_len (n_new=%d tail_len=%d)", n_new,
+                tail_len);
+  const int g = cfg->n_q_heads / cfg->n_kv_heads;
+  const int R = g * n_new;
+  std::vector<char> seen(nb, 0);
+  int64_t total_keys = 0;
+  gp.max_pos = 0;
+  for (int q = 0; q < nq; ++q) {
+    const int32_t a = sel_ptr[q], e = sel_ptr[q + 1];
+    if (e <= a) return fail(DBSA_ERR_INVALID_ARG, "query %d selects no block", q);
+    if (sel[a] != 0) return fail(DBSA_ERR_INVALID_ARG, "query %d: first block must be the sink (0)", q);
+    S2Query qi;
+    std::memset(&qi, 0, sizeof qi);
+    qi.seg_begin = (int32_t)gp.segs.size();
+    qi.n_seg = e - a;
+    int64_t p = 0;
+    for (int32_t i = a; i < e; ++i) {
+      const int32_t b = sel[i];
+      if (b < 0 || b >= nb) return fail(DBSA_ERR_INVALID_ARG, "query %d: block %d out of range", q, b);
+      if (seen[b]) return fail(DBSA_ERR_INVALID_ARG, "query %d: block %d selected twice", q, b);
+      seen[b] = 1;
+      S2Segment s;
+      s.cache_row0 = offs[b];
+      s.pos0 = (int32_t)p;
+      s.len = offs[b + 1] - offs[b];
+      s.pad = 0;
+      gp.segs.push_back(s);
+      p += s.len;
+    }
+    for (int32_t i = a; i < e; ++i) seen[sel[i]] = 0;
+    if (p + tail_len > (1 << 30)) return fail(DBSA_ERR_INVALID_ARG, "gathered context too long");
+    qi.n_gathered = (int32_t)p;
+    total_keys += p + tail_len;
+    gp.max_pos = std::max<int32_t>(gp.max_pos, (int32_t)(p + tail_len));
+    gp.queries.push_back(qi);
+  }
+  // split size: >= 33 keys per query row (bounds the partial-result traffic
+  // to ~3 % of the K/V bytes) and enough CTAs for ~4 waves at 2 CTAs / SM
+  const int zdim = (R <= 16) ? 1 : (R + kS2MaxRows - 1) / kS2MaxRows;
+  const int64_t min_chunk = std::max<int64_t>(256, (int64_t)33 * R);
+  const int64_t want_ctas = (int64_t)8 * num_sms();
+  const int64_t par_chunk =
+      (total_keys * cfg->n_kv_heads * zdim + want_ctas - 1) / std::max<int64_t>(1, want_ctas);
+  int64_t chunk = std::max(min_chunk, par_chunk);
+  chunk = (chunk + kS2Keys - 1) / kS2Keys * kS2Keys;
+  for (int q = 0; q < nq; ++q) {
+    S2Query &qi = gp.queries[q];
+    const int64_t K = (int64_t)qi.n_gathered + tail_len;
+    const int64_t n_split = std::max<int64_t>(1, (K + chunk - 1) / chunk);
+    int64_t per = (K + n_split - 1) / n_split;
+    per = (per + kS2Keys - 1) / kS2Keys * kS2Keys;
+    qi.item_begin = (int32_t)gp.items.size();
+    for (int64_t s0 = 0; s0 < K; s0 += per) {
+      S2Item it;
+      it.query = q;
+      it.p_begin = (int32_t)s0;
+      it.p_end = (int32_t)std::min<int64_t>(K, s0 + per);
+      it.pad = 0;
+      gp.items.push_back(it);
+    }
+    qi.n_items = (int32_t)gp.items.size() - qi.item_begin;
+  }
+  return DBSA_OK;
+}
+
+// -------------------------------------------------------------- workspace layouts
+struct S1Layout {
+  size_t hi, lo, items, q_rot, k_rot, v_bf16, total;
+  int32_t n_hi;
+};
+S1Layout s1_layout(const dbsa_config *cfg, int64_t max_pos, int64_t n_items, int64_t q_rows,
+                   int64_t k_rows) {
+  S1Layout l;
+  Carve cv;
+  const int64_t half = cfg->head_dim / 2;
+  l.n_hi = (int32_t)(std::max<int64_t>(max_pos - 1, 0) / kRopeLo + 1);
+  l.hi = cv.take((size_t)l.n_hi * half * sizeof(float2));
+  l.lo = cv.take((size_t)kRopeLo * half * sizeof(float2));
+  l.items = cv.take((size_t)n_items * sizeof(dbsa_tile_item));
+  l.q_rot = cv.take((size_t)cfg->n_q_heads * q_rows * cfg->head_dim * 2);
+  l.k_rot = cv.take((size_t)cfg->n_kv_heads * k_rows * cfg->head_dim * 2);
+  l.v_bf16 = cfg->dtype == DBSA_F32 ? cv.take((size_t)cfg->n_kv_heads * k_rows * cfg->head_dim * 2)
+                                    : 0;
+  l.total = cv.total();
+  return l;
+}
+
+struct S2Layout {
+  size_t hi, lo, queries, segs, items, part_acc, part_ml, total;
+  int32_t n_hi;
+};
+S2Layout s2_layout(const dbsa_config *cfg, const GatherPlan &gp, int32_t n_new) {
+  S2Layout l;
+  Carve cv;
+  const int64_t half = cfg->head_dim / 2;
+  l.n_hi = (int32_t)(std::max<int64_t>(gp.max_pos - 1, 0) / kRopeLo + 1);
+  l.hi = cv.take((size_t)l.n_hi * half * sizeof(float2));
+  l.lo = cv.take((size_t)kRopeLo * half * sizeof(float2));
+  l.queries = cv.take(gp.queries.size() * sizeof(S2Query));
+  l.segs = cv.take(gp.segs.size() * sizeof(S2Segment));
+  l.items = cv.take(gp.items.size() * sizeof(S2Item));
+  const size_t rows = gp.items.size() * (size_t)cfg->n_q_heads * n_new;
+  l.part_acc = cv.take(rows * cfg->head_dim * sizeof(float));
+  l.part_ml = cv.take(rows * sizeof(float2));
+  l.total = cv.total();
+  return l;
+}
+
+dbsa_status check_ws(void *ws, size_t ws_bytes, size_t need) {
+  if (ws == nullptr) return fail(DBSA_ERR_WORKSPACE, "workspace is NULL");
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+    return fail(DBSA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  if (ws_bytes < need)
+    return fail(DBSA_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", ws_bytes, need);
+  return DBSA_OK;
+}
+
+template <typename T>
+T *at(void *ws, size_t off) {
+  return reinterpret_cast<T *>(static_cast<uint8_t *>(ws) + off);
+}
+
+RopeTables tables_at(void *ws, size_t hi, size_t lo, int32_t n_hi) {
+  RopeTables t;
+  t.hi = at<float2>(ws, hi);
+  t.lo = at<float2>(ws, lo);
+  t.n_hi = n_hi;
+  return t;
+}
+
+int64_t encode_item_bound(const dbsa_config *cfg, int64_t T, int32_t nb) {
+  return (int64_t)cfg->n_q_heads * ((T + kTileRows - 1) / kTileRows + nb);
+}
+
+}  // namespace
+
+// ============================================================== public ABI
+extern "C" {
+
+const char *dbsa_version(void) { return "dbsa-b200 0.1 (sm_100a)"; }
+
+const char *dbsa_last_error(void) { return g_err.c_str(); }
+
+int64_t dbsa_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
+void dbsa_set_profile_events(void *start, void *stop) {
+  g_prof_start = static_cast<cudaEvent_t>(start);
+  g_prof_stop = static_cast<cudaEvent_t>(stop);
+}
+
+int32_t dbsa_group_blocks(const int32_t *demo_len, int32_t n_demos, int32_t k, int32_t *offs_out) {
+  if (demo_len == nullptr || offs_out == nullptr || n_demos <= 0 || k <= 0) {
+    fail(DBSA_ERR_INVALID_ARG, "group_blocks: bad arguments");
+    return -1;
+  }
+  const int32_t nb = (n_demos + k - 1) / k;
+  int64_t acc = 0;
+  offs_out[0] = 0;
+  for (int32_t i = 0; i < n_demos; ++i) {
+    if (demo_len[i] < 1) {
+      fail(DBSA_ERR_INVALID_ARG, "group_blocks: demonstration %d has no tokens", i);
+      return -1;
+    }
+    acc += demo_len[i];
+    if (acc > (1 << 30)) {
+      fail(DBSA_ERR_INVALID_ARG, "group_blocks: context too long");
+      return -1;
+    }
+    if ((i + 1) % k == 0 || i + 1 == n_demos) offs_out[(i + k) / k] = (int32_t)acc;
+  }
+  return nb;
+}
+
+int64_t dbsa_stage1_plan(const dbsa_config *cfg, const int32_t *offs_host, int32_t nb,
+                         dbsa_tile_item *items, int64_t max_items) {
+  if (check_cfg(cfg) != DBSA_OK || check_offs(offs_host, nb) != DBSA_OK) return -1;
+  std::vector<dbsa_tile_item> v;
+  encode_items(cfg, offs_host, nb, v);
+  if (items != nullptr)
+    std::memcpy(items, v.data(), sizeof(dbsa_tile_item) * (size_t)std::min<int64_t>(max_items, v.size()));
+  return (int64_t)v.size();
+}
+
+int64_t dbsa_stage1_tile_count(const dbsa_config *cfg, const int32_t *offs_host, int32_t nb) {
+  if (check_cfg(cfg) != DBSA_OK || check_offs(offs_host, nb) != DBSA_OK) return -1;
+  std::vector<dbsa_tile_item> v;
+  encode_items(cfg, offs_host, nb, v);
+  int64_t n = 0;
+  for (const auto &it : v) n += tiles_of(it);
+  return n;
+}
+
+size_t dbsa_encode_workspace_size(const dbsa_config *cfg, int64_t n_tokens, int32_t nb) {
+  if (check_cfg(cfg) != DBSA_OK || n_tokens <= 0 || nb <= 0) return 0;
+  return s1_layout(cfg, n_tokens, encode_item_bound(cfg, n_tokens, nb), n_tokens, n_tokens).total;
+}
+
+dbsa_status dbsa_encode_blocks(const dbsa_config *cfg, const void *q, const void *k,
+                               const void *v, const int32_t *offs_host, int32_t nb,
+                               void *k_cache, void *v_cache, int64_t cap, void *out,
+                               void *workspace, size_t ws_bytes, void *stream) {
+  dbsa_status s = check_cfg(cfg);
+  if (s != DBSA_OK) return s;
+  if ((s = check_offs(offs_host, nb)) != DBSA_OK) return s;
+  if (!q || !k || !v || !k_cache || !v_cache || !out)
+    return fail(DBSA_ERR_INVALID_ARG, "a tensor pointer is NULL");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(k_cache) ||
+      !aligned16(v_cache) || !aligned16(out))
+    return fail(DBSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  const int64_t T = offs_host[nb];
+  if (cap < T) return fail(DBSA_ERR_CAPACITY, "cache capacity %lld < %lld tokens", (long long)cap,
+                           (long long)T);
+  std::vector<dbsa_tile_item> items;
+  encode_items(cfg, offs_host, nb, items);
+  const S1Layout L = s1_layout(cfg, T, encode_item_bound(cfg, T, nb), T, T);
+  if ((s = check_ws(workspace, ws_bytes, L.total)) != DBSA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool f32 = cfg->dtype == DBSA_F32;
+  cudaError_t e;
+  if ((e = cudaMemsetAsync(workspace, 0, kStatusBytes, st)) != cudaSuccess)
+    return cuda_fail(e, "status clear");
+  const RopeTables rope = tables_at(workspace, L.hi, L.lo, L.n_hi);
+  if ((e = launch_rope_tables(const_cast<float2 *>(rope.hi), L.n_hi,
+                              const_cast<float2 *>(rope.lo), cfg->head_dim, cfg->rope_theta, st)) !=
+      cudaSuccess)
+    return cuda_fail(e, "rope tables");
+  count_launches(1);
+  if ((e = cudaMemcpyAsync(at<void>(workspace, L.items), items.data(),
+                           items.size() * sizeof(dbsa_tile_item), cudaMemcpyHostToDevice, st)) !=
+      cudaSuccess)
+    return cuda_fail(e, "tile list upload");
+  IngestArgs ia;
+  ia.q = q;
+  ia.k = k;
+  ia.v = v;
+  ia.n_tok = (int32_t)T;
+  ia.pos0 = 0;
+  ia.Hq = cfg->n_q_heads;
+  ia.Hkv = cfg->n_kv_heads;
+  ia.q_rot = at<void>(workspace, L.q_rot);
+  ia.q_rows = T;
+  ia.q_row_base = 0;
+  ia.k_rot = at<void>(workspace, L.k_rot);
+  ia.k_rows = T;
+  ia.k_row_base = 0;
+  ia.v_bf16 = f32 ? at<void>(workspace, L.v_bf16) : nullptr;
+  ia.k_cache = k_cache;
+  ia.v_cache = v_cache;
+  ia.cap = cap;
+  ia.rope = rope;
+  if ((e = launch_ingest(ia, cfg->head_dim, f32, st)) != cudaSuccess) return cuda_fail(e, "ingest");
+  count_launches(1);
+  Stage1Args sa;
+  sa.q_rot = ia.q_rot;
+  sa.q_rows = T;
+  sa.k_rot = ia.k_rot;
+  sa.k_rows = T;
+  sa.v = f32 ? ia.v_bf16 : v_cache;
+  sa.v_rows = T;
+  sa.v_head_stride = f32 ? T : cap;
+  sa.out = out;
+  sa.Hq = cfg->n_q_heads;
+  sa.Hkv = cfg->n_kv_heads;
+  sa.items = at<dbsa_tile_item>(workspace, L.items);
+  sa.n_items = (int32_t)items.size();
+  sa.scale_log2 = scale_log2(cfg);
+  sa.status = at<int>(workspace, 0);
+  {
+    ProfileScope prof(st);
+    e = launch_stage1(sa, cfg->head_dim, f32, num_sms(), st);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "stage-1 attention");
+  count_launches(1);
+  return DBSA_OK;
+}
+
+size_t dbsa_append_workspace_size(const dbsa_config *cfg, const int32_t *offs_host, int32_t nb,
+                                  int32_t L) {
+  if (check_cfg(cfg) != DBSA_OK || check_offs(offs_host, nb) != DBSA_OK || L < 1) return 0;
+  const AppendPlan ap = append_plan(cfg, offs_host, nb, L);
+  const int64_t n_items = (int64_t)cfg->n_q_heads * ((L + kTileRows - 1) / kTileRows);
+  return s1_layout(cfg, (int64_t)offs_host[nb] + L, n_items, L, ap.k_rows).total;
+}
+
+dbsa_status dbsa_append_block(const dbsa_config *cfg, const void *q, const void *k, const void *v,
+                              int32_t L, const int32_t *offs_host, int32_t nb, void *k_cache,
+                              void *v_cache, int64_t cap, void *out, void *workspace,
+                              size_t ws_bytes, void *stream) {
+  dbsa_status s = check_cfg(cfg);
+  if (s != DBSA_OK) return s;
+  if ((s = check_offs(offs_host, nb)) != DBSA_OK) return s;
+  if (L < 1) return fail(DBSA_ERR_INVALID_ARG, "the new block needs at least one token");
+  if (!q || !k || !v || !k_cache || !v_cache || !out)
+    return fail(DBSA_ERR_INVALID_ARG, "a tensor pointer is NULL");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(k_cache) ||
+      !aligned16(v_cache) || !aligned16(out))
+    return fail(DBSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  const int64_t T0 = offs_host[nb];
+  if (T0 + L > (1 << 30)) return fail(DBSA_ERR_INVALID_ARG, "context too long");
+  if (cap < T0 + L)
+    return fail(DBSA_ERR_CAPACITY, "cache capacity %lld < %lld tokens", (long long)cap,
+                (long long)(T0 + L));
+  const AppendPlan ap = append_plan(cfg, offs_host, nb, L);
+  const bool f32 = cfg->dtype == DBSA_F32;
+  std::vector<dbsa_tile_item> items;
+  {
+    int32_t krow[2] = {ap.cs[0], ap.cs[1]};
+    int32_t vrow[2];
+    for (int r = 0; r < 2; ++r) vrow[r] = f32 ? ap.cs[r] : ap.rs[r];
+    block_items(cfg, ap.offs.data(), nb, (int32_t)T0, krow, vrow, ap.nr, ap.rs, ap.re, items);
+  }
+  const int64_t n_items_bound = (int64_t)cfg->n_q_heads * ((L + kTileRows - 1) / kTileRows);
+  const S1Layout Ly = s1_layout(cfg, T0 + L, n_items_bound, L, ap.k_rows);
+  if ((s = check_ws(workspace, ws_bytes, Ly.total)) != DBSA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if ((e = cudaMemsetAsync(workspace, 0, kStatusBytes, st)) != cudaSuccess)
+    return cuda_fail(e, "status clear");
+  const RopeTables rope = tables_at(workspace, Ly.hi, Ly.lo, Ly.n_hi);
+  if ((e = launch_rope_tables(const_cast<float2 *>(rope.hi), Ly.n_hi,
+                              const_cast<float2 *>(rope.lo), cfg->head_dim, cfg->rope_theta, st)) !=
+      cudaSuccess)
+    return cuda_fail(e, "rope tables");
+  count_launches(1);
+  if ((e = cudaMemcpyAsync(at<void>(workspace, Ly.items), items.data(),
+                           items.size() * sizeof(dbsa_tile_item), cudaMemcpyHostToDevice, st)) !=
+      cudaSuccess)
+    return cuda_fail(e, "tile list upload");
+  void *k_rot = at<void>(workspace, Ly.k_rot);
+  void *v_bf16 = f32 ? at<void>(workspace, Ly.v_bf16) : nullptr;
+  // window rows already in the cache
+  for (int r = 0; r < ap.nr; ++r) {
+    const int32_t e_in_cache = std::min<int32_t>(ap.re[r], (int32_t)T0);
+    if (e_in_cache <= ap.rs[r]) continue;
+    WindowArgs wa;
+    wa.k_cache = k_cache;
+    wa.v_cache = v_cache;
+    wa.cap = cap;
+    wa.Hkv = cfg->n_kv_heads;
+    wa.row0 = ap.rs[r];
+    wa.n = e_in_cache - ap.rs[r];
+    wa.k_rot = k_rot;
+    wa.k_rows = ap.k_rows;
+    wa.dst_row0 = ap.cs[r];
+    wa.v_bf16 = v_bf16;
+    wa.rope = rope;
+    if ((e = launch_window(wa, cfg->head_dim, f32, st)) != cudaSuccess)
+      return cuda_fail(e, "window rotation");
+    count_launches(1);
+  }
+  IngestArgs ia;
+  ia.q = q;
+  ia.k = k;
+  ia.v = v;
+  ia.n_tok = L;
+  ia.pos0 = (int32_t)T0;
+  ia.Hq = cfg->n_q_heads;
+  ia.Hkv = cfg->n_kv_heads;
+  ia.q_rot = at<void>(workspace, Ly.q_rot);
+  ia.q_rows = L;
+  ia.q_row_base = 0;
+  ia.k_rot = k_rot;
+  ia.k_rows = ap.k_rows;
+  ia.k_row_base = ap.new_row;
+  ia.v_bf16 = v_bf16;
+  ia.k_cache = k_cache;
+  ia.v_cache = v_cache;
+  ia.cap = cap;
+  ia.rope = rope;
+  if ((e = launch_ingest(ia, cfg->head_dim, f32, st)) != cudaSuccess) return cuda_fail(e, "ingest");
+  count_launches(1);
+  Stage1Args sa;
+  sa.q_rot = ia.q_rot;
+  sa.q_rows = L;
+  sa.k_rot = k_rot;
+  sa.k_rows = ap.k_rows;
+  sa.v = f32 ? v_bf16 : v_cache;
+  sa.v_rows = f32 ? ap.k_rows : T0 + L;
+  sa.v_head_stride = f32 ? ap.k_rows : cap;
+  sa.out = out;
+  sa.Hq = cfg->n_q_heads;
+  sa.Hkv = cfg->n_kv_heads;
+  sa.items = at<dbsa_tile_item>(workspace, Ly.items);
+  sa.n_items = (int32_t)items.size();
+  sa.scale_log2 = scale_log2(cfg);
+  sa.status = at<int>(workspace, 0);
+  {
+    ProfileScope prof(st);
+    e = launch_stage1(sa, cfg->head_dim, f32, num_sms(), st);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "stage-1 attention");
+  count_launches(1);
+  return DBSA_OK;
+}
+
+size_t dbsa_gather_workspace_size(const dbsa_config *cfg, const int32_t *offs_host, int32_t nb,
+                                  int32_t nq, const int32_t *sel_ptr_host,
+                                  const int32_t *sel_blocks_host, int32_t n_new,
+                                  int32_t tail_len) {
+  if (check_cfg(cfg) != DBSA_OK || check_offs(offs_host, nb) != DBSA_OK) return 0;
+  GatherPlan gp;
+  if (gather_plan(cfg, offs_host, nb, nq, sel_ptr_host, sel_blocks_host, n_new, tail_len, gp) !=
+      DBSA_OK)
+    return 0;
+  return s2_layout(cfg, gp, n_new).total;
+}
+
+dbsa_status dbsa_gather_rope_attend(const dbsa_config *cfg, const void *k_cache,
+                                    const void *v_cache, int64_t cap, const int32_t *offs_host,
+                                    int32_t nb, int32_t nq, const int32_t *sel_ptr_host,
+                                    const int32_t *sel_blocks_host, const void *q_new,
+                                    int32_t n_new, const void *k_tail, const void *v_tail,
+                                    int32_t tail_len, int32_t tail_cap, void *out,
+                                    int32_t *dbg_map, int64_t dbg_cap, void *workspace,
+                                    size_t ws_bytes, void *stream) {
+  dbsa_status s = check_cfg(cfg);
+  if (s != DBSA_OK) return s;
+  if ((s = check_offs(offs_host, nb)) != DBSA_OK) return s;
+  if (!k_cache || !v_cache || !q_new || !k_tail || !v_tail || !out)
+    return fail(DBSA_ERR_INVALID_ARG, "a tensor pointer is NULL");
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(q_new) || !aligned16(k_tail) ||
+      !aligned16(v_tail) || !aligned16(out))
+    return fail(DBSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  if (tail_len > tail_cap)
+    return fail(DBSA_ERR_INVALID_ARG, "tail_len %d > tail_cap %d", tail_len, tail_cap);
+  if (offs_host[nb] > cap)
+    return fail(DBSA_ERR_CAPACITY, "offsets reach %d rows but cap is %lld", offs_host[nb],
+                (long long)cap);
+  GatherPlan gp;
+  if ((s = gather_plan(cfg, offs_host, nb, nq, sel_ptr_host, sel_blocks_host, n_new, tail_len,
+                       gp)) != DBSA_OK)
+    return s;
+  if (dbg_map != nullptr) {
+    if ((reinterpret_cast<uintptr_t>(dbg_map) & 7u) != 0)
+      return fail(DBSA_ERR_INVALID_ARG, "dbg_map must be 8-byte aligned");
+    for (const auto &qi : gp.queries)
+      if (qi.n_gathered > dbg_cap)
+        return fail(DBSA_ERR_INVALID_ARG, "dbg_cap %lld < gathered tokens %d", (long long)dbg_cap,
+                    qi.n_gathered);
+  }
+  const S2Layout L = s2_layout(cfg, gp, n_new);
+  if ((s = check_ws(workspace, ws_bytes, L.total)) != DBSA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if ((e = cudaMemsetAsync(workspace, 0, kStatusBytes, st)) != cudaSuccess)
+    return cuda_fail(e, "status clear");
+  const RopeTables rope = tables_at(workspace, L.hi, L.lo, L.n_hi);
+  if ((e = launch_rope_tables(const_cast<float2 *>(rope.hi), L.n_hi,
+                              const_cast<float2 *>(rope.lo), cfg->head_dim, cfg->rope_theta, st)) !=
+      cudaSuccess)
+    return cuda_fail(e, "rope tables");
+  count_launches(1);
+  // one upload of the three small plan arrays (they are contiguous in the carve)
+  {
+    std::vector<uint8_t> blob(L.part_acc - L.queries, 0);
+    std::memcpy(blob.data(), gp.queries.data(), gp.queries.size() * sizeof(S2Query));
+    std::memcpy(blob.data() + (L.segs - L.queries), gp.segs.data(),
+                gp.segs.size() * sizeof(S2Segment));
+    std::memcpy(blob.data() + (L.items - L.queries), gp.items.data(),
+                gp.items.size() * sizeof(S2Item));
+    if ((e = cudaMemcpyAsync(at<void>(workspace, L.queries), blob.data(), blob.size(),
+                             cudaMemcpyHostToDevice, st)) != cudaSuccess)
+      return cuda_fail(e, "gather plan upload");
+  }
+  Stage2Args a;
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+  a.cap = cap;
+  a.q_new = q_new;
+  a.k_tail = k_tail;
+  a.v_tail = v_tail;
+  a.tail_len = tail_len;
+  a.tail_cap = tail_cap;
+  a.n_new = n_new;
+  a.Hq = cfg->n_q_heads;
+  a.Hkv = cfg->n_kv_heads;
+  a.queries = at<S2Query>(workspace, L.queries);
+  a.segs = at<S2Segment>(workspace, L.segs);
+  a.items = at<S2Item>(workspace, L.items);
+  a.n_items = (int32_t)gp.items.size();
+  a.n_queries = nq;
+  a.part_acc = at<float>(workspace, L.part_acc);
+  a.part_ml = at<float2>(workspace, L.part_ml);
+  a.out = out;
+  a.dbg_map = dbg_map;
+  a.dbg_cap = dbg_cap;
+  a.scale_log2 = scale_log2(cfg);
+  a.rope = rope;
+  {
+    ProfileScope prof(st);
+    e = launch_stage2_main(a, cfg->head_dim, cfg->dtype == DBSA_F32, st);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "stage-2 attention");
+  count_launches(1);
+  if ((e = launch_stage2_merge(a, cfg->head_dim, cfg->dtype == DBSA_F32, st)) != cudaSuccess)
+    return cuda_fail(e, "stage-2 merge");
+  count_launches(1);
+  return DBSA_OK;
+}
+
+dbsa_status dbsa_read_status(const void *workspace, void *stream) {
+  if (workspace == nullptr) return fail(DBSA_ERR_INVALID_ARG, "workspace is NULL");
+  int word = 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof word, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "status read");
+  if (word == DBSA_ERR_TIMEOUT) {
+    fail(DBSA_ERR_TIMEOUT, "a device-side wait expired");
+    return DBSA_ERR_TIMEOUT;
+  }
+  return word == 0 ? DBSA_OK : (dbsa_status)word;
+}
+
+}  // extern "C"

@@ -1,0 +1,134 @@
+// Internal declarations of the DBSA library: device-visible plan structs and
+// the launchers each kernel file provides.  Not part of the public ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+#include "../../include/dbsa.h"
+
+namespace dbsa {
+
+constexpr int kTileRows = 128;   // Stage-1 query rows per tile (tcgen05 M)
+constexpr int kTileKeys = 128;   // Stage-1 keys per score tile (tcgen05 N)
+constexpr int kRopeLo = 64;      // positions per RoPE "hi" table step
+constexpr int kS2Keys = 64;      // Stage-2 keys per tile
+constexpr int kS2MaxRows = 64;   // Stage-2 query rows per CTA (4 warps x 16)
+
+// Head of every workspace: the device status word (cleared by each call).
+constexpr size_t kStatusBytes = 256;
+
+// RoPE angle factors, built on the device in fp64 and stored as fp32
+// (cos, sin) pairs: hi[a][i] = e^{i * 64a * w_i}, lo[r][i] = e^{i * r * w_i},
+// w_i = theta^(-2i/D).  Position p uses hi[p >> 6] * lo[p & 63].
+struct RopeTables {
+  const float2 *hi;
+  const float2 *lo;
+  int32_t n_hi;
+};
+
+// Stage 2: per-query metadata, gathered segments and split items.
+struct S2Segment {
+  int32_t cache_row0;  // first cache row of the block
+  int32_t pos0;        // fresh position of its first token
+  int32_t len;         // tokens
+  int32_t pad;
+};
+struct S2Query {
+  int32_t seg_begin;   // index into the segment array
+  int32_t n_seg;
+  int32_t n_gathered;  // T'_q
+  int32_t item_begin;  // first split item of this query
+  int32_t n_items;
+  int32_t pad[3];
+};
+struct S2Item {
+  int32_t query;
+  int32_t p_begin;     // key positions [p_begin, p_end) of the query's key sequence
+  int32_t p_end;
+  int32_t pad;
+};
+
+// ---- launchers (each returns cudaGetLastError() after enqueueing) ----
+
+cudaError_t launch_rope_tables(float2 *hi, int32_t n_hi, float2 *lo, int32_t head_dim,
+                               double theta, cudaStream_t st);
+
+// Rotate Q and K of n_tok token-major input rows (positions pos0..), copy the
+// raw K/V into the cache rows pos0.., and (f32 inputs) write bf16 V.
+struct IngestArgs {
+  const void *q, *k, *v;           // [n_tok][H][D] input dtype
+  int32_t n_tok, pos0;
+  int32_t Hq, Hkv;
+  void *q_rot;                     // bf16 [Hq][q_rows][D], row q_row_base + t
+  int64_t q_rows;
+  int32_t q_row_base;
+  void *k_rot;                     // bf16 [Hkv][k_rows][D], row k_row_base + t
+  int64_t k_rows;
+  int32_t k_row_base;
+  void *v_bf16;                    // bf16 [Hkv][k_rows][D] (f32 inputs only) or null
+  void *k_cache, *v_cache;         // input dtype [Hkv][cap][D], row pos0 + t
+  int64_t cap;
+  RopeTables rope;
+};
+cudaError_t launch_ingest(const IngestArgs &a, int head_dim, bool f32, cudaStream_t st);
+
+// Rotate cache rows [row0, row0+n) (positions = rows) into k_rot rows
+// dst_row0.. and (f32) convert the V rows to bf16 scratch rows.
+struct WindowArgs {
+  const void *k_cache, *v_cache;
+  int64_t cap;
+  int32_t Hkv;
+  int32_t row0, n;
+  void *k_rot;
+  int64_t k_rows;
+  int32_t dst_row0;
+  void *v_bf16;
+  RopeTables rope;
+};
+cudaError_t launch_window(const WindowArgs &a, int head_dim, bool f32, cudaStream_t st);
+
+// Stage-1 tcgen05 attention over a tile list.
+struct Stage1Args {
+  const void *q_rot;      // bf16 [Hq][q_rows][D]
+  int64_t q_rows;
+  const void *k_rot;      // bf16 [Hkv][k_rows][D]
+  int64_t k_rows;
+  const void *v;          // bf16 [Hkv][v_rows] rows, head stride v_head_stride rows
+  int64_t v_rows, v_head_stride;
+  void *out;              // [out_rows][Hq][D], bf16 or f32
+  int32_t Hq, Hkv;
+  const dbsa_tile_item *items;
+  int32_t n_items;
+  float scale_log2;       // softmax scale * log2(e)
+  int *status;
+};
+cudaError_t launch_stage1(const Stage1Args &a, int head_dim, bool out_f32, int num_sms,
+                          cudaStream_t st);
+
+// Stage-2 split-KV gather + re-RoPE + attention, then the split merge.
+struct Stage2Args {
+  const void *k_cache, *v_cache;   // [Hkv][cap][D]
+  int64_t cap;
+  const void *q_new;               // [nq][n_new][Hq][D]
+  const void *k_tail, *v_tail;     // [nq][tail_cap][Hkv][D]
+  int32_t tail_len, tail_cap, n_new;
+  int32_t Hq, Hkv;
+  const S2Query *queries;
+  const S2Segment *segs;
+  const S2Item *items;
+  int32_t n_items, n_queries;
+  float *part_acc;                 // [n_items][Hq][n_new][D]
+  float2 *part_ml;                 // [n_items][Hq][n_new] (m in log2 units, l)
+  void *out;                       // [nq][n_new][Hq][D]
+  int32_t *dbg_map;                // [nq][dbg_cap][2] or null
+  int64_t dbg_cap;
+  float scale_log2;
+  RopeTables rope;
+};
+cudaError_t launch_stage2_main(const Stage2Args &a, int head_dim, bool f32, cudaStream_t st);
+cudaError_t launch_stage2_merge(const Stage2Args &a, int head_dim, bool f32, cudaStream_t st);
+
+}  // namespace dbsa

@@ -1,0 +1,176 @@
+// RoPE angle tables and the Stage-1 preparation kernels.
+//
+// [DBSA notes] §Stage 1, item 3: queries and keys are rotated at sequential
+// positions, while the cache keeps K/V BEFORE the rotary transform.  The
+// preparation pass therefore (a) copies the raw K/V into the head-major cache,
+// (b) writes a rotated bf16 copy of Q and K into the workspace for the
+// tensor-core kernel, and for fp32 inputs (c) a bf16 copy of V.  It is pure
+// streaming work (HBM-bound); the angle factors come from two small tables
+// built once per call in fp64.
+#include <cuda_bf16.h>
+
+#include "dbsa_internal.h"
+#include "vec8.cuh"
+
+namespace dbsa {
+namespace {
+
+__global__ void rope_tables_kernel(float2 *hi, int32_t n_hi, float2 *lo, int32_t half,
+                                   double theta) {
+  const int64_t n = (int64_t)(n_hi + kRopeLo) * half;
+  for (int64_t u = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; u < n;
+       u += (int64_t)gridDim.x * blockDim.x) {
+    const int32_t i = (int32_t)(u % half);
+    const int64_t row = u / half;
+    const double w = pow(theta, -2.0 * (double)i / (double)(2 * half));
+    double s, c;
+    if (row < n_hi) {
+      sincos((double)(row * kRopeLo) * w, &s, &c);
+      hi[row * half + i] = make_float2((float)c, (float)s);
+    } else {
+      const int64_t r = row - n_hi;
+      sincos((double)r * w, &s, &c);
+      lo[r * half + i] = make_float2((float)c, (float)s);
+    }
+  }
+}
+
+// One work unit = (token t, head slot hh, chunk cp): elements [8cp, 8cp+8) of
+// the first half and the matching 8 of the second half.
+template <int D, typename T>
+__global__ void __launch_bounds__(256) ingest_kernel(IngestArgs a) {
+  constexpr int H = D / 2;
+  constexpr int CP = H / 8;
+  const int slots = a.Hq + 2 * a.Hkv;
+  const int64_t n_units = (int64_t)a.n_tok * slots * CP;
+  const T *q = static_cast<const T *>(a.q);
+  const T *k = static_cast<const T *>(a.k);
+  const T *v = static_cast<const T *>(a.v);
+  for (int64_t u = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; u < n_units;
+       u += (int64_t)gridDim.x * blockDim.x) {
+    const int cp = (int)(u % CP);
+    const int hh = (int)((u / CP) % slots);
+    const int64_t t = u / ((int64_t)CP * slots);
+    const int64_t pos = a.pos0 + t;
+    const int i0 = cp * 8;
+    float lo[8], hi[8];
+    if (hh < a.Hq) {  // query head: rotate into q_rot
+      const T *src = q + (t * a.Hq + hh) * D;
+      load8(src + i0, lo);
+      load8(src + H + i0, hi);
+      float c[8], s[8];
+      rope_cs8(a.rope, pos, i0, H, c, s);
+      rotate8(lo, hi, c, s);
+      bf16 *dst = static_cast<bf16 *>(a.q_rot) + ((int64_t)hh * a.q_rows + a.q_row_base + t) * D;
+      store8_bf16(dst + i0, lo);
+      store8_bf16(dst + H + i0, hi);
+    } else if (hh < a.Hq + a.Hkv) {  // key head: cache the raw key, rotate into k_rot
+      const int c_ = hh - a.Hq;
+      const T *src = k + (t * a.Hkv + c_) * D;
+      T *cache = static_cast<T *>(a.k_cache) + ((int64_t)c_ * a.cap + pos) * D;
+      copy8(src + i0, cache + i0);
+      copy8(src + H + i0, cache + H + i0);
+      load8(src + i0, lo);
+      load8(src + H + i0, hi);
+      float c[8], s[8];
+      rope_cs8(a.rope, pos, i0, H, c, s);
+      rotate8(lo, hi, c, s);
+      bf16 *dst = static_cast<bf16 *>(a.k_rot) + ((int64_t)c_ * a.k_rows + a.k_row_base + t) * D;
+      store8_bf16(dst + i0, lo);
+      store8_bf16(dst + H + i0, hi);
+    } else {  // value head: cache the raw value (and a bf16 copy for fp32 inputs)
+      const int c_ = hh - a.Hq - a.Hkv;
+      const T *src = v + (t * a.Hkv + c_) * D;
+      T *cache = static_cast<T *>(a.v_cache) + ((int64_t)c_ * a.cap + pos) * D;
+      copy8(src + i0, cache + i0);
+      copy8(src + H + i0, cache + H + i0);
+      if (a.v_bf16 != nullptr) {
+        load8(src + i0, lo);
+        load8(src + H + i0, hi);
+        bf16 *dst =
+            static_cast<bf16 *>(a.v_bf16) + ((int64_t)c_ * a.k_rows + a.k_row_base + t) * D;
+        store8_bf16(dst + i0, lo);
+        store8_bf16(dst + H + i0, hi);
+      }
+    }
+  }
+}
+
+// Cache rows [row0, row0+n) of every KV head, at positions equal to the row.
+template <int D, typename T>
+__global__ void __launch_bounds__(256) window_kernel(WindowArgs a) {
+  constexpr int H = D / 2;
+  constexpr int CP = H / 8;
+  const int64_t n_units = (int64_t)a.n * a.Hkv * CP;
+  for (int64_t u = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; u < n_units;
+       u += (int64_t)gridDim.x * blockDim.x) {
+    const int cp = (int)(u % CP);
+    const int c_ = (int)((u / CP) % a.Hkv);
+    const int64_t r = u / ((int64_t)CP * a.Hkv);
+    const int64_t pos = a.row0 + r;
+    const int i0 = cp * 8;
+    float lo[8], hi[8], c[8], s[8];
+    const T *src = static_cast<const T *>(a.k_cache) + ((int64_t)c_ * a.cap + pos) * D;
+    load8(src + i0, lo);
+    load8(src + H + i0, hi);
+    rope_cs8(a.rope, pos, i0, H, c, s);
+    rotate8(lo, hi, c, s);
+    bf16 *dst = static_cast<bf16 *>(a.k_rot) + ((int64_t)c_ * a.k_rows + a.dst_row0 + r) * D;
+    store8_bf16(dst + i0, lo);
+    store8_bf16(dst + H + i0, hi);
+    if (a.v_bf16 != nullptr) {
+      const T *vs = static_cast<const T *>(a.v_cache) + ((int64_t)c_ * a.cap + pos) * D;
+      load8(vs + i0, lo);
+      load8(vs + H + i0, hi);
+      bf16 *vd = static_cast<bf16 *>(a.v_bf16) + ((int64_t)c_ * a.k_rows + a.dst_row0 + r) * D;
+      store8_bf16(vd + i0, lo);
+      store8_bf16(vd + H + i0, hi);
+    }
+  }
+}
+
+int grid_for(int64_t n_units, int block) {
+  int64_t g = (n_units + block - 1) / block;
+  if (g > 148 * 16) g = 148 * 16;
+  if (g < 1) g = 1;
+  return (int)g;
+}
+
+}  // namespace
+
+cudaError_t launch_rope_tables(float2 *hi, int32_t n_hi, float2 *lo, int32_t head_dim,
+                               double theta, cudaStream_t st) {
+  const int half = head_dim / 2;
+  const int64_t n = (int64_t)(n_hi + kRopeLo) * half;
+  rope_tables_kernel<<<grid_for(n, 256), 256, 0, st>>>(hi, n_hi, lo, half, theta);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ingest(const IngestArgs &a, int head_dim, bool f32, cudaStream_t st) {
+  const int64_t n = (int64_t)a.n_tok * (a.Hq + 2 * a.Hkv) * (head_dim / 16);
+  const int g = grid_for(n, 256);
+  if (head_dim == 128) {
+    if (f32) ingest_kernel<128, float><<<g, 256, 0, st>>>(a);
+    else ingest_kernel<128, bf16><<<g, 256, 0, st>>>(a);
+  } else {
+    if (f32) ingest_kernel<64, float><<<g, 256, 0, st>>>(a);
+    else ingest_kernel<64, bf16><<<g, 256, 0, st>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_window(const WindowArgs &a, int head_dim, bool f32, cudaStream_t st) {
+  if (a.n <= 0) return cudaSuccess;
+  const int64_t n = (int64_t)a.n * a.Hkv * (head_dim / 16);
+  const int g = grid_for(n, 256);
+  if (head_dim == 128) {
+    if (f32) window_kernel<128, float><<<g, 256, 0, st>>>(a);
+    else window_kernel<128, bf16><<<g, 256, 0, st>>>(a);
+  } else {
+    if (f32) window_kernel<64, float><<<g, 256, 0, st>>>(a);
+    else window_kernel<64, bf16><<<g, 256, 0, st>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace dbsa

@@ -1,0 +1,515 @@
+// Stage-1 block-sparse streaming attention on the 5th-generation tensor core.
+//
+// [DBSA notes] §Stage 1, item 2: every token of block b_i attends to the sink
+// block b_1, the previous j blocks and (causally) its own block.  The host
+// planner turns this pattern into a tile list: one item per (query head,
+// 128-row query tile inside one block), each with at most two contiguous key
+// ranges (the sink, then the window up to the diagonal).  Masked tiles are
+// never enumerated (the page's implementation skipped masked blocks with
+// Flex Attention for a speed-up proportional to the sparsity; here the list
+// holds only the tiles that contain an allowed pair).
+//
+// One persistent CTA per SM walks items round-robin.  Warp roles:
+//   warp 0      TMA producer: Q tile, then K and V tiles (2-stage ring)
+//   warp 1      TMEM owner and tcgen05.mma issuer (one thread)
+//   warps 2..5  softmax: one thread per query row (TMEM lane), fp32 online
+//               softmax with a lazy rescale threshold, P written to shared
+//               memory as bf16, final O / l epilogue
+// S = Q K^T lives in TMEM (two 128-column buffers so that the next tile's
+// QK^T overlaps this tile's softmax), O in TMEM (D columns).  Q and K arrive
+// already rotated (bf16) from the preparation pass; V is read straight from
+// the pre-RoPE cache.  Every wait is bounded and reports DBSA_ERR_TIMEOUT.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <mutex>
+
+#include "dbsa_internal.h"
+#include "sm100.cuh"
+
+namespace dbsa {
+namespace {
+
+using namespace sm100;
+
+constexpr uint64_t kWaitLimitNs = 4000000000ull;   // 4 s: far above any legitimate wait
+constexpr uint64_t kDrainLimitNs = 200000000ull;   // 0.2 s for the exit drain
+constexpr uint32_t kFull = 0xFFFFFFFFu;
+
+enum Bar {
+  B_Q_FULL = 0, B_Q_EMPTY = 1, B_K_FULL = 2, B_K_EMPTY = 4, B_V_FULL = 6, B_V_EMPTY = 8,
+  B_S_FULL = 10, B_S_FREE = 12, B_P_FULL = 14, B_PV_DONE = 16, B_O_FREE = 18, B_DRAIN = 19,
+  B_COUNT = 20
+};
+
+struct Item {
+  int head, q_row0, q_pos0, n_rows, n_ranges;
+  int k_row0[2], v_row0[2], pos0[2], len[2];
+  int nt0, ntiles;
+};
+
+__device__ __forceinline__ Item load_item(const dbsa_tile_item *items, int idx) {
+  const dbsa_tile_item *s = items + idx;
+  Item it;
+  it.head = __ldg(&s->head);
+  it.q_row0 = __ldg(&s->q_row0);
+  it.q_pos0 = __ldg(&s->q_pos0);
+  it.n_rows = __ldg(&s->n_rows);
+  it.n_ranges = __ldg(&s->n_ranges);
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    it.k_row0[r] = __ldg(&s->k_row0[r]);
+    it.v_row0[r] = __ldg(&s->v_row0[r]);
+    it.pos0[r] = __ldg(&s->pos0[r]);
+    it.len[r] = it.n_ranges > r ? __ldg(&s->len[r]) : 0;
+  }
+  it.nt0 = (it.len[0] + kTileKeys - 1) / kTileKeys;
+  it.ntiles = it.nt0 + (it.len[1] + kTileKeys - 1) / kTileKeys;
+  return it;
+}
+
+__device__ __forceinline__ void tile_of(const Item &it, int t, int &r, int &kt) {
+  if (t < it.nt0) {
+    r = 0;
+    kt = t * kTileKeys;
+  } else {
+    r = 1;
+    kt = (t - it.nt0) * kTileKeys;
+  }
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Bounded wait used on the way out: ignores the abort flag.
+__device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kDrainLimitNs) return;
+  }
+}
+
+struct Params {
+  const dbsa_tile_item *items;
+  int n_items;
+  int group;  // Hq / Hkv
+  int Hq;
+  void *out;
+  float scale_log2;
+  int *status;
+};
+
+template <int D, bool OUT_F32>
+__global__ void __launch_bounds__(192, 1)
+    stage1_attn_kernel(const __grid_constant__ CUtensorMap tmQ,
+                       const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const Params p) {
+  constexpr uint32_t HALF = 128 * 64 * 2;        // one 128-row x 64-column swizzled atom column
+  constexpr uint32_t TILE = 128 * D * 2;         // Q / K / V tile
+  constexpr uint32_t PTILE = 128 * 128 * 2;      // P tile (128 rows x 128 keys)
+  constexpr int NH = D / 64;                     // 64-column halves per row
+  constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, false);
+  constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, true);
+  constexpr uint32_t TMEM_COLS = 512;
+  constexpr uint32_t COL_S = 0, COL_O = 256;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *base = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *sQ = base;
+  uint8_t *sK = sQ + TILE;
+  uint8_t *sV = sK + 2 * TILE;
+  uint8_t *sP = sV + 2 * TILE;
+  uint64_t *bar = reinterpret_cast<uint64_t *>(sP + 2 * PTILE);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + B_COUNT);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bar[B_Q_FULL], 1);
+    mbar_init(&bar[B_Q_EMPTY], 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar[B_K_FULL + s], 1);
+      mbar_init(&bar[B_K_EMPTY + s], 1);
+      mbar_init(&bar[B_V_FULL + s], 1);
+      mbar_init(&bar[B_V_EMPTY + s], 1);
+      mbar_init(&bar[B_S_FULL + s], 1);
+      mbar_init(&bar[B_S_FREE + s], 128);
+      mbar_init(&bar[B_P_FULL + s], 128);
+      mbar_init(&bar[B_PV_DONE + s], 1);
+    }
+    mbar_init(&bar[B_O_FREE], 128);
+    mbar_init(&bar[B_DRAIN], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ producer
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    uint32_t kv_it = 0, item_no = 0;
+    int armed_q = -1, armed_k[2] = {-1, -1}, armed_v[2] = {-1, -1};
+    bool ok = true;
+    for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x, ++item_no) {
+      const Item it = load_item(p.items, idx);
+      const int kvh = it.head / p.group;
+      if (item_no > 0) ok = mbar_wait(&bar[B_Q_EMPTY], (item_no - 1) & 1, abort_flag, p.status,
+                                      kWaitLimitNs, DBSA_ERR_TIMEOUT);
+      if (!ok) break;
+      mbar_arrive_expect_tx(&bar[B_Q_FULL], TILE);
+#pragma unroll
+      for (int h = 0; h < NH; ++h)
+        tma_load_3d(sQ + h * HALF, &tmQ, &bar[B_Q_FULL], h * 64, it.q_row0, it.head);
+      armed_q = item_no & 1;
+      for (int t = 0; t < it.ntiles; ++t, ++kv_it) {
+        int r, kt;
+        tile_of(it, t, r, kt);
+        const uint32_t st = kv_it & 1, n = kv_it >> 1;
+        if (n > 0) ok = mbar_wait(&bar[B_K_EMPTY + st], (n - 1) & 1, abort_flag, p.status,
+                                  kWaitLimitNs, DBSA_ERR_TIMEOUT);
+        if (!ok) break;
+        mbar_arrive_expect_tx(&bar[B_K_FULL + st], TILE);
+#pragma unroll
+        for (int h = 0; h < NH; ++h)
+          tma_load_3d(sK + st * TILE + h * HALF, &tmK, &bar[B_K_FULL + st], h * 64,
+                      it.k_row0[r] + kt, kvh);
+        armed_k[st] = n & 1;
+        if (n > 0) ok = mbar_wait(&bar[B_V_EMPTY + st], (n - 1) & 1, abort_flag, p.status,
+                                  kWaitLimitNs, DBSA_ERR_TIMEOUT);
+        if (!ok) break;
+        mbar_arrive_expect_tx(&bar[B_V_FULL + st], TILE);
+#pragma unroll
+        for (int h = 0; h < NH; ++h)
+          tma_load_3d(sV + st * TILE + h * HALF, &tmV, &bar[B_V_FULL + st], h * 64,
+                      it.v_row0[r] + kt, kvh);
+        armed_v[st] = n & 1;
+      }
+    }
+    // Every load this thread issued must land before the CTA exits.
+    if (armed_q >= 0) drain_wait(&bar[B_Q_FULL], (uint32_t)armed_q);
+    for (int s = 0; s < 2; ++s) {
+      if (armed_k[s] >= 0) drain_wait(&bar[B_K_FULL + s], (uint32_t)armed_k[s]);
+      if (armed_v[s] >= 0) drain_wait(&bar[B_V_FULL + s], (uint32_t)armed_v[s]);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------------ MMA issuer
+    const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP);
+    uint32_t kv_it = 0, s_it = 0, pv_it = 0, item_no = 0;
+    bool ok = true;
+    for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x, ++item_no) {
+      const Item it = load_item(p.items, idx);
+      ok = mbar_wait(&bar[B_Q_FULL], item_no & 1, abort_flag, p.status, kWaitLimitNs,
+                     DBSA_ERR_TIMEOUT);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t kv_base = kv_it;
+      auto issue_pv = [&](int t) -> bool {
+        const uint32_t pb = pv_it & 1, np = pv_it >> 1;
+        if (!mbar_wait(&bar[B_P_FULL + pb], np & 1, abort_flag, p.status, kWaitLimitNs,
+                       DBSA_ERR_TIMEOUT))
+          return false;
+        const uint32_t kvt = kv_base + t, st = kvt & 1;
+        if (!mbar_wait(&bar[B_V_FULL + st], (kvt >> 1) & 1, abort_flag, p.status, kWaitLimitNs,
+                       DBSA_ERR_TIMEOUT))
+          return false;
+        if (t == 0 && item_no > 0 &&
+            !mbar_wait(&bar[B_O_FREE], (item_no - 1) & 1, abort_flag, p.status, kWaitLimitNs,
+                       DBSA_ERR_TIMEOUT))
+          return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t da = sdesc_sw128(aP + pb * PTILE + (kk >> 2) * HALF + (kk & 3) * 32,
+                                          16, 1024);
+          const uint64_t db = sdesc_sw128(aV + st * TILE + kk * 2048, HALF, 1024);
+          mma_bf16_ss(tmem + COL_O, da, db, IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(&bar[B_V_EMPTY + st]);
+        mma_commit(&bar[B_PV_DONE + pb]);
+        ++pv_it;
+        return true;
+      };
+      for (int t = 0; ok && t < it.ntiles; ++t) {
+        const uint32_t st = kv_it & 1, n = kv_it >> 1;
+        ok = mbar_wait(&bar[B_K_FULL + st], n & 1, abort_flag, p.status, kWaitLimitNs,
+                       DBSA_ERR_TIMEOUT);
+        if (!ok) break;
+        const uint32_t sb = s_it & 1, ns = s_it >> 1;
+        if (ns > 0) ok = mbar_wait(&bar[B_S_FREE + sb], (ns - 1) & 1, abort_flag, p.status,
+                                   kWaitLimitNs, DBSA_ERR_TIMEOUT);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * HALF + (kk & 3) * 32;
+          const uint64_t da = sdesc_sw128(aQ + off, 16, 1024);
+          const uint64_t db = sdesc_sw128(aK + st * TILE + off, 16, 1024);
+          mma_bf16_ss(tmem + COL_S + sb * 128, da, db, IDESC_QK, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&bar[B_S_FULL + sb]);
+        mma_commit(&bar[B_K_EMPTY + st]);
+        if (t == it.ntiles - 1) mma_commit(&bar[B_Q_EMPTY]);
+        ++kv_it;
+        ++s_it;
+        if (t > 0) ok = issue_pv(t - 1);
+      }
+      if (ok) ok = issue_pv(it.ntiles - 1);
+    }
+    // All issued MMAs must finish before TMEM is released.
+    mma_commit(&bar[B_DRAIN]);
+    drain_wait(&bar[B_DRAIN], 0);
+  } else if (warp >= 2) {
+    // ------------------------------------------------------------ softmax
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const float sl2 = p.scale_log2;
+    uint32_t s_it = 0, item_no = 0;
+    bool ok = true;
+    for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x, ++item_no) {
+      const Item it = load_item(p.items, idx);
+      const int qpos = it.q_pos0 + row;
+      float m_ref = -INFINITY, l = 0.f;
+      for (int t = 0; t < it.ntiles; ++t, ++s_it) {
+        int r, kt;
+        tile_of(it, t, r, kt);
+        const uint32_t sb = s_it & 1, ns = s_it >> 1;
+        ok = __all_sync(kFull, mbar_wait(&bar[B_S_FULL + sb], ns & 1, abort_flag, p.status,
+                                         kWaitLimitNs, DBSA_ERR_TIMEOUT));
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t v[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_off + COL_S + sb * 128 + c * 32, v[c]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_wait_ld(v[c]);
+        tc_fence_before();
+        mbar_arrive(&bar[B_S_FREE + sb]);
+
+        const int klim = it.len[r] - kt;
+        const int kpos0 = it.pos0[r] + kt;
+        if (klim < kTileKeys || kpos0 + kTileKeys - 1 > it.q_pos0) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const int k = c * 32 + e;
+              if (k >= klim || kpos0 + k > qpos) v[c][e] = __float_as_uint(-INFINITY);
+            }
+        }
+        float mt0 = -INFINITY, mt1 = -INFINITY, mt2 = -INFINITY, mt3 = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          mt0 = fmaxf(mt0, __uint_as_float(v[0][e]));
+          mt1 = fmaxf(mt1, __uint_as_float(v[1][e]));
+          mt2 = fmaxf(mt2, __uint_as_float(v[2][e]));
+          mt3 = fmaxf(mt3, __uint_as_float(v[3][e]));
+        }
+        const float mt_x = fmaxf(fmaxf(mt0, mt1), fmaxf(mt2, mt3)) * sl2;
+        if (t == 0) {
+          m_ref = mt_x;
+        } else {
+          const bool need = mt_x > m_ref + 8.0f;
+          if (__any_sync(kFull, need)) {
+            // O must hold every earlier tile before it is rescaled.
+            const uint32_t prev = s_it - 1;
+            ok = __all_sync(kFull, mbar_wait(&bar[B_PV_DONE + (prev & 1)], (prev >> 1) & 1,
+                                             abort_flag, p.status, kWaitLimitNs,
+                                             DBSA_ERR_TIMEOUT));
+            if (!ok) break;
+            tc_fence_after();
+            const float m_new = fmaxf(m_ref, mt_x);
+            const float alpha = (m_new == -INFINITY) ? 1.f : ex2(m_ref - m_new);
+            l *= alpha;
+            m_ref = m_new;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t o[32];
+              tmem_ld32(tmem + lane_off + COL_O + c * 32, o);
+              tmem_wait_ld(o);
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+              tmem_st32(tmem + lane_off + COL_O + c * 32, o);
+            }
+            tmem_wait_st();
+          }
+        }
+        const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
+        float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const float p0 = ex2(fmaf(__uint_as_float(v[c][e]), sl2, -mu));
+            const float p1 = ex2(fmaf(__uint_as_float(v[c][e + 1]), sl2, -mu));
+            sum0 += p0;
+            sum1 += p1;
+            __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
+            v[c][e >> 1] = *reinterpret_cast<uint32_t *>(&h);  // packed pairs in v[c][0..15]
+          }
+        l += sum0 + sum1;
+        if (s_it >= 2) {
+          ok = __all_sync(kFull, mbar_wait(&bar[B_PV_DONE + sb], ((s_it - 2) >> 1) & 1, abort_flag,
+                                           p.status, kWaitLimitNs, DBSA_ERR_TIMEOUT));
+          if (!ok) break;
+        }
+        uint8_t *prow = sP + sb * PTILE + row * 128;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int kc = c * 4 + j;  // 8-key chunk index 0..15
+            const uint32_t addr = (kc >> 3) * HALF + ((((kc & 7) ^ (row & 7))) << 4);
+            *reinterpret_cast<uint4 *>(prow + addr) =
+                make_uint4(v[c][4 * j], v[c][4 * j + 1], v[c][4 * j + 2], v[c][4 * j + 3]);
+          }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&bar[B_P_FULL + sb]);
+      }
+      if (!ok) break;
+      // ---- epilogue: O / l of this row
+      const uint32_t last = s_it - 1;
+      ok = __all_sync(kFull, mbar_wait(&bar[B_PV_DONE + (last & 1)], (last >> 1) & 1, abort_flag,
+                                       p.status, kWaitLimitNs, DBSA_ERR_TIMEOUT));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t o[D / 32][32];
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) tmem_ld32(tmem + lane_off + COL_O + c * 32, o[c]);
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) tmem_wait_ld(o[c]);
+      tc_fence_before();
+      mbar_arrive(&bar[B_O_FREE]);
+      if (row < it.n_rows) {
+        const float inv = 1.f / l;
+        const int64_t orow = ((int64_t)(it.q_row0 + row) * p.Hq + it.head) * D;
+        if (OUT_F32) {
+          float *dst = static_cast<float *>(p.out) + orow;
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c)
+#pragma unroll
+            for (int e = 0; e < 32; e += 4)
+              *reinterpret_cast<float4 *>(dst + c * 32 + e) =
+                  make_float4(__uint_as_float(o[c][e]) * inv, __uint_as_float(o[c][e + 1]) * inv,
+                              __uint_as_float(o[c][e + 2]) * inv,
+                              __uint_as_float(o[c][e + 3]) * inv);
+        } else {
+          __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.out) + orow;
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c)
+#pragma unroll
+            for (int e = 0; e < 32; e += 8) {
+              uint32_t w[4];
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(o[c][e + 2 * q]) * inv,
+                                                         __uint_as_float(o[c][e + 2 * q + 1]) * inv);
+                w[q] = *reinterpret_cast<uint32_t *>(&h);
+              }
+              *reinterpret_cast<uint4 *>(dst + c * 32 + e) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+        }
+      }
+    }
+  }
+  __syncwarp();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// [heads][rows][D] bf16 view (head stride in rows), 128-row x 64-column boxes.
+bool make_map(CUtensorMap *m, const void *ptr, int D, int64_t rows, int64_t heads,
+              int64_t head_stride_rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)heads};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)head_stride_rows * D * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D>
+constexpr size_t smem_bytes() {
+  return 1024 + (size_t)128 * D * 2 * 5 + (size_t)128 * 128 * 2 * 2 + B_COUNT * 8 + 16;
+}
+
+template <int D, bool F32>
+cudaError_t launch_t(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                     const Params &p, int grid, cudaStream_t st) {
+  constexpr size_t smem = smem_bytes<D>();
+  static_assert(smem <= 232448, "shared memory budget");
+  static_assert(smem > 232448 / 2, "one CTA per SM (the kernel owns all 512 TMEM columns)");
+  cudaError_t e = cudaFuncSetAttribute(stage1_attn_kernel<D, F32>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  stage1_attn_kernel<D, F32><<<grid, 192, smem, st>>>(mq, mk, mv, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_stage1(const Stage1Args &a, int head_dim, bool out_f32, int num_sms,
+                          cudaStream_t st) {
+  if (a.n_items <= 0) return cudaSuccess;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, a.q_rot, head_dim, a.q_rows, a.Hq, a.q_rows) ||
+      !make_map(&mk, a.k_rot, head_dim, a.k_rows, a.Hkv, a.k_rows) ||
+      !make_map(&mv, a.v, head_dim, a.v_rows, a.Hkv, a.v_head_stride))
+    return cudaErrorInvalidValue;
+  Params p;
+  p.items = a.items;
+  p.n_items = a.n_items;
+  p.group = a.Hq / a.Hkv;
+  p.Hq = a.Hq;
+  p.out = a.out;
+  p.scale_log2 = a.scale_log2;
+  p.status = a.status;
+  const int grid = a.n_items < num_sms ? a.n_items : num_sms;
+  if (head_dim == 128)
+    return out_f32 ? launch_t<128, true>(mq, mk, mv, p, grid, st)
+                   : launch_t<128, false>(mq, mk, mv, p, grid, st);
+  return out_f32 ? launch_t<64, true>(mq, mk, mv, p, grid, st)
+                 : launch_t<64, false>(mq, mk, mv, p, grid, st);
+}
+
+}  // namespace dbsa

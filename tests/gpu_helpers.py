@@ -1,0 +1,82 @@
+"""Shared helpers of the GPU tests: run the library through its binding on
+seeded inputs and compare with the oracle on the same values."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from many_shot_icl_b200 import dbsa
+
+ATOL = 2e-2      # max-abs bound on attention outputs (bf16 inputs, fp32 accumulate)
+RTOL_FRO = 2e-2  # relative Frobenius error bound per head
+# "Peaky" variant (queries scaled x4, sharp softmax).  The tensor cores take
+# the rotated q and k as bf16 (relative rounding <= 2^-9 per element), which
+# moves a score by about sqrt(2d) * s_q * s_k * 2^-9 / sqrt(d) ~= 0.011 for
+# s_q = 4, s_k = 1; with |v| up to ~3.5 a sharp softmax turns that into up to
+# ~0.04 on an output element, plus half a bf16 ulp of the output (<= 0.008).
+ATOL_PEAKY = 6e-2
+
+
+def tdtype(dtype: str):
+    return torch.float32 if dtype == "f32" else torch.bfloat16
+
+
+def rand(shape, seed, dtype, scale=1.0, device="cuda"):
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    x = torch.randn(tuple(shape), generator=g, dtype=torch.float32) * scale
+    return x.to(tdtype(dtype)).to(device)
+
+
+def host_f32(t) -> np.ndarray:
+    return t.detach().float().cpu().numpy()
+
+
+def compare(got: np.ndarray, want: np.ndarray, head_axis: int, what: str, atol: float = ATOL):
+    """max-abs <= atol and, per head, relative Frobenius error <= RTOL_FRO."""
+    got = np.asarray(got, dtype=np.float64)
+    err = np.abs(got - want)
+    assert np.isfinite(got).all(), what + ": non-finite output"
+    assert err.max() <= atol, "%s: max-abs %.3e > %.1e" % (what, err.max(), atol)
+    g = np.moveaxis(got, head_axis, 0).reshape(got.shape[head_axis], -1)
+    w = np.moveaxis(want, head_axis, 0).reshape(want.shape[head_axis], -1)
+    rel = np.linalg.norm(g - w, axis=1) / np.maximum(np.linalg.norm(w, axis=1), 1e-30)
+    assert rel.max() <= RTOL_FRO, "%s: relative Frobenius %.3e > %.1e" % (what, rel.max(), RTOL_FRO)
+    return float(err.max()), float(rel.max())
+
+
+def offsets(lens) -> np.ndarray:
+    return np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+
+
+class Stage1Run:
+    """Inputs, cache and output of one dbsa_encode_blocks call."""
+
+    def __init__(self, cfg: dbsa.DbsaConfig, offs, seed=0, cap_extra=0, q_scale=1.0):
+        self.cfg, self.offs = cfg, np.asarray(offs, np.int32)
+        T = int(self.offs[-1])
+        self.T = T
+        Hq, Hkv, D = cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim
+        self.q = rand((T, Hq, D), seed * 10 + 1, cfg.dtype, q_scale)
+        self.k = rand((T, Hkv, D), seed * 10 + 2, cfg.dtype)
+        self.v = rand((T, Hkv, D), seed * 10 + 3, cfg.dtype)
+        self.cap = T + cap_extra
+        self.kc = torch.full((Hkv, self.cap, D), float("nan"), dtype=tdtype(cfg.dtype), device="cuda")
+        self.vc = torch.full((Hkv, self.cap, D), float("nan"), dtype=tdtype(cfg.dtype), device="cuda")
+        self.out = torch.full((T, Hq, D), float("nan"), dtype=tdtype(cfg.dtype), device="cuda")
+        nbytes = dbsa.encode_workspace_size(cfg, T, len(self.offs) - 1)
+        self.ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+
+    def run(self):
+        dbsa.encode_blocks(self.cfg, self.q, self.k, self.v, self.offs, self.kc, self.vc, self.out,
+                           self.ws)
+        assert dbsa.read_status(self.ws) == dbsa.OK
+        return self
+
+    def oracle_rows(self, heads, toks, pattern=None):
+        cfg = self.cfg
+        return oracle.stage1_rows(host_f32(self.q), host_f32(self.k), host_f32(self.v), self.offs,
+                                  cfg.window_j, cfg.rope_theta, heads, toks,
+                                  pattern=cfg.pattern if pattern is None else pattern,
+                                  scale=cfg.softmax_scale)

@@ -1,0 +1,121 @@
+"""Stage-2 parity on a B200: dbsa_gather_rope_attend against the CPU oracle
+on the same seeded inputs.  Gathered cache rows and fresh positions are
+compared exactly (dbg_map); attention outputs within the stated tolerance."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from many_shot_icl_b200 import dbsa, inputs
+from tests.gpu_helpers import ATOL, ATOL_PEAKY, compare, host_f32, offsets, rand, tdtype
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from many_shot_icl_b200 import build
+    build.build()
+    dbsa.load()
+    assert torch.cuda.is_available()
+
+
+class Stage2Run:
+    def __init__(self, cfg, offs, sels, n_new, tail_len, seed=0, tail_cap=None, q_scale=1.0,
+                 cap_extra=3):
+        self.cfg, self.offs, self.sels = cfg, np.asarray(offs, np.int32), sels
+        Hq, Hkv, D = cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim
+        T = int(self.offs[-1])
+        self.cap = T + cap_extra
+        self.nq = len(sels)
+        self.n_new, self.tail_len = n_new, tail_len
+        self.tail_cap = tail_cap or tail_len + 2
+        self.kc = rand((Hkv, self.cap, D), seed * 10 + 1, cfg.dtype)
+        self.vc = rand((Hkv, self.cap, D), seed * 10 + 2, cfg.dtype)
+        self.q_new = rand((self.nq, n_new, Hq, D), seed * 10 + 3, cfg.dtype, q_scale)
+        self.kt = rand((self.nq, self.tail_cap, Hkv, D), seed * 10 + 4, cfg.dtype)
+        self.vt = rand((self.nq, self.tail_cap, Hkv, D), seed * 10 + 5, cfg.dtype)
+        self.sel_ptr, self.sel = dbsa.selection_csr(sels)
+        self.out = torch.full((self.nq, n_new, Hq, D), float("nan"), dtype=tdtype(cfg.dtype),
+                              device="cuda")
+        Tmax = max(int(sum(self.offs[b + 1] - self.offs[b] for b in s)) for s in sels)
+        self.dbg = torch.full((self.nq, Tmax, 2), -1, dtype=torch.int32, device="cuda")
+        nbytes = dbsa.gather_workspace_size(cfg, self.offs, self.sel_ptr, self.sel, n_new, tail_len)
+        assert nbytes > 0, dbsa.last_error()
+        self.ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+
+    def run(self):
+        dbsa.gather_rope_attend(self.cfg, self.kc, self.vc, self.offs, self.sel_ptr, self.sel,
+                                self.q_new, self.kt, self.vt, self.tail_len, self.out, self.ws,
+                                dbg_map=self.dbg)
+        assert dbsa.read_status(self.ws) == dbsa.OK
+        return self
+
+    def check(self, what, queries=None, atol=ATOL):
+        kc, vc = host_f32(self.kc), host_f32(self.vc)
+        qn, kt, vt = host_f32(self.q_new), host_f32(self.kt), host_f32(self.vt)
+        out = host_f32(self.out)
+        dbg = self.dbg.cpu().numpy()
+        for q in (range(self.nq) if queries is None else queries):
+            m = oracle.stage2_gather_map(self.offs, self.sels[q])
+            np.testing.assert_array_equal(dbg[q, :len(m)], m, err_msg="%s: gather map q%d" % (what, q))
+            want = oracle.stage2_all(kc, vc, self.offs, self.sels[q], qn[q],
+                                     kt[q, :self.tail_len], vt[q, :self.tail_len],
+                                     self.cfg.rope_theta, scale=self.cfg.softmax_scale)
+            compare(out[q], want, head_axis=1, what="%s q%d" % (what, q), atol=atol)
+
+
+def test_tiny_workload_fp32():
+    w = inputs.TINY
+    offs = oracle.group_blocks(inputs.demo_lengths(w), w.demos_per_block)
+    sels = inputs.selections(w)
+    cfg = dbsa.DbsaConfig(w.n_q_heads, w.n_kv_heads, w.head_dim, "f32", w.rope_theta, w.window_j)
+    Stage2Run(cfg, offs, sels, n_new=w.query_tokens, tail_len=w.query_tokens, seed=1).run().check("tiny")
+
+
+@pytest.mark.parametrize("Hq,Hkv,D", [(8, 2, 128), (4, 4, 128), (4, 1, 64)])
+@pytest.mark.parametrize("n_new,tail_len", [(1, 1), (1, 9), (3, 7), (40, 40), (17, 20)])
+def test_bf16_prefill_and_decode(Hq, Hkv, D, n_new, tail_len):
+    rng = np.random.default_rng(Hq * 100 + n_new)
+    lens = rng.integers(40, 400, size=9)
+    offs = offsets(lens)
+    sels = [np.array([0, 2, 5, 7]), np.array([0, 8, 1]), np.array([0]), np.array([0, 3, 4, 6, 8, 1])]
+    cfg = dbsa.DbsaConfig(Hq, Hkv, D, "bf16", 5e5, 2)
+    Stage2Run(cfg, offs, sels, n_new, tail_len, seed=2).run().check(
+        "Hq%d Hkv%d D%d n%d t%d" % (Hq, Hkv, D, n_new, tail_len))
+
+
+def test_long_gather_many_splits_peaky():
+    # long selections force several splits per query; Q x 4 sharpens the softmax
+    rng = np.random.default_rng(5)
+    lens = rng.integers(900, 1600, size=12)
+    offs = offsets(lens)
+    sels = [np.concatenate([[0], np.sort(rng.choice(np.arange(1, 12), 8, replace=False))])
+            for _ in range(3)]
+    sels.append(np.concatenate([[0], rng.permutation(np.arange(1, 12))]))   # non-encoding order
+    cfg = dbsa.DbsaConfig(8, 2, 128, "bf16", 5e5, 2)
+    for n_new, tail_len in ((1, 41), (40, 40)):
+        Stage2Run(cfg, offs, sels, n_new, tail_len, seed=3, q_scale=4.0).run().check(
+            "long n%d" % n_new, atol=ATOL_PEAKY)
+        Stage2Run(cfg, offs, sels, n_new, tail_len, seed=13).run().check("long n%d" % n_new)
+
+
+def test_all_blocks_in_order_equals_stage1_positions():
+    # selecting every block in encoding order reproduces the original positions
+    lens = [100, 130, 90]
+    offs = offsets(lens)
+    cfg = dbsa.DbsaConfig(2, 1, 64, "bf16", 1e4, 2)
+    r = Stage2Run(cfg, offs, [np.array([0, 1, 2])], 4, 4, seed=4).run()
+    dbg = r.dbg.cpu().numpy()[0]
+    np.testing.assert_array_equal(dbg[:, 0], np.arange(320))
+    np.testing.assert_array_equal(dbg[:, 1], np.arange(320))
+    r.check("all blocks")
+
+
+def test_deterministic():
+    lens = [300, 200, 250, 270]
+    cfg = dbsa.DbsaConfig(8, 2, 128, "bf16", 5e5, 2)
+    r = Stage2Run(cfg, offsets(lens), [np.array([0, 2, 3])], 1, 5, seed=6).run()
+    o1 = r.out.clone()
+    r.run()
+    assert torch.equal(o1, r.out)

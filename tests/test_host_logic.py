@@ -1,0 +1,178 @@
+"""Host-side logic of libdbsa.so, CPU only (no kernel runs here).
+
+- the library loads and exports every function include/dbsa.h declares;
+- the block table equals the oracle's;
+- the Stage-1 tile list covers exactly the oracle's allowed (row, key) pairs,
+  once each, for every pattern of the sparse-pattern ablation;
+- invalid arguments are rejected with the documented status before any
+  device work.
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from many_shot_icl_b200 import dbsa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from many_shot_icl_b200 import build
+    build.build()
+    return dbsa.load()
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "dbsa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(dbsa_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = header_functions()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(dbsa.SYMBOLS)
+    assert "sm_100a" in dbsa.version()
+
+
+def test_group_blocks_matches_oracle(lib):
+    rng = np.random.default_rng(0)
+    for n, k in ((1, 1), (7, 3), (1000, 50), (173, 50), (50, 50)):
+        lens = rng.integers(15, 46, size=n).astype(np.int32)
+        np.testing.assert_array_equal(dbsa.group_blocks(lens, k), oracle.group_blocks(lens, k))
+    with pytest.raises(dbsa.DbsaError):
+        dbsa.group_blocks(np.array([3, 0, 4], np.int32), 2)
+
+
+def covered_pairs(items, head):
+    pairs = set()
+    for it in items:
+        if it.head != head:
+            continue
+        assert 1 <= it.n_rows <= 128 and it.n_ranges in (1, 2)
+        for t in range(it.q_pos0, it.q_pos0 + it.n_rows):
+            for r in range(it.n_ranges):
+                for s in range(it.pos0[r], it.pos0[r] + it.len[r]):
+                    if s <= t:
+                        assert (t, s) not in pairs, "pair covered twice"
+                        pairs.add((t, s))
+    return pairs
+
+
+@pytest.mark.parametrize("pattern", range(4))
+@pytest.mark.parametrize("j", [0, 1, 2, 5])
+def test_stage1_plan_covers_exactly_the_mask(lib, pattern, j):
+    rng = np.random.default_rng(10 + j)
+    lens = rng.integers(1, 300, size=7)
+    offs = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    T = int(offs[-1])
+    cfg = dbsa.DbsaConfig(4, 2, 64, window_j=j, pattern=pattern)
+    items = dbsa.stage1_plan(cfg, offs)
+    # rows: every token of every head exactly once, tiles never straddle a block
+    for h in range(4):
+        rows = sorted(t for it in items if it.head == h
+                      for t in range(it.q_pos0, it.q_pos0 + it.n_rows))
+        assert rows == list(range(T))
+    for it in items:
+        b = int(np.searchsorted(offs, it.q_pos0, side="right") - 1)
+        assert it.block == b and it.q_pos0 + it.n_rows <= offs[b + 1]
+        assert it.q_row0 == it.q_pos0 and list(it.k_row0)[:it.n_ranges] == list(it.pos0)[:it.n_ranges]
+    # pairs: exactly the oracle's explicit mask (sampled rows, all keys)
+    got = covered_pairs(items, head=1)
+    sample = sorted(set(rng.integers(0, T, size=40).tolist()) | {0, T - 1} |
+                    set(int(o) for o in offs[:-1]))
+    for t in sample:
+        want = {s for s in range(t + 1) if oracle.stage1_allowed(offs, j, t, s, pattern)}
+        have = {s for (tt, s) in got if tt == t}
+        assert have == want, (t, sorted(want ^ have)[:10])
+    # the tile count is the sum of the items' key tiles
+    assert dbsa.stage1_tile_count(cfg, offs) == sum(
+        sum((it.len[r] + 127) // 128 for r in range(it.n_ranges)) for it in items)
+
+
+def test_stage1_plan_allowed_count_matches_oracle(lib):
+    rng = np.random.default_rng(3)
+    lens = rng.integers(1, 200, size=9)
+    offs = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    cfg = dbsa.DbsaConfig(2, 1, 64, window_j=2)
+    pairs = covered_pairs(dbsa.stage1_plan(cfg, offs), head=0)
+    cnt = np.zeros(int(offs[-1]), np.int64)
+    for t, _ in pairs:
+        cnt[t] += 1
+    np.testing.assert_array_equal(cnt, oracle.stage1_allowed_counts(offs, 2))
+
+
+def _cfgp(cfg):
+    c = cfg.c()
+    return c, ctypes.byref(c)
+
+
+def test_invalid_arguments_are_rejected_before_device_work(lib):
+    fake = ctypes.c_void_p(4096)  # aligned, never dereferenced: validation fails first
+    offs = np.array([0, 5, 9, 20], np.int32)
+    ok_cfg = dbsa.DbsaConfig(4, 2, 128)
+    ws = ctypes.c_void_p(1 << 20)
+
+    def gather(cfg, sel_ptr, sel, n_new=1, tail_len=1, tail_cap=4, offs=offs, cap=64):
+        c, cp = _cfgp(cfg)
+        sp, sb = np.asarray(sel_ptr, np.int32), np.asarray(sel, np.int32)
+        return lib.dbsa_gather_rope_attend(
+            cp, fake, fake, cap, offs.ctypes.data_as(ctypes.c_void_p), len(offs) - 1, len(sp) - 1,
+            sp.ctypes.data_as(ctypes.c_void_p), sb.ctypes.data_as(ctypes.c_void_p), fake, n_new,
+            fake, fake, tail_len, tail_cap, fake, None, 0, ws, 1 << 30, None)
+
+    assert gather(ok_cfg, [0, 2], [1, 0]) == dbsa.ERR_INVALID_ARG       # sink not first
+    assert "sink" in dbsa.last_error()
+    assert gather(ok_cfg, [0, 3], [0, 2, 2]) == dbsa.ERR_INVALID_ARG    # duplicate
+    assert gather(ok_cfg, [0, 2], [0, 3]) == dbsa.ERR_INVALID_ARG       # out of range
+    assert gather(ok_cfg, [0, 0], []) == dbsa.ERR_INVALID_ARG           # empty selection
+    assert gather(ok_cfg, [0, 1], [0], n_new=3, tail_len=2) == dbsa.ERR_INVALID_ARG
+    assert gather(ok_cfg, [0, 1], [0], tail_len=5, tail_cap=4) == dbsa.ERR_INVALID_ARG
+    assert gather(ok_cfg, [0, 1], [0], cap=10) == dbsa.ERR_CAPACITY
+    assert gather(dbsa.DbsaConfig(4, 3, 128), [0, 1], [0]) == dbsa.ERR_UNSUPPORTED
+    assert gather(dbsa.DbsaConfig(4, 2, 96), [0, 1], [0]) == dbsa.ERR_UNSUPPORTED
+    bad_offs = np.array([0, 5, 5, 20], np.int32)
+    assert gather(ok_cfg, [0, 1], [0], offs=bad_offs) == dbsa.ERR_INVALID_ARG
+
+    def encode(cfg, offs=offs, cap=64, ws_bytes=1 << 30, q=fake, ws=ws):
+        c, cp = _cfgp(cfg)
+        return lib.dbsa_encode_blocks(cp, q, fake, fake, offs.ctypes.data_as(ctypes.c_void_p),
+                                      len(offs) - 1, fake, fake, cap, fake, ws, ws_bytes, None)
+
+    assert encode(ok_cfg, cap=19) == dbsa.ERR_CAPACITY
+    assert encode(ok_cfg, offs=np.array([1, 5], np.int32)) == dbsa.ERR_INVALID_ARG
+    assert encode(ok_cfg, q=ctypes.c_void_p(4097)) == dbsa.ERR_INVALID_ARG   # misaligned
+    assert encode(ok_cfg, q=None) == dbsa.ERR_INVALID_ARG
+    assert encode(ok_cfg, ws_bytes=100) == dbsa.ERR_WORKSPACE
+    assert encode(ok_cfg, ws=ctypes.c_void_p(4096 + 16)) == dbsa.ERR_WORKSPACE
+    assert encode(dbsa.DbsaConfig(4, 2, 128, rope_theta=0.5)) == dbsa.ERR_INVALID_ARG
+    assert encode(dbsa.DbsaConfig(4, 2, 128, window_j=-1)) == dbsa.ERR_INVALID_ARG
+    assert encode(dbsa.DbsaConfig(4, 2, 128, pattern=7)) == dbsa.ERR_INVALID_ARG
+
+    c, cp = _cfgp(ok_cfg)
+    assert lib.dbsa_append_block(cp, fake, fake, fake, 0, offs.ctypes.data_as(ctypes.c_void_p),
+                                 3, fake, fake, 64, fake, ws, 1 << 30, None) == dbsa.ERR_INVALID_ARG
+    assert lib.dbsa_append_block(cp, fake, fake, fake, 50, offs.ctypes.data_as(ctypes.c_void_p),
+                                 3, fake, fake, 64, fake, ws, 1 << 30, None) == dbsa.ERR_CAPACITY
+
+
+def test_workspace_sizes(lib):
+    cfg = dbsa.DbsaConfig(32, 8, 128, rope_theta=5e5)
+    offs = np.arange(0, 61 * 1500, 1500, dtype=np.int32)
+    T = int(offs[-1])
+    ws = dbsa.encode_workspace_size(cfg, T, 60)
+    # q_rot + k_rot dominate: (32 + 8) heads x T x 128 x 2 bytes
+    assert 40 * T * 256 <= ws < 40 * T * 256 * 1.05
+    wa = dbsa.append_workspace_size(cfg, offs, 1500)
+    assert 0 < wa < ws / 10
+    sel_ptr, sel = dbsa.selection_csr([np.array([0, 3, 9]), np.array([0, 1])])
+    wg = dbsa.gather_workspace_size(cfg, offs, sel_ptr, sel, 40, 40)
+    assert wg > 0
+    assert dbsa.gather_workspace_size(cfg, offs, sel_ptr, np.array([2, 3, 9, 0, 1]), 40, 40) == 0
