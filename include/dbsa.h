@@ -205,6 +205,36 @@ dbsa_status dbsa_gather_rope_attend(
     int64_t dbg_cap, void *workspace, size_t ws_bytes, void *stream);
 
 /* ---------------------------------------------------------------------------
+ * Stage 2 without a workspace.  The paper has no counterpart: this is a
+ * calling convention of this library, not a step of the method.
+ *
+ * For callers that cannot allocate device memory when they call in, such as
+ * code that runs inside another framework's fixed memory budget or a host
+ * thread that must not call cudaMalloc (it may synchronise the device).
+ * Same arguments, results and errors as dbsa_gather_rope_attend, minus the
+ * workspace.  The scratch is one array of 16 MiB in the library's device
+ * memory, held by every GPU that loads the library until the process exits.
+ *  - A batch whose dbsa_gather_workspace_size() exceeds 16 MiB is rejected
+ *    with DBSA_ERR_WORKSPACE and a message naming both sizes; nothing runs.
+ *  - The first call on a device looks up the array's device address (with
+ *    that device current) and keeps it; make that first call before any
+ *    stream capture.
+ *  - Every call on a device shares the one array and leaves its contents
+ *    behind; the call clears the status word it needs at zero.  Calls whose
+ *    work overlaps on the GPU (other streams, other host threads) race on the
+ *    array: serialise them.
+ *  - dbsa_read_status() does not apply (there is no caller workspace).
+ * It allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ * ------------------------------------------------------------------------ */
+dbsa_status dbsa_gather_rope_attend_noalloc(
+    const dbsa_config *cfg, const void *k_cache, const void *v_cache,
+    int64_t cap, const int32_t *offs_host, int32_t nb, int32_t nq,
+    const int32_t *sel_ptr_host, const int32_t *sel_blocks_host,
+    const void *q_new, int32_t n_new, const void *k_tail, const void *v_tail,
+    int32_t tail_len, int32_t tail_cap, void *out, int32_t *dbg_map,
+    int64_t dbg_cap, void *stream);
+
+/* ---------------------------------------------------------------------------
  * Status and introspection.
  * ------------------------------------------------------------------------ */
 

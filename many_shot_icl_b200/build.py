@@ -21,7 +21,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libdbsa.so")
-SOURCES = ["dbsa_api.cu", "rope.cu", "stage1_attn.cu", "stage2_attn.cu"]
+SOURCES = ["dbsa_api.cu", "rope.cu", "stage1_attn.cu", "stage2_attn.cu", "noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -372,6 +372,8 @@ int64_t encode_item_bound(const dbsa_config *cfg, int64_t T, int32_t nb) {
 
 }  // namespace
 
+void dbsa::set_last_error(const char *msg) { g_err = msg; }
+
 // ============================================================== public ABI
 extern "C" {
 

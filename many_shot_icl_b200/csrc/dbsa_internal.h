@@ -128,6 +128,9 @@ struct Stage2Args {
   float scale_log2;
   RopeTables rope;
 };
+// Sets the message dbsa_last_error() returns on this thread.
+void set_last_error(const char *msg);
+
 cudaError_t launch_stage2_main(const Stage2Args &a, int head_dim, bool f32, cudaStream_t st);
 cudaError_t launch_stage2_merge(const Stage2Args &a, int head_dim, bool f32, cudaStream_t st);
 

@@ -26,6 +26,7 @@ SYMBOLS = (
     "dbsa_append_workspace_size", "dbsa_append_block", "dbsa_gather_workspace_size",
     "dbsa_gather_rope_attend", "dbsa_last_error", "dbsa_read_status", "dbsa_stage1_plan",
     "dbsa_stage1_tile_count", "dbsa_version", "dbsa_kernel_launches", "dbsa_set_profile_events",
+    "dbsa_gather_rope_attend_noalloc",
 )
 
 
@@ -96,6 +97,9 @@ def load(path: str = LIB_PATH):
     lib.dbsa_gather_rope_attend.argtypes = [cfgp, vp, vp, i64, vp, i32, i32, vp, vp, vp, i32, vp,
                                             vp, i32, i32, vp, vp, i64, vp, sz, vp]
     lib.dbsa_gather_rope_attend.restype = ctypes.c_int
+    lib.dbsa_gather_rope_attend_noalloc.argtypes = [cfgp, vp, vp, i64, vp, i32, i32, vp, vp, vp,
+                                                    i32, vp, vp, i32, i32, vp, vp, i64, vp]
+    lib.dbsa_gather_rope_attend_noalloc.restype = ctypes.c_int
     lib.dbsa_last_error.argtypes = []
     lib.dbsa_last_error.restype = ctypes.c_char_p
     lib.dbsa_read_status.argtypes = [vp, vp]
@@ -237,6 +241,21 @@ def set_profile_events(start, stop):
             ev.record()
         return ev.cuda_event
     load().dbsa_set_profile_events(handle(start), handle(stop))
+
+
+def gather_rope_attend_noalloc(cfg: DbsaConfig, k_cache, v_cache, offs, sel_ptr, sel_blocks,
+                               q_new, k_tail, v_tail, tail_len: int, out, dbg_map=None,
+                               stream=None):
+    """Stage 2 without a workspace: for callers that cannot allocate device
+    memory.  Scratch is the library's fixed 16 MiB per-device array, shared
+    by every call (serialise calls that would overlap on the GPU)."""
+    o, sp, sb = _i32(offs), _i32(sel_ptr), _i32(sel_blocks)
+    c = cfg.c()
+    _check(load().dbsa_gather_rope_attend_noalloc(
+        ctypes.byref(c), _dp(k_cache), _dp(v_cache), k_cache.shape[1], _hp(o), len(o) - 1,
+        len(sp) - 1, _hp(sp), _hp(sb), _dp(q_new), q_new.shape[1], _dp(k_tail), _dp(v_tail),
+        tail_len, k_tail.shape[1], _dp(out), _dp(dbg_map),
+        0 if dbg_map is None else dbg_map.shape[1], _stream(stream)))
 
 
 def read_status(workspace, stream=None) -> int:
