@@ -244,6 +244,34 @@ def e2e_step_time(wl: Workload, host, steps: int):
     return t1 / steps, t2 / steps
 
 
+def profile_only(wl: Workload, args):
+    """Stage 1 or Stage 2 alone, W + K times (for ncu captures).  Stage 2 first
+    runs one Stage-1 pass to fill the caches it reads."""
+    import torch
+    from many_shot_icl_b200 import dbsa
+
+    def stage1():
+        for l in range(wl.layers):
+            dbsa.encode_blocks(wl.cfg, wl.q[l], wl.k[l], wl.v[l], wl.offs, wl.kc[l], wl.vc[l],
+                               wl.out[l], wl.ws)
+
+    def stage2():
+        for n_new, tail_len in wl.passes():
+            for l in range(wl.layers):
+                qn, out = (wl.qp[l], wl.out_p) if n_new > 1 else (wl.qd[l], wl.out_d)
+                dbsa.gather_rope_attend(wl.cfg, wl.kc[l], wl.vc[l], wl.offs, wl.sel_ptr, wl.sel,
+                                        qn, wl.kt[l], wl.vt[l], tail_len, out, wl.ws)
+
+    if args.profile_only == "stage2":
+        stage1()
+    for _ in range(args.warmup + args.steps):
+        stage1() if args.profile_only == "stage1" else stage2()
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_only": args.profile_only, "layers": wl.layers,
+                      "steps": args.warmup + args.steps, "ok": True}))
+    return 0
+
+
 def pinned_host_buffers(wl: Workload):
     import torch
     p = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t.cpu())
@@ -411,6 +439,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=16.0)
     ap.add_argument("--ref-budget", type=float, default=60.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-only", choices=["stage1", "stage2"], default=None,
+                    help="run W + K steps of one stage only and exit (for ncu captures)")
     args = ap.parse_args()
     world, rank, local = dist_setup()
     if args.impl == "reference":
@@ -433,6 +463,8 @@ def main():
     room = (n_appends + 1) * w.demos_per_block * w.demo_len_hi if n_appends else 0
     wl = Workload(w, layers, "cuda", rank=rank, append_room=room)
     torch.cuda.synchronize()
+    if args.profile_only:
+        return profile_only(wl, args)
 
     for _ in range(args.warmup):
         run_step(wl)
@@ -519,8 +551,11 @@ def main():
     s2_tok_s = q_tokens * world / t_s2
 
     # end to end from pinned host memory (rank-local)
-    host = pinned_host_buffers(wl)
-    e2e_t1, e2e_t2 = e2e_step_time(wl, host, args.e2e_steps)
+    if args.e2e_steps > 0:
+        host = pinned_host_buffers(wl)
+        e2e_t1, e2e_t2 = e2e_step_time(wl, host, args.e2e_steps)
+    else:
+        e2e_t1 = e2e_t2 = float("nan")
     e2e_t1 = max_over_ranks(e2e_t1, world)
     e2e_t2 = max_over_ranks(e2e_t2, world)
     elt = 2 if w.dtype == "bf16" else 4
