@@ -272,11 +272,14 @@ dbsa_status gather_plan(const dbsa_config *cfg, const int32_t *offs, int32_t nb,
     gp.max_pos = std::max<int32_t>(gp.max_pos, (int32_t)(p + tail_len));
     gp.queries.push_back(qi);
   }
-  // split size: >= 33 keys per query row (bounds the partial-result traffic
-  // to ~3 % of the K/V bytes) and enough CTAs for ~4 waves at 2 CTAs / SM
-  const int zdim = (R <= 16) ? 1 : (R + kS2MaxRows - 1) / kS2MaxRows;
-  const int64_t min_chunk = std::max<int64_t>(256, (int64_t)33 * R);
-  const int64_t want_ctas = (int64_t)8 * num_sms();
+  // Split size: >= 33 keys per query row of a CTA (bounds the partial-result
+  // traffic to ~3 % of the K/V bytes) and enough CTAs for ~4 waves at one
+  // CTA per SM.  Rows per CTA follow the kernel's shape table (16, 32, 64,
+  // 128, else row groups of 160).
+  const int rows_cta = (R <= 16) ? 16 : (R <= 32) ? 32 : (R <= 64) ? 64 : (R <= 128) ? 128 : 160;
+  const int zdim = (R + rows_cta - 1) / rows_cta;
+  const int64_t min_chunk = std::max<int64_t>(256, (int64_t)33 * std::min(R, rows_cta));
+  const int64_t want_ctas = (int64_t)4 * num_sms();
   const int64_t par_chunk =
       (total_keys * cfg->n_kv_heads * zdim + want_ctas - 1) / std::max<int64_t>(1, want_ctas);
   int64_t chunk = std::max(min_chunk, par_chunk);
@@ -303,17 +306,15 @@ dbsa_status gather_plan(const dbsa_config *cfg, const int32_t *offs, int32_t nb,
 
 // -------------------------------------------------------------- workspace layouts
 struct S1Layout {
-  size_t hi, lo, items, q_rot, k_rot, v_bf16, total;
+  size_t rope, items, q_rot, k_rot, v_bf16, total;
   int32_t n_hi;
 };
 S1Layout s1_layout(const dbsa_config *cfg, int64_t max_pos, int64_t n_items, int64_t q_rows,
                    int64_t k_rows) {
   S1Layout l;
   Carve cv;
-  const int64_t half = cfg->head_dim / 2;
   l.n_hi = (int32_t)(std::max<int64_t>(max_pos - 1, 0) / kRopeLo + 1);
-  l.hi = cv.take((size_t)l.n_hi * half * sizeof(float2));
-  l.lo = cv.take((size_t)kRopeLo * half * sizeof(float2));
+  l.rope = cv.take(rope_table_bytes(l.n_hi, cfg->head_dim));
   l.items = cv.take((size_t)n_items * sizeof(dbsa_tile_item));
   l.q_rot = cv.take((size_t)cfg->n_q_heads * q_rows * cfg->head_dim * 2);
   l.k_rot = cv.take((size_t)cfg->n_kv_heads * k_rows * cfg->head_dim * 2);
@@ -324,16 +325,14 @@ S1Layout s1_layout(const dbsa_config *cfg, int64_t max_pos, int64_t n_items, int
 }
 
 struct S2Layout {
-  size_t hi, lo, queries, segs, items, part_acc, part_ml, total;
+  size_t rope, queries, segs, items, part_acc, part_ml, total;
   int32_t n_hi;
 };
 S2Layout s2_layout(const dbsa_config *cfg, const GatherPlan &gp, int32_t n_new) {
   S2Layout l;
   Carve cv;
-  const int64_t half = cfg->head_dim / 2;
   l.n_hi = (int32_t)(std::max<int64_t>(gp.max_pos - 1, 0) / kRopeLo + 1);
-  l.hi = cv.take((size_t)l.n_hi * half * sizeof(float2));
-  l.lo = cv.take((size_t)kRopeLo * half * sizeof(float2));
+  l.rope = cv.take(rope_table_bytes(l.n_hi, cfg->head_dim));
   l.queries = cv.take(gp.queries.size() * sizeof(S2Query));
   l.segs = cv.take(gp.segs.size() * sizeof(S2Segment));
   l.items = cv.take(gp.items.size() * sizeof(S2Item));
@@ -358,12 +357,12 @@ T *at(void *ws, size_t off) {
   return reinterpret_cast<T *>(static_cast<uint8_t *>(ws) + off);
 }
 
-RopeTables tables_at(void *ws, size_t hi, size_t lo, int32_t n_hi) {
-  RopeTables t;
-  t.hi = at<float2>(ws, hi);
-  t.lo = at<float2>(ws, lo);
-  t.n_hi = n_hi;
-  return t;
+// Builds the RoPE tables at `off` in the workspace (enqueued) and returns them.
+cudaError_t build_tables(void *ws, size_t off, int32_t n_hi, const dbsa_config *cfg,
+                         cudaStream_t st, RopeTables *out) {
+  float *base = at<float>(ws, off);
+  *out = rope_tables_at(base, n_hi, cfg->head_dim);
+  return launch_rope_tables(base, n_hi, cfg->head_dim, cfg->rope_theta, st);
 }
 
 int64_t encode_item_bound(const dbsa_config *cfg, int64_t T, int32_t nb) {
@@ -459,10 +458,8 @@ dbsa_status dbsa_encode_blocks(const dbsa_config *cfg, const void *q, const void
   cudaError_t e;
   if ((e = cudaMemsetAsync(workspace, 0, kStatusBytes, st)) != cudaSuccess)
     return cuda_fail(e, "status clear");
-  const RopeTables rope = tables_at(workspace, L.hi, L.lo, L.n_hi);
-  if ((e = launch_rope_tables(const_cast<float2 *>(rope.hi), L.n_hi,
-                              const_cast<float2 *>(rope.lo), cfg->head_dim, cfg->rope_theta, st)) !=
-      cudaSuccess)
+  RopeTables rope;
+  if ((e = build_tables(workspace, L.rope, L.n_hi, cfg, st, &rope)) != cudaSuccess)
     return cuda_fail(e, "rope tables");
   count_launches(1);
   if ((e = cudaMemcpyAsync(at<void>(workspace, L.items), items.data(),
@@ -556,10 +553,8 @@ dbsa_status dbsa_append_block(const dbsa_config *cfg, const void *q, const void 
   cudaError_t e;
   if ((e = cudaMemsetAsync(workspace, 0, kStatusBytes, st)) != cudaSuccess)
     return cuda_fail(e, "status clear");
-  const RopeTables rope = tables_at(workspace, Ly.hi, Ly.lo, Ly.n_hi);
-  if ((e = launch_rope_tables(const_cast<float2 *>(rope.hi), Ly.n_hi,
-                              const_cast<float2 *>(rope.lo), cfg->head_dim, cfg->rope_theta, st)) !=
-      cudaSuccess)
+  RopeTables rope;
+  if ((e = build_tables(workspace, Ly.rope, Ly.n_hi, cfg, st, &rope)) != cudaSuccess)
     return cuda_fail(e, "rope tables");
   count_launches(1);
   if ((e = cudaMemcpyAsync(at<void>(workspace, Ly.items), items.data(),
@@ -684,10 +679,8 @@ dbsa_status dbsa_gather_rope_attend(const dbsa_config *cfg, const void *k_cache,
   cudaError_t e;
   if ((e = cudaMemsetAsync(workspace, 0, kStatusBytes, st)) != cudaSuccess)
     return cuda_fail(e, "status clear");
-  const RopeTables rope = tables_at(workspace, L.hi, L.lo, L.n_hi);
-  if ((e = launch_rope_tables(const_cast<float2 *>(rope.hi), L.n_hi,
-                              const_cast<float2 *>(rope.lo), cfg->head_dim, cfg->rope_theta, st)) !=
-      cudaSuccess)
+  RopeTables rope;
+  if ((e = build_tables(workspace, L.rope, L.n_hi, cfg, st, &rope)) != cudaSuccess)
     return cuda_fail(e, "rope tables");
   count_launches(1);
   // one upload of the three small plan arrays (they are contiguous in the carve)

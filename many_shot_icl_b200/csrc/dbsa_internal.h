@@ -13,19 +13,20 @@ namespace dbsa {
 
 constexpr int kTileRows = 128;   // Stage-1 query rows per tile (tcgen05 M)
 constexpr int kTileKeys = 128;   // Stage-1 keys per score tile (tcgen05 N)
-constexpr int kRopeLo = 64;      // positions per RoPE "hi" table step
-constexpr int kS2Keys = 64;      // Stage-2 keys per tile
-constexpr int kS2MaxRows = 64;   // Stage-2 query rows per CTA (4 warps x 16)
+constexpr int kRopeLo = 16;      // positions per RoPE "hi" table step
+constexpr int kRopeShift = 4;    // log2(kRopeLo)
+constexpr int kS2Keys = 64;      // Stage-2 split boundaries are multiples of this
 
 // Head of every workspace: the device status word (cleared by each call).
 constexpr size_t kStatusBytes = 256;
 
-// RoPE angle factors, built on the device in fp64 and stored as fp32
-// (cos, sin) pairs: hi[a][i] = e^{i * 64a * w_i}, lo[r][i] = e^{i * r * w_i},
-// w_i = theta^(-2i/D).  Position p uses hi[p >> 6] * lo[p & 63].
+// RoPE angle factors, built on the device in fp64 and stored as fp32 in
+// planar form: hc/hs[a][i] = cos/sin(16a * w_i), lc/ls[r][i] = cos/sin(r * w_i)
+// (r < 16), w_i = theta^(-2i/D), each [rows][D/2].  Position p uses the
+// complex product hi[p >> 4] * lo[p & 15].
 struct RopeTables {
-  const float2 *hi;
-  const float2 *lo;
+  const float *hc, *hs;
+  const float *lc, *ls;
   int32_t n_hi;
 };
 
@@ -53,8 +54,12 @@ struct S2Item {
 
 // ---- launchers (each returns cudaGetLastError() after enqueueing) ----
 
-cudaError_t launch_rope_tables(float2 *hi, int32_t n_hi, float2 *lo, int32_t head_dim,
-                               double theta, cudaStream_t st);
+// Fills the four tables (laid out back to back from `base`: hc, hs, lc, ls).
+cudaError_t launch_rope_tables(float *base, int32_t n_hi, int32_t head_dim, double theta,
+                               cudaStream_t st);
+// Table pointers inside a block of rope_table_bytes() starting at `base`.
+RopeTables rope_tables_at(const float *base, int32_t n_hi, int32_t head_dim);
+size_t rope_table_bytes(int32_t n_hi, int32_t head_dim);
 
 // Rotate Q and K of n_tok token-major input rows (positions pos0..), copy the
 // raw K/V into the cache rows pos0.., and (f32 inputs) write bf16 V.

@@ -15,22 +15,25 @@
 namespace dbsa {
 namespace {
 
-__global__ void rope_tables_kernel(float2 *hi, int32_t n_hi, float2 *lo, int32_t half,
-                                   double theta) {
+__global__ void rope_tables_kernel(float *base, int32_t n_hi, int32_t half, double theta) {
   const int64_t n = (int64_t)(n_hi + kRopeLo) * half;
+  float *hc = base, *hs = hc + (int64_t)n_hi * half;
+  float *lc = hs + (int64_t)n_hi * half, *ls = lc + (int64_t)kRopeLo * half;
   for (int64_t u = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; u < n;
        u += (int64_t)gridDim.x * blockDim.x) {
     const int32_t i = (int32_t)(u % half);
     const int64_t row = u / half;
     const double w = pow(theta, -2.0 * (double)i / (double)(2 * half));
-    double s, c;
+    double sn, cs;
     if (row < n_hi) {
-      sincos((double)(row * kRopeLo) * w, &s, &c);
-      hi[row * half + i] = make_float2((float)c, (float)s);
+      sincos((double)(row * kRopeLo) * w, &sn, &cs);
+      hc[row * half + i] = (float)cs;
+      hs[row * half + i] = (float)sn;
     } else {
       const int64_t r = row - n_hi;
-      sincos((double)r * w, &s, &c);
-      lo[r * half + i] = make_float2((float)c, (float)s);
+      sincos((double)r * w, &sn, &cs);
+      lc[r * half + i] = (float)cs;
+      ls[r * half + i] = (float)sn;
     }
   }
 }
@@ -138,11 +141,26 @@ int grid_for(int64_t n_units, int block) {
 
 }  // namespace
 
-cudaError_t launch_rope_tables(float2 *hi, int32_t n_hi, float2 *lo, int32_t head_dim,
-                               double theta, cudaStream_t st) {
+size_t rope_table_bytes(int32_t n_hi, int32_t head_dim) {
+  return (size_t)2 * (n_hi + kRopeLo) * (head_dim / 2) * sizeof(float);
+}
+
+RopeTables rope_tables_at(const float *base, int32_t n_hi, int32_t head_dim) {
+  const int64_t half = head_dim / 2;
+  RopeTables t;
+  t.hc = base;
+  t.hs = t.hc + n_hi * half;
+  t.lc = t.hs + n_hi * half;
+  t.ls = t.lc + kRopeLo * half;
+  t.n_hi = n_hi;
+  return t;
+}
+
+cudaError_t launch_rope_tables(float *base, int32_t n_hi, int32_t head_dim, double theta,
+                               cudaStream_t st) {
   const int half = head_dim / 2;
   const int64_t n = (int64_t)(n_hi + kRopeLo) * half;
-  rope_tables_kernel<<<grid_for(n, 256), 256, 0, st>>>(hi, n_hi, lo, half, theta);
+  rope_tables_kernel<<<grid_for(n, 256), 256, 0, st>>>(base, n_hi, half, theta);
   return cudaGetLastError();
 }
 

@@ -82,43 +82,34 @@ __device__ __forceinline__ uint32_t soff(int row, int chunk) {
   return (uint32_t)(row * (D * 2) + ((chunk ^ (row & 7)) << 4));
 }
 
-template <int D, typename CT>
-__device__ __forceinline__ void zero_chunk_row(uint8_t *tile, int row, int ch0, int nch) {
-  for (int ch = ch0; ch < ch0 + nch; ++ch)
-    *reinterpret_cast<uint4 *>(tile + soff<D>(row, ch)) = make_uint4(0, 0, 0, 0);
-}
-
-template <int D, typename CT>
-__device__ __forceinline__ void fetch_row(uint8_t *tile, int row, int ch0, int nch,
-                                          const CT *src) {
-  if constexpr (sizeof(CT) == 2) {
-    for (int ch = ch0; ch < ch0 + nch; ++ch) cp_async16(tile + soff<D>(row, ch), src + ch * 8);
-  } else {
-    for (int ch = ch0; ch < ch0 + nch; ++ch) {
-      float f[8];
-      load8(src + ch * 8, f);
-      store8_bf16(reinterpret_cast<bf16 *>(tile + soff<D>(row, ch)), f);
-    }
-  }
-}
-
-// KW = keys of each 64-key tile handled by one warp: 64 (each warp owns 16
-// query rows) or 16 (<= 16 rows; the four warps split the tile's keys).
-template <int D, typename CT, int KW>
-__global__ void __launch_bounds__(128) stage2_attn_kernel(const Stage2Args a) {
+// Warps form KG key groups of RT warps.  A key group streams the sub-tiles
+// j = kg, kg + KG, ... (KT keys each) of its split through its own NST-stage
+// cp.async ring; the group's RT warps own the CTA's 16-row query tiles and
+// all read the same keys, so every key is fetched from HBM and rotated once
+// per (query, KV head, row group).  Each warp keeps an online-softmax state
+// for its 16 rows; the key groups' states are merged through shared memory at
+// the end and written as one split partial.
+template <int D, typename CT, int RT, int KG, int KT, int NST>
+__global__ void __launch_bounds__(32 * RT * KG, 1) stage2_attn_kernel(const Stage2Args a) {
   constexpr int H = D / 2;
   constexpr int CH = D / 8;                 // 16-byte chunks per row
   constexpr int ROWB = D * 2;
-  constexpr int TILEB = kS2Keys * ROWB;
-  constexpr int MROWS = (KW == 64) ? 64 : 16;
-  constexpr int NB = KW / 8;                // n8 key blocks per warp
+  constexpr int NT = 32 * RT;               // threads of one key group
+  constexpr int NTOT = NT * KG;
+  constexpr int MROWS = 16 * RT;            // query rows of the CTA
+  constexpr int NB = KT / 8;                // n8 key blocks per sub-tile
   constexpr int ND = D / 8;                 // n8 dim blocks
+  static_assert(NB % 2 == 0 && KT % RT == 0, "tile shape");
+  constexpr uint32_t STAGEB = KT * ROWB;
   extern __shared__ __align__(128) uint8_t sm[];
   uint8_t *sQ = sm;
-  uint8_t *sK = sQ + MROWS * ROWB;
-  uint8_t *sV = sK + 2 * TILEB;
+  float *sLc = reinterpret_cast<float *>(sQ + MROWS * ROWB);  // RoPE lo table, [16][H] x 2
+  float *sLs = sLc + kRopeLo * H;
+  uint8_t *sRing = reinterpret_cast<uint8_t *>(sLs + kRopeLo * H);  // [KG][NST][K, V][KT][D]
 
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int kg = warp / RT, wr = warp % RT;
   const int c = blockIdx.y;
   const S2Item item = a.items[blockIdx.x];
   const S2Query qi = a.queries[item.query];
@@ -127,14 +118,26 @@ __global__ void __launch_bounds__(128) stage2_attn_kernel(const Stage2Args a) {
   const int R = g * a.n_new;
   const int Tq = qi.n_gathered;
   const int pos_first = Tq + a.tail_len - a.n_new;  // position of query token 0
-  const int row_base = (KW == 64) ? blockIdx.z * 64 : 0;
+  const int row_base = blockIdx.z * MROWS;
   const CT *kc = static_cast<const CT *>(a.k_cache);
   const CT *vc = static_cast<const CT *>(a.v_cache);
   const CT *kt = static_cast<const CT *>(a.k_tail);
   const CT *vt = static_cast<const CT *>(a.v_tail);
 
+  auto group_sync = [&]() {
+    if constexpr (RT == 1) {
+      __syncwarp();
+    } else {
+      asm volatile("bar.sync %0, %1;" ::"r"(1 + kg), "r"(NT) : "memory");
+    }
+  };
+
+  for (int u = tid; u < kRopeLo * H; u += NTOT) {
+    sLc[u] = __ldg(a.rope.lc + u);
+    sLs[u] = __ldg(a.rope.ls + u);
+  }
   // ---- query rows: rotate at their positions, store bf16 (swizzled)
-  for (int u = threadIdx.x; u < MROWS * (H / 8); u += blockDim.x) {
+  for (int u = tid; u < MROWS * (H / 8); u += NTOT) {
     const int rr = u / (H / 8), cp = u % (H / 8);
     const int r = row_base + rr;
     float lo[8], hi[8];
@@ -155,64 +158,86 @@ __global__ void __launch_bounds__(128) stage2_attn_kernel(const Stage2Args a) {
     store8_bf16(reinterpret_cast<bf16 *>(sQ + soff<D>(rr, cp + H / 8)), hi);
   }
 
-  // ---- gather: thread t fetches row (t >> 1) of every tile, chunk half (t & 1)
-  const int frow = threadIdx.x >> 1;
-  const int fch0 = (threadIdx.x & 1) * (CH / 2);
-  int seg = 0;  // per-thread segment cursor (positions only grow)
-  const int n_tiles = (item.p_end - item.p_begin + kS2Keys - 1) / kS2Keys;
-  auto issue_tile = [&](int j) {
-    const int p = item.p_begin + j * kS2Keys + frow;
-    uint8_t *dk = sK + (j & 1) * TILEB;
-    uint8_t *dv = sV + (j & 1) * TILEB;
-    if (p >= item.p_end) {
-      zero_chunk_row<D, CT>(dk, frow, fch0, CH / 2);
-      zero_chunk_row<D, CT>(dv, frow, fch0, CH / 2);
-      return;
-    }
-    const CT *ks, *vs;
-    if (p < Tq) {
-      while (seg + 1 < qi.n_seg && __ldg(&a.segs[qi.seg_begin + seg + 1].pos0) <= p) ++seg;
-      const S2Segment sg = a.segs[qi.seg_begin + seg];
-      const int64_t crow = (int64_t)sg.cache_row0 + (p - sg.pos0);
-      ks = kc + ((int64_t)c * a.cap + crow) * D;
-      vs = vc + ((int64_t)c * a.cap + crow) * D;
-      if (a.dbg_map != nullptr && c == 0 && blockIdx.z == 0 && fch0 == 0) {
-        int32_t *m = a.dbg_map + ((int64_t)q * a.dbg_cap + p) * 2;
-        m[0] = (int32_t)crow;
-        m[1] = p;
+  // ---- gather: warp wr of a key group loads (and later rotates) rows
+  // [wr * RPW, (wr + 1) * RPW) of each sub-tile.  Lane l (l < RPW) resolves
+  // the cache row of row l for K, lane 16 + l the same row for V; then every
+  // copy instruction moves one whole K row (lanes 0-15) and one whole V row
+  // (lanes 16-31), 256 contiguous bytes each.
+  constexpr int RPW = KT / RT;
+  static_assert(RPW <= 16 && CH <= 16, "one row per half-warp");
+  const int n_sub = (item.p_end - item.p_begin + KT - 1) / KT;
+  const int n_local = kg < n_sub ? (n_sub - kg + KG - 1) / KG : 0;
+  const int half_id = lane >> 4, hl = lane & 15;  // half-warp: 0 = K, 1 = V
+  int seg = 0;  // segment cursor: this lane's positions only grow
+  auto stage_ptr = [&](int jl, int kv) -> uint8_t * {
+    return sRing + ((size_t)(kg * NST + jl % NST) * 2 + kv) * STAGEB;
+  };
+  auto issue = [&](int jl) {
+    const int p0 = item.p_begin + (kg + jl * KG) * KT + wr * RPW;
+    // this lane's row pointer (lanes hl < RPW); null past the split end
+    const CT *my = nullptr;
+    if (hl < RPW) {
+      const int p = p0 + hl;
+      if (p < item.p_end) {
+        if (p < Tq) {
+          while (seg + 1 < qi.n_seg && __ldg(&a.segs[qi.seg_begin + seg + 1].pos0) <= p) ++seg;
+          const int64_t crow = (int64_t)__ldg(&a.segs[qi.seg_begin + seg].cache_row0) +
+                               (p - __ldg(&a.segs[qi.seg_begin + seg].pos0));
+          my = (half_id ? vc : kc) + ((int64_t)c * a.cap + crow) * D;
+          if (a.dbg_map != nullptr && c == 0 && blockIdx.z == 0 && half_id == 0) {
+            int32_t *m = a.dbg_map + ((int64_t)q * a.dbg_cap + p) * 2;
+            m[0] = (int32_t)crow;
+            m[1] = p;
+          }
+        } else {
+          const int64_t w = p - Tq;
+          my = (half_id ? vt : kt) + (((int64_t)q * a.tail_cap + w) * a.Hkv + c) * D;
+        }
       }
-    } else {
-      const int64_t w = p - Tq;
-      ks = kt + (((int64_t)q * a.tail_cap + w) * a.Hkv + c) * D;
-      vs = vt + (((int64_t)q * a.tail_cap + w) * a.Hkv + c) * D;
     }
-    fetch_row<D, CT>(dk, frow, fch0, CH / 2, ks);
-    fetch_row<D, CT>(dv, frow, fch0, CH / 2, vs);
+    uint8_t *dst = stage_ptr(jl, half_id);
+#pragma unroll 4
+    for (int r = 0; r < RPW; ++r) {
+      const CT *src = reinterpret_cast<const CT *>(
+          __shfl_sync(0xFFFFFFFFu, reinterpret_cast<unsigned long long>(my), (half_id << 4) + r));
+      if (hl < CH) {
+        uint8_t *d = dst + soff<D>(wr * RPW + r, hl);
+        if (src == nullptr) {
+          *reinterpret_cast<uint4 *>(d) = make_uint4(0, 0, 0, 0);
+        } else if constexpr (sizeof(CT) == 2) {
+          cp_async16(d, src + hl * 8);
+        } else {
+          float f[8];
+          load8(src + hl * 8, f);
+          store8_bf16(reinterpret_cast<bf16 *>(d), f);
+        }
+      }
+    }
   };
 
-  if (n_tiles > 0) issue_tile(0);
-  cp_async_commit();
-  __syncthreads();
+#pragma unroll
+  for (int s0 = 0; s0 < NST - 1; ++s0) {
+    if (s0 < n_local) issue(s0);
+    cp_async_commit();
+  }
+  __syncthreads();  // sQ complete
 
-  // ---- Q fragments (A operand), kept in registers for the whole split
-  const int wrow = (KW == 64) ? warp * 16 : 0;  // first query row of this warp (in sQ)
+  // ---- Q fragments (A operand) of this warp's 16 rows, kept in registers
   uint32_t qf[D / 16][4];
   {
-    const int r = wrow + (lane & 7) + ((lane >> 3) & 1) * 8;
+    const int r = wr * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
     for (int ks = 0; ks < D / 16; ++ks)
       ldsm_x4(smem_u32(sQ) + soff<D>(r, 2 * ks + (lane >> 4)), qf[ks][0], qf[ks][1], qf[ks][2],
               qf[ks][3]);
   }
-  // positions of this thread's two rows (g and g + 8 of the warp's 16)
   const int gq = lane >> 2, tq = lane & 3;
   int qpos[2];
 #pragma unroll
   for (int h2 = 0; h2 < 2; ++h2) {
-    const int r = row_base + wrow + gq + 8 * h2;
+    const int r = row_base + wr * 16 + gq + 8 * h2;
     qpos[h2] = (r < R) ? pos_first + r / g : INT_MAX;
   }
-  const int kw0 = (KW == 64) ? 0 : warp * 16;  // this warp's keys inside a tile
 
   float o[ND][4];
 #pragma unroll
@@ -220,35 +245,61 @@ __global__ void __launch_bounds__(128) stage2_attn_kernel(const Stage2Args a) {
   float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
   const float sl2 = a.scale_log2;
 
-  for (int j = 0; j < n_tiles; ++j) {
-    if (j + 1 < n_tiles) issue_tile(j + 1);
+  for (int jl = 0; jl < n_local; ++jl) {
+    cp_async_wait<NST - 2>();
+    group_sync();
+    if (jl + NST - 1 < n_local) issue(jl + NST - 1);
     cp_async_commit();
-    cp_async_wait<1>();
-    __syncthreads();
-    const int p0 = item.p_begin + j * kS2Keys;
-    uint8_t *tk = sK + (j & 1) * TILEB;
-    uint8_t *tv = sV + (j & 1) * TILEB;
-    // ---- re-rotate the raw keys at their fresh positions p0 + row
+    const int p0 = item.p_begin + (kg + jl * KG) * KT;
+    uint8_t *tk = stage_ptr(jl, 0);
+    uint8_t *tv = stage_ptr(jl, 1);
+    // ---- re-rotate this warp's rows of the sub-tile at their fresh positions
+    // p0 + row.  Lane = frequency pair(s); the rows of one warp share one
+    // 16-position group, hence one "hi" factor, and the "lo" factors come
+    // from shared memory.
     {
-      const int row = threadIdx.x >> 1;
-      const int i_base = (threadIdx.x & 1) * (H / 2);
-#pragma unroll
-      for (int cc = 0; cc < H / 16; ++cc) {
-        const int i0 = i_base + cc * 8;
-        bf16 *plo = reinterpret_cast<bf16 *>(tk + soff<D>(row, i0 / 8));
-        bf16 *phi = reinterpret_cast<bf16 *>(tk + soff<D>(row, (H + i0) / 8));
-        float lo[8], hi[8], cs[8], sn[8];
-        load8(plo, lo);
-        load8(phi, hi);
-        rope_cs8(a.rope, (int64_t)p0 + row, i0, H, cs, sn);
-        rotate8(lo, hi, cs, sn);
-        store8_bf16(plo, lo);
-        store8_bf16(phi, hi);
+      static_assert(RPW <= kRopeLo && kRopeLo % RPW == 0, "a warp's rows share one hi factor");
+      const int r0 = wr * RPW;
+      const int64_t hoff = (int64_t)((p0 + r0) >> kRopeShift) * H;
+      if constexpr (H == 64) {
+        const int i = 2 * lane;
+        const f32x2 hcos = *reinterpret_cast<const f32x2 *>(a.rope.hc + hoff + i);
+        const f32x2 hsin = *reinterpret_cast<const f32x2 *>(a.rope.hs + hoff + i);
+        const f32x2 nhsin = f2_neg(hsin);
+#pragma unroll 4
+        for (int r = r0; r < r0 + RPW; ++r) {
+          const int lr = (p0 + r) & (kRopeLo - 1);
+          const f32x2 lcos = *reinterpret_cast<const f32x2 *>(sLc + lr * H + i);
+          const f32x2 lsin = *reinterpret_cast<const f32x2 *>(sLs + lr * H + i);
+          const f32x2 cs = f2_fma(hcos, lcos, f2_mul(nhsin, lsin));
+          const f32x2 sn = f2_fma(hcos, lsin, f2_mul(hsin, lcos));
+          uint32_t *plo = reinterpret_cast<uint32_t *>(tk + soff<D>(r, i >> 3) + (i & 7) * 2);
+          uint32_t *phi = reinterpret_cast<uint32_t *>(tk + soff<D>(r, (H + i) >> 3) + (i & 7) * 2);
+          const f32x2 xl = f2_from_bf16x2(*plo), xh = f2_from_bf16x2(*phi);
+          *plo = f2_to_bf16x2(f2_fma(xl, cs, f2_mul(f2_neg(xh), sn)));
+          *phi = f2_to_bf16x2(f2_fma(xh, cs, f2_mul(xl, sn)));
+        }
+      } else {
+        static_assert(H == 32, "head_dim 64 or 128");
+        const int i = lane;
+        const float hcos = a.rope.hc[hoff + i], hsin = a.rope.hs[hoff + i];
+#pragma unroll 4
+        for (int r = r0; r < r0 + RPW; ++r) {
+          const int lr = (p0 + r) & (kRopeLo - 1);
+          const float lcos = sLc[lr * H + i], lsin = sLs[lr * H + i];
+          const float cs = __fmaf_rn(hcos, lcos, __fmul_rn(-hsin, lsin));
+          const float sn = __fmaf_rn(hcos, lsin, __fmul_rn(hsin, lcos));
+          bf16 *plo = reinterpret_cast<bf16 *>(tk + soff<D>(r, i >> 3)) + (i & 7);
+          bf16 *phi = reinterpret_cast<bf16 *>(tk + soff<D>(r, (H + i) >> 3)) + (i & 7);
+          const float xl = __bfloat162float(*plo), xh = __bfloat162float(*phi);
+          *plo = __float2bfloat16_rn(__fmaf_rn(xl, cs, __fmul_rn(-xh, sn)));
+          *phi = __float2bfloat16_rn(__fmaf_rn(xh, cs, __fmul_rn(xl, sn)));
+        }
       }
     }
-    __syncthreads();
+    group_sync();
 
-    // ---- S = Q K^T for this warp's 16 rows x KW keys
+    // ---- S = Q K^T for this warp's 16 rows x KT keys
     float s[NB][4];
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb) s[nb][0] = s[nb][1] = s[nb][2] = s[nb][3] = 0.f;
@@ -257,15 +308,15 @@ __global__ void __launch_bounds__(128) stage2_attn_kernel(const Stage2Args a) {
 #pragma unroll
       for (int nb = 0; nb < NB; nb += 2) {
         const int mi = lane >> 3;
-        const int krow = kw0 + (nb + (mi >> 1)) * 8 + (lane & 7);
+        const int krow = (nb + (mi >> 1)) * 8 + (lane & 7);
         uint32_t b0, b1, b2, b3;
         ldsm_x4(smem_u32(tk) + soff<D>(krow, 2 * ks + (mi & 1)), b0, b1, b2, b3);
         mma16816(s[nb], qf[ks], b0, b1);
         mma16816(s[nb + 1], qf[ks], b2, b3);
       }
     }
-    // ---- mask (split end, causal inside the query's own tail), online softmax
-    const bool need_mask = (p0 + kS2Keys > item.p_end) || (p0 + kS2Keys - 1 > pos_first);
+    // ---- mask (split end; causal inside the query's own tail), online softmax
+    const bool need_mask = (p0 + KT > item.p_end) || (p0 + KT - 1 > pos_first);
     float tmax[2] = {-INFINITY, -INFINITY};
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb)
@@ -273,29 +324,32 @@ __global__ void __launch_bounds__(128) stage2_attn_kernel(const Stage2Args a) {
       for (int e = 0; e < 4; ++e) {
         float x = s[nb][e] * sl2;
         if (need_mask) {
-          const int kp = p0 + kw0 + nb * 8 + 2 * tq + (e & 1);
+          const int kp = p0 + nb * 8 + 2 * tq + (e & 1);
           if (kp >= item.p_end || kp > qpos[e >> 1]) x = -INFINITY;
         }
         s[nb][e] = x;
         tmax[e >> 1] = fmaxf(tmax[e >> 1], x);
       }
-    float alpha[2], mu[2];
+    // Lazy rescale: the running max only moves (and O, l are rescaled) when
+    // a row's new scores exceed it by more than 2^8; until then the stale max
+    // keeps every exponent <= 2^8, which fp32 and bf16 P hold without loss.
+    float mu[2];
 #pragma unroll
     for (int h2 = 0; h2 < 2; ++h2) {
       tmax[h2] = fmaxf(tmax[h2], __shfl_xor_sync(0xFFFFFFFFu, tmax[h2], 1));
       tmax[h2] = fmaxf(tmax[h2], __shfl_xor_sync(0xFFFFFFFFu, tmax[h2], 2));
-      const float mn = fmaxf(m_run[h2], tmax[h2]);
-      alpha[h2] = (mn == -INFINITY) ? 1.f : ex2(m_run[h2] - mn);
-      m_run[h2] = mn;
-      mu[h2] = (mn == -INFINITY) ? 0.f : mn;
-      l_run[h2] *= alpha[h2];
-    }
+      if (tmax[h2] > m_run[h2] + 8.0f) {
+        const float mn = tmax[h2];
+        const float alpha = (m_run[h2] == -INFINITY) ? 0.f : ex2(m_run[h2] - mn);
+        m_run[h2] = mn;
+        l_run[h2] *= alpha;
 #pragma unroll
-    for (int nd = 0; nd < ND; ++nd) {
-      o[nd][0] *= alpha[0];
-      o[nd][1] *= alpha[0];
-      o[nd][2] *= alpha[1];
-      o[nd][3] *= alpha[1];
+        for (int nd = 0; nd < ND; ++nd) {
+          o[nd][2 * h2] *= alpha;
+          o[nd][2 * h2 + 1] *= alpha;
+        }
+      }
+      mu[h2] = (m_run[h2] == -INFINITY) ? 0.f : m_run[h2];
     }
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb)
@@ -307,14 +361,14 @@ __global__ void __launch_bounds__(128) stage2_attn_kernel(const Stage2Args a) {
       }
     // ---- O += P V
 #pragma unroll
-    for (int kk = 0; kk < KW / 16; ++kk) {
+    for (int kk = 0; kk < KT / 16; ++kk) {
       uint32_t pa[4];
       pa[0] = pack_bf16(s[2 * kk][0], s[2 * kk][1]);
       pa[1] = pack_bf16(s[2 * kk][2], s[2 * kk][3]);
       pa[2] = pack_bf16(s[2 * kk + 1][0], s[2 * kk + 1][1]);
       pa[3] = pack_bf16(s[2 * kk + 1][2], s[2 * kk + 1][3]);
       const int mi = lane >> 3;
-      const int vrow = kw0 + kk * 16 + (mi & 1) * 8 + (lane & 7);
+      const int vrow = kk * 16 + (mi & 1) * 8 + (lane & 7);
 #pragma unroll
       for (int nd = 0; nd < ND; nd += 2) {
         uint32_t b0, b1, b2, b3;
@@ -323,7 +377,6 @@ __global__ void __launch_bounds__(128) stage2_attn_kernel(const Stage2Args a) {
         mma16816(o[nd + 1], pa, b2, b3);
       }
     }
-    __syncthreads();  // tile j's buffers may be refilled by iteration j + 1
   }
   cp_async_wait<0>();
 
@@ -333,16 +386,15 @@ __global__ void __launch_bounds__(128) stage2_attn_kernel(const Stage2Args a) {
     l_run[h2] += __shfl_xor_sync(0xFFFFFFFFu, l_run[h2], 1);
     l_run[h2] += __shfl_xor_sync(0xFFFFFFFFu, l_run[h2], 2);
   }
-
-  auto part_index = [&](int r) -> int64_t {  // r = query row (GQA row) index
+  auto part_index = [&](int r) -> int64_t {  // r = GQA row index (token-major)
     const int tok = r / g, h = c * g + r % g;
     return ((int64_t)blockIdx.x * a.Hq + h) * a.n_new + tok;
   };
 
-  if constexpr (KW == 64) {
+  if constexpr (KG == 1) {
 #pragma unroll
     for (int h2 = 0; h2 < 2; ++h2) {
-      const int r = row_base + wrow + gq + 8 * h2;
+      const int r = row_base + wr * 16 + gq + 8 * h2;
       if (r >= R) continue;
       const int64_t pi = part_index(r);
       float *acc = a.part_acc + pi * D;
@@ -353,43 +405,43 @@ __global__ void __launch_bounds__(128) stage2_attn_kernel(const Stage2Args a) {
       if (tq == 0) a.part_ml[pi] = make_float2(m_run[h2], l_run[h2]);
     }
   } else {
-    // merge the four warps' partial states for the 16 rows through shared memory
+    // merge the key groups' states for the CTA's rows through shared memory
     __syncthreads();
-    float *so = reinterpret_cast<float *>(sK);          // [4][16][D]
-    float2 *sml = reinterpret_cast<float2 *>(so + 4 * 16 * D);  // [4][16]
+    float *so = reinterpret_cast<float *>(sRing);                  // [KG][MROWS][D]
+    float2 *sml = reinterpret_cast<float2 *>(so + KG * MROWS * D);  // [KG][MROWS]
 #pragma unroll
     for (int h2 = 0; h2 < 2; ++h2) {
-      const int r = gq + 8 * h2;
+      const int rr = wr * 16 + gq + 8 * h2;
 #pragma unroll
       for (int nd = 0; nd < ND; ++nd)
-        *reinterpret_cast<float2 *>(so + (warp * 16 + r) * D + nd * 8 + 2 * tq) =
+        *reinterpret_cast<float2 *>(so + ((size_t)kg * MROWS + rr) * D + nd * 8 + 2 * tq) =
             make_float2(o[nd][2 * h2], o[nd][2 * h2 + 1]);
-      if (tq == 0) sml[warp * 16 + r] = make_float2(m_run[h2], l_run[h2]);
+      if (tq == 0) sml[kg * MROWS + rr] = make_float2(m_run[h2], l_run[h2]);
     }
     __syncthreads();
-    // 128 threads: row = t / 8, dims [(t % 8) * D/8, +D/8)
-    const int r = threadIdx.x >> 3;
-    const int d0 = (threadIdx.x & 7) * (D / 8);
-    if (r < R) {
+    for (int idx = tid; idx < MROWS * (D / 4); idx += NTOT) {
+      const int rr = idx / (D / 4), d0 = (idx % (D / 4)) * 4;
+      const int r = row_base + rr;
+      if (r >= R) continue;
       float M = -INFINITY;
 #pragma unroll
-      for (int w = 0; w < 4; ++w) M = fmaxf(M, sml[w * 16 + r].x);
-      float wgt[4], L = 0.f;
+      for (int k = 0; k < KG; ++k) M = fmaxf(M, sml[k * MROWS + rr].x);
+      float L = 0.f;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        const float2 ml = sml[w * 16 + r];
-        wgt[w] = (ml.x == -INFINITY) ? 0.f : ex2(ml.x - M);
-        L += ml.y * wgt[w];
+      for (int k = 0; k < KG; ++k) {
+        const float2 ml = sml[k * MROWS + rr];
+        const float w = (ml.x == -INFINITY) ? 0.f : ex2(ml.x - M);
+        L += w * ml.y;
+        const float4 x = *reinterpret_cast<const float4 *>(so + ((size_t)k * MROWS + rr) * D + d0);
+        acc.x += w * x.x;
+        acc.y += w * x.y;
+        acc.z += w * x.z;
+        acc.w += w * x.w;
       }
       const int64_t pi = part_index(r);
-      float *acc = a.part_acc + pi * D;
-      for (int d = d0; d < d0 + D / 8; ++d) {
-        float x = 0.f;
-#pragma unroll
-        for (int w = 0; w < 4; ++w) x += wgt[w] * so[(w * 16 + r) * D + d];
-        acc[d] = x;
-      }
-      if ((threadIdx.x & 7) == 0) a.part_ml[pi] = make_float2(M, L);
+      *reinterpret_cast<float4 *>(a.part_acc + pi * D + d0) = acc;
+      if (d0 == 0) a.part_ml[pi] = make_float2(M, L);
     }
   }
 }
@@ -436,26 +488,35 @@ __global__ void __launch_bounds__(128) stage2_merge_kernel(const Stage2Args a) {
   }
 }
 
-template <int D, typename CT, int KW>
+template <int D, typename CT, int RT, int KG, int KT>
 cudaError_t launch_main(const Stage2Args &a, cudaStream_t st) {
-  constexpr int MROWS = (KW == 64) ? 64 : 16;
-  constexpr size_t smem = (size_t)MROWS * D * 2 + 4 * (size_t)kS2Keys * D * 2;
-  static_assert(KW == 64 || smem >= 4 * 16 * D * 4 + 4 * 16 * 8, "merge scratch fits");
-  cudaError_t e = cudaFuncSetAttribute(stage2_attn_kernel<D, CT, KW>,
+  constexpr int NST = 3;
+  constexpr int MROWS = 16 * RT;
+  constexpr size_t ring = (size_t)KG * NST * 2 * KT * D * 2;
+  constexpr size_t merge = KG > 1 ? (size_t)KG * MROWS * (D * 4 + 8) : 0;
+  constexpr size_t lo_tables = (size_t)2 * kRopeLo * (D / 2) * sizeof(float);
+  constexpr size_t smem = (size_t)MROWS * D * 2 + lo_tables + (ring > merge ? ring : merge);
+  static_assert(smem <= 232448, "shared memory budget");
+  cudaError_t e = cudaFuncSetAttribute(stage2_attn_kernel<D, CT, RT, KG, KT, NST>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const int g = a.Hq / a.Hkv;
-  const int R = g * a.n_new;
-  const int zdim = (KW == 64) ? (R + 63) / 64 : 1;
-  dim3 grid(a.n_items, a.Hkv, zdim);
-  stage2_attn_kernel<D, CT, KW><<<grid, 128, smem, st>>>(a);
+  const int R = (a.Hq / a.Hkv) * a.n_new;
+  dim3 grid(a.n_items, a.Hkv, (R + MROWS - 1) / MROWS);
+  stage2_attn_kernel<D, CT, RT, KG, KT, NST><<<grid, 32 * RT * KG, smem, st>>>(a);
   return cudaGetLastError();
 }
 
+// Rows per CTA by pass shape (kept in step with the host split planner):
+// <= 16 rows (decode): 8 key groups of 1 warp; <= 32: 4 x 2; <= 64: 2 x 4;
+// <= 128: 1 x 8; larger: 1 x 10 warps (160 rows) per row group.
 template <int D, typename CT>
 cudaError_t launch_d(const Stage2Args &a, cudaStream_t st) {
   const int R = (a.Hq / a.Hkv) * a.n_new;
-  return (R <= 16) ? launch_main<D, CT, 16>(a, st) : launch_main<D, CT, 64>(a, st);
+  if (R <= 16) return launch_main<D, CT, 1, 8, 16>(a, st);
+  if (R <= 32) return launch_main<D, CT, 2, 4, 32>(a, st);
+  if (R <= 64) return launch_main<D, CT, 4, 2, 64>(a, st);
+  if (R <= 128) return launch_main<D, CT, 8, 1, 64>(a, st);
+  return launch_main<D, CT, 10, 1, 80>(a, st);
 }
 
 template <int D, typename CT>

@@ -11,18 +11,24 @@ namespace dbsa {
 
 using bf16 = __nv_bfloat16;
 
-// (cos, sin) of p * w_i for the 8 frequencies i0..i0+7, as hi[p >> 6] * lo[p & 63].
+// (cos, sin) of p * w_i for the 8 frequencies i0..i0+7, as the complex
+// product hi[p >> 4] * lo[p & 15] (rounding pinned as in cmul below).
 __device__ __forceinline__ void rope_cs8(const RopeTables &t, int64_t p, int i0, int half,
                                          float (&c)[8], float (&s)[8]) {
-  const float4 *h4 = reinterpret_cast<const float4 *>(t.hi + (p >> 6) * half + i0);
-  const float4 *l4 = reinterpret_cast<const float4 *>(t.lo + (p & 63) * half + i0);
+  const int64_t hoff = (p >> kRopeShift) * half + i0, loff = (p & (kRopeLo - 1)) * half + i0;
 #pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const float4 a = __ldg(h4 + e), b = __ldg(l4 + e);
-    c[2 * e] = __fmaf_rn(a.x, b.x, __fmul_rn(-a.y, b.y));
-    s[2 * e] = __fmaf_rn(a.x, b.y, __fmul_rn(a.y, b.x));
-    c[2 * e + 1] = __fmaf_rn(a.z, b.z, __fmul_rn(-a.w, b.w));
-    s[2 * e + 1] = __fmaf_rn(a.z, b.w, __fmul_rn(a.w, b.z));
+  for (int e = 0; e < 2; ++e) {
+    const float4 hc = __ldg(reinterpret_cast<const float4 *>(t.hc + hoff) + e);
+    const float4 hs = __ldg(reinterpret_cast<const float4 *>(t.hs + hoff) + e);
+    const float4 lc = __ldg(reinterpret_cast<const float4 *>(t.lc + loff) + e);
+    const float4 ls = __ldg(reinterpret_cast<const float4 *>(t.ls + loff) + e);
+    const float ac[4] = {hc.x, hc.y, hc.z, hc.w}, as[4] = {hs.x, hs.y, hs.z, hs.w};
+    const float bc[4] = {lc.x, lc.y, lc.z, lc.w}, bs[4] = {ls.x, ls.y, ls.z, ls.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      c[4 * e + k] = __fmaf_rn(ac[k], bc[k], __fmul_rn(-as[k], bs[k]));
+      s[4 * e + k] = __fmaf_rn(ac[k], bs[k], __fmul_rn(as[k], bc[k]));
+    }
   }
 }
 
@@ -58,6 +64,39 @@ __device__ __forceinline__ void copy8(const bf16 *src, bf16 *dst) {
 __device__ __forceinline__ void copy8(const float *src, float *dst) {
   reinterpret_cast<float4 *>(dst)[0] = reinterpret_cast<const float4 *>(src)[0];
   reinterpret_cast<float4 *>(dst)[1] = reinterpret_cast<const float4 *>(src)[1];
+}
+
+// Packed pairs of fp32 (sm_100 f32x2 arithmetic: two independent IEEE fp32
+// operations per instruction, each rounded exactly like its scalar form).
+using f32x2 = unsigned long long;
+__device__ __forceinline__ f32x2 f2_pack(float a, float b) {
+  f32x2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(f32x2 r, float &a, float &b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ f32x2 f2_fma(f32x2 a, f32x2 b, f32x2 c) {
+  f32x2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ f32x2 f2_mul(f32x2 a, f32x2 b) {
+  f32x2 d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f32x2 f2_neg(f32x2 a) { return a ^ 0x8000000080000000ull; }
+// bf16 pair (low half = first element) <-> packed fp32 pair
+__device__ __forceinline__ f32x2 f2_from_bf16x2(uint32_t w) {
+  return f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+__device__ __forceinline__ uint32_t f2_to_bf16x2(f32x2 v) {
+  float a, b;
+  f2_unpack(v, a, b);
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t *>(&h);
 }
 
 // y_i = x_i c - x_{i+h} s ; y_{i+h} = x_{i+h} c + x_i s  (rotate-half RoPE).
