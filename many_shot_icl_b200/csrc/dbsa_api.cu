@@ -227,7 +227,16 @@ struct GatherPlan {
   std::vector<S2Segment> segs;
   std::vector<S2Item> items;
   int32_t max_pos;  // largest key / query position + 1
+  // block-major mode (single-token passes): per (block, query group) entries;
+  // the per-query kernel then runs only the tail items listed in run_items
+  bool block_major = false;
+  std::vector<S2BEntry> bm_entries;
+  std::vector<S2BSlot> bm_slots;
+  std::vector<int32_t> run_items;
 };
+
+// Queries (rows) per block-major entry: the kernel's CTA holds 64 rows.
+constexpr int kBMRows = 64;
 
 dbsa_status gather_plan(const dbsa_config *cfg, const int32_t *offs, int32_t nb, int32_t nq,
                         const int32_t *sel_ptr, const int32_t *sel, int32_t n_new,
@@ -284,6 +293,54 @@ dbsa_status gather_plan(const dbsa_config *cfg, const int32_t *offs, int32_t nb,
       (total_keys * cfg->n_kv_heads * zdim + want_ctas - 1) / std::max<int64_t>(1, want_ctas);
   int64_t chunk = std::max(min_chunk, par_chunk);
   chunk = (chunk + kS2Keys - 1) / kS2Keys * kS2Keys;
+  if (R <= 16) {
+    // Single-token passes: block-major.  Items per query = one per selected
+    // block (filled by the block-major kernel) + one for its own tail tokens
+    // (per-query kernel).  Entries group the queries that selected a block.
+    gp.block_major = true;
+    std::vector<std::vector<S2BSlot>> per_block(nb);
+    for (int q = 0; q < nq; ++q) {
+      S2Query &qi = gp.queries[q];
+      qi.item_begin = (int32_t)gp.items.size();
+      for (int sgi = 0; sgi < qi.n_seg; ++sgi) {
+        const S2Segment &sg = gp.segs[qi.seg_begin + sgi];
+        S2Item it;
+        it.query = q;
+        it.p_begin = sg.pos0;
+        it.p_end = sg.pos0 + sg.len;
+        it.p_lo = sg.pos0;
+        S2BSlot sl;
+        sl.query = q;
+        sl.pos0 = sg.pos0;
+        sl.item = (int32_t)gp.items.size();
+        sl.pad = 0;
+        per_block[sel[sel_ptr[q] + sgi]].push_back(sl);
+        gp.items.push_back(it);
+      }
+      S2Item tail;
+      tail.query = q;
+      tail.p_begin = qi.n_gathered & ~(kRopeLo - 1);  // aligned start; keys below
+      tail.p_end = qi.n_gathered + tail_len;          // n_gathered are masked
+      tail.p_lo = qi.n_gathered;
+      gp.run_items.push_back((int32_t)gp.items.size());
+      gp.items.push_back(tail);
+      qi.n_items = (int32_t)gp.items.size() - qi.item_begin;
+    }
+    const int qpc = std::max(1, kBMRows / R);
+    for (int b = 0; b < nb; ++b) {
+      const auto &v = per_block[b];
+      for (size_t i0 = 0; i0 < v.size(); i0 += qpc) {
+        S2BEntry e;
+        e.cache_row0 = offs[b];
+        e.len = offs[b + 1] - offs[b];
+        e.slot_begin = (int32_t)gp.bm_slots.size();
+        e.n_slots = (int32_t)std::min<size_t>(qpc, v.size() - i0);
+        for (int k = 0; k < e.n_slots; ++k) gp.bm_slots.push_back(v[i0 + k]);
+        gp.bm_entries.push_back(e);
+      }
+    }
+    return DBSA_OK;
+  }
   for (int q = 0; q < nq; ++q) {
     S2Query &qi = gp.queries[q];
     const int64_t K = (int64_t)qi.n_gathered + tail_len;
@@ -296,7 +353,7 @@ dbsa_status gather_plan(const dbsa_config *cfg, const int32_t *offs, int32_t nb,
       it.query = q;
       it.p_begin = (int32_t)s0;
       it.p_end = (int32_t)std::min<int64_t>(K, s0 + per);
-      it.pad = 0;
+      it.p_lo = it.p_begin;
       gp.items.push_back(it);
     }
     qi.n_items = (int32_t)gp.items.size() - qi.item_begin;
@@ -325,7 +382,7 @@ S1Layout s1_layout(const dbsa_config *cfg, int64_t max_pos, int64_t n_items, int
 }
 
 struct S2Layout {
-  size_t rope, queries, segs, items, part_acc, part_ml, total;
+  size_t rope, queries, segs, items, bm_entries, bm_slots, run_items, part_acc, part_ml, total;
   int32_t n_hi;
 };
 S2Layout s2_layout(const dbsa_config *cfg, const GatherPlan &gp, int32_t n_new) {
@@ -336,6 +393,9 @@ S2Layout s2_layout(const dbsa_config *cfg, const GatherPlan &gp, int32_t n_new) 
   l.queries = cv.take(gp.queries.size() * sizeof(S2Query));
   l.segs = cv.take(gp.segs.size() * sizeof(S2Segment));
   l.items = cv.take(gp.items.size() * sizeof(S2Item));
+  l.bm_entries = cv.take(gp.bm_entries.size() * sizeof(S2BEntry));
+  l.bm_slots = cv.take(gp.bm_slots.size() * sizeof(S2BSlot));
+  l.run_items = cv.take(gp.run_items.size() * sizeof(int32_t));
   const size_t rows = gp.items.size() * (size_t)cfg->n_q_heads * n_new;
   l.part_acc = cv.take(rows * cfg->head_dim * sizeof(float));
   l.part_ml = cv.take(rows * sizeof(float2));
@@ -691,6 +751,14 @@ dbsa_status dbsa_gather_rope_attend(const dbsa_config *cfg, const void *k_cache,
                 gp.segs.size() * sizeof(S2Segment));
     std::memcpy(blob.data() + (L.items - L.queries), gp.items.data(),
                 gp.items.size() * sizeof(S2Item));
+    if (gp.block_major) {
+      std::memcpy(blob.data() + (L.bm_entries - L.queries), gp.bm_entries.data(),
+                  gp.bm_entries.size() * sizeof(S2BEntry));
+      std::memcpy(blob.data() + (L.bm_slots - L.queries), gp.bm_slots.data(),
+                  gp.bm_slots.size() * sizeof(S2BSlot));
+      std::memcpy(blob.data() + (L.run_items - L.queries), gp.run_items.data(),
+                  gp.run_items.size() * sizeof(int32_t));
+    }
     if ((e = cudaMemcpyAsync(at<void>(workspace, L.queries), blob.data(), blob.size(),
                              cudaMemcpyHostToDevice, st)) != cudaSuccess)
       return cuda_fail(e, "gather plan upload");
@@ -712,6 +780,11 @@ dbsa_status dbsa_gather_rope_attend(const dbsa_config *cfg, const void *k_cache,
   a.items = at<S2Item>(workspace, L.items);
   a.n_items = (int32_t)gp.items.size();
   a.n_queries = nq;
+  a.run_items = gp.block_major ? at<int32_t>(workspace, L.run_items) : nullptr;
+  a.n_run = (int32_t)gp.run_items.size();
+  a.bm_entries = gp.block_major ? at<S2BEntry>(workspace, L.bm_entries) : nullptr;
+  a.bm_slots = gp.block_major ? at<S2BSlot>(workspace, L.bm_slots) : nullptr;
+  a.n_bm_entries = (int32_t)gp.bm_entries.size();
   a.part_acc = at<float>(workspace, L.part_acc);
   a.part_ml = at<float2>(workspace, L.part_ml);
   a.out = out;

@@ -89,7 +89,13 @@ __device__ __forceinline__ uint32_t soff(int row, int chunk) {
 // per (query, KV head, row group).  Each warp keeps an online-softmax state
 // for its 16 rows; the key groups' states are merged through shared memory at
 // the end and written as one split partial.
-template <int D, typename CT, int RT, int KG, int KT, int NST>
+//
+// BM (block-major) selects the single-token pass layout: the CTA's keys are
+// one selected block (positions r = 0..L-1 relative to the block, rotated
+// by r), its rows are the g * n_new rows of each query in the entry's slot
+// list (each rotated by its position minus the block's fresh start), and
+// there is no causal limit (every gathered key precedes the query tokens).
+template <int D, typename CT, int RT, int KG, int KT, int NST, bool BM>
 __global__ void __launch_bounds__(32 * RT * KG, 1) stage2_attn_kernel(const Stage2Args a) {
   constexpr int H = D / 2;
   constexpr int CH = D / 8;                 // 16-byte chunks per row
@@ -111,13 +117,30 @@ __global__ void __launch_bounds__(32 * RT * KG, 1) stage2_attn_kernel(const Stag
   const int warp = tid >> 5, lane = tid & 31;
   const int kg = warp / RT, wr = warp % RT;
   const int c = blockIdx.y;
-  const S2Item item = a.items[blockIdx.x];
-  const S2Query qi = a.queries[item.query];
-  const int q = item.query;
   const int g = a.Hq / a.Hkv;
-  const int R = g * a.n_new;
-  const int Tq = qi.n_gathered;
-  const int pos_first = Tq + a.tail_len - a.n_new;  // position of query token 0
+  const int RQ = g * a.n_new;                      // rows of one query
+  // per-query mode: one split item; block-major mode: one (block, queries) entry
+  int it_idx = 0, q = 0, Tq = 0, k_begin, k_end, k_lo, R;
+  S2Query qi;
+  S2BEntry be;
+  if constexpr (!BM) {
+    it_idx = a.run_items ? a.run_items[blockIdx.x] : (int)blockIdx.x;
+    const S2Item item = a.items[it_idx];
+    qi = a.queries[item.query];
+    q = item.query;
+    Tq = qi.n_gathered;
+    k_begin = item.p_begin;
+    k_end = item.p_end;
+    k_lo = item.p_lo;
+    R = RQ;
+  } else {
+    be = a.bm_entries[blockIdx.x];
+    k_begin = 0;
+    k_end = be.len;
+    k_lo = 0;
+    R = be.n_slots * RQ;
+  }
+  const int pos_first = Tq + a.tail_len - a.n_new;  // position of query token 0 (per query)
   const int row_base = blockIdx.z * MROWS;
   const CT *kc = static_cast<const CT *>(a.k_cache);
   const CT *vc = static_cast<const CT *>(a.v_cache);
@@ -142,13 +165,26 @@ __global__ void __launch_bounds__(32 * RT * KG, 1) stage2_attn_kernel(const Stag
     const int r = row_base + rr;
     float lo[8], hi[8];
     if (r < R) {
-      const int tok = r / g, h = c * g + r % g;
+      int qq = q, tok, h, pos;
+      if constexpr (!BM) {
+        tok = r / g;
+        h = c * g + r % g;
+        pos = pos_first + tok;
+      } else {
+        const S2BSlot sl = a.bm_slots[be.slot_begin + r / RQ];
+        const int within = r % RQ;
+        qq = sl.query;
+        tok = within / g;
+        h = c * g + within % g;
+        // query token position minus the block's fresh start
+        pos = a.queries[qq].n_gathered + a.tail_len - a.n_new + tok - sl.pos0;
+      }
       const CT *src = static_cast<const CT *>(a.q_new) +
-                      (((int64_t)q * a.n_new + tok) * a.Hq + h) * D;
+                      (((int64_t)qq * a.n_new + tok) * a.Hq + h) * D;
       load8(src + cp * 8, lo);
       load8(src + H + cp * 8, hi);
       float cs[8], sn[8];
-      rope_cs8(a.rope, pos_first + tok, cp * 8, H, cs, sn);
+      rope_cs8(a.rope, pos, cp * 8, H, cs, sn);
       rotate8(lo, hi, cs, sn);
     } else {
 #pragma unroll
@@ -165,7 +201,7 @@ __global__ void __launch_bounds__(32 * RT * KG, 1) stage2_attn_kernel(const Stag
   // (lanes 16-31), 256 contiguous bytes each.
   constexpr int RPW = KT / RT;
   static_assert(RPW <= 16 && CH <= 16, "one row per half-warp");
-  const int n_sub = (item.p_end - item.p_begin + KT - 1) / KT;
+  const int n_sub = (k_end - k_begin + KT - 1) / KT;
   const int n_local = kg < n_sub ? (n_sub - kg + KG - 1) / KG : 0;
   const int half_id = lane >> 4, hl = lane & 15;  // half-warp: 0 = K, 1 = V
   int seg = 0;  // segment cursor: this lane's positions only grow
@@ -173,13 +209,24 @@ __global__ void __launch_bounds__(32 * RT * KG, 1) stage2_attn_kernel(const Stag
     return sRing + ((size_t)(kg * NST + jl % NST) * 2 + kv) * STAGEB;
   };
   auto issue = [&](int jl) {
-    const int p0 = item.p_begin + (kg + jl * KG) * KT + wr * RPW;
+    const int p0 = k_begin + (kg + jl * KG) * KT + wr * RPW;
     // this lane's row pointer (lanes hl < RPW); null past the split end
     const CT *my = nullptr;
     if (hl < RPW) {
       const int p = p0 + hl;
-      if (p < item.p_end) {
-        if (p < Tq) {
+      if (p < k_end && p >= k_lo) {
+        if constexpr (BM) {
+          const int64_t crow = (int64_t)be.cache_row0 + p;
+          my = (half_id ? vc : kc) + ((int64_t)c * a.cap + crow) * D;
+          if (a.dbg_map != nullptr && c == 0 && blockIdx.z == 0 && half_id == 0) {
+            for (int sl = 0; sl < be.n_slots; ++sl) {
+              const S2BSlot slot = a.bm_slots[be.slot_begin + sl];
+              int32_t *m = a.dbg_map + ((int64_t)slot.query * a.dbg_cap + slot.pos0 + p) * 2;
+              m[0] = (int32_t)crow;
+              m[1] = slot.pos0 + p;
+            }
+          }
+        } else if (p < Tq) {
           while (seg + 1 < qi.n_seg && __ldg(&a.segs[qi.seg_begin + seg + 1].pos0) <= p) ++seg;
           const int64_t crow = (int64_t)__ldg(&a.segs[qi.seg_begin + seg].cache_row0) +
                                (p - __ldg(&a.segs[qi.seg_begin + seg].pos0));
@@ -222,13 +269,15 @@ __global__ void __launch_bounds__(32 * RT * KG, 1) stage2_attn_kernel(const Stag
   }
   __syncthreads();  // sQ complete
 
-  // ---- Q fragments (A operand) of this warp's 16 rows, kept in registers
-  uint32_t qf[D / 16][4];
-  {
-    const int r = wr * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+  // ---- Q fragments (A operand) of this warp's 16 rows: kept in registers,
+  // or (large CTAs, where registers are scarce) re-read from shared memory
+  constexpr bool kQRegs = RT < 8;
+  const int qfrow = wr * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+  uint32_t qf[kQRegs ? D / 16 : 1][4];
+  if constexpr (kQRegs) {
 #pragma unroll
     for (int ks = 0; ks < D / 16; ++ks)
-      ldsm_x4(smem_u32(sQ) + soff<D>(r, 2 * ks + (lane >> 4)), qf[ks][0], qf[ks][1], qf[ks][2],
+      ldsm_x4(smem_u32(sQ) + soff<D>(qfrow, 2 * ks + (lane >> 4)), qf[ks][0], qf[ks][1], qf[ks][2],
               qf[ks][3]);
   }
   const int gq = lane >> 2, tq = lane & 3;
@@ -236,7 +285,7 @@ __global__ void __launch_bounds__(32 * RT * KG, 1) stage2_attn_kernel(const Stag
 #pragma unroll
   for (int h2 = 0; h2 < 2; ++h2) {
     const int r = row_base + wr * 16 + gq + 8 * h2;
-    qpos[h2] = (r < R) ? pos_first + r / g : INT_MAX;
+    qpos[h2] = (!BM && r < R) ? pos_first + r / g : INT_MAX;
   }
 
   float o[ND][4];
@@ -250,7 +299,7 @@ __global__ void __launch_bounds__(32 * RT * KG, 1) stage2_attn_kernel(const Stag
     group_sync();
     if (jl + NST - 1 < n_local) issue(jl + NST - 1);
     cp_async_commit();
-    const int p0 = item.p_begin + (kg + jl * KG) * KT;
+    const int p0 = k_begin + (kg + jl * KG) * KT;
     uint8_t *tk = stage_ptr(jl, 0);
     uint8_t *tv = stage_ptr(jl, 1);
     // ---- re-rotate this warp's rows of the sub-tile at their fresh positions
@@ -262,19 +311,25 @@ __global__ void __launch_bounds__(32 * RT * KG, 1) stage2_attn_kernel(const Stag
       const int r0 = wr * RPW;
       const int64_t hoff = (int64_t)((p0 + r0) >> kRopeShift) * H;
       if constexpr (H == 64) {
+        // p0 is a multiple of 16 and r0 a multiple of 8, so row r0 + k sits at
+        // position offset (r0 & 15) + k of its 16-group and at swizzle phase
+        // k & 7: every address below is a per-lane base plus a constant.
+        static_assert(RPW % 8 == 0, "rows per warp keep the swizzle phase");
         const int i = 2 * lane;
         const f32x2 hcos = *reinterpret_cast<const f32x2 *>(a.rope.hc + hoff + i);
         const f32x2 hsin = *reinterpret_cast<const f32x2 *>(a.rope.hs + hoff + i);
         const f32x2 nhsin = f2_neg(hsin);
-#pragma unroll 4
-        for (int r = r0; r < r0 + RPW; ++r) {
-          const int lr = (p0 + r) & (kRopeLo - 1);
-          const f32x2 lcos = *reinterpret_cast<const f32x2 *>(sLc + lr * H + i);
-          const f32x2 lsin = *reinterpret_cast<const f32x2 *>(sLs + lr * H + i);
+        const float *lcb = sLc + (r0 & (kRopeLo - 1)) * H + i;
+        const float *lsb = sLs + (r0 & (kRopeLo - 1)) * H + i;
+        uint8_t *rowb = tk + r0 * ROWB + (i & 7) * 2;
+#pragma unroll
+        for (int k = 0; k < RPW; ++k) {
+          const f32x2 lcos = *reinterpret_cast<const f32x2 *>(lcb + k * H);
+          const f32x2 lsin = *reinterpret_cast<const f32x2 *>(lsb + k * H);
           const f32x2 cs = f2_fma(hcos, lcos, f2_mul(nhsin, lsin));
           const f32x2 sn = f2_fma(hcos, lsin, f2_mul(hsin, lcos));
-          uint32_t *plo = reinterpret_cast<uint32_t *>(tk + soff<D>(r, i >> 3) + (i & 7) * 2);
-          uint32_t *phi = reinterpret_cast<uint32_t *>(tk + soff<D>(r, (H + i) >> 3) + (i & 7) * 2);
+          uint32_t *plo = reinterpret_cast<uint32_t *>(rowb + k * ROWB + (((i >> 3) ^ (k & 7)) << 4));
+          uint32_t *phi = plo + (H / 8) * 4;  // second half: chunk + H/8, same swizzle
           const f32x2 xl = f2_from_bf16x2(*plo), xh = f2_from_bf16x2(*phi);
           *plo = f2_to_bf16x2(f2_fma(xl, cs, f2_mul(f2_neg(xh), sn)));
           *phi = f2_to_bf16x2(f2_fma(xh, cs, f2_mul(xl, sn)));
@@ -305,18 +360,24 @@ __global__ void __launch_bounds__(32 * RT * KG, 1) stage2_attn_kernel(const Stag
     for (int nb = 0; nb < NB; ++nb) s[nb][0] = s[nb][1] = s[nb][2] = s[nb][3] = 0.f;
 #pragma unroll
     for (int ks = 0; ks < D / 16; ++ks) {
+      uint32_t qa[4];
+      if constexpr (kQRegs) {
+        qa[0] = qf[ks][0]; qa[1] = qf[ks][1]; qa[2] = qf[ks][2]; qa[3] = qf[ks][3];
+      } else {
+        ldsm_x4(smem_u32(sQ) + soff<D>(qfrow, 2 * ks + (lane >> 4)), qa[0], qa[1], qa[2], qa[3]);
+      }
 #pragma unroll
       for (int nb = 0; nb < NB; nb += 2) {
         const int mi = lane >> 3;
         const int krow = (nb + (mi >> 1)) * 8 + (lane & 7);
         uint32_t b0, b1, b2, b3;
         ldsm_x4(smem_u32(tk) + soff<D>(krow, 2 * ks + (mi & 1)), b0, b1, b2, b3);
-        mma16816(s[nb], qf[ks], b0, b1);
-        mma16816(s[nb + 1], qf[ks], b2, b3);
+        mma16816(s[nb], qa, b0, b1);
+        mma16816(s[nb + 1], qa, b2, b3);
       }
     }
     // ---- mask (split end; causal inside the query's own tail), online softmax
-    const bool need_mask = (p0 + KT > item.p_end) || (p0 + KT - 1 > pos_first);
+    const bool need_mask = (p0 + KT > k_end) || (p0 < k_lo) || (!BM && p0 + KT - 1 > pos_first);
     float tmax[2] = {-INFINITY, -INFINITY};
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb)
@@ -325,7 +386,7 @@ __global__ void __launch_bounds__(32 * RT * KG, 1) stage2_attn_kernel(const Stag
         float x = s[nb][e] * sl2;
         if (need_mask) {
           const int kp = p0 + nb * 8 + 2 * tq + (e & 1);
-          if (kp >= item.p_end || kp > qpos[e >> 1]) x = -INFINITY;
+          if (kp >= k_end || kp < k_lo || kp > qpos[e >> 1]) x = -INFINITY;
         }
         s[nb][e] = x;
         tmax[e >> 1] = fmaxf(tmax[e >> 1], x);
@@ -386,9 +447,14 @@ __global__ void __launch_bounds__(32 * RT * KG, 1) stage2_attn_kernel(const Stag
     l_run[h2] += __shfl_xor_sync(0xFFFFFFFFu, l_run[h2], 1);
     l_run[h2] += __shfl_xor_sync(0xFFFFFFFFu, l_run[h2], 2);
   }
-  auto part_index = [&](int r) -> int64_t {  // r = GQA row index (token-major)
-    const int tok = r / g, h = c * g + r % g;
-    return ((int64_t)blockIdx.x * a.Hq + h) * a.n_new + tok;
+  auto part_index = [&](int r) -> int64_t {  // r = row index of the CTA (token-major)
+    if constexpr (BM) {
+      const int item = a.bm_slots[be.slot_begin + r / RQ].item;
+      const int within = r % RQ;
+      return ((int64_t)item * a.Hq + c * g + within % g) * a.n_new + within / g;
+    } else {
+      return ((int64_t)it_idx * a.Hq + c * g + r % g) * a.n_new + r / g;
+    }
   };
 
   if constexpr (KG == 1) {
@@ -488,7 +554,7 @@ __global__ void __launch_bounds__(128) stage2_merge_kernel(const Stage2Args a) {
   }
 }
 
-template <int D, typename CT, int RT, int KG, int KT>
+template <int D, typename CT, int RT, int KG, int KT, bool BM = false>
 cudaError_t launch_main(const Stage2Args &a, cudaStream_t st) {
   constexpr int NST = 3;
   constexpr int MROWS = 16 * RT;
@@ -497,12 +563,15 @@ cudaError_t launch_main(const Stage2Args &a, cudaStream_t st) {
   constexpr size_t lo_tables = (size_t)2 * kRopeLo * (D / 2) * sizeof(float);
   constexpr size_t smem = (size_t)MROWS * D * 2 + lo_tables + (ring > merge ? ring : merge);
   static_assert(smem <= 232448, "shared memory budget");
-  cudaError_t e = cudaFuncSetAttribute(stage2_attn_kernel<D, CT, RT, KG, KT, NST>,
+  cudaError_t e = cudaFuncSetAttribute(stage2_attn_kernel<D, CT, RT, KG, KT, NST, BM>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int R = (a.Hq / a.Hkv) * a.n_new;
-  dim3 grid(a.n_items, a.Hkv, (R + MROWS - 1) / MROWS);
-  stage2_attn_kernel<D, CT, RT, KG, KT, NST><<<grid, 32 * RT * KG, smem, st>>>(a);
+  // block-major entries hold at most MROWS rows (the host packs them so)
+  const int n_x = BM ? a.n_bm_entries : (a.run_items ? a.n_run : a.n_items);
+  if (n_x <= 0) return cudaSuccess;
+  dim3 grid(n_x, a.Hkv, BM ? 1 : (R + MROWS - 1) / MROWS);
+  stage2_attn_kernel<D, CT, RT, KG, KT, NST, BM><<<grid, 32 * RT * KG, smem, st>>>(a);
   return cudaGetLastError();
 }
 
@@ -512,6 +581,12 @@ cudaError_t launch_main(const Stage2Args &a, cudaStream_t st) {
 template <int D, typename CT>
 cudaError_t launch_d(const Stage2Args &a, cudaStream_t st) {
   const int R = (a.Hq / a.Hkv) * a.n_new;
+  if (a.bm_entries != nullptr) {
+    // block-major pass: entries of up to 64 rows (4 warps, 32-key sub-tiles,
+    // two CTAs per SM), then the per-query tail items
+    cudaError_t e = launch_main<D, CT, 4, 1, 32, true>(a, st);
+    if (e != cudaSuccess) return e;
+  }
   if (R <= 16) return launch_main<D, CT, 1, 8, 16>(a, st);
   if (R <= 32) return launch_main<D, CT, 2, 4, 32>(a, st);
   if (R <= 64) return launch_main<D, CT, 4, 2, 64>(a, st);
