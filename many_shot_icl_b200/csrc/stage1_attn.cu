@@ -12,13 +12,18 @@
 // One persistent CTA per SM walks items round-robin.  Warp roles:
 //   warp 0      TMA producer: Q tile, then K and V tiles (2-stage ring)
 //   warp 1      TMEM owner and tcgen05.mma issuer (one thread)
-//   warps 2..5  softmax: one thread per query row (TMEM lane), fp32 online
-//               softmax with a lazy rescale threshold, P written to shared
-//               memory as bf16, final O / l epilogue
+//   warps 2..9  softmax, two warpgroups: warpgroup h owns keys 64h..64h+63
+//               of every 128-key score tile, one thread per query row (TMEM
+//               lane).  Each half keeps its own fp32 running max and sum
+//               (lazy rescale threshold) and its own O accumulator
+//               (O_h += P[:, half h] V[half h, :]); the halves are combined
+//               once, in the epilogue.  Exponentials are the scarce resource
+//               (one MUFU op per score), so two warps per scheduler feed them.
 // S = Q K^T lives in TMEM (two 128-column buffers so that the next tile's
-// QK^T overlaps this tile's softmax), O in TMEM (D columns).  Q and K arrive
-// already rotated (bf16) from the preparation pass; V is read straight from
-// the pre-RoPE cache.  Every wait is bounded and reports DBSA_ERR_TIMEOUT.
+// QK^T overlaps this tile's softmax), O_0 and O_1 in TMEM (D columns each):
+// 512 columns in all.  Q and K arrive already rotated (bf16) from the
+// preparation pass; V is read straight from the pre-RoPE cache.  Every wait
+// is bounded and reports DBSA_ERR_TIMEOUT.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
@@ -40,9 +45,17 @@ constexpr uint32_t kFull = 0xFFFFFFFFu;
 
 enum Bar {
   B_Q_FULL = 0, B_Q_EMPTY = 1, B_K_FULL = 2, B_K_EMPTY = 4, B_V_FULL = 6, B_V_EMPTY = 8,
-  B_S_FULL = 10, B_S_FREE = 12, B_P_FULL = 14, B_PV_DONE = 16, B_O_FREE = 18, B_DRAIN = 19,
-  B_COUNT = 20
+  B_S_FULL = 10, B_S_FREE = 12,
+  B_P_FULL = 14,   // [key half][buffer]: 14..17
+  B_PV_DONE = 18,  // [key half][buffer]: 18..21
+  B_O_FREE = 22, B_DRAIN = 23,
+  B_ML_READY = 24,  // epilogue (m, l) exchange written by all softmax threads
+  B_ML_DONE = 25,   // ... and read by all of them (P buffer 0 reusable)
+  B_COUNT = 26
 };
+
+constexpr int kSoftmaxThreads = 256;              // warps 2..9: two warpgroups
+constexpr int kThreads = 64 + kSoftmaxThreads;    // + TMA warp + MMA warp
 
 struct Item {
   int head, q_row0, q_pos0, n_rows, n_ranges;
@@ -105,7 +118,7 @@ struct Params {
 };
 
 template <int D, bool OUT_F32>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     stage1_attn_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const Params p) {
@@ -116,7 +129,8 @@ __global__ void __launch_bounds__(192, 1)
   constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, false);
   constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, true);
   constexpr uint32_t TMEM_COLS = 512;
-  constexpr uint32_t COL_S = 0, COL_O = 256;
+  constexpr uint32_t COL_S = 0;                  // two S buffers, 128 columns each
+  constexpr uint32_t COL_O = 256;                // O of key half h at COL_O + h * D
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>(
@@ -126,6 +140,10 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t *sV = sK + 2 * TILE;
   uint8_t *sP = sV + 2 * TILE;
   uint64_t *bar = reinterpret_cast<uint64_t *>(sP + 2 * PTILE);
+  // Epilogue exchange of (m, l) between the two key halves of a row, [2][128].
+  // It reuses P buffer 0: the epilogue runs after the item's last PV has read
+  // P, and no thread writes P again before both halves are past the exchange.
+  float2 *sML = reinterpret_cast<float2 *>(sP);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + B_COUNT);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -141,12 +159,16 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&bar[B_V_FULL + s], 1);
       mbar_init(&bar[B_V_EMPTY + s], 1);
       mbar_init(&bar[B_S_FULL + s], 1);
-      mbar_init(&bar[B_S_FREE + s], 128);
-      mbar_init(&bar[B_P_FULL + s], 128);
-      mbar_init(&bar[B_PV_DONE + s], 1);
+      mbar_init(&bar[B_S_FREE + s], kSoftmaxThreads);
+      for (int h = 0; h < 2; ++h) {
+        mbar_init(&bar[B_P_FULL + 2 * h + s], 128);
+        mbar_init(&bar[B_PV_DONE + 2 * h + s], 1);
+      }
     }
-    mbar_init(&bar[B_O_FREE], 128);
+    mbar_init(&bar[B_O_FREE], kSoftmaxThreads);
     mbar_init(&bar[B_DRAIN], 1);
+    mbar_init(&bar[B_ML_READY], kSoftmaxThreads);
+    mbar_init(&bar[B_ML_DONE], kSoftmaxThreads);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -220,11 +242,9 @@ __global__ void __launch_bounds__(192, 1)
       if (!ok) break;
       tc_fence_after();
       const uint32_t kv_base = kv_it;
+      // O_h (+)= P[:, 64h : 64h+64] V[64h : 64h+64, :] for both key halves of tile t
       auto issue_pv = [&](int t) -> bool {
         const uint32_t pb = pv_it & 1, np = pv_it >> 1;
-        if (!mbar_wait(&bar[B_P_FULL + pb], np & 1, abort_flag, p.status, kWaitLimitNs,
-                       DBSA_ERR_TIMEOUT))
-          return false;
         const uint32_t kvt = kv_base + t, st = kvt & 1;
         if (!mbar_wait(&bar[B_V_FULL + st], (kvt >> 1) & 1, abort_flag, p.status, kWaitLimitNs,
                        DBSA_ERR_TIMEOUT))
@@ -233,16 +253,21 @@ __global__ void __launch_bounds__(192, 1)
             !mbar_wait(&bar[B_O_FREE], (item_no - 1) & 1, abort_flag, p.status, kWaitLimitNs,
                        DBSA_ERR_TIMEOUT))
           return false;
-        tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t da = sdesc_sw128(aP + pb * PTILE + (kk >> 2) * HALF + (kk & 3) * 32,
-                                          16, 1024);
-          const uint64_t db = sdesc_sw128(aV + st * TILE + kk * 2048, HALF, 1024);
-          mma_bf16_ss(tmem + COL_O, da, db, IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
+        for (int h = 0; h < 2; ++h) {
+          if (!mbar_wait(&bar[B_P_FULL + 2 * h + pb], np & 1, abort_flag, p.status, kWaitLimitNs,
+                         DBSA_ERR_TIMEOUT))
+            return false;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t da = sdesc_sw128(aP + pb * PTILE + h * HALF + kk * 32, 16, 1024);
+            const uint64_t db = sdesc_sw128(aV + st * TILE + (4 * h + kk) * 2048, HALF, 1024);
+            mma_bf16_ss(tmem + COL_O + h * D, da, db, IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&bar[B_PV_DONE + 2 * h + pb]);
         }
         mma_commit(&bar[B_V_EMPTY + st]);
-        mma_commit(&bar[B_PV_DONE + pb]);
         ++pv_it;
         return true;
       };
@@ -277,9 +302,13 @@ __global__ void __launch_bounds__(192, 1)
     drain_wait(&bar[B_DRAIN], 0);
   } else if (warp >= 2) {
     // ------------------------------------------------------------ softmax
+    // Two warpgroups: kh = key half of every S row (keys 64 kh .. 64 kh + 63),
+    // each with its own running max / sum and its own O accumulator.
+    const int kh = (warp - 2) >> 2;
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const uint32_t col_o = COL_O + kh * D;
     const float sl2 = p.scale_log2;
     uint32_t s_it = 0, item_no = 0;
     bool ok = true;
@@ -295,19 +324,20 @@ __global__ void __launch_bounds__(192, 1)
                                          kWaitLimitNs, DBSA_ERR_TIMEOUT));
         if (!ok) break;
         tc_fence_after();
-        uint32_t v[4][32];
+        uint32_t v[2][32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_off + COL_S + sb * 128 + c * 32, v[c]);
+        for (int c = 0; c < 2; ++c)
+          tmem_ld32(tmem + lane_off + COL_S + sb * 128 + kh * 64 + c * 32, v[c]);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_wait_ld(v[c]);
+        for (int c = 0; c < 2; ++c) tmem_wait_ld(v[c]);
         tc_fence_before();
         mbar_arrive(&bar[B_S_FREE + sb]);
 
-        const int klim = it.len[r] - kt;
-        const int kpos0 = it.pos0[r] + kt;
-        if (klim < kTileKeys || kpos0 + kTileKeys - 1 > it.q_pos0) {
+        const int klim = it.len[r] - kt - kh * 64;    // valid keys of this half
+        const int kpos0 = it.pos0[r] + kt + kh * 64;
+        if (klim < 64 || kpos0 + 63 > it.q_pos0) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
+          for (int c = 0; c < 2; ++c)
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
               const int k = c * 32 + e;
@@ -316,11 +346,11 @@ __global__ void __launch_bounds__(192, 1)
         }
         float mt0 = -INFINITY, mt1 = -INFINITY, mt2 = -INFINITY, mt3 = -INFINITY;
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
+        for (int e = 0; e < 32; e += 2) {
           mt0 = fmaxf(mt0, __uint_as_float(v[0][e]));
-          mt1 = fmaxf(mt1, __uint_as_float(v[1][e]));
-          mt2 = fmaxf(mt2, __uint_as_float(v[2][e]));
-          mt3 = fmaxf(mt3, __uint_as_float(v[3][e]));
+          mt1 = fmaxf(mt1, __uint_as_float(v[0][e + 1]));
+          mt2 = fmaxf(mt2, __uint_as_float(v[1][e]));
+          mt3 = fmaxf(mt3, __uint_as_float(v[1][e + 1]));
         }
         const float mt_x = fmaxf(fmaxf(mt0, mt1), fmaxf(mt2, mt3)) * sl2;
         if (t == 0) {
@@ -328,10 +358,10 @@ __global__ void __launch_bounds__(192, 1)
         } else {
           const bool need = mt_x > m_ref + 8.0f;
           if (__any_sync(kFull, need)) {
-            // O must hold every earlier tile before it is rescaled.
+            // this half's O must hold every earlier tile before it is rescaled
             const uint32_t prev = s_it - 1;
-            ok = __all_sync(kFull, mbar_wait(&bar[B_PV_DONE + (prev & 1)], (prev >> 1) & 1,
-                                             abort_flag, p.status, kWaitLimitNs,
+            ok = __all_sync(kFull, mbar_wait(&bar[B_PV_DONE + 2 * kh + (prev & 1)],
+                                             (prev >> 1) & 1, abort_flag, p.status, kWaitLimitNs,
                                              DBSA_ERR_TIMEOUT));
             if (!ok) break;
             tc_fence_after();
@@ -342,11 +372,11 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
               uint32_t o[32];
-              tmem_ld32(tmem + lane_off + COL_O + c * 32, o);
+              tmem_ld32(tmem + lane_off + col_o + c * 32, o);
               tmem_wait_ld(o);
 #pragma unroll
               for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-              tmem_st32(tmem + lane_off + COL_O + c * 32, o);
+              tmem_st32(tmem + lane_off + col_o + c * 32, o);
             }
             tmem_wait_st();
           }
@@ -354,80 +384,102 @@ __global__ void __launch_bounds__(192, 1)
         const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
         float sum0 = 0.f, sum1 = 0.f;
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
+        for (int c = 0; c < 2; ++c)
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
             const float p0 = ex2(fmaf(__uint_as_float(v[c][e]), sl2, -mu));
             const float p1 = ex2(fmaf(__uint_as_float(v[c][e + 1]), sl2, -mu));
             sum0 += p0;
             sum1 += p1;
-            __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
-            v[c][e >> 1] = *reinterpret_cast<uint32_t *>(&h);  // packed pairs in v[c][0..15]
+            __nv_bfloat162 hh = __floats2bfloat162_rn(p0, p1);
+            v[c][e >> 1] = *reinterpret_cast<uint32_t *>(&hh);  // packed pairs in v[c][0..15]
           }
         l += sum0 + sum1;
         if (s_it >= 2) {
-          ok = __all_sync(kFull, mbar_wait(&bar[B_PV_DONE + sb], ((s_it - 2) >> 1) & 1, abort_flag,
+          ok = __all_sync(kFull, mbar_wait(&bar[B_PV_DONE + 2 * kh + sb], ((s_it - 2) >> 1) & 1,
+                                           abort_flag, p.status, kWaitLimitNs, DBSA_ERR_TIMEOUT));
+          if (!ok) break;
+        }
+        if (t == 0 && item_no > 0) {  // the previous epilogue's exchange lives in P buffer 0
+          ok = __all_sync(kFull, mbar_wait(&bar[B_ML_DONE], (item_no - 1) & 1, abort_flag,
                                            p.status, kWaitLimitNs, DBSA_ERR_TIMEOUT));
           if (!ok) break;
         }
-        uint8_t *prow = sP + sb * PTILE + row * 128;
+        // this half's 64 keys = the P tile's swizzled 64-column block kh
+        uint8_t *prow = sP + sb * PTILE + kh * HALF + row * 128;
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
+        for (int c = 0; c < 2; ++c)
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            const int kc = c * 4 + j;  // 8-key chunk index 0..15
-            const uint32_t addr = (kc >> 3) * HALF + ((((kc & 7) ^ (row & 7))) << 4);
-            *reinterpret_cast<uint4 *>(prow + addr) =
+            const int kc = c * 4 + j;  // 8-key chunk index 0..7 within the half
+            *reinterpret_cast<uint4 *>(prow + ((kc ^ (row & 7)) << 4)) =
                 make_uint4(v[c][4 * j], v[c][4 * j + 1], v[c][4 * j + 2], v[c][4 * j + 3]);
           }
         fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(&bar[B_P_FULL + sb]);
+        mbar_arrive(&bar[B_P_FULL + 2 * kh + sb]);
       }
       if (!ok) break;
-      // ---- epilogue: O / l of this row
+      // ---- epilogue: O = (O_0 e^{m_0 - M} + O_1 e^{m_1 - M}) / (l_0 e^{m_0 - M} + ...)
       const uint32_t last = s_it - 1;
-      ok = __all_sync(kFull, mbar_wait(&bar[B_PV_DONE + (last & 1)], (last >> 1) & 1, abort_flag,
-                                       p.status, kWaitLimitNs, DBSA_ERR_TIMEOUT));
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        ok = ok && __all_sync(kFull, mbar_wait(&bar[B_PV_DONE + 2 * h + (last & 1)],
+                                               (last >> 1) & 1, abort_flag, p.status,
+                                               kWaitLimitNs, DBSA_ERR_TIMEOUT));
+      }
       if (!ok) break;
+      sML[kh * 128 + row] = make_float2(m_ref, l);
+      mbar_arrive(&bar[B_ML_READY]);
+      ok = __all_sync(kFull, mbar_wait(&bar[B_ML_READY], item_no & 1, abort_flag, p.status,
+                                       kWaitLimitNs, DBSA_ERR_TIMEOUT));
+      if (!ok) break;
+      const float2 mine = sML[kh * 128 + row], other = sML[(kh ^ 1) * 128 + row];
+      mbar_arrive(&bar[B_ML_DONE]);
+      const float2 ml0 = kh == 0 ? mine : other, ml1 = kh == 0 ? other : mine;
+      const float M = fmaxf(ml0.x, ml1.x);
+      const float w0 = (ml0.x == -INFINITY) ? 0.f : ex2(ml0.x - M);
+      const float w1 = (ml1.x == -INFINITY) ? 0.f : ex2(ml1.x - M);
+      const float inv = 1.f / (ml0.y * w0 + ml1.y * w1);
       tc_fence_after();
-      uint32_t o[D / 32][32];
+      // this thread writes output columns [kh * D/2, kh * D/2 + D/2) of its row
+      constexpr int HC = D / 2 / 32;   // 32-column chunks per half row
+      const int64_t orow = ((int64_t)(it.q_row0 + row) * p.Hq + it.head) * D;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) tmem_ld32(tmem + lane_off + COL_O + c * 32, o[c]);
+      for (int c = 0; c < HC; ++c) {
+        const int col = kh * (D / 2) + c * 32;
+        uint32_t o0[32], o1[32];
+        tmem_ld32(tmem + lane_off + COL_O + col, o0);
+        tmem_ld32(tmem + lane_off + COL_O + D + col, o1);
+        tmem_wait_ld(o0);
+        tmem_wait_ld(o1);
+        if (row < it.n_rows) {
+          float f[32];
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) tmem_wait_ld(o[c]);
-      tc_fence_before();
-      mbar_arrive(&bar[B_O_FREE]);
-      if (row < it.n_rows) {
-        const float inv = 1.f / l;
-        const int64_t orow = ((int64_t)(it.q_row0 + row) * p.Hq + it.head) * D;
-        if (OUT_F32) {
-          float *dst = static_cast<float *>(p.out) + orow;
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c)
+          for (int e = 0; e < 32; ++e)
+            f[e] = (__uint_as_float(o0[e]) * w0 + __uint_as_float(o1[e]) * w1) * inv;
+          if (OUT_F32) {
+            float *dst = static_cast<float *>(p.out) + orow + col;
 #pragma unroll
             for (int e = 0; e < 32; e += 4)
-              *reinterpret_cast<float4 *>(dst + c * 32 + e) =
-                  make_float4(__uint_as_float(o[c][e]) * inv, __uint_as_float(o[c][e + 1]) * inv,
-                              __uint_as_float(o[c][e + 2]) * inv,
-                              __uint_as_float(o[c][e + 3]) * inv);
-        } else {
-          __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.out) + orow;
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c)
+              *reinterpret_cast<float4 *>(dst + e) = make_float4(f[e], f[e + 1], f[e + 2], f[e + 3]);
+          } else {
+            __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.out) + orow + col;
 #pragma unroll
             for (int e = 0; e < 32; e += 8) {
               uint32_t w[4];
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
-                __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(o[c][e + 2 * q]) * inv,
-                                                         __uint_as_float(o[c][e + 2 * q + 1]) * inv);
-                w[q] = *reinterpret_cast<uint32_t *>(&h);
+                __nv_bfloat162 hh = __floats2bfloat162_rn(f[e + 2 * q], f[e + 2 * q + 1]);
+                w[q] = *reinterpret_cast<uint32_t *>(&hh);
               }
-              *reinterpret_cast<uint4 *>(dst + c * 32 + e) = make_uint4(w[0], w[1], w[2], w[3]);
+              *reinterpret_cast<uint4 *>(dst + e) = make_uint4(w[0], w[1], w[2], w[3]);
             }
+          }
         }
       }
+      tc_fence_before();
+      mbar_arrive(&bar[B_O_FREE]);
     }
   }
   __syncwarp();
@@ -482,7 +534,7 @@ cudaError_t launch_t(const CUtensorMap &mq, const CUtensorMap &mk, const CUtenso
   cudaError_t e = cudaFuncSetAttribute(stage1_attn_kernel<D, F32>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  stage1_attn_kernel<D, F32><<<grid, 192, smem, st>>>(mq, mk, mv, p);
+  stage1_attn_kernel<D, F32><<<grid, kThreads, smem, st>>>(mq, mk, mv, p);
   return cudaGetLastError();
 }
 
