@@ -50,8 +50,7 @@ enum Bar {
   B_PV_DONE = 18,  // [key half][buffer]: 18..21
   B_O_FREE = 22, B_DRAIN = 23,
   B_ML_READY = 24,  // epilogue (m, l) exchange written by all softmax threads
-  B_ML_DONE = 25,   // ... and read by all of them (P buffer 0 reusable)
-  B_COUNT = 26
+  B_COUNT = 25
 };
 
 constexpr int kSoftmaxThreads = 256;              // warps 2..9: two warpgroups
@@ -124,7 +123,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                        const __grid_constant__ CUtensorMap tmV, const Params p) {
   constexpr uint32_t HALF = 128 * 64 * 2;        // one 128-row x 64-column swizzled atom column
   constexpr uint32_t TILE = 128 * D * 2;         // Q / K / V tile
-  constexpr uint32_t PTILE = 128 * 128 * 2;      // P tile (128 rows x 128 keys)
   constexpr int NH = D / 64;                     // 64-column halves per row
   constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, false);
   constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, true);
@@ -138,12 +136,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *sQ = base;
   uint8_t *sK = sQ + TILE;
   uint8_t *sV = sK + 2 * TILE;
-  uint8_t *sP = sV + 2 * TILE;
-  uint64_t *bar = reinterpret_cast<uint64_t *>(sP + 2 * PTILE);
-  // Epilogue exchange of (m, l) between the two key halves of a row, [2][128].
-  // It reuses P buffer 0: the epilogue runs after the item's last PV has read
-  // P, and no thread writes P again before both halves are past the exchange.
-  float2 *sML = reinterpret_cast<float2 *>(sP);
+  float2 *sML = reinterpret_cast<float2 *>(sV + 2 * TILE);  // epilogue (m, l), [2][128]
+  uint64_t *bar = reinterpret_cast<uint64_t *>(sML + 256);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + B_COUNT);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -168,7 +162,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bar[B_O_FREE], kSoftmaxThreads);
     mbar_init(&bar[B_DRAIN], 1);
     mbar_init(&bar[B_ML_READY], kSoftmaxThreads);
-    mbar_init(&bar[B_ML_DONE], kSoftmaxThreads);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -232,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
-    const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP);
+    const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
     uint32_t kv_it = 0, s_it = 0, pv_it = 0, item_no = 0;
     bool ok = true;
     for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x, ++item_no) {
@@ -261,9 +254,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t da = sdesc_sw128(aP + pb * PTILE + h * HALF + kk * 32, 16, 1024);
+            // P of this half: 64 keys packed two per column in the first 32
+            // columns of the half's own S region; 8 columns per 16 keys
+            const uint32_t ta = tmem + COL_S + pb * 128 + h * 64 + kk * 8;
             const uint64_t db = sdesc_sw128(aV + st * TILE + (4 * h + kk) * 2048, HALF, 1024);
-            mma_bf16_ss(tmem + COL_O + h * D, da, db, IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
+            mma_bf16_ts(tmem + COL_O + h * D, ta, db, IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(&bar[B_PV_DONE + 2 * h + pb]);
         }
@@ -395,27 +390,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             v[c][e >> 1] = *reinterpret_cast<uint32_t *>(&hh);  // packed pairs in v[c][0..15]
           }
         l += sum0 + sum1;
-        if (s_it >= 2) {
-          ok = __all_sync(kFull, mbar_wait(&bar[B_PV_DONE + 2 * kh + sb], ((s_it - 2) >> 1) & 1,
-                                           abort_flag, p.status, kWaitLimitNs, DBSA_ERR_TIMEOUT));
-          if (!ok) break;
-        }
-        if (t == 0 && item_no > 0) {  // the previous epilogue's exchange lives in P buffer 0
-          ok = __all_sync(kFull, mbar_wait(&bar[B_ML_DONE], (item_no - 1) & 1, abort_flag,
-                                           p.status, kWaitLimitNs, DBSA_ERR_TIMEOUT));
-          if (!ok) break;
-        }
-        // this half's 64 keys = the P tile's swizzled 64-column block kh
-        uint8_t *prow = sP + sb * PTILE + kh * HALF + row * 128;
+        // P of this half (64 keys, bf16 pairs) over the first 32 columns of the
+        // half's own S region, which this thread has already read.  The S(t+2)
+        // that next writes this buffer is issued after PV(t), and the tensor
+        // core runs one thread's MMAs in order.
+        {
+          uint32_t pw[32];
 #pragma unroll
-        for (int c = 0; c < 2; ++c)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int kc = c * 4 + j;  // 8-key chunk index 0..7 within the half
-            *reinterpret_cast<uint4 *>(prow + ((kc ^ (row & 7)) << 4)) =
-                make_uint4(v[c][4 * j], v[c][4 * j + 1], v[c][4 * j + 2], v[c][4 * j + 3]);
+          for (int e = 0; e < 16; ++e) {
+            pw[e] = v[0][e];
+            pw[16 + e] = v[1][e];
           }
-        fence_proxy_async_smem();
+          tmem_st32(tmem + lane_off + COL_S + sb * 128 + kh * 64, pw);
+          tmem_wait_st();
+        }
         tc_fence_before();
         mbar_arrive(&bar[B_P_FULL + 2 * kh + sb]);
       }
@@ -435,7 +423,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                                        kWaitLimitNs, DBSA_ERR_TIMEOUT));
       if (!ok) break;
       const float2 mine = sML[kh * 128 + row], other = sML[(kh ^ 1) * 128 + row];
-      mbar_arrive(&bar[B_ML_DONE]);
       const float2 ml0 = kh == 0 ? mine : other, ml1 = kh == 0 ? other : mine;
       const float M = fmaxf(ml0.x, ml1.x);
       const float w0 = (ml0.x == -INFINITY) ? 0.f : ex2(ml0.x - M);
@@ -522,7 +509,12 @@ bool make_map(CUtensorMap *m, const void *ptr, int D, int64_t rows, int64_t head
 
 template <int D>
 constexpr size_t smem_bytes() {
-  return 1024 + (size_t)128 * D * 2 * 5 + (size_t)128 * 128 * 2 * 2 + B_COUNT * 8 + 16;
+  // + 1 KB for the manual 1024-byte alignment of the swizzled tiles.  The
+  // request is padded above half an SM's shared memory so that no two CTAs
+  // share an SM: each one allocates all 512 TMEM columns.
+  constexpr size_t need = 1024 + (size_t)128 * D * 2 * 5 + 256 * sizeof(float2) + B_COUNT * 8 + 16;
+  constexpr size_t one_per_sm = 232448 / 2 + 1024;
+  return need > one_per_sm ? need : one_per_sm;
 }
 
 template <int D, bool F32>
