@@ -34,6 +34,29 @@ METRIC = "Stage-1 encode tok/s & Stage-2 query tok/s (L3.1-8B shape, 90k); % roo
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from the ncu
+# captures summarised under profiles/, valid only for the kernel sources they were taken
+# on (sha256 of the files, first 16 hex digits); reported as null once a source changes.
+TRAFFIC = {
+    "stage1_attn": {"bytes": 2.561486e9, "sources": ("stage1_attn.cu", "sm100.cuh"),
+                    "sha": "7394b9ad15d9d6c1"},
+    "stage2_prompt": {"bytes": 0.865528e9, "sources": ("stage2_attn.cu", "vec8.cuh"),
+                      "sha": "1d6cc9d81c9c6a1a"},
+    "stage2_decode": {"bytes": 0.402878e9, "sources": ("stage2_attn.cu", "vec8.cuh"),
+                      "sha": "1d6cc9d81c9c6a1a"},
+}
+
+
+def traffic_for(name):
+    import hashlib
+    t = TRAFFIC[name]
+    h = hashlib.sha256()
+    for f in t["sources"]:
+        with open(os.path.join(ROOT, "many_shot_icl_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return t["bytes"] if h.hexdigest()[:16] == t["sha"] else None
+
+
 def load_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -550,7 +573,7 @@ def main():
         r = {"kernel": kernel, "launch_ms": round(ms, 4), "flop_per_launch": fl,
              "unique_bytes_per_launch": ub, "intensity_flop_per_unique_byte": round(fl / ub, 1),
              "per_query_bytes_per_launch": pb,
-             "per_query_bytes_gbs": round(pb / sec / 1e9, 1), "traffic": None}
+             "per_query_bytes_gbs": round(pb / sec / 1e9, 1)}
         if fl / ub >= ridge:
             r.update({"bound": "tensor", "achieved": round(fl / sec / 1e12, 1), "peak": peak_tf,
                       "unit": "TFLOP/s", "frac": round(fl / sec / 1e12 / peak_tf, 4),
@@ -572,6 +595,11 @@ def main():
                              p_pass[:1], s2p_ms)
     roof_s2d = (pass_roofline("stage2_attn_kernel (block-major + tail, decode step)",
                               p_pass[1:], s2d_ms) if len(p_pass) > 1 else None)
+    if w.name == inputs.L31_8B_90K.name:   # the captures were taken on this workload
+        roof_s1["traffic"] = traffic_for("stage1_attn")
+        roof_s2p["traffic"] = traffic_for("stage2_prompt")
+        if roof_s2d:
+            roof_s2d["traffic"] = traffic_for("stage2_decode")
     shares = {"stage1_attn": s1_ms * layers, "stage2_prompt": s2p_ms * layers,
               "stage2_decode": (s2d_ms * (len(p_pass) - 1) * layers) if roof_s2d else 0.0}
     by_name = {"stage1_attn": roof_s1, "stage2_prompt": roof_s2p, "stage2_decode": roof_s2d}

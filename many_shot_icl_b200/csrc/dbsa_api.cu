@@ -797,7 +797,7 @@ dbsa_status dbsa_gather_rope_attend(const dbsa_config *cfg, const void *k_cache,
     e = launch_stage2_main(a, cfg->head_dim, cfg->dtype == DBSA_F32, st);
   }
   if (e != cudaSuccess) return cuda_fail(e, "stage-2 attention");
-  count_launches(1);
+  count_launches(gp.block_major ? 2 : 1);  // block-major: block kernel + tail kernel
   if ((e = launch_stage2_merge(a, cfg->head_dim, cfg->dtype == DBSA_F32, st)) != cudaSuccess)
     return cuda_fail(e, "stage-2 merge");
   count_launches(1);
