@@ -233,7 +233,18 @@ struct GatherPlan {
   std::vector<S2BEntry> bm_entries;
   std::vector<S2BSlot> bm_slots;
   std::vector<int32_t> run_items;
+  // tensor-core block-major mode (multi-token passes): the query rows of all
+  // (query, block) items packed block by block, and the tile list of the
+  // tensor-core kernel over them
+  bool tc = false;
+  int32_t tc_rows = 0;
+  int32_t nb = 0;
+  int64_t cache_rows = 0;  // offs[nb]
+  std::vector<int32_t> row_item, item_row0;
+  std::vector<dbsa_tile_item> tc_tiles;
 };
+
+int32_t offs_count(const GatherPlan &gp) { return gp.nb + 1; }
 
 // Queries (rows) per block-major entry: the kernel's CTA holds 64 rows.
 constexpr int kBMRows = 64;
@@ -241,6 +252,8 @@ constexpr int kBMRows = 64;
 dbsa_status gather_plan(const dbsa_config *cfg, const int32_t *offs, int32_t nb, int32_t nq,
                         const int32_t *sel_ptr, const int32_t *sel, int32_t n_new,
                         int32_t tail_len, GatherPlan &gp) {
+  gp.nb = nb;
+  gp.cache_rows = offs[nb];
   if (nq < 1) return fail(DBSA_ERR_INVALID_ARG, "nq must be >= 1");
   if (sel_ptr == nullptr || sel == nullptr) return fail(DBSA_ERR_INVALID_ARG, "selection is NULL");
   if (sel_ptr[0] != 0) return fail(DBSA_ERR_INVALID_ARG, "sel_ptr[0] must be 0");
@@ -293,6 +306,66 @@ dbsa_status gather_plan(const dbsa_config *cfg, const int32_t *offs, int32_t nb,
       (total_keys * cfg->n_kv_heads * zdim + want_ctas - 1) / std::max<int64_t>(1, want_ctas);
   int64_t chunk = std::max(min_chunk, par_chunk);
   chunk = (chunk + kS2Keys - 1) / kS2Keys * kS2Keys;
+  if (R > 16) {
+    // Multi-token passes: tensor-core block-major.  Items per query = one
+    // per selected block + one for its own tail tokens (per-query kernel);
+    // the rows of the block items are packed block by block (queries in
+    // order, token-major rows within an item) and cut into 128-row tiles
+    // that all read the same block of rotated keys.
+    gp.tc = true;
+    std::vector<std::vector<int32_t>> per_block(nb);   // item ids selecting block b
+    for (int q = 0; q < nq; ++q) {
+      S2Query &qi = gp.queries[q];
+      qi.item_begin = (int32_t)gp.items.size();
+      for (int sgi = 0; sgi < qi.n_seg; ++sgi) {
+        const S2Segment &sg = gp.segs[qi.seg_begin + sgi];
+        S2Item it;
+        it.query = q;
+        it.p_begin = sg.pos0;  // the block's fresh start P
+        it.p_end = sg.pos0 + sg.len;
+        it.p_lo = sg.pos0;
+        per_block[sel[sel_ptr[q] + sgi]].push_back((int32_t)gp.items.size());
+        gp.items.push_back(it);
+      }
+      S2Item tail;
+      tail.query = q;
+      tail.p_begin = qi.n_gathered & ~(kRopeLo - 1);
+      tail.p_end = qi.n_gathered + tail_len;
+      tail.p_lo = qi.n_gathered;
+      gp.run_items.push_back((int32_t)gp.items.size());
+      gp.items.push_back(tail);
+      qi.n_items = (int32_t)gp.items.size() - qi.item_begin;
+    }
+    gp.item_row0.assign(gp.items.size(), -1);
+    std::vector<int32_t> block_row0(nb, 0), block_rows(nb, 0);
+    for (int b = 0; b < nb; ++b) {
+      block_row0[b] = gp.tc_rows;
+      for (int32_t it : per_block[b]) {
+        gp.item_row0[it] = gp.tc_rows;
+        for (int r = 0; r < R; ++r) gp.row_item.push_back(it);
+        gp.tc_rows += R;
+      }
+      block_rows[b] = gp.tc_rows - block_row0[b];
+    }
+    for (int c = 0; c < cfg->n_kv_heads; ++c)
+      for (int b = 0; b < nb; ++b)
+        for (int m = 0; m < block_rows[b]; m += kTileRows) {
+          dbsa_tile_item t;
+          std::memset(&t, 0, sizeof t);
+          t.head = c;
+          t.q_row0 = block_row0[b] + m;
+          t.q_pos0 = 1 << 30;  // after every gathered key: no causal limit
+          t.n_rows = std::min(kTileRows, block_rows[b] - m);
+          t.n_ranges = 1;
+          t.block = b;
+          t.k_row0[0] = offs[b];
+          t.v_row0[0] = offs[b];
+          t.pos0[0] = 0;
+          t.len[0] = offs[b + 1] - offs[b];
+          gp.tc_tiles.push_back(t);
+        }
+    return DBSA_OK;
+  }
   if (R <= 16) {
     // Single-token passes: block-major.  Items per query = one per selected
     // block (filled by the block-major kernel) + one for its own tail tokens
@@ -382,7 +455,8 @@ S1Layout s1_layout(const dbsa_config *cfg, int64_t max_pos, int64_t n_items, int
 }
 
 struct S2Layout {
-  size_t rope, queries, segs, items, bm_entries, bm_slots, run_items, part_acc, part_ml, total;
+  size_t rope, queries, segs, items, bm_entries, bm_slots, run_items, row_item, item_row0,
+      tc_tiles, offs, blob_end, k_hat, v_hat, q_hat, part_acc, part_ml, total;
   int32_t n_hi;
 };
 S2Layout s2_layout(const dbsa_config *cfg, const GatherPlan &gp, int32_t n_new) {
@@ -396,6 +470,16 @@ S2Layout s2_layout(const dbsa_config *cfg, const GatherPlan &gp, int32_t n_new) 
   l.bm_entries = cv.take(gp.bm_entries.size() * sizeof(S2BEntry));
   l.bm_slots = cv.take(gp.bm_slots.size() * sizeof(S2BSlot));
   l.run_items = cv.take(gp.run_items.size() * sizeof(int32_t));
+  l.row_item = cv.take(gp.row_item.size() * sizeof(int32_t));
+  l.item_row0 = cv.take(gp.item_row0.size() * sizeof(int32_t));
+  l.tc_tiles = cv.take(gp.tc_tiles.size() * sizeof(dbsa_tile_item));
+  l.offs = cv.take(gp.tc ? (size_t)(offs_count(gp)) * sizeof(int32_t) : 0);
+  l.blob_end = cv.take(0);
+  const int64_t T = gp.cache_rows;
+  l.k_hat = cv.take(gp.tc ? (size_t)cfg->n_kv_heads * T * cfg->head_dim * 2 : 0);
+  l.v_hat = cv.take(gp.tc && cfg->dtype == DBSA_F32 ? (size_t)cfg->n_kv_heads * T * cfg->head_dim * 2
+                                                     : 0);
+  l.q_hat = cv.take(gp.tc ? (size_t)cfg->n_kv_heads * gp.tc_rows * cfg->head_dim * 2 : 0);
   const size_t rows = gp.items.size() * (size_t)cfg->n_q_heads * n_new;
   l.part_acc = cv.take(rows * cfg->head_dim * sizeof(float));
   l.part_ml = cv.take(rows * sizeof(float2));
@@ -526,7 +610,7 @@ dbsa_status dbsa_encode_blocks(const dbsa_config *cfg, const void *q, const void
                            items.size() * sizeof(dbsa_tile_item), cudaMemcpyHostToDevice, st)) !=
       cudaSuccess)
     return cuda_fail(e, "tile list upload");
-  IngestArgs ia;
+  IngestArgs ia{};
   ia.q = q;
   ia.k = k;
   ia.v = v;
@@ -547,7 +631,7 @@ dbsa_status dbsa_encode_blocks(const dbsa_config *cfg, const void *q, const void
   ia.rope = rope;
   if ((e = launch_ingest(ia, cfg->head_dim, f32, st)) != cudaSuccess) return cuda_fail(e, "ingest");
   count_launches(1);
-  Stage1Args sa;
+  Stage1Args sa{};
   sa.q_rot = ia.q_rot;
   sa.q_rows = T;
   sa.k_rot = ia.k_rot;
@@ -627,7 +711,7 @@ dbsa_status dbsa_append_block(const dbsa_config *cfg, const void *q, const void 
   for (int r = 0; r < ap.nr; ++r) {
     const int32_t e_in_cache = std::min<int32_t>(ap.re[r], (int32_t)T0);
     if (e_in_cache <= ap.rs[r]) continue;
-    WindowArgs wa;
+    WindowArgs wa{};
     wa.k_cache = k_cache;
     wa.v_cache = v_cache;
     wa.cap = cap;
@@ -643,7 +727,7 @@ dbsa_status dbsa_append_block(const dbsa_config *cfg, const void *q, const void 
       return cuda_fail(e, "window rotation");
     count_launches(1);
   }
-  IngestArgs ia;
+  IngestArgs ia{};
   ia.q = q;
   ia.k = k;
   ia.v = v;
@@ -664,7 +748,7 @@ dbsa_status dbsa_append_block(const dbsa_config *cfg, const void *q, const void 
   ia.rope = rope;
   if ((e = launch_ingest(ia, cfg->head_dim, f32, st)) != cudaSuccess) return cuda_fail(e, "ingest");
   count_launches(1);
-  Stage1Args sa;
+  Stage1Args sa{};
   sa.q_rot = ia.q_rot;
   sa.q_rows = L;
   sa.k_rot = k_rot;
@@ -745,7 +829,7 @@ dbsa_status dbsa_gather_rope_attend(const dbsa_config *cfg, const void *k_cache,
   count_launches(1);
   // one upload of the three small plan arrays (they are contiguous in the carve)
   {
-    std::vector<uint8_t> blob(L.part_acc - L.queries, 0);
+    std::vector<uint8_t> blob(L.blob_end - L.queries, 0);
     std::memcpy(blob.data(), gp.queries.data(), gp.queries.size() * sizeof(S2Query));
     std::memcpy(blob.data() + (L.segs - L.queries), gp.segs.data(),
                 gp.segs.size() * sizeof(S2Segment));
@@ -759,11 +843,22 @@ dbsa_status dbsa_gather_rope_attend(const dbsa_config *cfg, const void *k_cache,
       std::memcpy(blob.data() + (L.run_items - L.queries), gp.run_items.data(),
                   gp.run_items.size() * sizeof(int32_t));
     }
+    if (gp.tc) {
+      std::memcpy(blob.data() + (L.run_items - L.queries), gp.run_items.data(),
+                  gp.run_items.size() * sizeof(int32_t));
+      std::memcpy(blob.data() + (L.row_item - L.queries), gp.row_item.data(),
+                  gp.row_item.size() * sizeof(int32_t));
+      std::memcpy(blob.data() + (L.item_row0 - L.queries), gp.item_row0.data(),
+                  gp.item_row0.size() * sizeof(int32_t));
+      std::memcpy(blob.data() + (L.tc_tiles - L.queries), gp.tc_tiles.data(),
+                  gp.tc_tiles.size() * sizeof(dbsa_tile_item));
+      std::memcpy(blob.data() + (L.offs - L.queries), offs_host, (size_t)(nb + 1) * sizeof(int32_t));
+    }
     if ((e = cudaMemcpyAsync(at<void>(workspace, L.queries), blob.data(), blob.size(),
                              cudaMemcpyHostToDevice, st)) != cudaSuccess)
       return cuda_fail(e, "gather plan upload");
   }
-  Stage2Args a;
+  Stage2Args a{};
   a.k_cache = k_cache;
   a.v_cache = v_cache;
   a.cap = cap;
@@ -780,7 +875,7 @@ dbsa_status dbsa_gather_rope_attend(const dbsa_config *cfg, const void *k_cache,
   a.items = at<S2Item>(workspace, L.items);
   a.n_items = (int32_t)gp.items.size();
   a.n_queries = nq;
-  a.run_items = gp.block_major ? at<int32_t>(workspace, L.run_items) : nullptr;
+  a.run_items = (gp.block_major || gp.tc) ? at<int32_t>(workspace, L.run_items) : nullptr;
   a.n_run = (int32_t)gp.run_items.size();
   a.bm_entries = gp.block_major ? at<S2BEntry>(workspace, L.bm_entries) : nullptr;
   a.bm_slots = gp.block_major ? at<S2BSlot>(workspace, L.bm_slots) : nullptr;
@@ -792,13 +887,87 @@ dbsa_status dbsa_gather_rope_attend(const dbsa_config *cfg, const void *k_cache,
   a.dbg_cap = dbg_cap;
   a.scale_log2 = scale_log2(cfg);
   a.rope = rope;
-  {
-    ProfileScope prof(st);
-    e = launch_stage2_main(a, cfg->head_dim, cfg->dtype == DBSA_F32, st);
+  const bool f32 = cfg->dtype == DBSA_F32;
+  if (gp.tc) {
+    // keys at block-relative positions, packed query rows, then the
+    // tensor-core kernel over (kv head, block, 128-row tile) in partial mode
+    RelRopeArgs ra{};
+    ra.k_cache = k_cache;
+    ra.v_cache = v_cache;
+    ra.cap = cap;
+    ra.Hkv = cfg->n_kv_heads;
+    ra.T = (int32_t)gp.cache_rows;
+    ra.nb = nb;
+    ra.offs = at<int32_t>(workspace, L.offs);
+    ra.k_hat = at<void>(workspace, L.k_hat);
+    ra.v_bf16 = f32 ? at<void>(workspace, L.v_hat) : nullptr;
+    ra.rope = rope;
+    if ((e = launch_rel_rope(ra, cfg->head_dim, f32, st)) != cudaSuccess)
+      return cuda_fail(e, "block-relative rotation");
+    QHatArgs qa{};
+    qa.q_new = q_new;
+    qa.n_new = n_new;
+    qa.tail_len = tail_len;
+    qa.Hq = cfg->n_q_heads;
+    qa.Hkv = cfg->n_kv_heads;
+    qa.queries = a.queries;
+    qa.items = a.items;
+    qa.row_item = at<int32_t>(workspace, L.row_item);
+    qa.item_row0 = at<int32_t>(workspace, L.item_row0);
+    qa.rows = gp.tc_rows;
+    qa.q_hat = at<void>(workspace, L.q_hat);
+    qa.rope = rope;
+    if ((e = launch_qhat(qa, cfg->head_dim, f32, st)) != cudaSuccess)
+      return cuda_fail(e, "query rotation");
+    count_launches(2);
+    if (dbg_map != nullptr) {
+      int32_t mx = 0;
+      for (const auto &qi : gp.queries) mx = std::max(mx, qi.n_gathered);
+      if ((e = launch_gather_map(a.queries, a.segs, nq, mx, dbg_map, dbg_cap, st)) != cudaSuccess)
+        return cuda_fail(e, "gather map");
+      count_launches(1);
+      a.dbg_map = nullptr;  // the per-query kernel below only sees tail keys
+    }
+    Stage1Args sa{};
+    sa.q_rot = qa.q_hat;
+    sa.q_rows = gp.tc_rows;
+    sa.k_rot = ra.k_hat;
+    sa.k_rows = gp.cache_rows;
+    sa.v = f32 ? ra.v_bf16 : v_cache;
+    sa.v_rows = gp.cache_rows;
+    sa.v_head_stride = f32 ? gp.cache_rows : cap;
+    sa.out = nullptr;
+    sa.Hq = cfg->n_kv_heads;  // packed rows are per kv head
+    sa.Hkv = cfg->n_kv_heads;
+    sa.items = at<dbsa_tile_item>(workspace, L.tc_tiles);
+    sa.n_items = (int32_t)gp.tc_tiles.size();
+    sa.scale_log2 = a.scale_log2;
+    sa.status = at<int>(workspace, 0);
+    sa.part.acc = a.part_acc;
+    sa.part.ml = a.part_ml;
+    sa.part.row_item = qa.row_item;
+    sa.part.item_row0 = qa.item_row0;
+    sa.part.group = cfg->n_q_heads / cfg->n_kv_heads;
+    sa.part.Hq = cfg->n_q_heads;
+    sa.part.n_new = n_new;
+    {
+      ProfileScope prof(st);
+      e = launch_stage1(sa, cfg->head_dim, false, num_sms(), st);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "stage-2 tensor-core attention");
+    count_launches(1);
+    if ((e = launch_stage2_main(a, cfg->head_dim, f32, st)) != cudaSuccess)  // tail items
+      return cuda_fail(e, "stage-2 tail attention");
+    count_launches(1);
+  } else {
+    {
+      ProfileScope prof(st);
+      e = launch_stage2_main(a, cfg->head_dim, f32, st);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "stage-2 attention");
+    count_launches(gp.block_major ? 2 : 1);  // block-major: block kernel + tail kernel
   }
-  if (e != cudaSuccess) return cuda_fail(e, "stage-2 attention");
-  count_launches(gp.block_major ? 2 : 1);  // block-major: block kernel + tail kernel
-  if ((e = launch_stage2_merge(a, cfg->head_dim, cfg->dtype == DBSA_F32, st)) != cudaSuccess)
+  if ((e = launch_stage2_merge(a, cfg->head_dim, f32, st)) != cudaSuccess)
     return cuda_fail(e, "stage-2 merge");
   count_launches(1);
   return DBSA_OK;

@@ -111,6 +111,55 @@ struct WindowArgs {
 };
 cudaError_t launch_window(const WindowArgs &a, int head_dim, bool f32, cudaStream_t st);
 
+// Partial-output mode of the tensor-core attention kernel (Stage 2, block-
+// major): row r of the packed query buffer belongs to split item row_item[r]
+// (rows of an item start at item_row0[item], token-major: u * group + local
+// head); the kernel writes (M, L) and the unnormalised accumulator to the
+// split-partial arrays, index ((item * Hq + head) * n_new + u).
+struct Stage1Partial {
+  float *acc;                  // null: plain mode
+  float2 *ml;
+  const int32_t *row_item;
+  const int32_t *item_row0;
+  int32_t group, Hq, n_new;
+};
+
+// Stage 2, block-major tensor-core passes: keys of every cache row rotated
+// at their position inside their own block (row s of block b at s - offs[b]);
+// fp32 caches also get a bf16 copy of V.
+struct RelRopeArgs {
+  const void *k_cache, *v_cache;   // [Hkv][cap][D], input dtype
+  int64_t cap;
+  int32_t Hkv, T, nb;
+  const int32_t *offs;             // device copy, [nb + 1]
+  void *k_hat;                     // bf16 [Hkv][T][D]
+  void *v_bf16;                    // bf16 [Hkv][T][D] (fp32 caches only) or null
+  RopeTables rope;
+};
+cudaError_t launch_rel_rope(const RelRopeArgs &a, int head_dim, bool f32, cudaStream_t st);
+
+// Packed query rows of the block-major pass: row r of kv head c is query
+// token u / local head hl of split item row_item[r] (a (query, block) pair),
+// rotated at (its position - the block's fresh start).  Also writes the
+// gather map when dbg_map is set.
+struct QHatArgs {
+  const void *q_new;               // [nq][n_new][Hq][D]
+  int32_t n_new, tail_len, Hq, Hkv;
+  const S2Query *queries;
+  const S2Item *items;             // block items: p_begin = fresh start P
+  const int32_t *row_item;
+  const int32_t *item_row0;
+  int32_t rows;                    // packed rows per kv head
+  void *q_hat;                     // bf16 [Hkv][rows][D]
+  RopeTables rope;
+};
+cudaError_t launch_qhat(const QHatArgs &a, int head_dim, bool f32, cudaStream_t st);
+
+// dbg_map[q][p] = (cache row, p) for every gathered token p of every query.
+cudaError_t launch_gather_map(const S2Query *queries, const S2Segment *segs, int32_t nq,
+                              int32_t max_tokens, int32_t *dbg_map, int64_t dbg_cap,
+                              cudaStream_t st);
+
 // Stage-1 tcgen05 attention over a tile list.
 struct Stage1Args {
   const void *q_rot;      // bf16 [Hq][q_rows][D]
@@ -125,6 +174,7 @@ struct Stage1Args {
   int32_t n_items;
   float scale_log2;       // softmax scale * log2(e)
   int *status;
+  Stage1Partial part;     // part.acc == null for Stage 1 itself
 };
 cudaError_t launch_stage1(const Stage1Args &a, int head_dim, bool out_f32, int num_sms,
                           cudaStream_t st);

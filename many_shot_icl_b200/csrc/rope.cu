@@ -132,6 +132,96 @@ __global__ void __launch_bounds__(256) window_kernel(WindowArgs a) {
   }
 }
 
+// Key rows at block-relative positions (row s of block b at s - offs[b]).
+template <int D, typename T>
+__global__ void __launch_bounds__(256) rel_rope_kernel(RelRopeArgs a) {
+  constexpr int H = D / 2;
+  constexpr int CP = H / 8;
+  const int64_t n_units = (int64_t)a.T * a.Hkv * CP;
+  for (int64_t u = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; u < n_units;
+       u += (int64_t)gridDim.x * blockDim.x) {
+    const int cp = (int)(u % CP);
+    const int c_ = (int)((u / CP) % a.Hkv);
+    const int32_t s = (int32_t)(u / ((int64_t)CP * a.Hkv));
+    int lo = 0, hi = a.nb;  // block of row s: offs[lo] <= s < offs[lo + 1]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (__ldg(a.offs + mid) <= s) lo = mid; else hi = mid;
+    }
+    const int64_t pos = s - __ldg(a.offs + lo);
+    const int i0 = cp * 8;
+    float xl[8], xh[8], c[8], sn[8];
+    const T *src = static_cast<const T *>(a.k_cache) + ((int64_t)c_ * a.cap + s) * D;
+    load8(src + i0, xl);
+    load8(src + H + i0, xh);
+    rope_cs8(a.rope, pos, i0, H, c, sn);
+    rotate8(xl, xh, c, sn);
+    bf16 *dst = static_cast<bf16 *>(a.k_hat) + ((int64_t)c_ * a.T + s) * D;
+    store8_bf16(dst + i0, xl);
+    store8_bf16(dst + H + i0, xh);
+    if (a.v_bf16 != nullptr) {
+      const T *vs = static_cast<const T *>(a.v_cache) + ((int64_t)c_ * a.cap + s) * D;
+      load8(vs + i0, xl);
+      load8(vs + H + i0, xh);
+      bf16 *vd = static_cast<bf16 *>(a.v_bf16) + ((int64_t)c_ * a.T + s) * D;
+      store8_bf16(vd + i0, xl);
+      store8_bf16(vd + H + i0, xh);
+    }
+  }
+}
+
+template <int D, typename T>
+__global__ void __launch_bounds__(256) qhat_kernel(QHatArgs a) {
+  constexpr int H = D / 2;
+  constexpr int CP = H / 8;
+  const int g = a.Hq / a.Hkv;
+  const int64_t n_units = (int64_t)a.rows * a.Hkv * CP;
+  for (int64_t u = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; u < n_units;
+       u += (int64_t)gridDim.x * blockDim.x) {
+    const int cp = (int)(u % CP);
+    const int c_ = (int)((u / CP) % a.Hkv);
+    const int32_t r = (int32_t)(u / ((int64_t)CP * a.Hkv));
+    const int item = __ldg(a.row_item + r);
+    const int w = r - __ldg(a.item_row0 + item);
+    const int tok = w / g, h = c_ * g + w % g;
+    const S2Item it = a.items[item];
+    const int q = it.query;
+    const int64_t pos =
+        (int64_t)a.queries[q].n_gathered + a.tail_len - a.n_new + tok - it.p_begin;
+    const int i0 = cp * 8;
+    float xl[8], xh[8], c[8], sn[8];
+    const T *src = static_cast<const T *>(a.q_new) + (((int64_t)q * a.n_new + tok) * a.Hq + h) * D;
+    load8(src + i0, xl);
+    load8(src + H + i0, xh);
+    rope_cs8(a.rope, pos, i0, H, c, sn);
+    rotate8(xl, xh, c, sn);
+    bf16 *dst = static_cast<bf16 *>(a.q_hat) + ((int64_t)c_ * a.rows + r) * D;
+    store8_bf16(dst + i0, xl);
+    store8_bf16(dst + H + i0, xh);
+  }
+}
+
+__global__ void gather_map_kernel(const S2Query *queries, const S2Segment *segs, int32_t nq,
+                                  int32_t max_tokens, int32_t *dbg, int64_t dbg_cap) {
+  const int64_t n = (int64_t)nq * max_tokens;
+  for (int64_t u = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; u < n;
+       u += (int64_t)gridDim.x * blockDim.x) {
+    const int q = (int)(u / max_tokens);
+    const int32_t p = (int32_t)(u % max_tokens);
+    const S2Query qi = queries[q];
+    if (p >= qi.n_gathered) continue;
+    int lo = 0, hi = qi.n_seg;  // segment holding fresh position p
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (segs[qi.seg_begin + mid].pos0 <= p) lo = mid; else hi = mid;
+    }
+    const S2Segment sg = segs[qi.seg_begin + lo];
+    int32_t *m = dbg + ((int64_t)q * dbg_cap + p) * 2;
+    m[0] = sg.cache_row0 + (p - sg.pos0);
+    m[1] = p;
+  }
+}
+
 int grid_for(int64_t n_units, int block) {
   int64_t g = (n_units + block - 1) / block;
   if (g > 148 * 16) g = 148 * 16;
@@ -140,6 +230,41 @@ int grid_for(int64_t n_units, int block) {
 }
 
 }  // namespace
+
+cudaError_t launch_rel_rope(const RelRopeArgs &a, int head_dim, bool f32, cudaStream_t st) {
+  if (a.T <= 0) return cudaSuccess;
+  const int g = grid_for((int64_t)a.T * a.Hkv * (head_dim / 16), 256);
+  if (head_dim == 128) {
+    if (f32) rel_rope_kernel<128, float><<<g, 256, 0, st>>>(a);
+    else rel_rope_kernel<128, bf16><<<g, 256, 0, st>>>(a);
+  } else {
+    if (f32) rel_rope_kernel<64, float><<<g, 256, 0, st>>>(a);
+    else rel_rope_kernel<64, bf16><<<g, 256, 0, st>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_qhat(const QHatArgs &a, int head_dim, bool f32, cudaStream_t st) {
+  if (a.rows <= 0) return cudaSuccess;
+  const int g = grid_for((int64_t)a.rows * a.Hkv * (head_dim / 16), 256);
+  if (head_dim == 128) {
+    if (f32) qhat_kernel<128, float><<<g, 256, 0, st>>>(a);
+    else qhat_kernel<128, bf16><<<g, 256, 0, st>>>(a);
+  } else {
+    if (f32) qhat_kernel<64, float><<<g, 256, 0, st>>>(a);
+    else qhat_kernel<64, bf16><<<g, 256, 0, st>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather_map(const S2Query *queries, const S2Segment *segs, int32_t nq,
+                              int32_t max_tokens, int32_t *dbg_map, int64_t dbg_cap,
+                              cudaStream_t st) {
+  if (nq <= 0 || max_tokens <= 0) return cudaSuccess;
+  gather_map_kernel<<<grid_for((int64_t)nq * max_tokens, 256), 256, 0, st>>>(
+      queries, segs, nq, max_tokens, dbg_map, dbg_cap);
+  return cudaGetLastError();
+}
 
 size_t rope_table_bytes(int32_t n_hi, int32_t head_dim) {
   return (size_t)2 * (n_hi + kRopeLo) * (head_dim / 2) * sizeof(float);

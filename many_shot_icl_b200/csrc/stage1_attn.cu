@@ -114,6 +114,7 @@ struct Params {
   void *out;
   float scale_log2;
   int *status;
+  Stage1Partial part;  // partial-output mode (part.acc != null)
 };
 
 template <int D, bool OUT_F32>
@@ -427,11 +428,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float M = fmaxf(ml0.x, ml1.x);
       const float w0 = (ml0.x == -INFINITY) ? 0.f : ex2(ml0.x - M);
       const float w1 = (ml1.x == -INFINITY) ? 0.f : ex2(ml1.x - M);
-      const float inv = 1.f / (ml0.y * w0 + ml1.y * w1);
+      const float L = ml0.y * w0 + ml1.y * w1;
+      // plain mode: normalised output; partial mode: (M, L) and the
+      // unnormalised accumulator relative to M, for a later LSE merge
+      const bool partial = p.part.acc != nullptr;
+      const float inv = partial ? 1.f : 1.f / L;
+      int64_t prow = 0;
+      if (partial && row < it.n_rows) {
+        const int grow = it.q_row0 + row;                 // row of the packed query buffer
+        const int item = __ldg(p.part.row_item + grow);
+        const int w = grow - __ldg(p.part.item_row0 + item);
+        const int h = it.head * p.part.group + w % p.part.group;
+        prow = ((int64_t)item * p.part.Hq + h) * p.part.n_new + w / p.part.group;
+        if (kh == 0) p.part.ml[prow] = make_float2(M, L);
+      }
       tc_fence_after();
       // this thread writes output columns [kh * D/2, kh * D/2 + D/2) of its row
       constexpr int HC = D / 2 / 32;   // 32-column chunks per half row
       const int64_t orow = ((int64_t)(it.q_row0 + row) * p.Hq + it.head) * D;
+      float *pacc = partial ? p.part.acc + prow * D : nullptr;
 #pragma unroll
       for (int c = 0; c < HC; ++c) {
         const int col = kh * (D / 2) + c * 32;
@@ -445,7 +460,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 32; ++e)
             f[e] = (__uint_as_float(o0[e]) * w0 + __uint_as_float(o1[e]) * w1) * inv;
-          if (OUT_F32) {
+          if (partial) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 4)
+              *reinterpret_cast<float4 *>(pacc + col + e) =
+                  make_float4(f[e], f[e + 1], f[e + 2], f[e + 3]);
+          } else if (OUT_F32) {
             float *dst = static_cast<float *>(p.out) + orow + col;
 #pragma unroll
             for (int e = 0; e < 32; e += 4)
@@ -548,6 +568,7 @@ cudaError_t launch_stage1(const Stage1Args &a, int head_dim, bool out_f32, int n
   p.out = a.out;
   p.scale_log2 = a.scale_log2;
   p.status = a.status;
+  p.part = a.part;
   const int grid = a.n_items < num_sms ? a.n_items : num_sms;
   if (head_dim == 128)
     return out_f32 ? launch_t<128, true>(mq, mk, mv, p, grid, st)
