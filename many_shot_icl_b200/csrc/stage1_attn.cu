@@ -43,14 +43,18 @@ constexpr uint64_t kWaitLimitNs = 4000000000ull;   // 4 s: far above any legitim
 constexpr uint64_t kDrainLimitNs = 200000000ull;   // 0.2 s for the exit drain
 constexpr uint32_t kFull = 0xFFFFFFFFu;
 
+constexpr int kStages = 3;   // K and V ring depth (tiles in flight per operand)
+
 enum Bar {
-  B_Q_FULL = 0, B_Q_EMPTY = 1, B_K_FULL = 2, B_K_EMPTY = 4, B_V_FULL = 6, B_V_EMPTY = 8,
-  B_S_FULL = 10, B_S_FREE = 12,
-  B_P_FULL = 14,   // [key half][buffer]: 14..17
-  B_PV_DONE = 18,  // [key half][buffer]: 18..21
-  B_O_FREE = 22, B_DRAIN = 23,
-  B_ML_READY = 24,  // epilogue (m, l) exchange written by all softmax threads
-  B_COUNT = 25
+  B_Q_FULL = 0, B_Q_EMPTY = 1,
+  B_K_FULL = 2, B_K_EMPTY = 2 + kStages, B_V_FULL = 2 + 2 * kStages, B_V_EMPTY = 2 + 3 * kStages,
+  B_S_FULL = 2 + 4 * kStages,  // [buffer]
+  B_P_FULL = B_S_FULL + 2,     // [buffer]: both key halves of P written (256 arrivals)
+  B_PV_DONE = B_P_FULL + 2,    // [buffer]: PV of both halves done
+  B_O_FREE = B_PV_DONE + 2, B_DRAIN = B_O_FREE + 1,
+  B_ML_A = B_DRAIN + 1,       // epilogue: key half 1 has published (m, l)
+  B_ML_B = B_ML_A + 1,        // epilogue: key half 0 has published the merge factors
+  B_COUNT = B_ML_B + 1
 };
 
 constexpr int kSoftmaxThreads = 256;              // warps 2..9: two warpgroups
@@ -131,14 +135,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr uint32_t COL_S = 0;                  // two S buffers, 128 columns each
   constexpr uint32_t COL_O = 256;                // O of key half h at COL_O + h * D
 
+  // Tiles (1024-byte aligned for the 128-byte swizzle): Q, kStages K, kStages V;
+  // then the epilogue exchange and the barriers.  The request leaves room for
+  // any alignment pad of the dynamic shared-memory base.
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t *sQ = base;
   uint8_t *sK = sQ + TILE;
-  uint8_t *sV = sK + 2 * TILE;
-  float2 *sML = reinterpret_cast<float2 *>(sV + 2 * TILE);  // epilogue (m, l), [2][128]
-  uint64_t *bar = reinterpret_cast<uint64_t *>(sML + 256);
+  uint8_t *sV = sK + kStages * TILE;
+  float2 *sML = reinterpret_cast<float2 *>(sV + kStages * TILE);  // epilogue exchange, [128]
+  uint64_t *bar = reinterpret_cast<uint64_t *>(sML + 128);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + B_COUNT);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -148,21 +155,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(&bar[B_Q_FULL], 1);
     mbar_init(&bar[B_Q_EMPTY], 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kStages; ++s) {
       mbar_init(&bar[B_K_FULL + s], 1);
       mbar_init(&bar[B_K_EMPTY + s], 1);
       mbar_init(&bar[B_V_FULL + s], 1);
       mbar_init(&bar[B_V_EMPTY + s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(&bar[B_S_FULL + s], 1);
-      mbar_init(&bar[B_S_FREE + s], kSoftmaxThreads);
-      for (int h = 0; h < 2; ++h) {
-        mbar_init(&bar[B_P_FULL + 2 * h + s], 128);
-        mbar_init(&bar[B_PV_DONE + 2 * h + s], 1);
-      }
+      mbar_init(&bar[B_P_FULL + s], kSoftmaxThreads);
+      mbar_init(&bar[B_PV_DONE + s], 1);
     }
     mbar_init(&bar[B_O_FREE], kSoftmaxThreads);
     mbar_init(&bar[B_DRAIN], 1);
-    mbar_init(&bar[B_ML_READY], kSoftmaxThreads);
+    mbar_init(&bar[B_ML_A], 128);
+    mbar_init(&bar[B_ML_B], 128);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -177,50 +184,99 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ producer
+    // Two independent cursors over the CTA's tile sequence: K tiles (each
+    // item's Q tile first) and V tiles.  A K slot frees when its QK^T has
+    // run, a V slot only when its PV has run, which happens about two tiles
+    // later; separate cursors keep the K loads from queueing behind V slots.
+    // Neither cursor blocks: the thread polls whichever slot it needs next.
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
-    uint32_t kv_it = 0, item_no = 0;
-    int armed_q = -1, armed_k[2] = {-1, -1}, armed_v[2] = {-1, -1};
-    bool ok = true;
-    for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x, ++item_no) {
-      const Item it = load_item(p.items, idx);
-      const int kvh = it.head / p.group;
-      if (item_no > 0) ok = mbar_wait(&bar[B_Q_EMPTY], (item_no - 1) & 1, abort_flag, p.status,
-                                      kWaitLimitNs, DBSA_ERR_TIMEOUT);
-      if (!ok) break;
-      mbar_arrive_expect_tx(&bar[B_Q_FULL], TILE);
+    int kidx = blockIdx.x, vidx = blockIdx.x, kt = 0, vt = 0;
+    Item kit, vit;
+    if (kidx < p.n_items) kit = vit = load_item(p.items, kidx);
+    bool need_q = kidx < p.n_items;
+    uint32_t qn = 0, kn = 0, vn = 0;          // Q, K, V tiles issued
+    int armed_q = -1, armed_k[kStages], armed_v[kStages];
 #pragma unroll
-      for (int h = 0; h < NH; ++h)
-        tma_load_3d(sQ + h * HALF, &tmQ, &bar[B_Q_FULL], h * 64, it.q_row0, it.head);
-      armed_q = item_no & 1;
-      for (int t = 0; t < it.ntiles; ++t, ++kv_it) {
-        int r, kt;
-        tile_of(it, t, r, kt);
-        const uint32_t st = kv_it & 1, n = kv_it >> 1;
-        if (n > 0) ok = mbar_wait(&bar[B_K_EMPTY + st], (n - 1) & 1, abort_flag, p.status,
-                                  kWaitLimitNs, DBSA_ERR_TIMEOUT);
-        if (!ok) break;
-        mbar_arrive_expect_tx(&bar[B_K_FULL + st], TILE);
+    for (int s = 0; s < kStages; ++s) armed_k[s] = armed_v[s] = -1;
+    uint64_t t_prog = globaltimer_ns();
+    uint32_t idle = 0;
+    while (kidx < p.n_items || vidx < p.n_items) {
+      bool prog = false;
+      if (kidx < p.n_items) {
+        const int kvh = kit.head / p.group;
+        if (need_q) {
+          if (qn == 0 || mbar_try_wait(&bar[B_Q_EMPTY], (qn - 1) & 1)) {
+            mbar_arrive_expect_tx(&bar[B_Q_FULL], TILE);
 #pragma unroll
-        for (int h = 0; h < NH; ++h)
-          tma_load_3d(sK + st * TILE + h * HALF, &tmK, &bar[B_K_FULL + st], h * 64,
-                      it.k_row0[r] + kt, kvh);
-        armed_k[st] = n & 1;
-        if (n > 0) ok = mbar_wait(&bar[B_V_EMPTY + st], (n - 1) & 1, abort_flag, p.status,
-                                  kWaitLimitNs, DBSA_ERR_TIMEOUT);
-        if (!ok) break;
-        mbar_arrive_expect_tx(&bar[B_V_FULL + st], TILE);
+            for (int h = 0; h < NH; ++h)
+              tma_load_3d(sQ + h * HALF, &tmQ, &bar[B_Q_FULL], h * 64, kit.q_row0, kit.head);
+            armed_q = qn & 1;
+            ++qn;
+            need_q = false;
+            prog = true;
+          }
+        } else {
+          const uint32_t st = kn % kStages, n = kn / kStages;
+          if (n == 0 || mbar_try_wait(&bar[B_K_EMPTY + st], (n - 1) & 1)) {
+            int r, k0;
+            tile_of(kit, kt, r, k0);
+            mbar_arrive_expect_tx(&bar[B_K_FULL + st], TILE);
 #pragma unroll
-        for (int h = 0; h < NH; ++h)
-          tma_load_3d(sV + st * TILE + h * HALF, &tmV, &bar[B_V_FULL + st], h * 64,
-                      it.v_row0[r] + kt, kvh);
-        armed_v[st] = n & 1;
+            for (int h = 0; h < NH; ++h)
+              tma_load_3d(sK + st * TILE + h * HALF, &tmK, &bar[B_K_FULL + st], h * 64,
+                          (r ? kit.k_row0[1] : kit.k_row0[0]) + k0, kvh);
+            armed_k[st] = n & 1;
+            ++kn;
+            prog = true;
+            if (++kt == kit.ntiles) {
+              kt = 0;
+              kidx += gridDim.x;
+              if (kidx < p.n_items) {
+                kit = load_item(p.items, kidx);
+                need_q = true;
+              }
+            }
+          }
+        }
+      }
+      if (vidx < p.n_items) {
+        const uint32_t st = vn % kStages, n = vn / kStages;
+        if (n == 0 || mbar_try_wait(&bar[B_V_EMPTY + st], (n - 1) & 1)) {
+          int r, k0;
+          tile_of(vit, vt, r, k0);
+          const int kvh = vit.head / p.group;
+          mbar_arrive_expect_tx(&bar[B_V_FULL + st], TILE);
+#pragma unroll
+          for (int h = 0; h < NH; ++h)
+            tma_load_3d(sV + st * TILE + h * HALF, &tmV, &bar[B_V_FULL + st], h * 64,
+                        (r ? vit.v_row0[1] : vit.v_row0[0]) + k0, kvh);
+          armed_v[st] = n & 1;
+          ++vn;
+          prog = true;
+          if (++vt == vit.ntiles) {
+            vt = 0;
+            vidx += gridDim.x;
+            if (vidx < p.n_items) vit = load_item(p.items, vidx);
+          }
+        }
+      }
+      if (prog) {
+        idle = 0;
+        t_prog = globaltimer_ns();
+      } else if ((++idle & 63u) == 0u) {
+        if (*abort_flag) break;
+        if (globaltimer_ns() - t_prog > kWaitLimitNs) {
+          *abort_flag = 1;
+          atomicExch(p.status, DBSA_ERR_TIMEOUT);
+          break;
+        }
       }
     }
     // Every load this thread issued must land before the CTA exits.
     if (armed_q >= 0) drain_wait(&bar[B_Q_FULL], (uint32_t)armed_q);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kStages; ++s) {
       if (armed_k[s] >= 0) drain_wait(&bar[B_K_FULL + s], (uint32_t)armed_k[s]);
       if (armed_v[s] >= 0) drain_wait(&bar[B_V_FULL + s], (uint32_t)armed_v[s]);
     }
@@ -236,46 +292,47 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const uint32_t kv_base = kv_it;
-      // O_h (+)= P[:, 64h : 64h+64] V[64h : 64h+64, :] for both key halves of tile t
+      // O_h (+)= P[:, 64h : 64h+64] V[64h : 64h+64, :] for both key halves of tile t.
+      // The waits are the minimum: V landed, O free (first tile of an item),
+      // P written by both softmax halves.
       auto issue_pv = [&](int t) -> bool {
         const uint32_t pb = pv_it & 1, np = pv_it >> 1;
-        const uint32_t kvt = kv_base + t, st = kvt & 1;
-        if (!mbar_wait(&bar[B_V_FULL + st], (kvt >> 1) & 1, abort_flag, p.status, kWaitLimitNs,
+        const uint32_t kvt = kv_base + t, st = kvt % kStages;
+        if (!mbar_wait(&bar[B_V_FULL + st], (kvt / kStages) & 1, abort_flag, p.status, kWaitLimitNs,
                        DBSA_ERR_TIMEOUT))
           return false;
         if (t == 0 && item_no > 0 &&
             !mbar_wait(&bar[B_O_FREE], (item_no - 1) & 1, abort_flag, p.status, kWaitLimitNs,
                        DBSA_ERR_TIMEOUT))
           return false;
+        if (!mbar_wait(&bar[B_P_FULL + pb], np & 1, abort_flag, p.status, kWaitLimitNs,
+                       DBSA_ERR_TIMEOUT))
+          return false;
+        tc_fence_after();
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          if (!mbar_wait(&bar[B_P_FULL + 2 * h + pb], np & 1, abort_flag, p.status, kWaitLimitNs,
-                         DBSA_ERR_TIMEOUT))
-            return false;
-          tc_fence_after();
+        for (int h = 0; h < 2; ++h)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            // P of this half: 64 keys packed two per column in the first 32
+            // P of half h: 64 keys packed two per column in the first 32
             // columns of the half's own S region; 8 columns per 16 keys
             const uint32_t ta = tmem + COL_S + pb * 128 + h * 64 + kk * 8;
             const uint64_t db = sdesc_sw128(aV + st * TILE + (4 * h + kk) * 2048, HALF, 1024);
             mma_bf16_ts(tmem + COL_O + h * D, ta, db, IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
           }
-          mma_commit(&bar[B_PV_DONE + 2 * h + pb]);
-        }
+        mma_commit(&bar[B_PV_DONE + pb]);
         mma_commit(&bar[B_V_EMPTY + st]);
         ++pv_it;
         return true;
       };
       for (int t = 0; ok && t < it.ntiles; ++t) {
-        const uint32_t st = kv_it & 1, n = kv_it >> 1;
+        const uint32_t st = kv_it % kStages, n = kv_it / kStages;
         ok = mbar_wait(&bar[B_K_FULL + st], n & 1, abort_flag, p.status, kWaitLimitNs,
                        DBSA_ERR_TIMEOUT);
         if (!ok) break;
-        const uint32_t sb = s_it & 1, ns = s_it >> 1;
-        if (ns > 0) ok = mbar_wait(&bar[B_S_FREE + sb], (ns - 1) & 1, abort_flag, p.status,
-                                   kWaitLimitNs, DBSA_ERR_TIMEOUT);
-        if (!ok) break;
+        // S[sb] last held P(t - 2), which PV(t - 2), issued before this QK,
+        // has consumed (the tensor core runs one thread's MMAs in order); the
+        // softmax read S(t - 2) before it signalled P_FULL(t - 2).
+        const uint32_t sb = s_it & 1;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -326,11 +383,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32(tmem + lane_off + COL_S + sb * 128 + kh * 64 + c * 32, v[c]);
 #pragma unroll
         for (int c = 0; c < 2; ++c) tmem_wait_ld(v[c]);
-        tc_fence_before();
-        mbar_arrive(&bar[B_S_FREE + sb]);
 
-        const int klim = it.len[r] - kt - kh * 64;    // valid keys of this half
-        const int kpos0 = it.pos0[r] + kt + kh * 64;
+        const int klim = (r ? it.len[1] : it.len[0]) - kt - kh * 64;    // valid keys of this half
+        const int kpos0 = (r ? it.pos0[1] : it.pos0[0]) + kt + kh * 64;
         if (klim < 64 || kpos0 + 63 > it.q_pos0) {
 #pragma unroll
           for (int c = 0; c < 2; ++c)
@@ -356,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (__any_sync(kFull, need)) {
             // this half's O must hold every earlier tile before it is rescaled
             const uint32_t prev = s_it - 1;
-            ok = __all_sync(kFull, mbar_wait(&bar[B_PV_DONE + 2 * kh + (prev & 1)],
+            ok = __all_sync(kFull, mbar_wait(&bar[B_PV_DONE + (prev & 1)],
                                              (prev >> 1) & 1, abort_flag, p.status, kWaitLimitNs,
                                              DBSA_ERR_TIMEOUT));
             if (!ok) break;
@@ -406,33 +461,52 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait_st();
         }
         tc_fence_before();
-        mbar_arrive(&bar[B_P_FULL + 2 * kh + sb]);
+        mbar_arrive(&bar[B_P_FULL + sb]);
       }
       if (!ok) break;
       // ---- epilogue: O = (O_0 e^{m_0 - M} + O_1 e^{m_1 - M}) / (l_0 e^{m_0 - M} + ...)
       const uint32_t last = s_it - 1;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        ok = ok && __all_sync(kFull, mbar_wait(&bar[B_PV_DONE + 2 * h + (last & 1)],
-                                               (last >> 1) & 1, abort_flag, p.status,
-                                               kWaitLimitNs, DBSA_ERR_TIMEOUT));
-      }
+      ok = __all_sync(kFull, mbar_wait(&bar[B_PV_DONE + (last & 1)], (last >> 1) & 1, abort_flag,
+                                       p.status, kWaitLimitNs, DBSA_ERR_TIMEOUT));
       if (!ok) break;
-      sML[kh * 128 + row] = make_float2(m_ref, l);
-      mbar_arrive(&bar[B_ML_READY]);
-      ok = __all_sync(kFull, mbar_wait(&bar[B_ML_READY], item_no & 1, abort_flag, p.status,
-                                       kWaitLimitNs, DBSA_ERR_TIMEOUT));
-      if (!ok) break;
-      const float2 mine = sML[kh * 128 + row], other = sML[(kh ^ 1) * 128 + row];
-      const float2 ml0 = kh == 0 ? mine : other, ml1 = kh == 0 ? other : mine;
-      const float M = fmaxf(ml0.x, ml1.x);
-      const float w0 = (ml0.x == -INFINITY) ? 0.f : ex2(ml0.x - M);
-      const float w1 = (ml1.x == -INFINITY) ? 0.f : ex2(ml1.x - M);
-      const float L = ml0.y * w0 + ml1.y * w1;
-      // plain mode: normalised output; partial mode: (M, L) and the
-      // unnormalised accumulator relative to M, for a later LSE merge
+      // Key half 1 publishes its (m, l); key half 0 merges the two states and
+      // publishes the factors (f0, f1) that both halves apply to O_0, O_1.
+      // Plain mode: f_h = e^{m_h - M} / L (normalised output); partial mode:
+      // f_h = e^{m_h - M} and (M, L) go to the split-partial arrays.
       const bool partial = p.part.acc != nullptr;
-      const float inv = partial ? 1.f : 1.f / L;
+      float f0, f1;
+      if (kh == 1) {
+        sML[row] = make_float2(m_ref, l);
+        mbar_arrive(&bar[B_ML_A]);
+        ok = __all_sync(kFull, mbar_wait(&bar[B_ML_B], item_no & 1, abort_flag, p.status,
+                                         kWaitLimitNs, DBSA_ERR_TIMEOUT));
+        if (!ok) break;
+        const float2 f = sML[row];
+        f0 = f.x;
+        f1 = f.y;
+      } else {
+        ok = __all_sync(kFull, mbar_wait(&bar[B_ML_A], item_no & 1, abort_flag, p.status,
+                                         kWaitLimitNs, DBSA_ERR_TIMEOUT));
+        if (!ok) break;
+        const float2 ml1 = sML[row];
+        const float M = fmaxf(m_ref, ml1.x);
+        const float w0 = (m_ref == -INFINITY) ? 0.f : ex2(m_ref - M);
+        const float w1 = (ml1.x == -INFINITY) ? 0.f : ex2(ml1.x - M);
+        const float L = l * w0 + ml1.y * w1;
+        const float inv = partial ? 1.f : 1.f / L;
+        f0 = w0 * inv;
+        f1 = w1 * inv;
+        sML[row] = make_float2(f0, f1);
+        mbar_arrive(&bar[B_ML_B]);
+        if (partial && row < it.n_rows) {
+          const int grow = it.q_row0 + row;
+          const int item = __ldg(p.part.row_item + grow);
+          const int w = grow - __ldg(p.part.item_row0 + item);
+          const int h = it.head * p.part.group + w % p.part.group;
+          p.part.ml[((int64_t)item * p.part.Hq + h) * p.part.n_new + w / p.part.group] =
+              make_float2(M, L);
+        }
+      }
       int64_t prow = 0;
       if (partial && row < it.n_rows) {
         const int grow = it.q_row0 + row;                 // row of the packed query buffer
@@ -440,7 +514,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int w = grow - __ldg(p.part.item_row0 + item);
         const int h = it.head * p.part.group + w % p.part.group;
         prow = ((int64_t)item * p.part.Hq + h) * p.part.n_new + w / p.part.group;
-        if (kh == 0) p.part.ml[prow] = make_float2(M, L);
       }
       tc_fence_after();
       // this thread writes output columns [kh * D/2, kh * D/2 + D/2) of its row
@@ -459,7 +532,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           float f[32];
 #pragma unroll
           for (int e = 0; e < 32; ++e)
-            f[e] = (__uint_as_float(o0[e]) * w0 + __uint_as_float(o1[e]) * w1) * inv;
+            f[e] = __uint_as_float(o0[e]) * f0 + __uint_as_float(o1[e]) * f1;
           if (partial) {
 #pragma unroll
             for (int e = 0; e < 32; e += 4)
@@ -529,10 +602,12 @@ bool make_map(CUtensorMap *m, const void *ptr, int D, int64_t rows, int64_t head
 
 template <int D>
 constexpr size_t smem_bytes() {
-  // + 1 KB for the manual 1024-byte alignment of the swizzled tiles.  The
-  // request is padded above half an SM's shared memory so that no two CTAs
-  // share an SM: each one allocates all 512 TMEM columns.
-  constexpr size_t need = 1024 + (size_t)128 * D * 2 * 5 + 256 * sizeof(float2) + B_COUNT * 8 + 16;
+  // tiles + epilogue exchange + barriers, + 1 KB for the manual 1024-byte
+  // alignment of the swizzled tiles.  The request is padded above half an
+  // SM's shared memory so that no two CTAs share an SM: each one allocates
+  // all 512 TMEM columns.
+  constexpr size_t need = 1024 + (size_t)128 * D * 2 * (1 + 2 * kStages) + 128 * sizeof(float2) +
+                          B_COUNT * 8 + 16;
   constexpr size_t one_per_sm = 232448 / 2 + 1024;
   return need > one_per_sm ? need : one_per_sm;
 }
