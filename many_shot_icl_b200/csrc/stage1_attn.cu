@@ -282,73 +282,79 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
-    const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
-    uint32_t kv_it = 0, s_it = 0, pv_it = 0, item_no = 0;
+    // The tensor core keeps only about one MMA queued, so every instruction
+    // this thread runs between two MMAs is tensor-core idle time: descriptors
+    // are precomputed (an operand's descriptor for a byte offset is the base
+    // descriptor plus offset / 16), ring stages advance incrementally, and a
+    // wait costs one try_wait when its phase is already complete.
+    const uint64_t dQ = sdesc_sw128(smem_u32(sQ), 16, 1024);
+    const uint64_t dK = sdesc_sw128(smem_u32(sK), 16, 1024);
+    const uint64_t dV = sdesc_sw128(smem_u32(sV), HALF, 1024);
+    constexpr uint64_t kTileDesc = TILE >> 4;
+    uint32_t kst = 0, kph = 0, vst = 0, vph = 0;   // ring stage / phase of the next QK, PV
+    uint32_t s_it = 0, pv_it = 0, item_no = 0;
     bool ok = true;
+    auto wait = [&](int b, uint32_t parity) -> bool {
+      return mbar_try_wait(&bar[b], parity) ||
+             mbar_wait(&bar[b], parity, abort_flag, p.status, kWaitLimitNs, DBSA_ERR_TIMEOUT);
+    };
     for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x, ++item_no) {
-      const Item it = load_item(p.items, idx);
-      ok = mbar_wait(&bar[B_Q_FULL], item_no & 1, abort_flag, p.status, kWaitLimitNs,
-                     DBSA_ERR_TIMEOUT);
+      const int ntiles = load_item(p.items, idx).ntiles;
+      ok = wait(B_Q_FULL, item_no & 1);
       if (!ok) break;
       tc_fence_after();
-      const uint32_t kv_base = kv_it;
-      // O_h (+)= P[:, 64h : 64h+64] V[64h : 64h+64, :] for both key halves of tile t.
-      // The waits are the minimum: V landed, O free (first tile of an item),
-      // P written by both softmax halves.
-      auto issue_pv = [&](int t) -> bool {
-        const uint32_t pb = pv_it & 1, np = pv_it >> 1;
-        const uint32_t kvt = kv_base + t, st = kvt % kStages;
-        if (!mbar_wait(&bar[B_V_FULL + st], (kvt / kStages) & 1, abort_flag, p.status, kWaitLimitNs,
-                       DBSA_ERR_TIMEOUT))
-          return false;
-        if (t == 0 && item_no > 0 &&
-            !mbar_wait(&bar[B_O_FREE], (item_no - 1) & 1, abort_flag, p.status, kWaitLimitNs,
-                       DBSA_ERR_TIMEOUT))
-          return false;
-        if (!mbar_wait(&bar[B_P_FULL + pb], np & 1, abort_flag, p.status, kWaitLimitNs,
-                       DBSA_ERR_TIMEOUT))
-          return false;
+      // O_h (+)= P[:, 64h : 64h+64] V[64h : 64h+64, :] for both key halves of
+      // the item's tile t: waits for V, for O (first tile of an item), for P.
+      auto issue_pv = [&](bool first) -> bool {
+        const uint32_t pb = pv_it & 1;
+        if (!wait(B_V_FULL + vst, vph)) return false;
+        if (first && item_no > 0 && !wait(B_O_FREE, (item_no - 1) & 1)) return false;
+        if (!wait(B_P_FULL + pb, (pv_it >> 1) & 1)) return false;
         tc_fence_after();
+        const uint64_t dv = dV + vst * kTileDesc;
+        const uint32_t ta = tmem + COL_S + pb * 128;
 #pragma unroll
         for (int h = 0; h < 2; ++h)
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
+          for (int kk = 0; kk < 4; ++kk)
             // P of half h: 64 keys packed two per column in the first 32
             // columns of the half's own S region; 8 columns per 16 keys
-            const uint32_t ta = tmem + COL_S + pb * 128 + h * 64 + kk * 8;
-            const uint64_t db = sdesc_sw128(aV + st * TILE + (4 * h + kk) * 2048, HALF, 1024);
-            mma_bf16_ts(tmem + COL_O + h * D, ta, db, IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
-          }
+            mma_bf16_ts(tmem + COL_O + h * D, ta + h * 64 + kk * 8, dv + (4 * h + kk) * 128,
+                        IDESC_PV, (kk > 0 || !first) ? 1u : 0u);
         mma_commit(&bar[B_PV_DONE + pb]);
-        mma_commit(&bar[B_V_EMPTY + st]);
+        mma_commit(&bar[B_V_EMPTY + vst]);
         ++pv_it;
+        if (++vst == kStages) {
+          vst = 0;
+          vph ^= 1;
+        }
         return true;
       };
-      for (int t = 0; ok && t < it.ntiles; ++t) {
-        const uint32_t st = kv_it % kStages, n = kv_it / kStages;
-        ok = mbar_wait(&bar[B_K_FULL + st], n & 1, abort_flag, p.status, kWaitLimitNs,
-                       DBSA_ERR_TIMEOUT);
-        if (!ok) break;
+      for (int t = 0; t < ntiles; ++t) {
         // S[sb] last held P(t - 2), which PV(t - 2), issued before this QK,
         // has consumed (the tensor core runs one thread's MMAs in order); the
         // softmax read S(t - 2) before it signalled P_FULL(t - 2).
-        const uint32_t sb = s_it & 1;
+        ok = wait(B_K_FULL + kst, kph);
+        if (!ok) break;
         tc_fence_after();
+        const uint32_t sb = s_it & 1;
+        const uint64_t dk = dK + kst * kTileDesc;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * HALF + (kk & 3) * 32;
-          const uint64_t da = sdesc_sw128(aQ + off, 16, 1024);
-          const uint64_t db = sdesc_sw128(aK + st * TILE + off, 16, 1024);
-          mma_bf16_ss(tmem + COL_S + sb * 128, da, db, IDESC_QK, kk > 0 ? 1u : 0u);
+          const uint32_t off16 = ((kk >> 2) * HALF + (kk & 3) * 32) >> 4;
+          mma_bf16_ss(tmem + COL_S + sb * 128, dQ + off16, dk + off16, IDESC_QK, kk > 0 ? 1u : 0u);
         }
         mma_commit(&bar[B_S_FULL + sb]);
-        mma_commit(&bar[B_K_EMPTY + st]);
-        if (t == it.ntiles - 1) mma_commit(&bar[B_Q_EMPTY]);
-        ++kv_it;
+        mma_commit(&bar[B_K_EMPTY + kst]);
+        if (t == ntiles - 1) mma_commit(&bar[B_Q_EMPTY]);
         ++s_it;
-        if (t > 0) ok = issue_pv(t - 1);
+        if (++kst == kStages) {
+          kst = 0;
+          kph ^= 1;
+        }
+        if (t > 0 && !(ok = issue_pv(t == 1))) break;
       }
-      if (ok) ok = issue_pv(it.ntiles - 1);
+      if (ok) ok = issue_pv(ntiles == 1);
     }
     // All issued MMAs must finish before TMEM is released.
     mma_commit(&bar[B_DRAIN]);
