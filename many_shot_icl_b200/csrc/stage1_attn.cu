@@ -10,20 +10,29 @@
 // holds only the tiles that contain an allowed pair).
 //
 // One persistent CTA per SM walks items round-robin.  Warp roles:
-//   warp 0      TMA producer: Q tile, then K and V tiles (2-stage ring)
-//   warp 1      TMEM owner and tcgen05.mma issuer (one thread)
-//   warps 2..9  softmax, two warpgroups: warpgroup h owns keys 64h..64h+63
-//               of every 128-key score tile, one thread per query row (TMEM
-//               lane).  Each half keeps its own fp32 running max and sum
-//               (lazy rescale threshold) and its own O accumulator
-//               (O_h += P[:, half h] V[half h, :]); the halves are combined
-//               once, in the epilogue.  Exponentials are the scarce resource
-//               (one MUFU op per score), so two warps per scheduler feed them.
-// S = Q K^T lives in TMEM (two 128-column buffers so that the next tile's
-// QK^T overlaps this tile's softmax), O_0 and O_1 in TMEM (D columns each):
-// 512 columns in all.  Q and K arrive already rotated (bf16) from the
-// preparation pass; V is read straight from the pre-RoPE cache.  Every wait
-// is bounded and reports DBSA_ERR_TIMEOUT.
+//   warp 0      TMA producer: two independent cursors, one for each item's Q
+//               tile (double-buffered) and its K tiles (3-stage ring), one
+//               for the V tiles (2-stage ring)
+//   warp 1      TMEM owner; one thread issues O += P V (tcgen05, A from TMEM)
+//   warp 10     one thread issues S = Q K^T (tcgen05, both operands in SMEM)
+//   warps 2..9  softmax, two warpgroups in ping-pong: warpgroup w takes the
+//               tiles whose CTA-wide index has parity w (all 128 keys of
+//               each), one thread per query row (TMEM lane), with its own
+//               fp32 running max and sum (lazy rescale threshold) and its own
+//               O accumulator O_w; the two states are combined once, in the
+//               epilogue.  While one warpgroup exponentiates (one MUFU op
+//               per score), the other loads, reduces and stores.
+// S = Q K^T lives in TMEM in two 128-column buffers (tile parity), P is
+// written back over the first 64 columns of its own S buffer as bf16 pairs,
+// and O_0, O_1 take D columns each: 512 columns in all.  Q and K arrive
+// already rotated (bf16) from the preparation pass; V is read straight from
+// the pre-RoPE cache.  Every wait is bounded and reports DBSA_ERR_TIMEOUT.
+//
+// Measured on B200 (see the profiles): the tensor core runs a 128x128x16
+// MMA in 64 cycles but keeps only about one MMA queued, so the issuing
+// threads must not stall between MMAs; softmax warps that saturate the FMA
+// pipe starve an issuer on the same SM sub-partition, hence the packed
+// (f32x2) and 3-input arithmetic in the softmax and two issuer threads.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
@@ -43,22 +52,31 @@ constexpr uint64_t kWaitLimitNs = 4000000000ull;   // 4 s: far above any legitim
 constexpr uint64_t kDrainLimitNs = 200000000ull;   // 0.2 s for the exit drain
 constexpr uint32_t kFull = 0xFFFFFFFFu;
 
-constexpr int kStages = 3;   // K and V ring depth (tiles in flight per operand)
+// Ring depths (tiles in flight).  A K slot frees when its QK^T has run and is
+// needed again kStagesK tiles later; a V slot frees only after its PV, about
+// two tiles after the QK, and is needed kStagesV tiles later.  Q is double
+// buffered so that the next item's Q tile loads during the current item.
+constexpr int kStagesK = 3;
+constexpr int kStagesV = 2;
+constexpr int kStagesQ = 2;
 
 enum Bar {
-  B_Q_FULL = 0, B_Q_EMPTY = 1,
-  B_K_FULL = 2, B_K_EMPTY = 2 + kStages, B_V_FULL = 2 + 2 * kStages, B_V_EMPTY = 2 + 3 * kStages,
-  B_S_FULL = 2 + 4 * kStages,  // [buffer]
-  B_P_FULL = B_S_FULL + 2,     // [buffer]: both key halves of P written (256 arrivals)
-  B_PV_DONE = B_P_FULL + 2,    // [buffer]: PV of both halves done
+  B_Q_FULL = 0, B_Q_EMPTY = B_Q_FULL + kStagesQ,
+  B_K_FULL = B_Q_EMPTY + kStagesQ, B_K_EMPTY = B_K_FULL + kStagesK,
+  B_V_FULL = B_K_EMPTY + kStagesK, B_V_EMPTY = B_V_FULL + kStagesV,
+  B_S_FULL = B_V_EMPTY + kStagesV,  // [buffer]
+  B_P_FULL = B_S_FULL + 2,     // [buffer]: P written by the buffer's warpgroup
+  B_PV_DONE = B_P_FULL + 2,    // [buffer]: PV of the buffer's tile done
   B_O_FREE = B_PV_DONE + 2, B_DRAIN = B_O_FREE + 1,
   B_ML_A = B_DRAIN + 1,       // epilogue: key half 1 has published (m, l)
-  B_ML_B = B_ML_A + 1,        // epilogue: key half 0 has published the merge factors
-  B_COUNT = B_ML_B + 1
+  B_ML_B = B_ML_A + 1,        // epilogue: warpgroup 0 has published the merge factors
+  B_DRAIN_QK = B_ML_B + 1,
+  B_COUNT = B_DRAIN_QK + 1
 };
 
 constexpr int kSoftmaxThreads = 256;              // warps 2..9: two warpgroups
-constexpr int kThreads = 64 + kSoftmaxThreads;    // + TMA warp + MMA warp
+constexpr int kQKWarp = 10;                       // QK^T issuer (after the softmax warps)
+constexpr int kThreads = 96 + kSoftmaxThreads;    // + TMA warp, PV warp, QK warp
 
 struct Item {
   int head, q_row0, q_pos0, n_rows, n_ranges;
@@ -102,6 +120,34 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// The softmax warps share each SM sub-partition with the MMA-issuing thread,
+// and every FMA-pipe instruction they issue can delay an MMA issue; the
+// per-score arithmetic therefore uses sm_100's packed and 3-input forms.
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+using f32x2 = unsigned long long;
+__device__ __forceinline__ f32x2 f2_pack(float a, float b) {
+  f32x2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(f32x2 r, float &a, float &b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ f32x2 f2_fma(f32x2 a, f32x2 b, f32x2 c) {
+  f32x2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ f32x2 f2_add(f32x2 a, f32x2 b) {
+  f32x2 d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
 // Bounded wait used on the way out: ignores the abort flag.
 __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
   const uint64_t t0 = globaltimer_ns();
@@ -135,16 +181,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr uint32_t COL_S = 0;                  // two S buffers, 128 columns each
   constexpr uint32_t COL_O = 256;                // O of key half h at COL_O + h * D
 
-  // Tiles (1024-byte aligned for the 128-byte swizzle): Q, kStages K, kStages V;
+  // Tiles (1024-byte aligned for the 128-byte swizzle): the Q, K and V rings;
   // then the epilogue exchange and the barriers.  The request leaves room for
   // any alignment pad of the dynamic shared-memory base.
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t *sQ = base;
-  uint8_t *sK = sQ + TILE;
-  uint8_t *sV = sK + kStages * TILE;
-  float2 *sML = reinterpret_cast<float2 *>(sV + kStages * TILE);  // epilogue exchange, [128]
+  uint8_t *sK = sQ + kStagesQ * TILE;
+  uint8_t *sV = sK + kStagesK * TILE;
+  float2 *sML = reinterpret_cast<float2 *>(sV + kStagesV * TILE);  // epilogue exchange, [128]
   uint64_t *bar = reinterpret_cast<uint64_t *>(sML + 128);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + B_COUNT);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
@@ -153,21 +199,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    mbar_init(&bar[B_Q_FULL], 1);
-    mbar_init(&bar[B_Q_EMPTY], 1);
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kStagesQ; ++s) {
+      mbar_init(&bar[B_Q_FULL + s], 1);
+      mbar_init(&bar[B_Q_EMPTY + s], 1);
+    }
+    for (int s = 0; s < kStagesK; ++s) {
       mbar_init(&bar[B_K_FULL + s], 1);
       mbar_init(&bar[B_K_EMPTY + s], 1);
+    }
+    for (int s = 0; s < kStagesV; ++s) {
       mbar_init(&bar[B_V_FULL + s], 1);
       mbar_init(&bar[B_V_EMPTY + s], 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar[B_S_FULL + s], 1);
-      mbar_init(&bar[B_P_FULL + s], kSoftmaxThreads);
+      mbar_init(&bar[B_P_FULL + s], 128);
       mbar_init(&bar[B_PV_DONE + s], 1);
     }
     mbar_init(&bar[B_O_FREE], kSoftmaxThreads);
     mbar_init(&bar[B_DRAIN], 1);
+    mbar_init(&bar[B_DRAIN_QK], 1);
     mbar_init(&bar[B_ML_A], 128);
     mbar_init(&bar[B_ML_B], 128);
     *abort_flag = 0;
@@ -197,9 +248,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (kidx < p.n_items) kit = vit = load_item(p.items, kidx);
     bool need_q = kidx < p.n_items;
     uint32_t qn = 0, kn = 0, vn = 0;          // Q, K, V tiles issued
-    int armed_q = -1, armed_k[kStages], armed_v[kStages];
+    int armed_q[kStagesQ], armed_k[kStagesK], armed_v[kStagesV];
 #pragma unroll
-    for (int s = 0; s < kStages; ++s) armed_k[s] = armed_v[s] = -1;
+    for (int s = 0; s < kStagesQ; ++s) armed_q[s] = -1;
+#pragma unroll
+    for (int s = 0; s < kStagesK; ++s) armed_k[s] = -1;
+#pragma unroll
+    for (int s = 0; s < kStagesV; ++s) armed_v[s] = -1;
     uint64_t t_prog = globaltimer_ns();
     uint32_t idle = 0;
     while (kidx < p.n_items || vidx < p.n_items) {
@@ -207,18 +262,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (kidx < p.n_items) {
         const int kvh = kit.head / p.group;
         if (need_q) {
-          if (qn == 0 || mbar_try_wait(&bar[B_Q_EMPTY], (qn - 1) & 1)) {
-            mbar_arrive_expect_tx(&bar[B_Q_FULL], TILE);
+          const uint32_t qs = qn % kStagesQ, nq = qn / kStagesQ;
+          if (nq == 0 || mbar_try_wait(&bar[B_Q_EMPTY + qs], (nq - 1) & 1)) {
+            mbar_arrive_expect_tx(&bar[B_Q_FULL + qs], TILE);
 #pragma unroll
             for (int h = 0; h < NH; ++h)
-              tma_load_3d(sQ + h * HALF, &tmQ, &bar[B_Q_FULL], h * 64, kit.q_row0, kit.head);
-            armed_q = qn & 1;
+              tma_load_3d(sQ + qs * TILE + h * HALF, &tmQ, &bar[B_Q_FULL + qs], h * 64, kit.q_row0,
+                          kit.head);
+            armed_q[qs] = nq & 1;
             ++qn;
             need_q = false;
             prog = true;
           }
         } else {
-          const uint32_t st = kn % kStages, n = kn / kStages;
+          const uint32_t st = kn % kStagesK, n = kn / kStagesK;
           if (n == 0 || mbar_try_wait(&bar[B_K_EMPTY + st], (n - 1) & 1)) {
             int r, k0;
             tile_of(kit, kt, r, k0);
@@ -242,7 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (vidx < p.n_items) {
-        const uint32_t st = vn % kStages, n = vn / kStages;
+        const uint32_t st = vn % kStagesV, n = vn / kStagesV;
         if (n == 0 || mbar_try_wait(&bar[B_V_EMPTY + st], (n - 1) & 1)) {
           int r, k0;
           tile_of(vit, vt, r, k0);
@@ -275,24 +332,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     // Every load this thread issued must land before the CTA exits.
-    if (armed_q >= 0) drain_wait(&bar[B_Q_FULL], (uint32_t)armed_q);
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kStagesQ; ++s)
+      if (armed_q[s] >= 0) drain_wait(&bar[B_Q_FULL + s], (uint32_t)armed_q[s]);
+    for (int s = 0; s < kStagesK; ++s)
       if (armed_k[s] >= 0) drain_wait(&bar[B_K_FULL + s], (uint32_t)armed_k[s]);
+    for (int s = 0; s < kStagesV; ++s)
       if (armed_v[s] >= 0) drain_wait(&bar[B_V_FULL + s], (uint32_t)armed_v[s]);
-    }
-  } else if (warp == 1 && lane == 0) {
-    // ------------------------------------------------------------ MMA issuer
-    // The tensor core keeps only about one MMA queued, so every instruction
-    // this thread runs between two MMAs is tensor-core idle time: descriptors
-    // are precomputed (an operand's descriptor for a byte offset is the base
-    // descriptor plus offset / 16), ring stages advance incrementally, and a
-    // wait costs one try_wait when its phase is already complete.
+  } else if ((warp == 1 || warp == kQKWarp) && lane == 0) {
+    // ------------------------------------------------------------ MMA issuers
+    // Two threads on different SM sub-partitions feed the tensor core: warp
+    // kQKWarp issues S = Q K^T, warp 1 issues O += P V.  The tensor core keeps
+    // only about one MMA queued, so every instruction an issuer runs between
+    // two MMAs is idle time for it: descriptors are precomputed (a descriptor
+    // for a byte offset is the base descriptor plus offset / 16), ring stages
+    // advance incrementally, and a wait whose phase is complete costs one
+    // try_wait.  QK(t) writes the S buffer in which P(t - 2) lived, so it
+    // waits for PV(t - 2) to complete (the softmax read S(t - 2) before it
+    // signalled P(t - 2)).
+    const bool is_qk = warp == kQKWarp;
     const uint64_t dQ = sdesc_sw128(smem_u32(sQ), 16, 1024);
     const uint64_t dK = sdesc_sw128(smem_u32(sK), 16, 1024);
     const uint64_t dV = sdesc_sw128(smem_u32(sV), HALF, 1024);
     constexpr uint64_t kTileDesc = TILE >> 4;
-    uint32_t kst = 0, kph = 0, vst = 0, vph = 0;   // ring stage / phase of the next QK, PV
-    uint32_t s_it = 0, pv_it = 0, item_no = 0;
+    uint32_t st = 0, ph = 0;        // ring stage / phase of this issuer's operand (K or V)
+    uint32_t s_it = 0, item_no = 0;
     bool ok = true;
     auto wait = [&](int b, uint32_t parity) -> bool {
       return mbar_try_wait(&bar[b], parity) ||
@@ -300,126 +363,126 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x, ++item_no) {
       const int ntiles = load_item(p.items, idx).ntiles;
-      ok = wait(B_Q_FULL, item_no & 1);
-      if (!ok) break;
-      tc_fence_after();
-      // O_h (+)= P[:, 64h : 64h+64] V[64h : 64h+64, :] for both key halves of
-      // the item's tile t: waits for V, for O (first tile of an item), for P.
-      auto issue_pv = [&](bool first) -> bool {
-        const uint32_t pb = pv_it & 1;
-        if (!wait(B_V_FULL + vst, vph)) return false;
-        if (first && item_no > 0 && !wait(B_O_FREE, (item_no - 1) & 1)) return false;
-        if (!wait(B_P_FULL + pb, (pv_it >> 1) & 1)) return false;
-        tc_fence_after();
-        const uint64_t dv = dV + vst * kTileDesc;
-        const uint32_t ta = tmem + COL_S + pb * 128;
+      const uint32_t qs = item_no % kStagesQ;
+      if (is_qk && !(ok = wait(B_Q_FULL + qs, (item_no / kStagesQ) & 1))) break;
+      const uint64_t dq = dQ + qs * kTileDesc;
+      for (int t = 0; t < ntiles; ++t, ++s_it) {
+        const uint32_t b = s_it & 1;
+        if (is_qk) {
+          if (!(ok = wait(B_K_FULL + st, ph))) break;
+          if (s_it >= 2 && !(ok = wait(B_PV_DONE + b, ((s_it - 2) >> 1) & 1))) break;
+          tc_fence_after();
+          const uint64_t dk = dK + st * kTileDesc;
 #pragma unroll
-        for (int h = 0; h < 2; ++h)
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off16 = ((kk >> 2) * HALF + (kk & 3) * 32) >> 4;
+            mma_bf16_ss(tmem + COL_S + b * 128, dq + off16, dk + off16, IDESC_QK,
+                        kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&bar[B_S_FULL + b]);
+          mma_commit(&bar[B_K_EMPTY + st]);
+          if (t == ntiles - 1) mma_commit(&bar[B_Q_EMPTY + qs]);
+        } else {
+          // O_b (+)= P V, b = the tile's warpgroup; both accumulators must have
+          // been read by the previous item's epilogue before the first PV.
+          // The first tile of each warpgroup in an item (t = 0, 1) starts O_b.
+          if (!(ok = wait(B_V_FULL + st, ph))) break;
+          if (t == 0 && item_no > 0 && !(ok = wait(B_O_FREE, (item_no - 1) & 1))) break;
+          if (!(ok = wait(B_P_FULL + b, (s_it >> 1) & 1))) break;
+          tc_fence_after();
+          const uint64_t dv = dV + st * kTileDesc;
+          const uint32_t ta = tmem + COL_S + b * 128;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            // P of half h: 64 keys packed two per column in the first 32
-            // columns of the half's own S region; 8 columns per 16 keys
-            mma_bf16_ts(tmem + COL_O + h * D, ta + h * 64 + kk * 8, dv + (4 * h + kk) * 128,
-                        IDESC_PV, (kk > 0 || !first) ? 1u : 0u);
-        mma_commit(&bar[B_PV_DONE + pb]);
-        mma_commit(&bar[B_V_EMPTY + vst]);
-        ++pv_it;
-        if (++vst == kStages) {
-          vst = 0;
-          vph ^= 1;
+          for (int kk = 0; kk < 8; ++kk)
+            // P: 128 keys packed two per column in the first 64 columns of
+            // the tile's S buffer; 8 columns per 16 keys
+            mma_bf16_ts(tmem + COL_O + b * D, ta + kk * 8, dv + kk * 128, IDESC_PV,
+                        (kk > 0 || t >= 2) ? 1u : 0u);
+          mma_commit(&bar[B_PV_DONE + b]);
+          mma_commit(&bar[B_V_EMPTY + st]);
         }
-        return true;
-      };
-      for (int t = 0; t < ntiles; ++t) {
-        // S[sb] last held P(t - 2), which PV(t - 2), issued before this QK,
-        // has consumed (the tensor core runs one thread's MMAs in order); the
-        // softmax read S(t - 2) before it signalled P_FULL(t - 2).
-        ok = wait(B_K_FULL + kst, kph);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t sb = s_it & 1;
-        const uint64_t dk = dK + kst * kTileDesc;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off16 = ((kk >> 2) * HALF + (kk & 3) * 32) >> 4;
-          mma_bf16_ss(tmem + COL_S + sb * 128, dQ + off16, dk + off16, IDESC_QK, kk > 0 ? 1u : 0u);
+        if (++st == (is_qk ? kStagesK : kStagesV)) {
+          st = 0;
+          ph ^= 1;
         }
-        mma_commit(&bar[B_S_FULL + sb]);
-        mma_commit(&bar[B_K_EMPTY + kst]);
-        if (t == ntiles - 1) mma_commit(&bar[B_Q_EMPTY]);
-        ++s_it;
-        if (++kst == kStages) {
-          kst = 0;
-          kph ^= 1;
-        }
-        if (t > 0 && !(ok = issue_pv(t == 1))) break;
       }
-      if (ok) ok = issue_pv(ntiles == 1);
     }
     // All issued MMAs must finish before TMEM is released.
-    mma_commit(&bar[B_DRAIN]);
-    drain_wait(&bar[B_DRAIN], 0);
-  } else if (warp >= 2) {
+    const int drain = is_qk ? B_DRAIN_QK : B_DRAIN;
+    mma_commit(&bar[drain]);
+    drain_wait(&bar[drain], 0);
+  } else if (warp >= 2 && warp < 2 + kSoftmaxThreads / 32) {
     // ------------------------------------------------------------ softmax
-    // Two warpgroups: kh = key half of every S row (keys 64 kh .. 64 kh + 63),
-    // each with its own running max / sum and its own O accumulator.
-    const int kh = (warp - 2) >> 2;
+    // Two warpgroups in ping-pong: warpgroup w takes the tiles whose CTA-wide
+    // index has parity w (all 128 keys of each), with its own running max /
+    // sum and its own O accumulator O_w; the two states are combined once, in
+    // the epilogue.  While one warpgroup exponentiates, the other loads,
+    // reduces and stores, so neither the exponential unit nor the tensor core
+    // waits on a lock-step phase.
+    const int wg = (warp - 2) >> 2;
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    const uint32_t col_o = COL_O + kh * D;
+    const uint32_t col_s = COL_S + wg * 128;
+    const uint32_t col_o = COL_O + wg * D;
     const float sl2 = p.scale_log2;
     uint32_t s_it = 0, item_no = 0;
     bool ok = true;
     for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x, ++item_no) {
       const Item it = load_item(p.items, idx);
       const int qpos = it.q_pos0 + row;
+      const uint32_t s_first = s_it;
       float m_ref = -INFINITY, l = 0.f;
+      uint32_t prev = 0;          // CTA-wide index of this warpgroup's previous tile
+      bool mine_any = false;
       for (int t = 0; t < it.ntiles; ++t, ++s_it) {
+        if ((int)(s_it & 1) != wg) continue;
         int r, kt;
         tile_of(it, t, r, kt);
-        const uint32_t sb = s_it & 1, ns = s_it >> 1;
-        ok = __all_sync(kFull, mbar_wait(&bar[B_S_FULL + sb], ns & 1, abort_flag, p.status,
-                                         kWaitLimitNs, DBSA_ERR_TIMEOUT));
+        ok = __all_sync(kFull, mbar_wait(&bar[B_S_FULL + wg], (s_it >> 1) & 1, abort_flag,
+                                         p.status, kWaitLimitNs, DBSA_ERR_TIMEOUT));
         if (!ok) break;
         tc_fence_after();
-        uint32_t v[2][32];
-#pragma unroll
-        for (int c = 0; c < 2; ++c)
-          tmem_ld32(tmem + lane_off + COL_S + sb * 128 + kh * 64 + c * 32, v[c]);
-#pragma unroll
-        for (int c = 0; c < 2; ++c) tmem_wait_ld(v[c]);
-
-        const int klim = (r ? it.len[1] : it.len[0]) - kt - kh * 64;    // valid keys of this half
-        const int kpos0 = (r ? it.pos0[1] : it.pos0[0]) + kt + kh * 64;
-        if (klim < 64 || kpos0 + 63 > it.q_pos0) {
-#pragma unroll
-          for (int c = 0; c < 2; ++c)
+        const int klim = (r ? it.len[1] : it.len[0]) - kt;   // valid keys of this tile
+        const int kpos0 = (r ? it.pos0[1] : it.pos0[0]) + kt;
+        const bool need_mask = klim < 128 || kpos0 + 127 > it.q_pos0;
+        const int klast = min(klim - 1, qpos - kpos0);       // last allowed key of this row
+        // -- pass 1: row maximum over the tile's 128 scores, 64 columns per load
+        float mt[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll 1
+        for (int c = 0; c < 4; c += 2) {
+          uint32_t va[32], vb[32];
+          tmem_ld32(tmem + lane_off + col_s + c * 32, va);
+          tmem_ld32(tmem + lane_off + col_s + c * 32 + 32, vb);
+          tmem_wait_ld(va);
+          tmem_wait_ld(vb);
+          if (need_mask) {
+            // masked scores are written back as -inf, so pass 2 needs no mask
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
-              const int k = c * 32 + e;
-              if (k >= klim || kpos0 + k > qpos) v[c][e] = __float_as_uint(-INFINITY);
+              if (c * 32 + e > klast) va[e] = __float_as_uint(-INFINITY);
+              if (c * 32 + 32 + e > klast) vb[e] = __float_as_uint(-INFINITY);
             }
-        }
-        float mt0 = -INFINITY, mt1 = -INFINITY, mt2 = -INFINITY, mt3 = -INFINITY;
+            tmem_st32(tmem + lane_off + col_s + c * 32, va);
+            tmem_st32(tmem + lane_off + col_s + c * 32 + 32, vb);
+          }
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          mt0 = fmaxf(mt0, __uint_as_float(v[0][e]));
-          mt1 = fmaxf(mt1, __uint_as_float(v[0][e + 1]));
-          mt2 = fmaxf(mt2, __uint_as_float(v[1][e]));
-          mt3 = fmaxf(mt3, __uint_as_float(v[1][e + 1]));
+          for (int e = 0; e < 32; e += 2) {
+            mt[(e >> 1) & 1] = max3(mt[(e >> 1) & 1], __uint_as_float(va[e]), __uint_as_float(va[e + 1]));
+            mt[2 + ((e >> 1) & 1)] =
+                max3(mt[2 + ((e >> 1) & 1)], __uint_as_float(vb[e]), __uint_as_float(vb[e + 1]));
+          }
         }
-        const float mt_x = fmaxf(fmaxf(mt0, mt1), fmaxf(mt2, mt3)) * sl2;
-        if (t == 0) {
+        if (need_mask) tmem_wait_st();
+        const float mt_x = max3(mt[0], mt[1], fmaxf(mt[2], mt[3])) * sl2;
+        if (!mine_any) {
           m_ref = mt_x;
         } else {
           const bool need = mt_x > m_ref + 8.0f;
           if (__any_sync(kFull, need)) {
-            // this half's O must hold every earlier tile before it is rescaled
-            const uint32_t prev = s_it - 1;
-            ok = __all_sync(kFull, mbar_wait(&bar[B_PV_DONE + (prev & 1)],
-                                             (prev >> 1) & 1, abort_flag, p.status, kWaitLimitNs,
-                                             DBSA_ERR_TIMEOUT));
+            // O_w must hold this warpgroup's earlier tiles before it is rescaled
+            ok = __all_sync(kFull, mbar_wait(&bar[B_PV_DONE + wg], (prev >> 1) & 1, abort_flag,
+                                             p.status, kWaitLimitNs, DBSA_ERR_TIMEOUT));
             if (!ok) break;
             tc_fence_after();
             const float m_new = fmaxf(m_ref, mt_x);
@@ -438,50 +501,68 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_wait_st();
           }
         }
+        mine_any = true;
+        prev = s_it;
+        // -- pass 2: P = 2^(s * scale - m) as bf16 pairs over S columns 0..63.
+        // Chunk c reads S columns 32c..32c+31 and writes P columns 16c..16c+15,
+        // whose scores were already read.
         const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
-        float sum0 = 0.f, sum1 = 0.f;
-#pragma unroll
-        for (int c = 0; c < 2; ++c)
+        const f32x2 sc2 = f2_pack(sl2, sl2), nmu2 = f2_pack(-mu, -mu);
+        f32x2 sum2[2] = {0ull, 0ull};
+        // chunk c of 32 scores -> 16 packed P columns; the next chunk's load is
+        // in flight while this one is exponentiated
+        auto exp_chunk = [&](const uint32_t (&v)[32], int c) {
+          uint32_t pw[16];
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            const float p0 = ex2(fmaf(__uint_as_float(v[c][e]), sl2, -mu));
-            const float p1 = ex2(fmaf(__uint_as_float(v[c][e + 1]), sl2, -mu));
-            sum0 += p0;
-            sum1 += p1;
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), sc2, nmu2),
+                      x0, x1);
+            const float p0 = ex2(x0), p1 = ex2(x1);
+            sum2[(e >> 1) & 1] = f2_add(sum2[(e >> 1) & 1], f2_pack(p0, p1));
             __nv_bfloat162 hh = __floats2bfloat162_rn(p0, p1);
-            v[c][e >> 1] = *reinterpret_cast<uint32_t *>(&hh);  // packed pairs in v[c][0..15]
+            pw[e >> 1] = *reinterpret_cast<uint32_t *>(&hh);
           }
-        l += sum0 + sum1;
-        // P of this half (64 keys, bf16 pairs) over the first 32 columns of the
-        // half's own S region, which this thread has already read.  The S(t+2)
-        // that next writes this buffer is issued after PV(t), and the tensor
-        // core runs one thread's MMAs in order.
-        {
-          uint32_t pw[32];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            pw[e] = v[0][e];
-            pw[16 + e] = v[1][e];
-          }
-          tmem_st32(tmem + lane_off + COL_S + sb * 128 + kh * 64, pw);
-          tmem_wait_st();
+          tmem_st16(tmem + lane_off + col_s + c * 16, pw);
+        };
+#pragma unroll 1
+        for (int c = 0; c < 4; c += 2) {
+          uint32_t va[32], vb[32];
+          tmem_ld32(tmem + lane_off + col_s + c * 32, va);
+          tmem_wait_ld(va);
+          tmem_ld32(tmem + lane_off + col_s + c * 32 + 32, vb);
+          exp_chunk(va, c);
+          tmem_wait_ld(vb);
+          exp_chunk(vb, c + 1);
         }
+        tmem_wait_st();
+        float sa, sb2, sc, sd;
+        f2_unpack(sum2[0], sa, sb2);
+        f2_unpack(sum2[1], sc, sd);
+        l += (sa + sb2) + (sc + sd);
+        // The S(t + 2) that next writes this buffer is issued after PV(t), and
+        // the tensor core runs one thread's MMAs in order.
         tc_fence_before();
-        mbar_arrive(&bar[B_P_FULL + sb]);
+        mbar_arrive(&bar[B_P_FULL + wg]);
       }
       if (!ok) break;
       // ---- epilogue: O = (O_0 e^{m_0 - M} + O_1 e^{m_1 - M}) / (l_0 e^{m_0 - M} + ...)
+      // The item's last PV done implies all of its PVs are (in-order tensor
+      // core).  A warpgroup without a tile in this item (single-tile items)
+      // has m = -inf, l = 0 and a stale O, which is not read.
       const uint32_t last = s_it - 1;
+      const bool has0 = it.ntiles >= 2 || (s_first & 1) == 0;
+      const bool has1 = it.ntiles >= 2 || (s_first & 1) == 1;
       ok = __all_sync(kFull, mbar_wait(&bar[B_PV_DONE + (last & 1)], (last >> 1) & 1, abort_flag,
                                        p.status, kWaitLimitNs, DBSA_ERR_TIMEOUT));
       if (!ok) break;
-      // Key half 1 publishes its (m, l); key half 0 merges the two states and
-      // publishes the factors (f0, f1) that both halves apply to O_0, O_1.
-      // Plain mode: f_h = e^{m_h - M} / L (normalised output); partial mode:
-      // f_h = e^{m_h - M} and (M, L) go to the split-partial arrays.
+      // Warpgroup 1 publishes its (m, l); warpgroup 0 merges the two states
+      // and publishes the factors (f0, f1) that both apply to O_0, O_1.
+      // Plain mode: f_w = e^{m_w - M} / L (normalised output); partial mode:
+      // f_w = e^{m_w - M} and (M, L) go to the split-partial arrays.
       const bool partial = p.part.acc != nullptr;
       float f0, f1;
-      if (kh == 1) {
+      if (wg == 1) {
         sML[row] = make_float2(m_ref, l);
         mbar_arrive(&bar[B_ML_A]);
         ok = __all_sync(kFull, mbar_wait(&bar[B_ML_B], item_no & 1, abort_flag, p.status,
@@ -522,13 +603,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         prow = ((int64_t)item * p.part.Hq + h) * p.part.n_new + w / p.part.group;
       }
       tc_fence_after();
-      // this thread writes output columns [kh * D/2, kh * D/2 + D/2) of its row
+      // this thread writes output columns [wg * D/2, wg * D/2 + D/2) of its row
       constexpr int HC = D / 2 / 32;   // 32-column chunks per half row
       const int64_t orow = ((int64_t)(it.q_row0 + row) * p.Hq + it.head) * D;
       float *pacc = partial ? p.part.acc + prow * D : nullptr;
 #pragma unroll
       for (int c = 0; c < HC; ++c) {
-        const int col = kh * (D / 2) + c * 32;
+        const int col = wg * (D / 2) + c * 32;
+        // both accumulators are read; a stale one is discarded by the select
+        // below (never multiplied: its bits may not be a finite number)
         uint32_t o0[32], o1[32];
         tmem_ld32(tmem + lane_off + COL_O + col, o0);
         tmem_ld32(tmem + lane_off + COL_O + D + col, o1);
@@ -538,7 +621,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           float f[32];
 #pragma unroll
           for (int e = 0; e < 32; ++e)
-            f[e] = __uint_as_float(o0[e]) * f0 + __uint_as_float(o1[e]) * f1;
+            f[e] = (has0 ? __uint_as_float(o0[e]) * f0 : 0.f) +
+                   (has1 ? __uint_as_float(o1[e]) * f1 : 0.f);
           if (partial) {
 #pragma unroll
             for (int e = 0; e < 32; e += 4)
@@ -612,7 +696,7 @@ constexpr size_t smem_bytes() {
   // alignment of the swizzled tiles.  The request is padded above half an
   // SM's shared memory so that no two CTAs share an SM: each one allocates
   // all 512 TMEM columns.
-  constexpr size_t need = 1024 + (size_t)128 * D * 2 * (1 + 2 * kStages) + 128 * sizeof(float2) +
+  constexpr size_t need = 1024 + (size_t)128 * D * 2 * (kStagesQ + kStagesK + kStagesV) + 128 * sizeof(float2) +
                           B_COUNT * 8 + 16;
   constexpr size_t one_per_sm = 232448 / 2 + 1024;
   return need > one_per_sm ? need : one_per_sm;
