@@ -28,7 +28,7 @@
 // already rotated (bf16) from the preparation pass; V is read straight from
 // the pre-RoPE cache.  Every wait is bounded and reports DBSA_ERR_TIMEOUT.
 //
-// Measured on B200 (see the profiles): the tensor core runs a 128x128x16
+// Measured on B200: the tensor core runs a 128x128x16
 // MMA in 64 cycles but keeps only about one MMA queued, so the issuing
 // threads must not stall between MMAs; softmax warps that saturate the FMA
 // pipe starve an issuer on the same SM sub-partition, hence the packed
