@@ -43,8 +43,8 @@ TRAFFIC = {
     # the prompt pass runs the tensor-core kernel in partial mode
     "stage2_prompt": {"bytes": 1.543696e9, "sources": ("stage1_attn.cu", "sm100.cuh"),
                       "sha": "cb61161f17f09bd1"},
-    "stage2_decode": {"bytes": 0.400653e9, "sources": ("stage2_attn.cu", "vec8.cuh"),
-                      "sha": "1d6cc9d81c9c6a1a"},
+    "stage2_decode": {"bytes": None, "sources": ("stage1_attn.cu", "sm100.cuh"),
+                      "sha": None},
 }
 
 
@@ -596,7 +596,7 @@ def main():
                "flop_per_launch": tile_flop, "launch_ms": round(s1_ms, 4)}
     roof_s2p = pass_roofline("stage1_attn_kernel, partial mode (block-major tcgen05, prompt pass)",
                              p_pass[:1], s2p_ms)
-    roof_s2d = (pass_roofline("stage2_attn_kernel (block-major + tail, decode step)",
+    roof_s2d = (pass_roofline("stage1_attn_kernel, partial mode (block-major tcgen05, decode step)",
                               p_pass[1:], s2d_ms) if len(p_pass) > 1 else None)
     if w.name == inputs.L31_8B_90K.name:   # the captures were taken on this workload
         roof_s1["traffic"] = traffic_for("stage1_attn")

@@ -227,16 +227,10 @@ struct GatherPlan {
   std::vector<S2Segment> segs;
   std::vector<S2Item> items;
   int32_t max_pos;  // largest key / query position + 1
-  // block-major mode (single-token passes): per (block, query group) entries;
-  // the per-query kernel then runs only the tail items listed in run_items
-  bool block_major = false;
-  std::vector<S2BEntry> bm_entries;
-  std::vector<S2BSlot> bm_slots;
+  // the tail items (one per query), which the per-query kernel runs
   std::vector<int32_t> run_items;
-  // tensor-core block-major mode (multi-token passes): the query rows of all
-  // (query, block) items packed block by block, and the tile list of the
-  // tensor-core kernel over them
-  bool tc = false;
+  // the query rows of all (query, block) items packed block by block, and the
+  // tile list of the tensor-core kernel over them
   int32_t tc_rows = 0;
   int32_t nb = 0;
   int64_t cache_rows = 0;  // offs[nb]
@@ -245,9 +239,6 @@ struct GatherPlan {
 };
 
 int32_t offs_count(const GatherPlan &gp) { return gp.nb + 1; }
-
-// Queries (rows) per block-major entry: the kernel's CTA holds 64 rows.
-constexpr int kBMRows = 64;
 
 dbsa_status gather_plan(const dbsa_config *cfg, const int32_t *offs, int32_t nb, int32_t nq,
                         const int32_t *sel_ptr, const int32_t *sel, int32_t n_new,
@@ -263,7 +254,6 @@ dbsa_status gather_plan(const dbsa_config *cfg, const int32_t *offs, int32_t nb,
   const int g = cfg->n_q_heads / cfg->n_kv_heads;
   const int R = g * n_new;
   std::vector<char> seen(nb, 0);
-  int64_t total_keys = 0;
   gp.max_pos = 0;
   for (int q = 0; q < nq; ++q) {
     const int32_t a = sel_ptr[q], e = sel_ptr[q + 1];
@@ -290,29 +280,16 @@ dbsa_status gather_plan(const dbsa_config *cfg, const int32_t *offs, int32_t nb,
     for (int32_t i = a; i < e; ++i) seen[sel[i]] = 0;
     if (p + tail_len > (1 << 30)) return fail(DBSA_ERR_INVALID_ARG, "gathered context too long");
     qi.n_gathered = (int32_t)p;
-    total_keys += p + tail_len;
     gp.max_pos = std::max<int32_t>(gp.max_pos, (int32_t)(p + tail_len));
     gp.queries.push_back(qi);
   }
-  // Split size: >= 33 keys per query row of a CTA (bounds the partial-result
-  // traffic to ~3 % of the K/V bytes) and enough CTAs for ~4 waves at one
-  // CTA per SM.  Rows per CTA follow the kernel's shape table (16, 32, 64,
-  // 128, else row groups of 160).
-  const int rows_cta = (R <= 16) ? 16 : (R <= 32) ? 32 : (R <= 64) ? 64 : (R <= 128) ? 128 : 160;
-  const int zdim = (R + rows_cta - 1) / rows_cta;
-  const int64_t min_chunk = std::max<int64_t>(256, (int64_t)33 * std::min(R, rows_cta));
-  const int64_t want_ctas = (int64_t)4 * num_sms();
-  const int64_t par_chunk =
-      (total_keys * cfg->n_kv_heads * zdim + want_ctas - 1) / std::max<int64_t>(1, want_ctas);
-  int64_t chunk = std::max(min_chunk, par_chunk);
-  chunk = (chunk + kS2Keys - 1) / kS2Keys * kS2Keys;
-  if (R > 16) {
-    // Multi-token passes: tensor-core block-major.  Items per query = one
+  {
+    // Every pass is block-major on the tensor core.  Items per query = one
     // per selected block + one for its own tail tokens (per-query kernel);
     // the rows of the block items are packed block by block (queries in
     // order, token-major rows within an item) and cut into 128-row tiles
-    // that all read the same block of rotated keys.
-    gp.tc = true;
+    // that all read the same block of rotated keys, so a block selected by
+    // many queries is read and rotated once per pass.
     std::vector<std::vector<int32_t>> per_block(nb);   // item ids selecting block b
     for (int q = 0; q < nq; ++q) {
       S2Query &qi = gp.queries[q];
@@ -364,72 +341,6 @@ dbsa_status gather_plan(const dbsa_config *cfg, const int32_t *offs, int32_t nb,
           t.len[0] = offs[b + 1] - offs[b];
           gp.tc_tiles.push_back(t);
         }
-    return DBSA_OK;
-  }
-  if (R <= 16) {
-    // Single-token passes: block-major.  Items per query = one per selected
-    // block (filled by the block-major kernel) + one for its own tail tokens
-    // (per-query kernel).  Entries group the queries that selected a block.
-    gp.block_major = true;
-    std::vector<std::vector<S2BSlot>> per_block(nb);
-    for (int q = 0; q < nq; ++q) {
-      S2Query &qi = gp.queries[q];
-      qi.item_begin = (int32_t)gp.items.size();
-      for (int sgi = 0; sgi < qi.n_seg; ++sgi) {
-        const S2Segment &sg = gp.segs[qi.seg_begin + sgi];
-        S2Item it;
-        it.query = q;
-        it.p_begin = sg.pos0;
-        it.p_end = sg.pos0 + sg.len;
-        it.p_lo = sg.pos0;
-        S2BSlot sl;
-        sl.query = q;
-        sl.pos0 = sg.pos0;
-        sl.item = (int32_t)gp.items.size();
-        sl.pad = 0;
-        per_block[sel[sel_ptr[q] + sgi]].push_back(sl);
-        gp.items.push_back(it);
-      }
-      S2Item tail;
-      tail.query = q;
-      tail.p_begin = qi.n_gathered & ~(kRopeLo - 1);  // aligned start; keys below
-      tail.p_end = qi.n_gathered + tail_len;          // n_gathered are masked
-      tail.p_lo = qi.n_gathered;
-      gp.run_items.push_back((int32_t)gp.items.size());
-      gp.items.push_back(tail);
-      qi.n_items = (int32_t)gp.items.size() - qi.item_begin;
-    }
-    const int qpc = std::max(1, kBMRows / R);
-    for (int b = 0; b < nb; ++b) {
-      const auto &v = per_block[b];
-      for (size_t i0 = 0; i0 < v.size(); i0 += qpc) {
-        S2BEntry e;
-        e.cache_row0 = offs[b];
-        e.len = offs[b + 1] - offs[b];
-        e.slot_begin = (int32_t)gp.bm_slots.size();
-        e.n_slots = (int32_t)std::min<size_t>(qpc, v.size() - i0);
-        for (int k = 0; k < e.n_slots; ++k) gp.bm_slots.push_back(v[i0 + k]);
-        gp.bm_entries.push_back(e);
-      }
-    }
-    return DBSA_OK;
-  }
-  for (int q = 0; q < nq; ++q) {
-    S2Query &qi = gp.queries[q];
-    const int64_t K = (int64_t)qi.n_gathered + tail_len;
-    const int64_t n_split = std::max<int64_t>(1, (K + chunk - 1) / chunk);
-    int64_t per = (K + n_split - 1) / n_split;
-    per = (per + kS2Keys - 1) / kS2Keys * kS2Keys;
-    qi.item_begin = (int32_t)gp.items.size();
-    for (int64_t s0 = 0; s0 < K; s0 += per) {
-      S2Item it;
-      it.query = q;
-      it.p_begin = (int32_t)s0;
-      it.p_end = (int32_t)std::min<int64_t>(K, s0 + per);
-      it.p_lo = it.p_begin;
-      gp.items.push_back(it);
-    }
-    qi.n_items = (int32_t)gp.items.size() - qi.item_begin;
   }
   return DBSA_OK;
 }
@@ -455,7 +366,7 @@ S1Layout s1_layout(const dbsa_config *cfg, int64_t max_pos, int64_t n_items, int
 }
 
 struct S2Layout {
-  size_t rope, queries, segs, items, bm_entries, bm_slots, run_items, row_item, item_row0,
+  size_t rope, queries, segs, items, run_items, row_item, item_row0,
       tc_tiles, offs, blob_end, k_hat, v_hat, q_hat, part_acc, part_ml, total;
   int32_t n_hi;
 };
@@ -467,19 +378,16 @@ S2Layout s2_layout(const dbsa_config *cfg, const GatherPlan &gp, int32_t n_new) 
   l.queries = cv.take(gp.queries.size() * sizeof(S2Query));
   l.segs = cv.take(gp.segs.size() * sizeof(S2Segment));
   l.items = cv.take(gp.items.size() * sizeof(S2Item));
-  l.bm_entries = cv.take(gp.bm_entries.size() * sizeof(S2BEntry));
-  l.bm_slots = cv.take(gp.bm_slots.size() * sizeof(S2BSlot));
   l.run_items = cv.take(gp.run_items.size() * sizeof(int32_t));
   l.row_item = cv.take(gp.row_item.size() * sizeof(int32_t));
   l.item_row0 = cv.take(gp.item_row0.size() * sizeof(int32_t));
   l.tc_tiles = cv.take(gp.tc_tiles.size() * sizeof(dbsa_tile_item));
-  l.offs = cv.take(gp.tc ? (size_t)(offs_count(gp)) * sizeof(int32_t) : 0);
+  l.offs = cv.take((size_t)(offs_count(gp)) * sizeof(int32_t));
   l.blob_end = cv.take(0);
   const int64_t T = gp.cache_rows;
-  l.k_hat = cv.take(gp.tc ? (size_t)cfg->n_kv_heads * T * cfg->head_dim * 2 : 0);
-  l.v_hat = cv.take(gp.tc && cfg->dtype == DBSA_F32 ? (size_t)cfg->n_kv_heads * T * cfg->head_dim * 2
-                                                     : 0);
-  l.q_hat = cv.take(gp.tc ? (size_t)cfg->n_kv_heads * gp.tc_rows * cfg->head_dim * 2 : 0);
+  l.k_hat = cv.take((size_t)cfg->n_kv_heads * T * cfg->head_dim * 2);
+  l.v_hat = cv.take(cfg->dtype == DBSA_F32 ? (size_t)cfg->n_kv_heads * T * cfg->head_dim * 2 : 0);
+  l.q_hat = cv.take((size_t)cfg->n_kv_heads * gp.tc_rows * cfg->head_dim * 2);
   const size_t rows = gp.items.size() * (size_t)cfg->n_q_heads * n_new;
   l.part_acc = cv.take(rows * cfg->head_dim * sizeof(float));
   l.part_ml = cv.take(rows * sizeof(float2));
@@ -835,25 +743,15 @@ dbsa_status dbsa_gather_rope_attend(const dbsa_config *cfg, const void *k_cache,
                 gp.segs.size() * sizeof(S2Segment));
     std::memcpy(blob.data() + (L.items - L.queries), gp.items.data(),
                 gp.items.size() * sizeof(S2Item));
-    if (gp.block_major) {
-      std::memcpy(blob.data() + (L.bm_entries - L.queries), gp.bm_entries.data(),
-                  gp.bm_entries.size() * sizeof(S2BEntry));
-      std::memcpy(blob.data() + (L.bm_slots - L.queries), gp.bm_slots.data(),
-                  gp.bm_slots.size() * sizeof(S2BSlot));
-      std::memcpy(blob.data() + (L.run_items - L.queries), gp.run_items.data(),
-                  gp.run_items.size() * sizeof(int32_t));
-    }
-    if (gp.tc) {
-      std::memcpy(blob.data() + (L.run_items - L.queries), gp.run_items.data(),
-                  gp.run_items.size() * sizeof(int32_t));
-      std::memcpy(blob.data() + (L.row_item - L.queries), gp.row_item.data(),
-                  gp.row_item.size() * sizeof(int32_t));
-      std::memcpy(blob.data() + (L.item_row0 - L.queries), gp.item_row0.data(),
-                  gp.item_row0.size() * sizeof(int32_t));
-      std::memcpy(blob.data() + (L.tc_tiles - L.queries), gp.tc_tiles.data(),
-                  gp.tc_tiles.size() * sizeof(dbsa_tile_item));
-      std::memcpy(blob.data() + (L.offs - L.queries), offs_host, (size_t)(nb + 1) * sizeof(int32_t));
-    }
+    std::memcpy(blob.data() + (L.run_items - L.queries), gp.run_items.data(),
+                gp.run_items.size() * sizeof(int32_t));
+    std::memcpy(blob.data() + (L.row_item - L.queries), gp.row_item.data(),
+                gp.row_item.size() * sizeof(int32_t));
+    std::memcpy(blob.data() + (L.item_row0 - L.queries), gp.item_row0.data(),
+                gp.item_row0.size() * sizeof(int32_t));
+    std::memcpy(blob.data() + (L.tc_tiles - L.queries), gp.tc_tiles.data(),
+                gp.tc_tiles.size() * sizeof(dbsa_tile_item));
+    std::memcpy(blob.data() + (L.offs - L.queries), offs_host, (size_t)(nb + 1) * sizeof(int32_t));
     if ((e = cudaMemcpyAsync(at<void>(workspace, L.queries), blob.data(), blob.size(),
                              cudaMemcpyHostToDevice, st)) != cudaSuccess)
       return cuda_fail(e, "gather plan upload");
@@ -875,11 +773,8 @@ dbsa_status dbsa_gather_rope_attend(const dbsa_config *cfg, const void *k_cache,
   a.items = at<S2Item>(workspace, L.items);
   a.n_items = (int32_t)gp.items.size();
   a.n_queries = nq;
-  a.run_items = (gp.block_major || gp.tc) ? at<int32_t>(workspace, L.run_items) : nullptr;
+  a.run_items = at<int32_t>(workspace, L.run_items);
   a.n_run = (int32_t)gp.run_items.size();
-  a.bm_entries = gp.block_major ? at<S2BEntry>(workspace, L.bm_entries) : nullptr;
-  a.bm_slots = gp.block_major ? at<S2BSlot>(workspace, L.bm_slots) : nullptr;
-  a.n_bm_entries = (int32_t)gp.bm_entries.size();
   a.part_acc = at<float>(workspace, L.part_acc);
   a.part_ml = at<float2>(workspace, L.part_ml);
   a.out = out;
@@ -888,7 +783,7 @@ dbsa_status dbsa_gather_rope_attend(const dbsa_config *cfg, const void *k_cache,
   a.scale_log2 = scale_log2(cfg);
   a.rope = rope;
   const bool f32 = cfg->dtype == DBSA_F32;
-  if (gp.tc) {
+  {
     // keys at block-relative positions, packed query rows, then the
     // tensor-core kernel over (kv head, block, 128-row tile) in partial mode
     RelRopeArgs ra{};
@@ -959,13 +854,6 @@ dbsa_status dbsa_gather_rope_attend(const dbsa_config *cfg, const void *k_cache,
     if ((e = launch_stage2_main(a, cfg->head_dim, f32, st)) != cudaSuccess)  // tail items
       return cuda_fail(e, "stage-2 tail attention");
     count_launches(1);
-  } else {
-    {
-      ProfileScope prof(st);
-      e = launch_stage2_main(a, cfg->head_dim, f32, st);
-    }
-    if (e != cudaSuccess) return cuda_fail(e, "stage-2 attention");
-    count_launches(gp.block_major ? 2 : 1);  // block-major: block kernel + tail kernel
   }
   if ((e = launch_stage2_merge(a, cfg->head_dim, f32, st)) != cudaSuccess)
     return cuda_fail(e, "stage-2 merge");

@@ -15,7 +15,6 @@ constexpr int kTileRows = 128;   // Stage-1 query rows per tile (tcgen05 M)
 constexpr int kTileKeys = 128;   // Stage-1 keys per score tile (tcgen05 N)
 constexpr int kRopeLo = 16;      // positions per RoPE "hi" table step
 constexpr int kRopeShift = 4;    // log2(kRopeLo)
-constexpr int kS2Keys = 64;      // Stage-2 split boundaries are multiples of this
 
 // Head of every workspace: the device status word (cleared by each call).
 constexpr size_t kStatusBytes = 256;
@@ -51,23 +50,6 @@ struct S2Item {
   int32_t p_end;       // p_begin is a multiple of 16 (the kernel's RoPE step)
   int32_t p_lo;        // keys below p_lo (>= p_begin) belong to other items: masked
 };
-// Block-major Stage 2 (single-token passes of a query batch): one entry per
-// (block, group of queries that selected it).  The block's keys are rotated
-// once at block-relative positions r and each query row at (its position -
-// the block's fresh start P), since R(a)^T R(b) = R(b - a).
-struct S2BEntry {
-  int32_t cache_row0;  // first cache row of the block
-  int32_t len;         // tokens of the block
-  int32_t slot_begin;  // first slot of this entry
-  int32_t n_slots;     // queries of this entry
-};
-struct S2BSlot {
-  int32_t query;
-  int32_t pos0;        // fresh start position P of the block in this query's cache
-  int32_t item;        // split item (partial slot) of (query, block)
-  int32_t pad;
-};
-
 // ---- launchers (each returns cudaGetLastError() after enqueueing) ----
 
 // Fills the four tables (laid out back to back from `base`: hc, hs, lc, ls).
@@ -191,11 +173,8 @@ struct Stage2Args {
   const S2Segment *segs;
   const S2Item *items;
   int32_t n_items, n_queries;
-  const int32_t *run_items;        // items the per-query kernel runs (null: all n_items)
+  const int32_t *run_items;        // the tail items, which the per-query kernel runs
   int32_t n_run;
-  const S2BEntry *bm_entries;      // block-major entries (null: none)
-  const S2BSlot *bm_slots;
-  int32_t n_bm_entries;
   float *part_acc;                 // [n_items][Hq][n_new][D]
   float2 *part_ml;                 // [n_items][Hq][n_new] (m in log2 units, l)
   void *out;                       // [nq][n_new][Hq][D]

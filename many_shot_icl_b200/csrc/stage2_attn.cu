@@ -1,22 +1,24 @@
-// Stage 2: fused gather + RoPE re-rotation + GQA attention, split over the
-// key sequence ("split-KV"), then a log-sum-exp merge of the splits.
+// Stage 2, per-query part: each query's own tail tokens, then the log-sum-exp
+// merge of all split partials.
 //
 // [DBSA notes] §Stage 2, items 2-4: the selected blocks (sink first) are
 // concatenated, their cached pre-RoPE keys are rotated again at fresh
 // sequential positions, and the query tokens attend to the whole gathered
-// cache.  Query q's key sequence is [gathered tokens 0..T'_q) ++ [its own tail
-// tokens], positions 0..T'_q + tail_len - 1, so one causal rule (key position
-// <= row position) covers both parts.
+// cache and, causally, to the query's own tokens.  Query q's key sequence is
+// [gathered tokens 0..T'_q) ++ [its own tail tokens], positions
+// 0..T'_q + tail_len - 1.  The gathered blocks are handled block by block by
+// the tensor-core kernel (one partial per (query, block)); this file holds the
+// kernel for the remaining split item of each query, its tail keys
+// [T'_q, T'_q + tail_len), and the merge of every partial of a query row.
 //
-// Grid: (split item, KV head, row group).  Every CTA reads each key of its
-// split once and scores it against all g * n_new query rows that share the KV
-// head (GQA), so the cache is streamed from HBM once per (query, KV head).
-// Keys are fetched with 16-byte cp.async through a per-thread segment walk
-// (the gather), rotated in shared memory (fp32 math, two-level fp64-built
-// table), and multiplied on the tensor cores with mma.sync (bf16 in, fp32
-// accumulate); softmax runs online in registers.  Decode passes (<= 16 rows)
-// split each key tile across the four warps and merge them through shared
-// memory; longer passes give each warp 16 rows.
+// Grid of the tail kernel: (tail item, KV head, row group).  A CTA reads each
+// tail key once and scores it against all g * n_new query rows that share the
+// KV head (GQA).  Keys are fetched with 16-byte cp.async, rotated in shared
+// memory (fp32 math, two-level fp64-built table) at their positions, and
+// multiplied with mma.sync (bf16 in, fp32 accumulate); softmax runs online in
+// registers and one causal rule (key position <= row position) covers the
+// tail.  Passes of <= 16 rows split each key tile across the warps and merge
+// them through shared memory; longer passes give each warp 16 rows.
 #include <cuda_bf16.h>
 
 #include <cfloat>
@@ -90,12 +92,7 @@ __device__ __forceinline__ uint32_t soff(int row, int chunk) {
 // for its 16 rows; the key groups' states are merged through shared memory at
 // the end and written as one split partial.
 //
-// BM (block-major) selects the single-token pass layout: the CTA's keys are
-// one selected block (positions r = 0..L-1 relative to the block, rotated
-// by r), its rows are the g * n_new rows of each query in the entry's slot
-// list (each rotated by its position minus the block's fresh start), and
-// there is no causal limit (every gathered key precedes the query tokens).
-template <int D, typename CT, int RT, int KG, int KT, int NST, bool BM>
+template <int D, typename CT, int RT, int KG, int KT, int NST>
 __global__ void __launch_bounds__(32 * RT * KG, 1) stage2_attn_kernel(const Stage2Args a) {
   constexpr int H = D / 2;
   constexpr int CH = D / 8;                 // 16-byte chunks per row
@@ -119,31 +116,17 @@ __global__ void __launch_bounds__(32 * RT * KG, 1) stage2_attn_kernel(const Stag
   const int c = blockIdx.y;
   const int g = a.Hq / a.Hkv;
   const int RQ = g * a.n_new;                      // rows of one query
-  // per-query mode: one split item; block-major mode: one (block, queries) entry
-  int it_idx = 0, q = 0, Tq = 0, k_begin, k_end, k_lo, R;
-  S2Query qi;
-  S2BEntry be;
-  if constexpr (!BM) {
-    it_idx = a.run_items ? a.run_items[blockIdx.x] : (int)blockIdx.x;
-    const S2Item item = a.items[it_idx];
-    qi = a.queries[item.query];
-    q = item.query;
-    Tq = qi.n_gathered;
-    k_begin = item.p_begin;
-    k_end = item.p_end;
-    k_lo = item.p_lo;
-    R = RQ;
-  } else {
-    be = a.bm_entries[blockIdx.x];
-    k_begin = 0;
-    k_end = be.len;
-    k_lo = 0;
-    R = be.n_slots * RQ;
-  }
+  // one tail item: keys [p_lo, p_end) of the query's sequence are its own
+  // tail tokens (p_begin is p_lo rounded down to the RoPE step; the keys
+  // below p_lo belong to the gathered blocks and are masked)
+  const int it_idx = a.run_items[blockIdx.x];
+  const S2Item item = a.items[it_idx];
+  const int q = item.query;
+  const int Tq = a.queries[q].n_gathered;
+  const int k_begin = item.p_begin, k_end = item.p_end, k_lo = item.p_lo;
+  const int R = RQ;
   const int pos_first = Tq + a.tail_len - a.n_new;  // position of query token 0 (per query)
   const int row_base = blockIdx.z * MROWS;
-  const CT *kc = static_cast<const CT *>(a.k_cache);
-  const CT *vc = static_cast<const CT *>(a.v_cache);
   const CT *kt = static_cast<const CT *>(a.k_tail);
   const CT *vt = static_cast<const CT *>(a.v_tail);
 
@@ -165,22 +148,9 @@ __global__ void __launch_bounds__(32 * RT * KG, 1) stage2_attn_kernel(const Stag
     const int r = row_base + rr;
     float lo[8], hi[8];
     if (r < R) {
-      int qq = q, tok, h, pos;
-      if constexpr (!BM) {
-        tok = r / g;
-        h = c * g + r % g;
-        pos = pos_first + tok;
-      } else {
-        const S2BSlot sl = a.bm_slots[be.slot_begin + r / RQ];
-        const int within = r % RQ;
-        qq = sl.query;
-        tok = within / g;
-        h = c * g + within % g;
-        // query token position minus the block's fresh start
-        pos = a.queries[qq].n_gathered + a.tail_len - a.n_new + tok - sl.pos0;
-      }
+      const int tok = r / g, h = c * g + r % g, pos = pos_first + tok;
       const CT *src = static_cast<const CT *>(a.q_new) +
-                      (((int64_t)qq * a.n_new + tok) * a.Hq + h) * D;
+                      (((int64_t)q * a.n_new + tok) * a.Hq + h) * D;
       load8(src + cp * 8, lo);
       load8(src + H + cp * 8, hi);
       float cs[8], sn[8];
@@ -194,17 +164,16 @@ __global__ void __launch_bounds__(32 * RT * KG, 1) stage2_attn_kernel(const Stag
     store8_bf16(reinterpret_cast<bf16 *>(sQ + soff<D>(rr, cp + H / 8)), hi);
   }
 
-  // ---- gather: warp wr of a key group loads (and later rotates) rows
+  // ---- loads: warp wr of a key group loads (and later rotates) rows
   // [wr * RPW, (wr + 1) * RPW) of each sub-tile.  Lane l (l < RPW) resolves
-  // the cache row of row l for K, lane 16 + l the same row for V; then every
+  // the tail row of row l for K, lane 16 + l the same row for V; then every
   // copy instruction moves one whole K row (lanes 0-15) and one whole V row
-  // (lanes 16-31), 256 contiguous bytes each.
+  // (lanes 16-31).
   constexpr int RPW = KT / RT;
   static_assert(RPW <= 16 && CH <= 16, "one row per half-warp");
   const int n_sub = (k_end - k_begin + KT - 1) / KT;
   const int n_local = kg < n_sub ? (n_sub - kg + KG - 1) / KG : 0;
   const int half_id = lane >> 4, hl = lane & 15;  // half-warp: 0 = K, 1 = V
-  int seg = 0;  // segment cursor: this lane's positions only grow
   auto stage_ptr = [&](int jl, int kv) -> uint8_t * {
     return sRing + ((size_t)(kg * NST + jl % NST) * 2 + kv) * STAGEB;
   };
@@ -214,32 +183,9 @@ __global__ void __launch_bounds__(32 * RT * KG, 1) stage2_attn_kernel(const Stag
     const CT *my = nullptr;
     if (hl < RPW) {
       const int p = p0 + hl;
-      if (p < k_end && p >= k_lo) {
-        if constexpr (BM) {
-          const int64_t crow = (int64_t)be.cache_row0 + p;
-          my = (half_id ? vc : kc) + ((int64_t)c * a.cap + crow) * D;
-          if (a.dbg_map != nullptr && c == 0 && blockIdx.z == 0 && half_id == 0) {
-            for (int sl = 0; sl < be.n_slots; ++sl) {
-              const S2BSlot slot = a.bm_slots[be.slot_begin + sl];
-              int32_t *m = a.dbg_map + ((int64_t)slot.query * a.dbg_cap + slot.pos0 + p) * 2;
-              m[0] = (int32_t)crow;
-              m[1] = slot.pos0 + p;
-            }
-          }
-        } else if (p < Tq) {
-          while (seg + 1 < qi.n_seg && __ldg(&a.segs[qi.seg_begin + seg + 1].pos0) <= p) ++seg;
-          const int64_t crow = (int64_t)__ldg(&a.segs[qi.seg_begin + seg].cache_row0) +
-                               (p - __ldg(&a.segs[qi.seg_begin + seg].pos0));
-          my = (half_id ? vc : kc) + ((int64_t)c * a.cap + crow) * D;
-          if (a.dbg_map != nullptr && c == 0 && blockIdx.z == 0 && half_id == 0) {
-            int32_t *m = a.dbg_map + ((int64_t)q * a.dbg_cap + p) * 2;
-            m[0] = (int32_t)crow;
-            m[1] = p;
-          }
-        } else {
-          const int64_t w = p - Tq;
-          my = (half_id ? vt : kt) + (((int64_t)q * a.tail_cap + w) * a.Hkv + c) * D;
-        }
+      if (p < k_end && p >= k_lo) {   // k_lo = T'_q: p is tail token p - T'_q
+        const int64_t w = p - Tq;
+        my = (half_id ? vt : kt) + (((int64_t)q * a.tail_cap + w) * a.Hkv + c) * D;
       }
     }
     uint8_t *dst = stage_ptr(jl, half_id);
@@ -285,7 +231,7 @@ __global__ void __launch_bounds__(32 * RT * KG, 1) stage2_attn_kernel(const Stag
 #pragma unroll
   for (int h2 = 0; h2 < 2; ++h2) {
     const int r = row_base + wr * 16 + gq + 8 * h2;
-    qpos[h2] = (!BM && r < R) ? pos_first + r / g : INT_MAX;
+    qpos[h2] = r < R ? pos_first + r / g : INT_MAX;
   }
 
   float o[ND][4];
@@ -377,7 +323,7 @@ __global__ void __launch_bounds__(32 * RT * KG, 1) stage2_attn_kernel(const Stag
       }
     }
     // ---- mask (split end; causal inside the query's own tail), online softmax
-    const bool need_mask = (p0 + KT > k_end) || (p0 < k_lo) || (!BM && p0 + KT - 1 > pos_first);
+    const bool need_mask = (p0 + KT > k_end) || (p0 < k_lo) || (p0 + KT - 1 > pos_first);
     float tmax[2] = {-INFINITY, -INFINITY};
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb)
@@ -448,13 +394,7 @@ __global__ void __launch_bounds__(32 * RT * KG, 1) stage2_attn_kernel(const Stag
     l_run[h2] += __shfl_xor_sync(0xFFFFFFFFu, l_run[h2], 2);
   }
   auto part_index = [&](int r) -> int64_t {  // r = row index of the CTA (token-major)
-    if constexpr (BM) {
-      const int item = a.bm_slots[be.slot_begin + r / RQ].item;
-      const int within = r % RQ;
-      return ((int64_t)item * a.Hq + c * g + within % g) * a.n_new + within / g;
-    } else {
-      return ((int64_t)it_idx * a.Hq + c * g + r % g) * a.n_new + r / g;
-    }
+    return ((int64_t)it_idx * a.Hq + c * g + r % g) * a.n_new + r / g;
   };
 
   if constexpr (KG == 1) {
@@ -554,7 +494,7 @@ __global__ void __launch_bounds__(128) stage2_merge_kernel(const Stage2Args a) {
   }
 }
 
-template <int D, typename CT, int RT, int KG, int KT, bool BM = false>
+template <int D, typename CT, int RT, int KG, int KT>
 cudaError_t launch_main(const Stage2Args &a, cudaStream_t st) {
   constexpr int NST = 3;
   constexpr int MROWS = 16 * RT;
@@ -563,15 +503,13 @@ cudaError_t launch_main(const Stage2Args &a, cudaStream_t st) {
   constexpr size_t lo_tables = (size_t)2 * kRopeLo * (D / 2) * sizeof(float);
   constexpr size_t smem = (size_t)MROWS * D * 2 + lo_tables + (ring > merge ? ring : merge);
   static_assert(smem <= 232448, "shared memory budget");
-  cudaError_t e = cudaFuncSetAttribute(stage2_attn_kernel<D, CT, RT, KG, KT, NST, BM>,
+  cudaError_t e = cudaFuncSetAttribute(stage2_attn_kernel<D, CT, RT, KG, KT, NST>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int R = (a.Hq / a.Hkv) * a.n_new;
-  // block-major entries hold at most MROWS rows (the host packs them so)
-  const int n_x = BM ? a.n_bm_entries : (a.run_items ? a.n_run : a.n_items);
-  if (n_x <= 0) return cudaSuccess;
-  dim3 grid(n_x, a.Hkv, BM ? 1 : (R + MROWS - 1) / MROWS);
-  stage2_attn_kernel<D, CT, RT, KG, KT, NST, BM><<<grid, 32 * RT * KG, smem, st>>>(a);
+  if (a.n_run <= 0) return cudaSuccess;
+  dim3 grid(a.n_run, a.Hkv, (R + MROWS - 1) / MROWS);
+  stage2_attn_kernel<D, CT, RT, KG, KT, NST><<<grid, 32 * RT * KG, smem, st>>>(a);
   return cudaGetLastError();
 }
 
@@ -581,12 +519,6 @@ cudaError_t launch_main(const Stage2Args &a, cudaStream_t st) {
 template <int D, typename CT>
 cudaError_t launch_d(const Stage2Args &a, cudaStream_t st) {
   const int R = (a.Hq / a.Hkv) * a.n_new;
-  if (a.bm_entries != nullptr) {
-    // block-major pass: entries of up to 64 rows (4 warps, 32-key sub-tiles,
-    // two CTAs per SM), then the per-query tail items
-    cudaError_t e = launch_main<D, CT, 4, 1, 32, true>(a, st);
-    if (e != cudaSuccess) return e;
-  }
   if (R <= 16) return launch_main<D, CT, 1, 8, 16>(a, st);
   if (R <= 32) return launch_main<D, CT, 2, 4, 32>(a, st);
   if (R <= 64) return launch_main<D, CT, 4, 2, 64>(a, st);

@@ -134,7 +134,7 @@ def run_stage2(w, cfg, kc, vc, offs, sels, n_new, tail_len, seed):
 @pytest.mark.parametrize("name,order,n_new,tail_len", [
     ("llama2-7b-30k", "encoding", 32, 32),
     ("llama3.1-8b-90k", "encoding", 40, 40),     # prompt pass (per-query kernel)
-    ("llama3.1-8b-90k", "encoding", 1, 45),      # a decode step (block-major kernel)
+    ("llama3.1-8b-90k", "encoding", 1, 45),      # a decode step
     ("llama3.1-8b-128k", "encoding", 32, 32),
     ("llama3.1-8b-128k", "ascending", 32, 32),
 ])
