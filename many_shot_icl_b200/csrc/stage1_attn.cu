@@ -19,9 +19,12 @@
 //               tiles whose CTA-wide index has parity w (all 128 keys of
 //               each), one thread per query row (TMEM lane), with its own
 //               fp32 running max and sum (lazy rescale threshold) and its own
-//               O accumulator O_w; the two states are combined once, in the
-//               epilogue.  While one warpgroup exponentiates (one MUFU op
-//               per score), the other loads, reduces and stores.
+//               O accumulator O_w.  While one warpgroup exponentiates (one
+//               MUFU op per score), the other loads, reduces and stores.  At
+//               an item's end they publish the merge factors of the two
+//               states and go on to the next item.
+//   warps 11..14 epilogue: combine O_0 and O_1 of the finished item, store
+//               the output, free O for the next item's first PV.
 // S = Q K^T lives in TMEM in two 128-column buffers (tile parity), P is
 // written back over the first 64 columns of its own S buffer as bf16 pairs,
 // and O_0, O_1 take D columns each: 512 columns in all.  Q and K arrive
@@ -68,15 +71,17 @@ enum Bar {
   B_P_FULL = B_S_FULL + 2,     // [buffer]: P written by the buffer's warpgroup
   B_PV_DONE = B_P_FULL + 2,    // [buffer]: PV of the buffer's tile done
   B_O_FREE = B_PV_DONE + 2, B_DRAIN = B_O_FREE + 1,
-  B_ML_A = B_DRAIN + 1,       // epilogue: key half 1 has published (m, l)
-  B_ML_B = B_ML_A + 1,        // epilogue: warpgroup 0 has published the merge factors
-  B_DRAIN_QK = B_ML_B + 1,
+  B_ML_A = B_DRAIN + 1,       // end of item: warpgroup 1 has published (m, l)
+  B_ML_B = B_ML_A + 1,        // end of item: warpgroup 0 has published the merge factors
+  B_ML_FREE = B_ML_B + 1,     // the epilogue warpgroup has read the merge factors
+  B_DRAIN_QK = B_ML_FREE + 1,
   B_COUNT = B_DRAIN_QK + 1
 };
 
 constexpr int kSoftmaxThreads = 256;              // warps 2..9: two warpgroups
 constexpr int kQKWarp = 10;                       // QK^T issuer (after the softmax warps)
-constexpr int kThreads = 96 + kSoftmaxThreads;    // + TMA warp, PV warp, QK warp
+constexpr int kEpiWarp0 = 11;                     // warps 11..14: epilogue warpgroup
+constexpr int kThreads = 32 * (kEpiWarp0 + 4);
 
 struct Item {
   int head, q_row0, q_pos0, n_rows, n_ranges;
@@ -216,11 +221,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bar[B_P_FULL + s], 128);
       mbar_init(&bar[B_PV_DONE + s], 1);
     }
-    mbar_init(&bar[B_O_FREE], kSoftmaxThreads);
+    mbar_init(&bar[B_O_FREE], 128);
     mbar_init(&bar[B_DRAIN], 1);
     mbar_init(&bar[B_DRAIN_QK], 1);
     mbar_init(&bar[B_ML_A], 128);
     mbar_init(&bar[B_ML_B], 128);
+    mbar_init(&bar[B_ML_FREE], 128);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -431,7 +437,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x, ++item_no) {
       const Item it = load_item(p.items, idx);
       const int qpos = it.q_pos0 + row;
-      const uint32_t s_first = s_it;
       float m_ref = -INFINITY, l = 0.f;
       uint32_t prev = 0;          // CTA-wide index of this warpgroup's previous tile
       bool mine_any = false;
@@ -546,31 +551,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&bar[B_P_FULL + wg]);
       }
       if (!ok) break;
-      // ---- epilogue: O = (O_0 e^{m_0 - M} + O_1 e^{m_1 - M}) / (l_0 e^{m_0 - M} + ...)
-      // The item's last PV done implies all of its PVs are (in-order tensor
-      // core).  A warpgroup without a tile in this item (single-tile items)
-      // has m = -inf, l = 0 and a stale O, which is not read.
-      const uint32_t last = s_it - 1;
-      const bool has0 = it.ntiles >= 2 || (s_first & 1) == 0;
-      const bool has1 = it.ntiles >= 2 || (s_first & 1) == 1;
-      ok = __all_sync(kFull, mbar_wait(&bar[B_PV_DONE + (last & 1)], (last >> 1) & 1, abort_flag,
-                                       p.status, kWaitLimitNs, DBSA_ERR_TIMEOUT));
-      if (!ok) break;
-      // Warpgroup 1 publishes its (m, l); warpgroup 0 merges the two states
-      // and publishes the factors (f0, f1) that both apply to O_0, O_1.
-      // Plain mode: f_w = e^{m_w - M} / L (normalised output); partial mode:
-      // f_w = e^{m_w - M} and (M, L) go to the split-partial arrays.
+      // ---- end of item: merge factors for O = (O_0 e^{m_0 - M} + O_1 e^{m_1 - M}) /
+      // (l_0 e^{m_0 - M} + l_1 e^{m_1 - M}).  Warpgroup 1 publishes its (m, l);
+      // warpgroup 0 merges the two states and publishes (f0, f1) for the
+      // epilogue warpgroup.  Plain mode: f_w = e^{m_w - M} / L (normalised
+      // output); partial mode: f_w = e^{m_w - M} and (M, L) go to the
+      // split-partial arrays.  Both warpgroups then go on to the next item.
       const bool partial = p.part.acc != nullptr;
-      float f0, f1;
       if (wg == 1) {
+        if (item_no > 0)
+          ok = __all_sync(kFull, mbar_wait(&bar[B_ML_FREE], (item_no - 1) & 1, abort_flag,
+                                           p.status, kWaitLimitNs, DBSA_ERR_TIMEOUT));
+        if (!ok) break;
         sML[row] = make_float2(m_ref, l);
         mbar_arrive(&bar[B_ML_A]);
-        ok = __all_sync(kFull, mbar_wait(&bar[B_ML_B], item_no & 1, abort_flag, p.status,
-                                         kWaitLimitNs, DBSA_ERR_TIMEOUT));
-        if (!ok) break;
-        const float2 f = sML[row];
-        f0 = f.x;
-        f1 = f.y;
       } else {
         ok = __all_sync(kFull, mbar_wait(&bar[B_ML_A], item_no & 1, abort_flag, p.status,
                                          kWaitLimitNs, DBSA_ERR_TIMEOUT));
@@ -581,9 +575,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float w1 = (ml1.x == -INFINITY) ? 0.f : ex2(ml1.x - M);
         const float L = l * w0 + ml1.y * w1;
         const float inv = partial ? 1.f : 1.f / L;
-        f0 = w0 * inv;
-        f1 = w1 * inv;
-        sML[row] = make_float2(f0, f1);
+        sML[row] = make_float2(w0 * inv, w1 * inv);
         mbar_arrive(&bar[B_ML_B]);
         if (partial && row < it.n_rows) {
           const int grow = it.q_row0 + row;
@@ -594,6 +586,36 @@ __global__ void __launch_bounds__(kThreads, 1)
               make_float2(M, L);
         }
       }
+    }
+  } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
+    // ------------------------------------------------------------ epilogue
+    // One thread per row (TMEM lane).  Per item: the merge factors, then, once
+    // the item's last PV is done (in-order tensor core: so are all of its
+    // PVs), O_0 and O_1 are read, combined and stored; O is then free for the
+    // next item's first PV.  A warpgroup without a tile in the item
+    // (single-tile items) left a stale O, which the selects discard.
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const bool partial = p.part.acc != nullptr;
+    uint32_t s_it = 0, item_no = 0;
+    bool ok = true;
+    for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x, ++item_no) {
+      const Item it = load_item(p.items, idx);
+      const uint32_t s_first = s_it;
+      s_it += it.ntiles;
+      const uint32_t last = s_it - 1;
+      const bool has0 = it.ntiles >= 2 || (s_first & 1) == 0;
+      const bool has1 = it.ntiles >= 2 || (s_first & 1) == 1;
+      ok = __all_sync(kFull, mbar_wait(&bar[B_ML_B], item_no & 1, abort_flag, p.status,
+                                       kWaitLimitNs, DBSA_ERR_TIMEOUT));
+      if (!ok) break;
+      const float2 fw = sML[row];
+      mbar_arrive(&bar[B_ML_FREE]);
+      ok = __all_sync(kFull, mbar_wait(&bar[B_PV_DONE + (last & 1)], (last >> 1) & 1, abort_flag,
+                                       p.status, kWaitLimitNs, DBSA_ERR_TIMEOUT));
+      if (!ok) break;
+      tc_fence_after();
       int64_t prow = 0;
       if (partial && row < it.n_rows) {
         const int grow = it.q_row0 + row;                 // row of the packed query buffer
@@ -602,37 +624,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int h = it.head * p.part.group + w % p.part.group;
         prow = ((int64_t)item * p.part.Hq + h) * p.part.n_new + w / p.part.group;
       }
-      tc_fence_after();
-      // this thread writes output columns [wg * D/2, wg * D/2 + D/2) of its row
-      constexpr int HC = D / 2 / 32;   // 32-column chunks per half row
       const int64_t orow = ((int64_t)(it.q_row0 + row) * p.Hq + it.head) * D;
       float *pacc = partial ? p.part.acc + prow * D : nullptr;
-#pragma unroll
-      for (int c = 0; c < HC; ++c) {
-        const int col = wg * (D / 2) + c * 32;
-        // both accumulators are read; a stale one is discarded by the select
-        // below (never multiplied: its bits may not be a finite number)
+#pragma unroll 1
+      for (int col = 0; col < D; col += 32) {
         uint32_t o0[32], o1[32];
         tmem_ld32(tmem + lane_off + COL_O + col, o0);
         tmem_ld32(tmem + lane_off + COL_O + D + col, o1);
         tmem_wait_ld(o0);
         tmem_wait_ld(o1);
         if (row < it.n_rows) {
-          float f[32];
 #pragma unroll
           for (int e = 0; e < 32; ++e)
-            f[e] = (has0 ? __uint_as_float(o0[e]) * f0 : 0.f) +
-                   (has1 ? __uint_as_float(o1[e]) * f1 : 0.f);
+            o0[e] = __float_as_uint((has0 ? __uint_as_float(o0[e]) * fw.x : 0.f) +
+                                    (has1 ? __uint_as_float(o1[e]) * fw.y : 0.f));
           if (partial) {
 #pragma unroll
             for (int e = 0; e < 32; e += 4)
-              *reinterpret_cast<float4 *>(pacc + col + e) =
-                  make_float4(f[e], f[e + 1], f[e + 2], f[e + 3]);
+              *reinterpret_cast<uint4 *>(pacc + col + e) =
+                  make_uint4(o0[e], o0[e + 1], o0[e + 2], o0[e + 3]);
           } else if (OUT_F32) {
             float *dst = static_cast<float *>(p.out) + orow + col;
 #pragma unroll
             for (int e = 0; e < 32; e += 4)
-              *reinterpret_cast<float4 *>(dst + e) = make_float4(f[e], f[e + 1], f[e + 2], f[e + 3]);
+              *reinterpret_cast<uint4 *>(dst + e) = make_uint4(o0[e], o0[e + 1], o0[e + 2], o0[e + 3]);
           } else {
             __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.out) + orow + col;
 #pragma unroll
@@ -640,7 +655,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               uint32_t w[4];
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
-                __nv_bfloat162 hh = __floats2bfloat162_rn(f[e + 2 * q], f[e + 2 * q + 1]);
+                __nv_bfloat162 hh = __floats2bfloat162_rn(__uint_as_float(o0[e + 2 * q]),
+                                                          __uint_as_float(o0[e + 2 * q + 1]));
                 w[q] = *reinterpret_cast<uint32_t *>(&hh);
               }
               *reinterpret_cast<uint4 *>(dst + e) = make_uint4(w[0], w[1], w[2], w[3]);
