@@ -205,6 +205,47 @@ dbsa_status dbsa_gather_rope_attend(
     int64_t dbg_cap, void *workspace, size_t ws_bytes, void *stream);
 
 /* ---------------------------------------------------------------------------
+ * Stage 2 with prepared block keys ([DBSA notes] §Stage 2, item 3: RoPE is
+ * re-applied to the cached keys at the gathered positions).
+ *
+ * Gathered token p of query q sits at P + r, where P is the fresh start of
+ * its block in that query and r its offset inside the block; since
+ * R(a)^T R(b) = R(b - a), the score of (query row, key) factors into the key
+ * rotated at r and the query row rotated at (its position - P).  The rotated
+ * keys R(r) k depend on the cache only, so one dbsa_block_keys() call serves
+ * every query batch and decode step until the cache changes (an encode or an
+ * append), and dbsa_gather_rope_attend_prepared() skips that rotation.
+ *
+ *   block_keys device, bk_bytes >= dbsa_block_keys_size(cfg, offs, nb),
+ *              256-byte aligned, owned by the caller: the keys of every cache
+ *              row s of block b rotated at s - offs[b] (bf16, [Hkv][T][D]),
+ *              a bf16 copy of V for DBSA_F32 caches, and the tables used.
+ *
+ * dbsa_gather_rope_attend_prepared takes the arguments of
+ * dbsa_gather_rope_attend plus block_keys, which must come from
+ * dbsa_block_keys() on the same cfg, cache contents, cap and offsets (not
+ * checked).  Results are bit-identical to dbsa_gather_rope_attend.  Its
+ * workspace may be the size dbsa_gather_workspace_size() returns (an upper
+ * bound: the rotated keys are not placed in it).
+ * Errors: as dbsa_gather_rope_attend; WORKSPACE also for a missing,
+ * misaligned or too small block_keys buffer.
+ * ------------------------------------------------------------------------ */
+size_t dbsa_block_keys_size(const dbsa_config *cfg, const int32_t *offs_host,
+                            int32_t nb);
+dbsa_status dbsa_block_keys(const dbsa_config *cfg, const void *k_cache,
+                            const void *v_cache, int64_t cap,
+                            const int32_t *offs_host, int32_t nb,
+                            void *block_keys, size_t bk_bytes, void *stream);
+dbsa_status dbsa_gather_rope_attend_prepared(
+    const dbsa_config *cfg, const void *k_cache, const void *v_cache,
+    int64_t cap, const int32_t *offs_host, int32_t nb, int32_t nq,
+    const int32_t *sel_ptr_host, const int32_t *sel_blocks_host,
+    const void *q_new, int32_t n_new, const void *k_tail, const void *v_tail,
+    int32_t tail_len, int32_t tail_cap, void *out, int32_t *dbg_map,
+    int64_t dbg_cap, const void *block_keys, size_t bk_bytes, void *workspace,
+    size_t ws_bytes, void *stream);
+
+/* ---------------------------------------------------------------------------
  * Stage 2 without a workspace.  The paper has no counterpart: this is a
  * calling convention of this library, not a step of the method.
  *

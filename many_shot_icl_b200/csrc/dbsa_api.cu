@@ -370,7 +370,10 @@ struct S2Layout {
       tc_tiles, offs, blob_end, k_hat, v_hat, q_hat, part_acc, part_ml, total;
   int32_t n_hi;
 };
-S2Layout s2_layout(const dbsa_config *cfg, const GatherPlan &gp, int32_t n_new) {
+// prepared: the block-relative keys (and bf16 V of fp32 caches) come from a
+// dbsa_block_keys() buffer instead of the workspace.
+S2Layout s2_layout(const dbsa_config *cfg, const GatherPlan &gp, int32_t n_new,
+                   bool prepared = false) {
   S2Layout l;
   Carve cv;
   l.n_hi = (int32_t)(std::max<int64_t>(gp.max_pos - 1, 0) / kRopeLo + 1);
@@ -385,12 +388,35 @@ S2Layout s2_layout(const dbsa_config *cfg, const GatherPlan &gp, int32_t n_new) 
   l.offs = cv.take((size_t)(offs_count(gp)) * sizeof(int32_t));
   l.blob_end = cv.take(0);
   const int64_t T = gp.cache_rows;
-  l.k_hat = cv.take((size_t)cfg->n_kv_heads * T * cfg->head_dim * 2);
-  l.v_hat = cv.take(cfg->dtype == DBSA_F32 ? (size_t)cfg->n_kv_heads * T * cfg->head_dim * 2 : 0);
+  l.k_hat = cv.take(prepared ? 0 : (size_t)cfg->n_kv_heads * T * cfg->head_dim * 2);
+  l.v_hat = cv.take(!prepared && cfg->dtype == DBSA_F32
+                        ? (size_t)cfg->n_kv_heads * T * cfg->head_dim * 2
+                        : 0);
   l.q_hat = cv.take((size_t)cfg->n_kv_heads * gp.tc_rows * cfg->head_dim * 2);
   const size_t rows = gp.items.size() * (size_t)cfg->n_q_heads * n_new;
   l.part_acc = cv.take(rows * cfg->head_dim * sizeof(float));
   l.part_ml = cv.take(rows * sizeof(float2));
+  l.total = cv.total();
+  return l;
+}
+
+// dbsa_block_keys() buffer: status word, RoPE tables for positions inside a
+// block, the offset table, K-hat [Hkv][T][D] bf16 and (fp32 caches) bf16 V.
+struct BKLayout {
+  size_t rope, offs, k_hat, v_hat, total;
+  int32_t n_hi;
+};
+BKLayout bk_layout(const dbsa_config *cfg, const int32_t *offs, int32_t nb) {
+  BKLayout l;
+  Carve cv;
+  int32_t max_len = 1;
+  for (int32_t b = 0; b < nb; ++b) max_len = std::max(max_len, offs[b + 1] - offs[b]);
+  l.n_hi = (max_len - 1) / kRopeLo + 1;
+  const int64_t T = offs[nb];
+  l.rope = cv.take(rope_table_bytes(l.n_hi, cfg->head_dim));
+  l.offs = cv.take((size_t)(nb + 1) * sizeof(int32_t));
+  l.k_hat = cv.take((size_t)cfg->n_kv_heads * T * cfg->head_dim * 2);
+  l.v_hat = cv.take(cfg->dtype == DBSA_F32 ? (size_t)cfg->n_kv_heads * T * cfg->head_dim * 2 : 0);
   l.total = cv.total();
   return l;
 }
@@ -692,14 +718,20 @@ size_t dbsa_gather_workspace_size(const dbsa_config *cfg, const int32_t *offs_ho
   return s2_layout(cfg, gp, n_new).total;
 }
 
-dbsa_status dbsa_gather_rope_attend(const dbsa_config *cfg, const void *k_cache,
-                                    const void *v_cache, int64_t cap, const int32_t *offs_host,
-                                    int32_t nb, int32_t nq, const int32_t *sel_ptr_host,
-                                    const int32_t *sel_blocks_host, const void *q_new,
-                                    int32_t n_new, const void *k_tail, const void *v_tail,
-                                    int32_t tail_len, int32_t tail_cap, void *out,
-                                    int32_t *dbg_map, int64_t dbg_cap, void *workspace,
-                                    size_t ws_bytes, void *stream) {
+}  // extern "C"
+
+namespace {
+
+// Stage 2 behind both entry points; block_keys = null rotates the cache keys
+// at block-relative positions into the workspace, else takes them from a
+// dbsa_block_keys() buffer.
+dbsa_status gather_impl(const dbsa_config *cfg, const void *k_cache, const void *v_cache,
+                        int64_t cap, const int32_t *offs_host, int32_t nb, int32_t nq,
+                        const int32_t *sel_ptr_host, const int32_t *sel_blocks_host,
+                        const void *q_new, int32_t n_new, const void *k_tail, const void *v_tail,
+                        int32_t tail_len, int32_t tail_cap, void *out, int32_t *dbg_map,
+                        int64_t dbg_cap, const void *block_keys, size_t bk_bytes, void *workspace,
+                        size_t ws_bytes, void *stream) {
   dbsa_status s = check_cfg(cfg);
   if (s != DBSA_OK) return s;
   if ((s = check_offs(offs_host, nb)) != DBSA_OK) return s;
@@ -725,8 +757,17 @@ dbsa_status dbsa_gather_rope_attend(const dbsa_config *cfg, const void *k_cache,
         return fail(DBSA_ERR_INVALID_ARG, "dbg_cap %lld < gathered tokens %d", (long long)dbg_cap,
                     qi.n_gathered);
   }
-  const S2Layout L = s2_layout(cfg, gp, n_new);
+  const bool prepared = block_keys != nullptr;
+  const S2Layout L = s2_layout(cfg, gp, n_new, prepared);
   if ((s = check_ws(workspace, ws_bytes, L.total)) != DBSA_OK) return s;
+  BKLayout B{};
+  if (prepared) {
+    B = bk_layout(cfg, offs_host, nb);
+    if ((reinterpret_cast<uintptr_t>(block_keys) & 255u) != 0)
+      return fail(DBSA_ERR_WORKSPACE, "block_keys must be 256-byte aligned");
+    if (bk_bytes < B.total)
+      return fail(DBSA_ERR_WORKSPACE, "block_keys too small: %zu < %zu bytes", bk_bytes, B.total);
+  }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   if ((e = cudaMemsetAsync(workspace, 0, kStatusBytes, st)) != cudaSuccess)
@@ -794,11 +835,15 @@ dbsa_status dbsa_gather_rope_attend(const dbsa_config *cfg, const void *k_cache,
     ra.T = (int32_t)gp.cache_rows;
     ra.nb = nb;
     ra.offs = at<int32_t>(workspace, L.offs);
-    ra.k_hat = at<void>(workspace, L.k_hat);
-    ra.v_bf16 = f32 ? at<void>(workspace, L.v_hat) : nullptr;
+    void *bk = const_cast<void *>(block_keys);
+    ra.k_hat = prepared ? at<void>(bk, B.k_hat) : at<void>(workspace, L.k_hat);
+    ra.v_bf16 = !f32 ? nullptr : prepared ? at<void>(bk, B.v_hat) : at<void>(workspace, L.v_hat);
     ra.rope = rope;
-    if ((e = launch_rel_rope(ra, cfg->head_dim, f32, st)) != cudaSuccess)
-      return cuda_fail(e, "block-relative rotation");
+    if (!prepared) {
+      if ((e = launch_rel_rope(ra, cfg->head_dim, f32, st)) != cudaSuccess)
+        return cuda_fail(e, "block-relative rotation");
+      count_launches(1);
+    }
     QHatArgs qa{};
     qa.q_new = q_new;
     qa.n_new = n_new;
@@ -814,7 +859,7 @@ dbsa_status dbsa_gather_rope_attend(const dbsa_config *cfg, const void *k_cache,
     qa.rope = rope;
     if ((e = launch_qhat(qa, cfg->head_dim, f32, st)) != cudaSuccess)
       return cuda_fail(e, "query rotation");
-    count_launches(2);
+    count_launches(1);
     if (dbg_map != nullptr) {
       int32_t mx = 0;
       for (const auto &qi : gp.queries) mx = std::max(mx, qi.n_gathered);
@@ -859,6 +904,82 @@ dbsa_status dbsa_gather_rope_attend(const dbsa_config *cfg, const void *k_cache,
     return cuda_fail(e, "stage-2 merge");
   count_launches(1);
   return DBSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+dbsa_status dbsa_gather_rope_attend(const dbsa_config *cfg, const void *k_cache,
+                                    const void *v_cache, int64_t cap, const int32_t *offs_host,
+                                    int32_t nb, int32_t nq, const int32_t *sel_ptr_host,
+                                    const int32_t *sel_blocks_host, const void *q_new,
+                                    int32_t n_new, const void *k_tail, const void *v_tail,
+                                    int32_t tail_len, int32_t tail_cap, void *out,
+                                    int32_t *dbg_map, int64_t dbg_cap, void *workspace,
+                                    size_t ws_bytes, void *stream) {
+  return gather_impl(cfg, k_cache, v_cache, cap, offs_host, nb, nq, sel_ptr_host,
+                     sel_blocks_host, q_new, n_new, k_tail, v_tail, tail_len, tail_cap, out,
+                     dbg_map, dbg_cap, nullptr, 0, workspace, ws_bytes, stream);
+}
+
+size_t dbsa_block_keys_size(const dbsa_config *cfg, const int32_t *offs_host, int32_t nb) {
+  if (check_cfg(cfg) != DBSA_OK || check_offs(offs_host, nb) != DBSA_OK) return 0;
+  return bk_layout(cfg, offs_host, nb).total;
+}
+
+dbsa_status dbsa_block_keys(const dbsa_config *cfg, const void *k_cache, const void *v_cache,
+                            int64_t cap, const int32_t *offs_host, int32_t nb, void *block_keys,
+                            size_t bk_bytes, void *stream) {
+  dbsa_status s = check_cfg(cfg);
+  if (s != DBSA_OK) return s;
+  if ((s = check_offs(offs_host, nb)) != DBSA_OK) return s;
+  if (!k_cache || !v_cache) return fail(DBSA_ERR_INVALID_ARG, "a tensor pointer is NULL");
+  if (!aligned16(k_cache) || !aligned16(v_cache))
+    return fail(DBSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  if (offs_host[nb] > cap)
+    return fail(DBSA_ERR_CAPACITY, "offsets reach %d rows but cap is %lld", offs_host[nb],
+                (long long)cap);
+  const BKLayout B = bk_layout(cfg, offs_host, nb);
+  if ((s = check_ws(block_keys, bk_bytes, B.total)) != DBSA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  RopeTables rope;
+  if ((e = build_tables(block_keys, B.rope, B.n_hi, cfg, st, &rope)) != cudaSuccess)
+    return cuda_fail(e, "rope tables");
+  count_launches(1);
+  if ((e = cudaMemcpyAsync(at<void>(block_keys, B.offs), offs_host,
+                           (size_t)(nb + 1) * sizeof(int32_t), cudaMemcpyHostToDevice, st)) !=
+      cudaSuccess)
+    return cuda_fail(e, "offset upload");
+  RelRopeArgs ra{};
+  ra.k_cache = k_cache;
+  ra.v_cache = v_cache;
+  ra.cap = cap;
+  ra.Hkv = cfg->n_kv_heads;
+  ra.T = offs_host[nb];
+  ra.nb = nb;
+  ra.offs = at<int32_t>(block_keys, B.offs);
+  ra.k_hat = at<void>(block_keys, B.k_hat);
+  ra.v_bf16 = cfg->dtype == DBSA_F32 ? at<void>(block_keys, B.v_hat) : nullptr;
+  ra.rope = rope;
+  if ((e = launch_rel_rope(ra, cfg->head_dim, cfg->dtype == DBSA_F32, st)) != cudaSuccess)
+    return cuda_fail(e, "block-relative rotation");
+  count_launches(1);
+  return DBSA_OK;
+}
+
+dbsa_status dbsa_gather_rope_attend_prepared(
+    const dbsa_config *cfg, const void *k_cache, const void *v_cache, int64_t cap,
+    const int32_t *offs_host, int32_t nb, int32_t nq, const int32_t *sel_ptr_host,
+    const int32_t *sel_blocks_host, const void *q_new, int32_t n_new, const void *k_tail,
+    const void *v_tail, int32_t tail_len, int32_t tail_cap, void *out, int32_t *dbg_map,
+    int64_t dbg_cap, const void *block_keys, size_t bk_bytes, void *workspace, size_t ws_bytes,
+    void *stream) {
+  if (block_keys == nullptr) return fail(DBSA_ERR_INVALID_ARG, "block_keys is NULL");
+  return gather_impl(cfg, k_cache, v_cache, cap, offs_host, nb, nq, sel_ptr_host,
+                     sel_blocks_host, q_new, n_new, k_tail, v_tail, tail_len, tail_cap, out,
+                     dbg_map, dbg_cap, block_keys, bk_bytes, workspace, ws_bytes, stream);
 }
 
 dbsa_status dbsa_read_status(const void *workspace, void *stream) {

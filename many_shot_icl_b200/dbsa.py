@@ -26,7 +26,8 @@ SYMBOLS = (
     "dbsa_append_workspace_size", "dbsa_append_block", "dbsa_gather_workspace_size",
     "dbsa_gather_rope_attend", "dbsa_last_error", "dbsa_read_status", "dbsa_stage1_plan",
     "dbsa_stage1_tile_count", "dbsa_version", "dbsa_kernel_launches", "dbsa_set_profile_events",
-    "dbsa_gather_rope_attend_noalloc",
+    "dbsa_gather_rope_attend_noalloc", "dbsa_block_keys_size", "dbsa_block_keys",
+    "dbsa_gather_rope_attend_prepared",
 )
 
 
@@ -100,6 +101,14 @@ def load(path: str = LIB_PATH):
     lib.dbsa_gather_rope_attend_noalloc.argtypes = [cfgp, vp, vp, i64, vp, i32, i32, vp, vp, vp,
                                                     i32, vp, vp, i32, i32, vp, vp, i64, vp]
     lib.dbsa_gather_rope_attend_noalloc.restype = ctypes.c_int
+    lib.dbsa_block_keys_size.argtypes = [cfgp, vp, i32]
+    lib.dbsa_block_keys_size.restype = sz
+    lib.dbsa_block_keys.argtypes = [cfgp, vp, vp, i64, vp, i32, vp, sz, vp]
+    lib.dbsa_block_keys.restype = ctypes.c_int
+    lib.dbsa_gather_rope_attend_prepared.argtypes = [cfgp, vp, vp, i64, vp, i32, i32, vp, vp, vp,
+                                                     i32, vp, vp, i32, i32, vp, vp, i64, vp, sz,
+                                                     vp, sz, vp]
+    lib.dbsa_gather_rope_attend_prepared.restype = ctypes.c_int
     lib.dbsa_last_error.argtypes = []
     lib.dbsa_last_error.restype = ctypes.c_char_p
     lib.dbsa_read_status.argtypes = [vp, vp]
@@ -216,16 +225,38 @@ def append_block(cfg: DbsaConfig, q, k, v, offs, k_cache, v_cache, out, workspac
 
 
 def gather_rope_attend(cfg: DbsaConfig, k_cache, v_cache, offs, sel_ptr, sel_blocks, q_new,
-                       k_tail, v_tail, tail_len: int, out, workspace, dbg_map=None, stream=None):
-    """Stage 2 for a batch of queries (see dbsa_gather_rope_attend)."""
+                       k_tail, v_tail, tail_len: int, out, workspace, dbg_map=None, stream=None,
+                       block_keys=None):
+    """Stage 2 for a batch of queries (see dbsa_gather_rope_attend); with
+    block_keys (from block_keys()), dbsa_gather_rope_attend_prepared."""
     o, sp, sb = _i32(offs), _i32(sel_ptr), _i32(sel_blocks)
     c = cfg.c()
-    _check(load().dbsa_gather_rope_attend(
+    args = [ctypes.byref(c), _dp(k_cache), _dp(v_cache), k_cache.shape[1], _hp(o), len(o) - 1,
+            len(sp) - 1, _hp(sp), _hp(sb), _dp(q_new), q_new.shape[1], _dp(k_tail), _dp(v_tail),
+            tail_len, k_tail.shape[1], _dp(out), _dp(dbg_map),
+            0 if dbg_map is None else dbg_map.shape[1]]
+    ws = [_dp(workspace), workspace.numel() * workspace.element_size(), _stream(stream)]
+    if block_keys is None:
+        _check(load().dbsa_gather_rope_attend(*args, *ws))
+    else:
+        _check(load().dbsa_gather_rope_attend_prepared(
+            *args, _dp(block_keys), block_keys.numel() * block_keys.element_size(), *ws))
+
+
+def block_keys_size(cfg: DbsaConfig, offs) -> int:
+    o = _i32(offs)
+    c = cfg.c()
+    return int(load().dbsa_block_keys_size(ctypes.byref(c), _hp(o), len(o) - 1))
+
+
+def block_keys(cfg: DbsaConfig, k_cache, v_cache, offs, buf, stream=None):
+    """Keys of every cache row rotated at their position inside their block,
+    into buf (uint8 device tensor of block_keys_size() bytes)."""
+    o = _i32(offs)
+    c = cfg.c()
+    _check(load().dbsa_block_keys(
         ctypes.byref(c), _dp(k_cache), _dp(v_cache), k_cache.shape[1], _hp(o), len(o) - 1,
-        len(sp) - 1, _hp(sp), _hp(sb), _dp(q_new), q_new.shape[1], _dp(k_tail), _dp(v_tail),
-        tail_len, k_tail.shape[1], _dp(out), _dp(dbg_map),
-        0 if dbg_map is None else dbg_map.shape[1], _dp(workspace),
-        workspace.numel() * workspace.element_size(), _stream(stream)))
+        _dp(buf), buf.numel() * buf.element_size(), _stream(stream)))
 
 
 def kernel_launches() -> int:

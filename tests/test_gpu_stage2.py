@@ -119,3 +119,43 @@ def test_deterministic():
     o1 = r.out.clone()
     r.run()
     assert torch.equal(o1, r.out)
+
+
+def _run_both(cfg, offs, sels, n_new, tail_len, seed):
+    """dbsa_gather_rope_attend and the prepared-keys path on the same inputs."""
+    plain = Stage2Run(cfg, offs, sels, n_new, tail_len, seed=seed).run()
+    bk = torch.empty(dbsa.block_keys_size(cfg, plain.offs), dtype=torch.uint8, device="cuda")
+    dbsa.block_keys(cfg, plain.kc, plain.vc, plain.offs, bk)
+    out = torch.full_like(plain.out, float("nan"))
+    dbg = torch.full_like(plain.dbg, -1)
+    dbsa.gather_rope_attend(cfg, plain.kc, plain.vc, plain.offs, plain.sel_ptr, plain.sel,
+                            plain.q_new, plain.kt, plain.vt, tail_len, out, plain.ws,
+                            dbg_map=dbg, block_keys=bk)
+    assert dbsa.read_status(plain.ws) == dbsa.OK
+    return plain, out, dbg, bk
+
+
+@pytest.mark.parametrize("dtype,Hq,Hkv,D,n_new,tail_len", [("bf16", 8, 2, 128, 40, 40),
+                                                          ("bf16", 8, 2, 128, 1, 41),
+                                                          ("f32", 2, 1, 64, 16, 16)])
+def test_prepared_block_keys_bit_identical(dtype, Hq, Hkv, D, n_new, tail_len):
+    """One dbsa_block_keys() call, then the prepared path gives the plain path's
+    bits (same kernels, same rotated keys) for prompt and decode passes, and
+    the prepared buffer serves a second pass with other queries."""
+    cfg = dbsa.DbsaConfig(Hq, Hkv, D, dtype, 5e5, 2)
+    offs = offsets(np.random.default_rng(7).integers(20, 150, size=9))
+    rng = np.random.default_rng(8)
+    sels = [np.concatenate([[0], rng.permutation(np.arange(1, 9))[:k]]) for k in (3, 5, 1, 8)]
+    plain, out, dbg, bk = _run_both(cfg, offs, sels, n_new, tail_len, seed=3)
+    assert torch.equal(out, plain.out)
+    assert torch.equal(dbg, plain.dbg)
+    plain.check("prepared", queries=[0, 3])
+    # the same block keys, another batch over the same cache
+    other = [np.array([0, 8, 2]), np.array([0, 1])]
+    run2 = Stage2Run(cfg, offs, other, n_new, tail_len, seed=3)
+    run2.kc, run2.vc = plain.kc, plain.vc
+    run2.run()
+    out2 = torch.full_like(run2.out, float("nan"))
+    dbsa.gather_rope_attend(cfg, run2.kc, run2.vc, run2.offs, run2.sel_ptr, run2.sel, run2.q_new,
+                            run2.kt, run2.vt, tail_len, out2, run2.ws, block_keys=bk)
+    assert torch.equal(out2, run2.out)

@@ -156,6 +156,29 @@ def test_invalid_arguments_are_rejected_before_device_work(lib):
     assert encode(dbsa.DbsaConfig(4, 2, 128, window_j=-1)) == dbsa.ERR_INVALID_ARG
     assert encode(dbsa.DbsaConfig(4, 2, 128, pattern=7)) == dbsa.ERR_INVALID_ARG
 
+    def prepared(bk, bk_bytes, cfg=ok_cfg):
+        c, cp = _cfgp(cfg)
+        sp, sb = np.array([0, 1], np.int32), np.array([0], np.int32)
+        return lib.dbsa_gather_rope_attend_prepared(
+            cp, fake, fake, 64, offs.ctypes.data_as(ctypes.c_void_p), len(offs) - 1, 1,
+            sp.ctypes.data_as(ctypes.c_void_p), sb.ctypes.data_as(ctypes.c_void_p), fake, 1,
+            fake, fake, 1, 4, fake, None, 0, bk, bk_bytes, ws, 1 << 30, None)
+
+    need = dbsa.block_keys_size(ok_cfg, offs)
+    assert prepared(None, need) == dbsa.ERR_INVALID_ARG                  # no block keys
+    assert prepared(ctypes.c_void_p(4096 + 16), need) == dbsa.ERR_WORKSPACE   # misaligned
+    assert prepared(ctypes.c_void_p(4096), need - 1) == dbsa.ERR_WORKSPACE    # too small
+    assert "block_keys" in dbsa.last_error()
+
+    def block_keys(cap=64, bk=ctypes.c_void_p(1 << 20), bk_bytes=1 << 30, k=fake):
+        c, cp = _cfgp(ok_cfg)
+        return lib.dbsa_block_keys(cp, k, fake, cap, offs.ctypes.data_as(ctypes.c_void_p),
+                                   len(offs) - 1, bk, bk_bytes, None)
+
+    assert block_keys(cap=19) == dbsa.ERR_CAPACITY
+    assert block_keys(k=None) == dbsa.ERR_INVALID_ARG
+    assert block_keys(bk_bytes=need - 1) == dbsa.ERR_WORKSPACE
+
     c, cp = _cfgp(ok_cfg)
     assert lib.dbsa_append_block(cp, fake, fake, fake, 0, offs.ctypes.data_as(ctypes.c_void_p),
                                  3, fake, fake, 64, fake, ws, 1 << 30, None) == dbsa.ERR_INVALID_ARG
@@ -176,3 +199,7 @@ def test_workspace_sizes(lib):
     wg = dbsa.gather_workspace_size(cfg, offs, sel_ptr, sel, 40, 40)
     assert wg > 0
     assert dbsa.gather_workspace_size(cfg, offs, sel_ptr, np.array([2, 3, 9, 0, 1]), 40, 40) == 0
+    # prepared block keys: K at block-relative positions, bf16 [Hkv][T][D], plus small tables
+    bk = dbsa.block_keys_size(cfg, offs)
+    assert 8 * T * 256 <= bk < 8 * T * 256 + (1 << 20)
+    assert dbsa.block_keys_size(dbsa.DbsaConfig(2, 1, 64, "f32"), offs) >= 2 * T * 128
