@@ -360,6 +360,97 @@ def append_series(wl: Workload, n_appends: int):
     return ms, flops
 
 
+# ------------------------------------------------------------------ comparators
+def comparators(wl: Workload, n_ret_queries: int = 4):
+    """Attention-level counterparts of the pages' baselines, on layer 0 of the
+    workload, scaled to all layers (every layer is identical work):
+      fixed ICL: setup = full causal prefill of the whole context; inference =
+        every query attends to every block (prompt pass + decode steps);
+      retrieval ICL: per query, a fresh causal prefill of its retrieved blocks
+        followed by its prompt tokens, then the decode steps over that private
+        cache (timed on n_ret_queries queries, scaled to the batch).
+    Device time with CUDA events; DBSA's own numbers come from the bench step."""
+    import dataclasses
+    import torch
+    from many_shot_icl_b200 import dbsa
+    w, L = wl.w, wl.layers
+    Hq, Hkv, D = w.n_q_heads, w.n_kv_heads, w.head_dim
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def timed(fn, reps=2):
+        fn()
+        torch.cuda.synchronize()
+        e0, e1 = ev(), ev()
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / 1e3 / reps
+
+    # fixed ICL setup: full causal attention over the context
+    full = dataclasses.replace(wl.cfg, pattern=dbsa.PATTERN_FULL)
+    fixed_setup = timed(lambda: dbsa.encode_blocks(full, wl.q[0], wl.k[0], wl.v[0], wl.offs, wl.kc[0],
+                                                   wl.vc[0], wl.out[0], wl.ws)) * L
+    # restore layer 0's DBSA cache contents (the same K/V, bit-identical rows)
+    dbsa.encode_blocks(wl.cfg, wl.q[0], wl.k[0], wl.v[0], wl.offs, wl.kc[0], wl.vc[0], wl.out[0],
+                       wl.ws)
+    # fixed ICL inference: every query selects every block
+    all_sel = [np.arange(wl.nb, dtype=np.int32) for _ in range(wl.nq)]
+    sp, sb = dbsa.selection_csr(all_sel)
+    wsz = max(dbsa.gather_workspace_size(wl.cfg, wl.offs, sp, sb, n, t) for n, t in wl.passes())
+    ws_all = torch.empty(wsz, dtype=torch.uint8, device="cuda")
+    out_p = torch.empty_like(wl.out_p)
+    out_d = torch.empty_like(wl.out_d)
+
+    def fixed_inference():
+        dbsa.block_keys(wl.cfg, wl.kc[0], wl.vc[0], wl.offs, wl.bk[0])
+        for n_new, tail_len in wl.passes():
+            qn, out = (wl.qp[0], out_p) if n_new > 1 else (wl.qd[0], out_d)
+            dbsa.gather_rope_attend(wl.cfg, wl.kc[0], wl.vc[0], wl.offs, sp, sb, qn, wl.kt[0],
+                                    wl.vt[0], tail_len, out, ws_all, block_keys=wl.bk[0])
+    fixed_inf = timed(fixed_inference, reps=1) * L / wl.nq
+    del ws_all
+    # retrieval ICL: per query, causal prefill of [retrieved blocks ; prompt], then decode
+    t_ret, nqs = 0.0, min(n_ret_queries, wl.nq)
+    for qi in range(nqs):
+        lens = [int(wl.offs[b + 1] - wl.offs[b]) for b in wl.sels[qi]] + [w.query_tokens]
+        offs_q = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+        Tq = int(offs_q[-1])
+        cap = Tq + w.decode_steps
+        seed = 90000 + qi
+        q = inputs.randn((Tq, Hq, D), seed, w.dtype, "cuda")
+        k = inputs.randn((Tq, Hkv, D), seed + 1, w.dtype, "cuda")
+        v = inputs.randn((Tq, Hkv, D), seed + 2, w.dtype, "cuda")
+        kc = torch.empty((Hkv, cap, D), dtype=wl.dt, device="cuda")
+        vc = torch.empty_like(kc)
+        out = torch.empty((Tq, Hq, D), dtype=wl.dt, device="cuda")
+        ws1 = torch.empty(dbsa.encode_workspace_size(full, Tq, len(lens)), dtype=torch.uint8,
+                          device="cuda")
+        sel1 = [np.arange(len(lens), dtype=np.int32)]
+        sp1, sb1 = dbsa.selection_csr(sel1)
+        kt = inputs.randn((1, w.decode_steps, Hkv, D), seed + 3, w.dtype, "cuda")
+        vt = inputs.randn((1, w.decode_steps, Hkv, D), seed + 4, w.dtype, "cuda")
+        qd = inputs.randn((1, 1, Hq, D), seed + 5, w.dtype, "cuda")
+        od = torch.empty((1, 1, Hq, D), dtype=wl.dt, device="cuda")
+        ws2 = torch.empty(max([1] + [dbsa.gather_workspace_size(wl.cfg, offs_q, sp1, sb1, 1, i)
+                                     for i in range(1, w.decode_steps + 1)]),
+                          dtype=torch.uint8, device="cuda")
+
+        def ret_query():
+            dbsa.encode_blocks(full, q, k, v, offs_q, kc, vc, out, ws1)
+            for i in range(1, w.decode_steps + 1):
+                dbsa.gather_rope_attend(wl.cfg, kc, vc, offs_q, sp1, sb1, qd, kt, vt, i, od, ws2)
+        t_ret += timed(ret_query, reps=1)
+        del q, k, v, kc, vc, out, ws1, ws2
+    ret_inf = t_ret / nqs * L
+    return {"note": "attention only; layer 0 timed and scaled to %d layers; retrieval ICL on %d "
+                    "queries; the pages' ratios are whole-model latencies on L40S/A100 (context "
+                    "only)" % (L, nqs),
+            "fixed_icl": {"setup_s": fixed_setup, "inference_s_per_query": fixed_inf},
+            "retrieval_icl": {"setup_s": 0.0, "inference_s_per_query": ret_inf}}
+
+
 # ------------------------------------------------------------------ oracle timing
 def oracle_sample(w: inputs.Workload, budget_s: float, threads: int | None = None):
     """Time the oracle on a bounded sample of the workload (layer 0 inputs):
@@ -482,6 +573,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=16.0)
     ap.add_argument("--ref-budget", type=float, default=60.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-compare", action="store_true",
+                    help="skip the retrieval-ICL / fixed-ICL attention comparators")
     ap.add_argument("--profile-only", choices=["stage1", "stage2"], default=None,
                     help="run W + K steps of one stage only and exit (for ncu captures)")
     args = ap.parse_args()
@@ -651,6 +744,17 @@ def main():
                "tflops": [round(f / (m * 1e-3) / 1e12, 1) for f, m in zip(fl, ms)],
                "slope_ms_per_append": round(float(np.polyfit(np.arange(len(ms)), ms, 1)[0]), 4)}
 
+    comp = None
+    if rank == 0 and world == 1 and not args.no_compare:
+        comp = comparators(wl)
+        dbsa_inf = t_s2 / wl.nq
+        comp["dbsa"] = {"setup_s": t_s1, "inference_s_per_query": dbsa_inf}
+        comp["inference_ratio_dbsa_over_retrieval_icl"] = \
+            dbsa_inf / comp["retrieval_icl"]["inference_s_per_query"]
+        comp["inference_ratio_fixed_icl_over_retrieval_icl"] = \
+            comp["fixed_icl"]["inference_s_per_query"] / comp["retrieval_icl"]["inference_s_per_query"]
+        comp["setup_ratio_dbsa_over_fixed_icl"] = t_s1 / comp["fixed_icl"]["setup_s"]
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         c1, c2, cores, desc, _ = oracle_sample(w, args.cpu_budget)
@@ -684,6 +788,7 @@ def main():
                     "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
             "cpu_baseline": cpu,
             "append": app,
+            "comparators": comp,
             "clocks": clocks,
             "gpu_launches": int(launches / args.steps),
             "gpu_launches_timed_region": int(launches),

@@ -513,13 +513,15 @@ cudaError_t launch_main(const Stage2Args &a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-// Rows per CTA by pass shape (kept in step with the host split planner):
-// <= 16 rows (decode): 8 key groups of 1 warp; <= 32: 4 x 2; <= 64: 2 x 4;
-// <= 128: 1 x 8; larger: 1 x 10 warps (160 rows) per row group.
+// Rows per CTA by pass shape: <= 16 rows (decode): 4 key groups of 1 warp;
+// <= 32: 4 x 2; <= 64: 2 x 4; <= 128: 1 x 8; larger: 1 x 10 warps (160 rows)
+// per row group.
 template <int D, typename CT>
 cudaError_t launch_d(const Stage2Args &a, cudaStream_t st) {
   const int R = (a.Hq / a.Hkv) * a.n_new;
-  if (R <= 16) return launch_main<D, CT, 1, 8, 16>(a, st);
+  // tail items span at most tail_len + 15 keys: 4 key groups of 16 keys cover
+  // a decode step's tail (<= 48 tokens) in one round at 2 CTAs per SM
+  if (R <= 16) return launch_main<D, CT, 1, 4, 16>(a, st);
   if (R <= 32) return launch_main<D, CT, 2, 4, 32>(a, st);
   if (R <= 64) return launch_main<D, CT, 4, 2, 64>(a, st);
   if (R <= 128) return launch_main<D, CT, 8, 1, 64>(a, st);
