@@ -444,11 +444,39 @@ def comparators(wl: Workload, n_ret_queries: int = 4):
         t_ret += timed(ret_query, reps=1)
         del q, k, v, kc, vc, out, ws1, ws2
     ret_inf = t_ret / nqs * L
+    # DBSA with a demonstration-granular selection: the same cache, Stage-2
+    # offsets with one block per demonstration after the sink block, and each
+    # query selecting the sink and the same share of demonstrations
+    lens = inputs.demo_lengths(w)
+    k_demo = w.demos_per_block
+    d_offs = np.concatenate([[0], [int(np.sum(lens[:k_demo]))],
+                             int(np.sum(lens[:k_demo])) + np.cumsum(lens[k_demo:])]).astype(np.int32)
+    assert int(d_offs[-1]) == wl.T
+    n_d = len(d_offs) - 1
+    rng = np.random.default_rng(77)
+    n_pick = int(round(w.retrieval_ratio * (n_d - 1)))
+    d_sels = [np.concatenate([[0], np.sort(rng.permutation(np.arange(1, n_d))[:n_pick])]).astype(
+        np.int32) for _ in range(wl.nq)]
+    dsp, dsb = dbsa.selection_csr(d_sels)
+    dws = torch.empty(max(dbsa.gather_workspace_size(wl.cfg, d_offs, dsp, dsb, n, t)
+                          for n, t in wl.passes()), dtype=torch.uint8, device="cuda")
+
+    def demo_inference():
+        for n_new, tail_len in wl.passes():
+            qn, out = (wl.qp[0], out_p) if n_new > 1 else (wl.qd[0], out_d)
+            dbsa.gather_rope_attend(wl.cfg, wl.kc[0], wl.vc[0], d_offs, dsp, dsb, qn, wl.kt[0],
+                                    wl.vt[0], tail_len, out, dws)
+    demo_inf = timed(demo_inference, reps=1) * L / wl.nq
+    d_tokens = float(np.mean([int(np.sum(np.diff(d_offs)[s_])) for s_ in d_sels]))
     return {"note": "attention only; layer 0 timed and scaled to %d layers; retrieval ICL on %d "
                     "queries; the pages' ratios are whole-model latencies on L40S/A100 (context "
                     "only)" % (L, nqs),
             "fixed_icl": {"setup_s": fixed_setup, "inference_s_per_query": fixed_inf},
-            "retrieval_icl": {"setup_s": 0.0, "inference_s_per_query": ret_inf}}
+            "retrieval_icl": {"setup_s": 0.0, "inference_s_per_query": ret_inf},
+            "dbsa_demo_granular": {"inference_s_per_query": demo_inf,
+                                   "demonstrations_per_query": n_pick,
+                                   "mean_gathered_tokens": d_tokens,
+                                   "path": "per-query split (segments shorter than a key tile)"}}
 
 
 # ------------------------------------------------------------------ oracle timing

@@ -227,8 +227,13 @@ struct GatherPlan {
   std::vector<S2Segment> segs;
   std::vector<S2Item> items;
   int32_t max_pos;  // largest key / query position + 1
-  // the tail items (one per query), which the per-query kernel runs
+  // items the per-query kernel runs: the tail items (one per query) in the
+  // block-major mode, every split item in the per-query mode
   std::vector<int32_t> run_items;
+  // per-query mode (short selected segments, e.g. single demonstrations):
+  // each query's key sequence is split into a few items that the per-query
+  // kernel gathers segment by segment; no packed rows, no tensor-core tiles
+  bool per_query = false;
   // the query rows of all (query, block) items packed block by block, and the
   // tile list of the tensor-core kernel over them
   int32_t tc_rows = 0;
@@ -255,6 +260,7 @@ dbsa_status gather_plan(const dbsa_config *cfg, const int32_t *offs, int32_t nb,
   const int R = g * n_new;
   std::vector<char> seen(nb, 0);
   gp.max_pos = 0;
+  int64_t total_keys = 0;
   for (int q = 0; q < nq; ++q) {
     const int32_t a = sel_ptr[q], e = sel_ptr[q + 1];
     if (e <= a) return fail(DBSA_ERR_INVALID_ARG, "query %d selects no block", q);
@@ -280,11 +286,51 @@ dbsa_status gather_plan(const dbsa_config *cfg, const int32_t *offs, int32_t nb,
     for (int32_t i = a; i < e; ++i) seen[sel[i]] = 0;
     if (p + tail_len > (1 << 30)) return fail(DBSA_ERR_INVALID_ARG, "gathered context too long");
     qi.n_gathered = (int32_t)p;
+    total_keys += p + tail_len;
     gp.max_pos = std::max<int32_t>(gp.max_pos, (int32_t)(p + tail_len));
     gp.queries.push_back(qi);
   }
+  // Selections of short segments (a demonstration-granular gather: blocks of
+  // one demonstration each) go per query: the block-major path keeps one
+  // partial per (query, segment) row, which would then outweigh the K/V.
+  int64_t gathered = 0;
+  for (const auto &qi : gp.queries) gathered += qi.n_gathered;
+  if (gathered < (int64_t)kTileKeys * (int64_t)gp.segs.size()) {
+    gp.per_query = true;
+    // Split size: >= 33 keys per query row of a CTA (bounds the partial
+    // traffic to ~3 % of the K/V bytes) and enough CTAs for ~4 waves.  Rows
+    // per CTA follow the per-query kernel's shape table.
+    constexpr int kSplitKeys = 64;
+    const int rows_cta = (R <= 16) ? 16 : (R <= 32) ? 32 : (R <= 64) ? 64 : (R <= 128) ? 128 : 160;
+    const int zdim = (R + rows_cta - 1) / rows_cta;
+    const int64_t min_chunk = std::max<int64_t>(256, (int64_t)33 * std::min(R, rows_cta));
+    const int64_t want_ctas = (int64_t)4 * num_sms();
+    const int64_t par_chunk =
+        (total_keys * cfg->n_kv_heads * zdim + want_ctas - 1) / std::max<int64_t>(1, want_ctas);
+    int64_t chunk = std::max(min_chunk, par_chunk);
+    chunk = (chunk + kSplitKeys - 1) / kSplitKeys * kSplitKeys;
+    for (int q = 0; q < nq; ++q) {
+      S2Query &qi = gp.queries[q];
+      const int64_t K = (int64_t)qi.n_gathered + tail_len;
+      const int64_t n_split = std::max<int64_t>(1, (K + chunk - 1) / chunk);
+      int64_t per = (K + n_split - 1) / n_split;
+      per = (per + kSplitKeys - 1) / kSplitKeys * kSplitKeys;
+      qi.item_begin = (int32_t)gp.items.size();
+      for (int64_t s0 = 0; s0 < K; s0 += per) {
+        S2Item it;
+        it.query = q;
+        it.p_begin = (int32_t)s0;
+        it.p_end = (int32_t)std::min<int64_t>(K, s0 + per);
+        it.p_lo = it.p_begin;
+        gp.run_items.push_back((int32_t)gp.items.size());
+        gp.items.push_back(it);
+      }
+      qi.n_items = (int32_t)gp.items.size() - qi.item_begin;
+    }
+    return DBSA_OK;
+  }
   {
-    // Every pass is block-major on the tensor core.  Items per query = one
+    // Block-major on the tensor core.  Items per query = one
     // per selected block + one for its own tail tokens (per-query kernel);
     // the rows of the block items are packed block by block (queries in
     // order, token-major rows within an item) and cut into 128-row tiles
@@ -388,8 +434,9 @@ S2Layout s2_layout(const dbsa_config *cfg, const GatherPlan &gp, int32_t n_new,
   l.offs = cv.take((size_t)(offs_count(gp)) * sizeof(int32_t));
   l.blob_end = cv.take(0);
   const int64_t T = gp.cache_rows;
-  l.k_hat = cv.take(prepared ? 0 : (size_t)cfg->n_kv_heads * T * cfg->head_dim * 2);
-  l.v_hat = cv.take(!prepared && cfg->dtype == DBSA_F32
+  const bool own_keys = !prepared && !gp.per_query;
+  l.k_hat = cv.take(own_keys ? (size_t)cfg->n_kv_heads * T * cfg->head_dim * 2 : 0);
+  l.v_hat = cv.take(own_keys && cfg->dtype == DBSA_F32
                         ? (size_t)cfg->n_kv_heads * T * cfg->head_dim * 2
                         : 0);
   l.q_hat = cv.take((size_t)cfg->n_kv_heads * gp.tc_rows * cfg->head_dim * 2);
@@ -824,7 +871,22 @@ dbsa_status gather_impl(const dbsa_config *cfg, const void *k_cache, const void 
   a.scale_log2 = scale_log2(cfg);
   a.rope = rope;
   const bool f32 = cfg->dtype == DBSA_F32;
-  {
+  if (gp.per_query) {
+    // gather map, then the per-query kernel over every split item
+    if (dbg_map != nullptr) {
+      int32_t mx = 0;
+      for (const auto &qi : gp.queries) mx = std::max(mx, qi.n_gathered);
+      if ((e = launch_gather_map(a.queries, a.segs, nq, mx, dbg_map, dbg_cap, st)) != cudaSuccess)
+        return cuda_fail(e, "gather map");
+      count_launches(1);
+    }
+    {
+      ProfileScope prof(st);
+      e = launch_stage2_main(a, cfg->head_dim, f32, st);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "stage-2 per-query attention");
+    count_launches(1);
+  } else {
     // keys at block-relative positions, packed query rows, then the
     // tensor-core kernel over (kv head, block, 128-row tile) in partial mode
     RelRopeArgs ra{};

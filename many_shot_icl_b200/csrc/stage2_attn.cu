@@ -1,4 +1,4 @@
-// Stage 2, per-query part: each query's own tail tokens, then the log-sum-exp
+// Stage 2, per-query part: the per-query split kernel, then the log-sum-exp
 // merge of all split partials.
 //
 // [DBSA notes] §Stage 2, items 2-4: the selected blocks (sink first) are
@@ -6,14 +6,16 @@
 // sequential positions, and the query tokens attend to the whole gathered
 // cache and, causally, to the query's own tokens.  Query q's key sequence is
 // [gathered tokens 0..T'_q) ++ [its own tail tokens], positions
-// 0..T'_q + tail_len - 1.  The gathered blocks are handled block by block by
-// the tensor-core kernel (one partial per (query, block)); this file holds the
-// kernel for the remaining split item of each query, its tail keys
-// [T'_q, T'_q + tail_len), and the merge of every partial of a query row.
+// 0..T'_q + tail_len - 1.  Normally the gathered blocks are handled block by
+// block by the tensor-core kernel (one partial per (query, block)) and this
+// kernel runs each query's tail keys [T'_q, T'_q + tail_len); for selections
+// of short segments (a demonstration-granular gather) it runs whole split
+// items [p_begin, p_end) of a query's key sequence, fetching the gathered
+// keys segment by segment.  The merge combines every partial of a row.
 //
-// Grid of the tail kernel: (tail item, KV head, row group).  A CTA reads each
-// tail key once and scores it against all g * n_new query rows that share the
-// KV head (GQA).  Keys are fetched with 16-byte cp.async, rotated in shared
+// Grid: (item, KV head, row group).  A CTA reads each key of its item once
+// and scores it against all g * n_new query rows that share the KV head
+// (GQA).  Keys are fetched with 16-byte cp.async, rotated in shared
 // memory (fp32 math, two-level fp64-built table) at their positions, and
 // multiplied with mma.sync (bf16 in, fp32 accumulate); softmax runs online in
 // registers and one causal rule (key position <= row position) covers the
@@ -116,17 +118,19 @@ __global__ void __launch_bounds__(32 * RT * KG, 1) stage2_attn_kernel(const Stag
   const int c = blockIdx.y;
   const int g = a.Hq / a.Hkv;
   const int RQ = g * a.n_new;                      // rows of one query
-  // one tail item: keys [p_lo, p_end) of the query's sequence are its own
-  // tail tokens (p_begin is p_lo rounded down to the RoPE step; the keys
-  // below p_lo belong to the gathered blocks and are masked)
+  // keys [p_lo, p_end) of the query's sequence (p_begin is a multiple of the
+  // RoPE step; keys in [p_begin, p_lo) belong to other items and are masked)
   const int it_idx = a.run_items[blockIdx.x];
   const S2Item item = a.items[it_idx];
   const int q = item.query;
-  const int Tq = a.queries[q].n_gathered;
+  const S2Query qi = a.queries[q];
+  const int Tq = qi.n_gathered;
   const int k_begin = item.p_begin, k_end = item.p_end, k_lo = item.p_lo;
   const int R = RQ;
   const int pos_first = Tq + a.tail_len - a.n_new;  // position of query token 0 (per query)
   const int row_base = blockIdx.z * MROWS;
+  const CT *kc = static_cast<const CT *>(a.k_cache);
+  const CT *vc = static_cast<const CT *>(a.v_cache);
   const CT *kt = static_cast<const CT *>(a.k_tail);
   const CT *vt = static_cast<const CT *>(a.v_tail);
 
@@ -164,14 +168,15 @@ __global__ void __launch_bounds__(32 * RT * KG, 1) stage2_attn_kernel(const Stag
     store8_bf16(reinterpret_cast<bf16 *>(sQ + soff<D>(rr, cp + H / 8)), hi);
   }
 
-  // ---- loads: warp wr of a key group loads (and later rotates) rows
+  // ---- gather: warp wr of a key group loads (and later rotates) rows
   // [wr * RPW, (wr + 1) * RPW) of each sub-tile.  Lane l (l < RPW) resolves
-  // the tail row of row l for K, lane 16 + l the same row for V; then every
-  // copy instruction moves one whole K row (lanes 0-15) and one whole V row
-  // (lanes 16-31).
+  // the cache or tail row of row l for K, lane 16 + l the same row for V;
+  // then every copy instruction moves one whole K row (lanes 0-15) and one
+  // whole V row (lanes 16-31).
   constexpr int RPW = KT / RT;
   static_assert(RPW <= 16 && CH <= 16, "one row per half-warp");
   const int n_sub = (k_end - k_begin + KT - 1) / KT;
+  int seg = 0;  // segment cursor: this lane's positions only grow
   const int n_local = kg < n_sub ? (n_sub - kg + KG - 1) / KG : 0;
   const int half_id = lane >> 4, hl = lane & 15;  // half-warp: 0 = K, 1 = V
   auto stage_ptr = [&](int jl, int kv) -> uint8_t * {
@@ -183,9 +188,16 @@ __global__ void __launch_bounds__(32 * RT * KG, 1) stage2_attn_kernel(const Stag
     const CT *my = nullptr;
     if (hl < RPW) {
       const int p = p0 + hl;
-      if (p < k_end && p >= k_lo) {   // k_lo = T'_q: p is tail token p - T'_q
-        const int64_t w = p - Tq;
-        my = (half_id ? vt : kt) + (((int64_t)q * a.tail_cap + w) * a.Hkv + c) * D;
+      if (p < k_end && p >= k_lo) {
+        if (p < Tq) {   // gathered token p: walk to the segment that holds it
+          while (seg + 1 < qi.n_seg && __ldg(&a.segs[qi.seg_begin + seg + 1].pos0) <= p) ++seg;
+          const int64_t crow = (int64_t)__ldg(&a.segs[qi.seg_begin + seg].cache_row0) +
+                               (p - __ldg(&a.segs[qi.seg_begin + seg].pos0));
+          my = (half_id ? vc : kc) + ((int64_t)c * a.cap + crow) * D;
+        } else {        // the query's own tail token p - T'_q
+          const int64_t w = p - Tq;
+          my = (half_id ? vt : kt) + (((int64_t)q * a.tail_cap + w) * a.Hkv + c) * D;
+        }
       }
     }
     uint8_t *dst = stage_ptr(jl, half_id);

@@ -16,6 +16,11 @@ RTOL_FRO = 2e-2  # relative Frobenius error bound per head
 # s_q = 4, s_k = 1; with |v| up to ~3.5 a sharp softmax turns that into up to
 # ~0.04 on an output element, plus half a bf16 ulp of the output (<= 0.008).
 ATOL_PEAKY = 6e-2
+# The same argument bounds the relative Frobenius error of a peaky row: its
+# output is close to one V row (elements ~N(0,1), norm ~sqrt(d)) and each
+# element may move by ~0.04, so up to ~4 % on a row; with few rows per head
+# (a decode step has one) nothing averages this out.
+RTOL_FRO_PEAKY = 4e-2
 
 
 def tdtype(dtype: str):
@@ -33,8 +38,12 @@ def host_f32(t) -> np.ndarray:
     return t.detach().float().cpu().numpy()
 
 
-def compare(got: np.ndarray, want: np.ndarray, head_axis: int, what: str, atol: float = ATOL):
-    """max-abs <= atol and, per head, relative Frobenius error <= RTOL_FRO."""
+def compare(got: np.ndarray, want: np.ndarray, head_axis: int, what: str, atol: float = ATOL,
+            rtol: float | None = None):
+    """max-abs <= atol and, per head, relative Frobenius error <= rtol (RTOL_FRO,
+    or RTOL_FRO_PEAKY when the peaky max-abs bound is in use)."""
+    if rtol is None:
+        rtol = RTOL_FRO_PEAKY if atol >= ATOL_PEAKY else RTOL_FRO
     got = np.asarray(got, dtype=np.float64)
     err = np.abs(got - want)
     assert np.isfinite(got).all(), what + ": non-finite output"
@@ -42,7 +51,7 @@ def compare(got: np.ndarray, want: np.ndarray, head_axis: int, what: str, atol: 
     g = np.moveaxis(got, head_axis, 0).reshape(got.shape[head_axis], -1)
     w = np.moveaxis(want, head_axis, 0).reshape(want.shape[head_axis], -1)
     rel = np.linalg.norm(g - w, axis=1) / np.maximum(np.linalg.norm(w, axis=1), 1e-30)
-    assert rel.max() <= RTOL_FRO, "%s: relative Frobenius %.3e > %.1e" % (what, rel.max(), RTOL_FRO)
+    assert rel.max() <= rtol, "%s: relative Frobenius %.3e > %.1e" % (what, rel.max(), rtol)
     return float(err.max()), float(rel.max())
 
 

@@ -159,3 +159,24 @@ def test_prepared_block_keys_bit_identical(dtype, Hq, Hkv, D, n_new, tail_len):
     dbsa.gather_rope_attend(cfg, run2.kc, run2.vc, run2.offs, run2.sel_ptr, run2.sel, run2.q_new,
                             run2.kt, run2.vt, tail_len, out2, run2.ws, block_keys=bk)
     assert torch.equal(out2, run2.out)
+
+
+@pytest.mark.parametrize("n_new,tail_len", [(16, 16), (1, 9)])
+def test_demonstration_granular_gather(n_new, tail_len):
+    """Example-level selection ([DBSA notes] §Ablations, selection granularity):
+    the offsets table makes every demonstration after the sink block its own
+    block, and each query selects the sink and single demonstrations.  Such
+    short segments go through the per-query split path (its workspace holds
+    no block-relative keys); checked against the oracle, gather maps exact."""
+    cfg = dbsa.DbsaConfig(8, 2, 128, "bf16", 5e5, 2)
+    rng = np.random.default_rng(21)
+    lens = np.concatenate([[200], rng.integers(8, 31, size=60)])
+    offs = offsets(lens)
+    nb = len(lens)
+    sels = [np.concatenate([[0], rng.permutation(np.arange(1, nb))[:k]]) for k in (18, 3, 40, 1)]
+    run = Stage2Run(cfg, offs, sels, n_new, tail_len, seed=5)
+    T = int(offs[-1])
+    assert run.ws.numel() < cfg.n_kv_heads * T * cfg.head_dim * 2
+    run.run().check("demo-granular")
+    peaky = Stage2Run(cfg, offs, sels[:2], n_new, tail_len, seed=6, q_scale=4.0).run()
+    peaky.check("demo-granular peaky", atol=ATOL_PEAKY)

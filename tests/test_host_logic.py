@@ -199,6 +199,13 @@ def test_workspace_sizes(lib):
     wg = dbsa.gather_workspace_size(cfg, offs, sel_ptr, sel, 40, 40)
     assert wg > 0
     assert dbsa.gather_workspace_size(cfg, offs, sel_ptr, np.array([2, 3, 9, 0, 1]), 40, 40) == 0
+    # a demonstration-granular selection (blocks of ~30 tokens) goes per query:
+    # its workspace holds no block-relative keys
+    lens = np.concatenate([[1500], np.full(100, 30)])
+    doffs = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    dsp, dsel = dbsa.selection_csr([np.arange(0, 101, 3)])
+    wd = dbsa.gather_workspace_size(cfg, doffs, dsp, dsel, 40, 40)
+    assert 0 < wd < 8 * int(doffs[-1]) * 256
     # prepared block keys: K at block-relative positions, bf16 [Hkv][T][D], plus small tables
     bk = dbsa.block_keys_size(cfg, offs)
     assert 8 * T * 256 <= bk < 8 * T * 256 + (1 << 20)
