@@ -531,6 +531,8 @@ def oracle_sample(w: inputs.Workload, budget_s: float, threads: int | None = Non
 
 # ------------------------------------------------------------------ main
 def dist_setup():
+    """Process group of a torchrun launch (one rank per GPU, NCCL); the host
+    logic also runs on gloo (DBSA_DIST_BACKEND=gloo) for CPU tests."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -538,19 +540,29 @@ def dist_setup():
         import datetime
         import torch
         import torch.distributed as tdist
-        torch.cuda.set_device(local)
-        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+        backend = os.environ.get("DBSA_DIST_BACKEND", "nccl")
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        tdist.init_process_group(backend, timeout=datetime.timedelta(seconds=600))
     return world, rank, local
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """Max of a per-rank device time over all ranks (the job's time)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as tdist
-    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    dev = "cuda" if tdist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], device=dev, dtype=torch.float64)
     tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
     return float(t.item())
+
+
+def weak_scaling_value(units_per_rank: float, world: int, t_max: float) -> float:
+    """Whole-job throughput: every rank processes its own batch of
+    units_per_rank, and the job takes the slowest rank's time."""
+    return units_per_rank * world / t_max
 
 
 def barrier(world):
@@ -749,8 +761,8 @@ def main():
 
     T = wl.T
     q_tokens = wl.nq * (w.query_tokens + w.decode_steps)
-    s1_tok_s = T * world / t_s1
-    s2_tok_s = q_tokens * world / t_s2
+    s1_tok_s = weak_scaling_value(T, world, t_s1)
+    s2_tok_s = weak_scaling_value(q_tokens, world, t_s2)
 
     # end to end from pinned host memory (rank-local)
     if args.e2e_steps > 0:
