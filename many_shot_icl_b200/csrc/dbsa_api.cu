@@ -441,7 +441,7 @@ S2Layout s2_layout(const dbsa_config *cfg, const GatherPlan &gp, int32_t n_new,
                         : 0);
   l.q_hat = cv.take((size_t)cfg->n_kv_heads * gp.tc_rows * cfg->head_dim * 2);
   const size_t rows = gp.items.size() * (size_t)cfg->n_q_heads * n_new;
-  l.part_acc = cv.take(rows * cfg->head_dim * sizeof(float));
+  l.part_acc = cv.take(rows * cfg->head_dim * sizeof(uint16_t));
   l.part_ml = cv.take(rows * sizeof(float2));
   l.total = cv.total();
   return l;
@@ -863,7 +863,7 @@ dbsa_status gather_impl(const dbsa_config *cfg, const void *k_cache, const void 
   a.n_queries = nq;
   a.run_items = at<int32_t>(workspace, L.run_items);
   a.n_run = (int32_t)gp.run_items.size();
-  a.part_acc = at<float>(workspace, L.part_acc);
+  a.part_acc = at<uint16_t>(workspace, L.part_acc);
   a.part_ml = at<float2>(workspace, L.part_ml);
   a.out = out;
   a.dbg_map = dbg_map;

@@ -93,13 +93,19 @@ struct WindowArgs {
 };
 cudaError_t launch_window(const WindowArgs &a, int head_dim, bool f32, cudaStream_t st);
 
+// Split partials (Stage 2): per (item, head, token) row, (M, L) in fp32 (M
+// the row's score maximum in log2 units, L the sum of 2^(s - M) over the
+// item's keys) and the item's normalised output O_item = sum p v / L as bf16
+// (a convex combination of V rows, so it keeps V's range).  The merge forms
+// O = sum_i 2^(M_i - M) L_i O_i / sum_i 2^(M_i - M) L_i.
+//
 // Partial-output mode of the tensor-core attention kernel (Stage 2, block-
 // major): row r of the packed query buffer belongs to split item row_item[r]
 // (rows of an item start at item_row0[item], token-major: u * group + local
-// head); the kernel writes (M, L) and the unnormalised accumulator to the
-// split-partial arrays, index ((item * Hq + head) * n_new + u).
+// head); the kernel writes the partial of each row at index
+// ((item * Hq + head) * n_new + u).
 struct Stage1Partial {
-  float *acc;                  // null: plain mode
+  uint16_t *acc;               // bf16 normalised outputs; null: plain mode
   float2 *ml;
   const int32_t *row_item;
   const int32_t *item_row0;
@@ -175,7 +181,7 @@ struct Stage2Args {
   int32_t n_items, n_queries;
   const int32_t *run_items;        // the tail items, which the per-query kernel runs
   int32_t n_run;
-  float *part_acc;                 // [n_items][Hq][n_new][D]
+  uint16_t *part_acc;              // bf16 [n_items][Hq][n_new][D], normalised (see above)
   float2 *part_ml;                 // [n_items][Hq][n_new] (m in log2 units, l)
   void *out;                       // [nq][n_new][Hq][D]
   int32_t *dbg_map;                // [nq][dbg_cap][2] or null

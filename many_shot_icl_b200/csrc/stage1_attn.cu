@@ -553,10 +553,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       // ---- end of item: merge factors for O = (O_0 e^{m_0 - M} + O_1 e^{m_1 - M}) /
       // (l_0 e^{m_0 - M} + l_1 e^{m_1 - M}).  Warpgroup 1 publishes its (m, l);
-      // warpgroup 0 merges the two states and publishes (f0, f1) for the
-      // epilogue warpgroup.  Plain mode: f_w = e^{m_w - M} / L (normalised
-      // output); partial mode: f_w = e^{m_w - M} and (M, L) go to the
-      // split-partial arrays.  Both warpgroups then go on to the next item.
+      // warpgroup 0 merges the two states and publishes f_w = e^{m_w - M} / L
+      // for the epilogue warpgroup (in partial mode (M, L) also go to the
+      // split-partial arrays).  Both warpgroups then go on to the next item.
       const bool partial = p.part.acc != nullptr;
       if (wg == 1) {
         if (item_no > 0)
@@ -574,7 +573,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float w0 = (m_ref == -INFINITY) ? 0.f : ex2(m_ref - M);
         const float w1 = (ml1.x == -INFINITY) ? 0.f : ex2(ml1.x - M);
         const float L = l * w0 + ml1.y * w1;
-        const float inv = partial ? 1.f : 1.f / L;
+        const float inv = L > 0.f ? 1.f / L : 0.f;
         sML[row] = make_float2(w0 * inv, w1 * inv);
         mbar_arrive(&bar[B_ML_B]);
         if (partial && row < it.n_rows) {
@@ -625,7 +624,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         prow = ((int64_t)item * p.part.Hq + h) * p.part.n_new + w / p.part.group;
       }
       const int64_t orow = ((int64_t)(it.q_row0 + row) * p.Hq + it.head) * D;
-      float *pacc = partial ? p.part.acc + prow * D : nullptr;
+      uint16_t *pacc = partial ? p.part.acc + prow * D : nullptr;
 #pragma unroll 1
       for (int col = 0; col < D; col += 32) {
         uint32_t o0[32], o1[32];
@@ -638,18 +637,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 32; ++e)
             o0[e] = __float_as_uint((has0 ? __uint_as_float(o0[e]) * fw.x : 0.f) +
                                     (has1 ? __uint_as_float(o1[e]) * fw.y : 0.f));
-          if (partial) {
-#pragma unroll
-            for (int e = 0; e < 32; e += 4)
-              *reinterpret_cast<uint4 *>(pacc + col + e) =
-                  make_uint4(o0[e], o0[e + 1], o0[e + 2], o0[e + 3]);
-          } else if (OUT_F32) {
+          if (OUT_F32 && !partial) {
             float *dst = static_cast<float *>(p.out) + orow + col;
 #pragma unroll
             for (int e = 0; e < 32; e += 4)
               *reinterpret_cast<uint4 *>(dst + e) = make_uint4(o0[e], o0[e + 1], o0[e + 2], o0[e + 3]);
           } else {
-            __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.out) + orow + col;
+            // bf16 output, or the bf16 normalised partial of the row
+            uint16_t *dst = partial ? pacc + col : static_cast<uint16_t *>(p.out) + orow + col;
 #pragma unroll
             for (int e = 0; e < 32; e += 8) {
               uint32_t w[4];

@@ -409,17 +409,19 @@ __global__ void __launch_bounds__(32 * RT * KG, 1) stage2_attn_kernel(const Stag
     return ((int64_t)it_idx * a.Hq + c * g + r % g) * a.n_new + r / g;
   };
 
+  // partials: (M, L) and the normalised output acc / L as bf16
   if constexpr (KG == 1) {
 #pragma unroll
     for (int h2 = 0; h2 < 2; ++h2) {
       const int r = row_base + wr * 16 + gq + 8 * h2;
       if (r >= R) continue;
       const int64_t pi = part_index(r);
-      float *acc = a.part_acc + pi * D;
+      const float inv = l_run[h2] > 0.f ? 1.f / l_run[h2] : 0.f;
+      uint16_t *acc = a.part_acc + pi * D;
 #pragma unroll
       for (int nd = 0; nd < ND; ++nd)
-        *reinterpret_cast<float2 *>(acc + nd * 8 + 2 * tq) =
-            make_float2(o[nd][2 * h2], o[nd][2 * h2 + 1]);
+        *reinterpret_cast<uint32_t *>(acc + nd * 8 + 2 * tq) =
+            pack_bf16(o[nd][2 * h2] * inv, o[nd][2 * h2 + 1] * inv);
       if (tq == 0) a.part_ml[pi] = make_float2(m_run[h2], l_run[h2]);
     }
   } else {
@@ -458,14 +460,16 @@ __global__ void __launch_bounds__(32 * RT * KG, 1) stage2_attn_kernel(const Stag
         acc.w += w * x.w;
       }
       const int64_t pi = part_index(r);
-      *reinterpret_cast<float4 *>(a.part_acc + pi * D + d0) = acc;
+      const float inv = L > 0.f ? 1.f / L : 0.f;
+      *reinterpret_cast<uint2 *>(a.part_acc + pi * D + d0) =
+          make_uint2(pack_bf16(acc.x * inv, acc.y * inv), pack_bf16(acc.z * inv, acc.w * inv));
       if (d0 == 0) a.part_ml[pi] = make_float2(M, L);
     }
   }
 }
 
 // One warp per output row (query q, token u, head h): combine the row's split
-// partials with their log-sum-exp weights.
+// partials, O = sum_i 2^(M_i - M) L_i O_i / sum_i 2^(M_i - M) L_i.
 template <int D, typename OT>
 __global__ void __launch_bounds__(128) stage2_merge_kernel(const Stage2Args a) {
   const int64_t row = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
@@ -489,11 +493,17 @@ __global__ void __launch_bounds__(128) stage2_merge_kernel(const Stage2Args a) {
   for (int i = 0; i < qi.n_items; ++i) {
     const int64_t pi = ((int64_t)(qi.item_begin + i) * a.Hq + h) * a.n_new + tok;
     const float2 ml = a.part_ml[pi];
-    const float w = (ml.x == -INFINITY) ? 0.f : ex2(ml.x - M);
-    L += w * ml.y;
-    const float *src = a.part_acc + pi * D + lane * PER;
+    const float w = (ml.x == -INFINITY) ? 0.f : ex2(ml.x - M) * ml.y;
+    L += w;
+    const uint16_t *src = a.part_acc + pi * D + lane * PER;
+    uint16_t v[PER];
+    if constexpr (PER == 4) {
+      *reinterpret_cast<uint2 *>(v) = *reinterpret_cast<const uint2 *>(src);
+    } else {
+      *reinterpret_cast<uint32_t *>(v) = *reinterpret_cast<const uint32_t *>(src);
+    }
 #pragma unroll
-    for (int e = 0; e < PER; ++e) acc[e] += w * src[e];
+    for (int e = 0; e < PER; ++e) acc[e] += w * __uint_as_float((uint32_t)v[e] << 16);
   }
   const float inv = 1.f / L;
   OT *dst = static_cast<OT *>(a.out) + (((int64_t)q * a.n_new + tok) * a.Hq + h) * D + lane * PER;
