@@ -133,7 +133,7 @@ def run_stage2(w, cfg, kc, vc, offs, sels, n_new, tail_len, seed):
 
 @pytest.mark.parametrize("name,order,n_new,tail_len", [
     ("llama2-7b-30k", "encoding", 32, 32),
-    ("llama3.1-8b-90k", "encoding", 40, 40),     # prompt pass (per-query kernel)
+    ("llama3.1-8b-90k", "encoding", 40, 40),     # prompt pass
     ("llama3.1-8b-90k", "encoding", 1, 45),      # a decode step
     ("llama3.1-8b-128k", "encoding", 32, 32),
     ("llama3.1-8b-128k", "ascending", 32, 32),
@@ -155,3 +155,63 @@ def test_stage2_full_batch_sampled(name, order, n_new, tail_len):
                                  host_f32(kt[qi, :tail_len]), host_f32(vt[qi, :tail_len]),
                                  w.rope_theta)
         compare(host_f32(out[qi]), want, head_axis=1, what="%s q%d" % (name, qi))
+
+
+def demo_granular(w, offs, seed):
+    """The same context as one block per demonstration after the sink block,
+    and per query the sink plus a seeded 30 % of the demonstrations."""
+    lens = inputs.demo_lengths(w)
+    k = w.demos_per_block
+    d_offs = np.concatenate([[0, offs[1]], offs[1] + np.cumsum(lens[k:])]).astype(np.int32)
+    assert d_offs[-1] == offs[-1]
+    n = len(d_offs) - 1
+    rng = np.random.default_rng(seed)
+    pick = int(round(w.retrieval_ratio * (n - 1)))
+    sels = [np.concatenate([[0], np.sort(rng.permutation(np.arange(1, n))[:pick])]).astype(np.int32)
+            for _ in range(w.n_queries)]
+    return d_offs, sels
+
+
+def test_stage2_demo_granular_full_size():
+    """90k cache, 64 queries selecting single demonstrations (~885 segments
+    each): the per-query split path, checked like the block-granular batches."""
+    w = inputs.L31_8B_90K
+    cfg, offs, q, k, v, kc, vc, _ = run_stage1(w)
+    del q, k, v
+    d_offs, sels = demo_granular(w, offs, seed=9)
+    n_new = tail_len = w.query_tokens
+    qn, kt, vt, out, dbg = run_stage2(w, cfg, kc, vc, d_offs, sels, n_new, tail_len,
+                                      seed=inputs.tensor_seed(w, 0, 3, 77))
+    dbg = dbg.cpu().numpy()
+    for qi, s in enumerate(sels):
+        m = oracle.stage2_gather_map(d_offs, s)
+        np.testing.assert_array_equal(dbg[qi, :len(m)], m)
+    kch, vch = host_f32(kc), host_f32(vc)
+    for qi in (0, len(sels) - 1):
+        want = oracle.stage2_all(kch, vch, d_offs, sels[qi], host_f32(qn[qi]),
+                                 host_f32(kt[qi, :tail_len]), host_f32(vt[qi, :tail_len]),
+                                 w.rope_theta)
+        compare(host_f32(out[qi]), want, head_axis=1, what="demo-granular q%d" % qi)
+
+
+def test_prepared_block_keys_full_size():
+    """90k cache, the bench's batch: dbsa_block_keys once, then the prompt pass
+    and a decode step through the prepared call, bit-identical to the plain
+    call."""
+    w = inputs.L31_8B_90K
+    cfg, offs, q, k, v, kc, vc, _ = run_stage1(w)
+    del q, k, v
+    sels = inputs.selections(w)
+    bk = torch.empty(dbsa.block_keys_size(cfg, offs), dtype=torch.uint8, device="cuda")
+    dbsa.block_keys(cfg, kc, vc, offs, bk)
+    sp, sb = dbsa.selection_csr(sels)
+    for n_new, tail_len in ((w.query_tokens, w.query_tokens), (1, w.query_tokens + 3)):
+        qn, kt, vt, out, _ = run_stage2(w, cfg, kc, vc, offs, sels, n_new, tail_len,
+                                        seed=inputs.tensor_seed(w, 0, 3, n_new))
+        ws = torch.empty(dbsa.gather_workspace_size(cfg, offs, sp, sb, n_new, tail_len),
+                         dtype=torch.uint8, device="cuda")
+        out2 = torch.full_like(out, float("nan"))
+        dbsa.gather_rope_attend(cfg, kc, vc, offs, sp, sb, qn, kt, vt, tail_len, out2, ws,
+                                block_keys=bk)
+        assert dbsa.read_status(ws) == dbsa.OK
+        assert torch.equal(out2, out), "prepared path differs at n_new=%d" % n_new
