@@ -245,42 +245,97 @@ def stage_times(wl: Workload):
 
 
 def e2e_step_time(wl: Workload, host, steps: int):
-    """Same step through the public API from pinned host buffers: per layer the
-    Q/K/V upload, the call and the output download are inside the timed region."""
+    """The same step through the public API from pinned host buffers: every
+    layer's Q/K/V upload, its calls and its output download are inside the
+    timed region.  Copies run on their own streams and overlap the kernels of
+    neighbouring layers (double-buffered device inputs and outputs, ordered
+    with events), as a serving loop would run them."""
     import torch
     from many_shot_icl_b200 import dbsa
-    dev_q, dev_k, dev_v, dev_o = wl.q[0], wl.k[0], wl.v[0], wl.out[0]
+    comp = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()
+    # Stage-1 double buffers: device inputs/outputs and host outputs
+    din = [(wl.q[0], wl.k[0], wl.v[0]), host["dev_in2"]]
+    dout = [wl.out[0], host["dev_out2"]]
+    hout = [host["o"], host["o2"]]
+    # Stage-2 double buffers for the outputs of consecutive calls
+    d2out = {True: [wl.out_p, host["dev_op2"]], False: [wl.out_d, host["dev_od2"]]}
+    h2out = {True: [host["op"], host["op2"]], False: [host["od"], host["od2"]]}
     t1 = t2 = 0.0
     for _ in range(steps):
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
         torch.cuda.synchronize()
-        ev[0].record()
+        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        e0.record(comp)
+        s_in.wait_stream(comp)
+        s_out.wait_stream(comp)
+        in_done, comp_done, out_done = [ev(), ev()], [None, None], [None, None]
         for l in range(wl.layers):
-            dev_q.copy_(host["q"], non_blocking=True)
-            dev_k.copy_(host["k"], non_blocking=True)
-            dev_v.copy_(host["v"], non_blocking=True)
-            dbsa.encode_blocks(wl.cfg, dev_q, dev_k, dev_v, wl.offs, wl.kc[l], wl.vc[l], dev_o,
-                               wl.ws)
-            host["o"].copy_(dev_o, non_blocking=True)
-        ev[1].record()
+            b = l & 1
+            with torch.cuda.stream(s_in):
+                if comp_done[b] is not None:
+                    s_in.wait_event(comp_done[b])       # buffer b's last reader is done
+                for d, h in zip(din[b], (host["q"], host["k"], host["v"])):
+                    d.copy_(h, non_blocking=True)
+                in_done[b].record(s_in)
+            comp.wait_event(in_done[b])
+            if out_done[b] is not None:
+                comp.wait_event(out_done[b])             # output b has been read back
+            dbsa.encode_blocks(wl.cfg, din[b][0], din[b][1], din[b][2], wl.offs, wl.kc[l],
+                               wl.vc[l], dout[b], wl.ws)
+            comp_done[b] = ev()
+            comp_done[b].record(comp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(comp_done[b])
+                hout[b].copy_(dout[b], non_blocking=True)
+                out_done[b] = ev()
+                out_done[b].record(s_out)
+        comp.wait_stream(s_out)
+        e1.record(comp)
+        s_in.wait_stream(comp)
+        s_out.wait_stream(comp)
         for l in range(wl.layers):
             dbsa.block_keys(wl.cfg, wl.kc[l], wl.vc[l], wl.offs, wl.bk[l])
+        layer_done = [None] * wl.layers
+        out_done2 = {True: [None, None], False: [None, None]}
+        k = 0
         for n_new, tail_len in wl.passes():
+            prompt = n_new > 1
             for l in range(wl.layers):
-                qn, out = (wl.qp[l], wl.out_p) if n_new > 1 else (wl.qd[l], wl.out_d)
-                hq, ho = (host["qp"], host["op"]) if n_new > 1 else (host["qd"], host["od"])
-                qn.copy_(hq, non_blocking=True)
-                # the pass's new tail tokens (K and V) arrive from the host too
-                wl.kt[l][:, tail_len - n_new:tail_len].copy_(host["kt"][:, :n_new], non_blocking=True)
-                wl.vt[l][:, tail_len - n_new:tail_len].copy_(host["vt"][:, :n_new], non_blocking=True)
+                b = k & 1
+                k += 1
+                qn = wl.qp[l] if prompt else wl.qd[l]
+                hq = host["qp"] if prompt else host["qd"]
+                done_in = ev()
+                with torch.cuda.stream(s_in):
+                    if layer_done[l] is not None:
+                        s_in.wait_event(layer_done[l])  # this layer's last call has read qn
+                    qn.copy_(hq, non_blocking=True)
+                    # the pass's new tail tokens (K and V) arrive from the host too
+                    wl.kt[l][:, tail_len - n_new:tail_len].copy_(host["kt"][:, :n_new],
+                                                                 non_blocking=True)
+                    wl.vt[l][:, tail_len - n_new:tail_len].copy_(host["vt"][:, :n_new],
+                                                                 non_blocking=True)
+                    done_in.record(s_in)
+                comp.wait_event(done_in)
+                if out_done2[prompt][b] is not None:
+                    comp.wait_event(out_done2[prompt][b])
+                out = d2out[prompt][b]
                 dbsa.gather_rope_attend(wl.cfg, wl.kc[l], wl.vc[l], wl.offs, wl.sel_ptr, wl.sel,
                                         qn, wl.kt[l], wl.vt[l], tail_len, out, wl.ws,
                                         block_keys=wl.bk[l])
-                ho.copy_(out, non_blocking=True)
-        ev[2].record()
+                layer_done[l] = ev()
+                layer_done[l].record(comp)
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(layer_done[l])
+                    h2out[prompt][b].copy_(out, non_blocking=True)
+                    out_done2[prompt][b] = ev()
+                    out_done2[prompt][b].record(s_out)
+        comp.wait_stream(s_out)
+        e2.record(comp)
         torch.cuda.synchronize()
-        t1 += ev[0].elapsed_time(ev[1]) / 1e3
-        t2 += ev[1].elapsed_time(ev[2]) / 1e3
+        t1 += e0.elapsed_time(e1) / 1e3
+        t2 += e1.elapsed_time(e2) / 1e3
     return t1 / steps, t2 / steps
 
 
@@ -318,11 +373,17 @@ def profile_only(wl: Workload, args):
 def pinned_host_buffers(wl: Workload):
     import torch
     p = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t.cpu())
+    pinned = lambda t: torch.empty(t.shape, dtype=wl.dt, pin_memory=True)
     h = {"q": p(wl.q[0]), "k": p(wl.k[0]), "v": p(wl.v[0]),
-         "o": torch.empty(wl.out[0].shape, dtype=wl.dt, pin_memory=True),
+         "o": pinned(wl.out[0]), "o2": pinned(wl.out[0]),
          "qp": p(wl.qp[0]), "qd": p(wl.qd[0]), "kt": p(wl.kt[0]), "vt": p(wl.vt[0]),
-         "op": torch.empty(wl.out_p.shape, dtype=wl.dt, pin_memory=True),
-         "od": torch.empty(wl.out_d.shape, dtype=wl.dt, pin_memory=True)}
+         "op": pinned(wl.out_p), "op2": pinned(wl.out_p),
+         "od": pinned(wl.out_d), "od2": pinned(wl.out_d),
+         # second device buffers of the overlapped end-to-end loop
+         "dev_in2": (torch.empty_like(wl.q[0]), torch.empty_like(wl.k[0]),
+                     torch.empty_like(wl.v[0])),
+         "dev_out2": torch.empty_like(wl.out[0]),
+         "dev_op2": torch.empty_like(wl.out_p), "dev_od2": torch.empty_like(wl.out_d)}
     return h
 
 
