@@ -914,6 +914,7 @@ dbsa_status gather_impl(const dbsa_config *cfg, const void *k_cache, const void 
     qa.Hkv = cfg->n_kv_heads;
     qa.queries = a.queries;
     qa.items = a.items;
+    qa.n_items = a.n_items;
     qa.row_item = at<int32_t>(workspace, L.row_item);
     qa.item_row0 = at<int32_t>(workspace, L.item_row0);
     qa.rows = gp.tc_rows;

@@ -135,6 +135,7 @@ struct QHatArgs {
   int32_t n_new, tail_len, Hq, Hkv;
   const S2Query *queries;
   const S2Item *items;             // block items: p_begin = fresh start P
+  int32_t n_items;                 // items (tail items have item_row0 = -1)
   const int32_t *row_item;
   const int32_t *item_row0;
   int32_t rows;                    // packed rows per kv head

@@ -172,32 +172,39 @@ __global__ void __launch_bounds__(256) rel_rope_kernel(RelRopeArgs a) {
 
 template <int D, typename T>
 __global__ void __launch_bounds__(256) qhat_kernel(QHatArgs a) {
+  // One thread per (block item, query token, 8-pair chunk): every query head
+  // of that token shares its position, so the rotation factors are built once
+  // and applied to all Hq rows (the packed row of head h lives in the plane of
+  // its kv head h / g, at the item's first row + token * g + h % g).
   constexpr int H = D / 2;
   constexpr int CP = H / 8;
   const int g = a.Hq / a.Hkv;
-  const int64_t n_units = (int64_t)a.rows * a.Hkv * CP;
+  const int64_t n_units = (int64_t)a.n_items * a.n_new * CP;
   for (int64_t u = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; u < n_units;
        u += (int64_t)gridDim.x * blockDim.x) {
     const int cp = (int)(u % CP);
-    const int c_ = (int)((u / CP) % a.Hkv);
-    const int32_t r = (int32_t)(u / ((int64_t)CP * a.Hkv));
-    const int item = __ldg(a.row_item + r);
-    const int w = r - __ldg(a.item_row0 + item);
-    const int tok = w / g, h = c_ * g + w % g;
+    const int tok = (int)((u / CP) % a.n_new);
+    const int item = (int)(u / ((int64_t)CP * a.n_new));
+    const int row0 = __ldg(a.item_row0 + item);
+    if (row0 < 0) continue;                      // a tail item: no packed rows
     const S2Item it = a.items[item];
     const int q = it.query;
     const int64_t pos =
         (int64_t)a.queries[q].n_gathered + a.tail_len - a.n_new + tok - it.p_begin;
     const int i0 = cp * 8;
-    float xl[8], xh[8], c[8], sn[8];
-    const T *src = static_cast<const T *>(a.q_new) + (((int64_t)q * a.n_new + tok) * a.Hq + h) * D;
-    load8(src + i0, xl);
-    load8(src + H + i0, xh);
+    float c[8], sn[8];
     rope_cs8(a.rope, pos, i0, H, c, sn);
-    rotate8(xl, xh, c, sn);
-    bf16 *dst = static_cast<bf16 *>(a.q_hat) + ((int64_t)c_ * a.rows + r) * D;
-    store8_bf16(dst + i0, xl);
-    store8_bf16(dst + H + i0, xh);
+    const T *src = static_cast<const T *>(a.q_new) + ((int64_t)q * a.n_new + tok) * a.Hq * D;
+    const int32_t r = row0 + tok * g;
+    for (int h = 0; h < a.Hq; ++h) {
+      float xl[8], xh[8];
+      load8(src + (int64_t)h * D + i0, xl);
+      load8(src + (int64_t)h * D + H + i0, xh);
+      rotate8(xl, xh, c, sn);
+      bf16 *dst = static_cast<bf16 *>(a.q_hat) + ((int64_t)(h / g) * a.rows + r + h % g) * D;
+      store8_bf16(dst + i0, xl);
+      store8_bf16(dst + H + i0, xh);
+    }
   }
 }
 
@@ -246,7 +253,7 @@ cudaError_t launch_rel_rope(const RelRopeArgs &a, int head_dim, bool f32, cudaSt
 
 cudaError_t launch_qhat(const QHatArgs &a, int head_dim, bool f32, cudaStream_t st) {
   if (a.rows <= 0) return cudaSuccess;
-  const int g = grid_for((int64_t)a.rows * a.Hkv * (head_dim / 16), 256);
+  const int g = grid_for((int64_t)a.n_items * a.n_new * (head_dim / 16), 256);
   if (head_dim == 128) {
     if (f32) qhat_kernel<128, float><<<g, 256, 0, st>>>(a);
     else qhat_kernel<128, bf16><<<g, 256, 0, st>>>(a);
