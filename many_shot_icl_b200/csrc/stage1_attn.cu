@@ -153,6 +153,37 @@ __device__ __forceinline__ f32x2 f2_add(f32x2 a, f32x2 b) {
   return d;
 }
 
+// 2^x for a pair of scores on the FMA pipe.  The exponential unit delivers 16
+// results per clock per SM, which for a 128x128 tile is as long as its two
+// MMAs; evaluating a share of P here keeps it off the critical path.  With
+// n = round(x) and f = x - n in [-1/2, 1/2], 2^x = 2^n * 2^f: n is added to the
+// exponent field and 2^f is a cubic fitted to it on that interval (weighted
+// least squares at Chebyshev nodes, reweighted toward equal ripple), with a
+// relative error below 7.5e-5, far under the half-ulp (2^-9) of the bf16 P it
+// feeds.  The rounding adds and subtracts 1.5 * 2^23, which leaves round(x) in
+// the low bits of the sum.  x is clamped at -125 so the exponent field stays
+// normal: a masked (-inf) score gives 2^-125 rather than 0.
+constexpr float kExp2C0 = 0.99992806f, kExp2C1 = 0.69326097f, kExp2C2 = 0.24261113f,
+                kExp2C3 = 0.05517166f;
+// Pairs (of the 16 in a 32-score chunk) whose P is evaluated by exp2_poly2.
+constexpr uint32_t kPolyPairMask = 0x8080u;
+__device__ __forceinline__ f32x2 exp2_poly2(f32x2 x) {
+  float x0, x1;
+  f2_unpack(x, x0, x1);
+  const f32x2 xc = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const f32x2 j = f2_add(xc, f2_pack(12582912.f, 12582912.f));
+  const f32x2 n = f2_add(j, f2_pack(-12582912.f, -12582912.f));
+  const f32x2 f = f2_fma(n, f2_pack(-1.f, -1.f), xc);
+  f32x2 q = f2_fma(f2_pack(kExp2C3, kExp2C3), f, f2_pack(kExp2C2, kExp2C2));
+  q = f2_fma(q, f, f2_pack(kExp2C1, kExp2C1));
+  q = f2_fma(q, f, f2_pack(kExp2C0, kExp2C0));
+  float j0, j1, q0, q1;
+  f2_unpack(j, j0, j1);
+  f2_unpack(q, q0, q1);
+  return f2_pack(__uint_as_float(__float_as_uint(q0) + (__float_as_uint(j0) << 23)),
+                 __uint_as_float(__float_as_uint(q1) + (__float_as_uint(j1) << 23)));
+}
+
 // Bounded wait used on the way out: ignores the abort flag.
 __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
   const uint64_t t0 = globaltimer_ns();
@@ -520,10 +551,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t pw[16];
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            float x0, x1;
-            f2_unpack(f2_fma(f2_pack(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), sc2, nmu2),
-                      x0, x1);
-            const float p0 = ex2(x0), p1 = ex2(x1);
+            const f32x2 x2 =
+                f2_fma(f2_pack(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), sc2, nmu2);
+            float p0, p1;
+            if ((kPolyPairMask >> (e >> 1)) & 1u) {
+              f2_unpack(exp2_poly2(x2), p0, p1);
+            } else {
+              float x0, x1;
+              f2_unpack(x2, x0, x1);
+              p0 = ex2(x0);
+              p1 = ex2(x1);
+            }
             sum2[(e >> 1) & 1] = f2_add(sum2[(e >> 1) & 1], f2_pack(p0, p1));
             __nv_bfloat162 hh = __floats2bfloat162_rn(p0, p1);
             pw[e >> 1] = *reinterpret_cast<uint32_t *>(&hh);

@@ -210,3 +210,30 @@ def test_workspace_sizes(lib):
     bk = dbsa.block_keys_size(cfg, offs)
     assert 8 * T * 256 <= bk < 8 * T * 256 + (1 << 20)
     assert dbsa.block_keys_size(dbsa.DbsaConfig(2, 1, 64, "f32"), offs) >= 2 * T * 128
+
+
+def test_softmax_polynomial_exp2_error_bound():
+    """The Stage-1 softmax evaluates part of P = 2^x with a cubic on the FMA
+    pipe.  Emulate its float32 steps (clamp at -125, round by adding and
+    subtracting 1.5 * 2^23, cubic in f = x - n, n added to the exponent field)
+    with the coefficients parsed from the kernel source, and check the result
+    against 2^x in fp64: relative error far below the bf16 half-ulp (2^-9) of
+    the P it feeds, positive and finite everywhere, masked scores tiny."""
+    src = open(os.path.join(ROOT, "many_shot_icl_b200", "csrc", "stage1_attn.cu")).read()
+    c = [np.float32(float(re.search(r"kExp2C%d = ([0-9.e+-]+)f" % i, src).group(1)))
+         for i in range(4)]
+    x = np.concatenate([np.linspace(-140, 9, 1_000_001, dtype=np.float32),
+                        np.float32([-np.inf, 0.0, -0.5, 0.5, 8.0, -125.0, -124.5])])
+    magic = np.float32(12582912.0)
+    xc = np.maximum(x, np.float32(-125.0))
+    j = (xc + magic).astype(np.float32)
+    n = (j - magic).astype(np.float32)
+    f = (xc - n).astype(np.float32)
+    assert np.all(np.abs(f) <= 0.5)
+    q = ((c[3] * f + c[2]) * f + c[1]) * f + c[0]
+    r = (q.view(np.uint32) + (j.view(np.uint32) << np.uint32(23))).view(np.float32)
+    assert np.all(np.isfinite(r)) and np.all(r > 0)
+    live = x >= -125
+    rel = np.abs(r[live].astype(np.float64) / np.exp2(x[live].astype(np.float64)) - 1.0)
+    assert rel.max() < 1e-4 < 2.0 ** -9
+    assert np.all(r[~live] < 1e-37)
