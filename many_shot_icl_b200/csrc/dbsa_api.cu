@@ -52,6 +52,85 @@ dbsa_status cuda_fail(cudaError_t e, const char *where) {
 constexpr size_t kAlign = 1024;
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Copies bytes from page-locked host memory (read over the bus by the SMs)
+// into device memory: 16-byte words while both sides allow, then bytes.
+__global__ void __launch_bounds__(256) copy_from_host_kernel(uint8_t *dst, const uint8_t *src,
+                                                             size_t bytes) {
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  const size_t i0 = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const bool vec = ((reinterpret_cast<uintptr_t>(dst) | reinterpret_cast<uintptr_t>(src)) & 15u) == 0;
+  const size_t words = vec ? bytes / 16 : 0;
+  for (size_t i = i0; i < words; i += stride)
+    reinterpret_cast<uint4 *>(dst)[i] = reinterpret_cast<const uint4 *>(src)[i];
+  for (size_t i = words * 16 + i0; i < bytes; i += stride) dst[i] = src[i];
+}
+
+// Host-built plans (tile lists, gather tables, block offsets) reach the device
+// through page-locked staging memory that a small kernel reads directly.  Two
+// things are avoided: from a pageable source cudaMemcpyAsync holds the calling
+// thread until the copy can be staged (stalling a caller that queues later
+// layers behind this call), and a copy-engine transfer can be queued behind
+// the caller's own large uploads on other streams (the next layer's inputs),
+// delaying this call by their whole duration.  Each thread keeps a ring of
+// staging slots; a slot is refilled only once the event recorded behind its
+// previous read has completed, so a read never sees a slot being rewritten.
+// The slots live until the process exits.
+class StagingRing {
+ public:
+  cudaError_t upload(void *dst, const void *src, size_t bytes, cudaStream_t st) {
+    if (bytes == 0) return cudaSuccess;
+    Slot &s = slots_[next_];
+    next_ = (next_ + 1) % kSlots;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (s.ev != nullptr) {
+      if ((e = cudaEventSynchronize(s.ev)) != cudaSuccess) return e;
+      if (s.dev != dev) {
+        cudaEventDestroy(s.ev);
+        s.ev = nullptr;
+      }
+    }
+    if (s.cap < bytes) {
+      if (s.p != nullptr) cudaFreeHost(s.p);  // its last copy has completed
+      s.p = nullptr;
+      const size_t cap = align_up(std::max(bytes, 2 * s.cap), size_t(1) << 16);
+      s.cap = 0;
+      if ((e = cudaHostAlloc(&s.p, cap, cudaHostAllocPortable | cudaHostAllocMapped)) !=
+          cudaSuccess)
+        return e;
+      s.cap = cap;
+    }
+    if (s.ev == nullptr) {
+      if ((e = cudaEventCreateWithFlags(&s.ev, cudaEventDisableTiming)) != cudaSuccess) return e;
+      s.dev = dev;
+    }
+    std::memcpy(s.p, src, bytes);
+    const int grid = (int)std::min<size_t>((bytes + 4095) / 4096, 148);
+    copy_from_host_kernel<<<grid, 256, 0, st>>>(static_cast<uint8_t *>(dst),
+                                               static_cast<const uint8_t *>(s.p), bytes);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    count_launches(1);
+    return cudaEventRecord(s.ev, st);
+  }
+
+ private:
+  struct Slot {
+    void *p = nullptr;
+    size_t cap = 0;
+    cudaEvent_t ev = nullptr;
+    int dev = -1;
+  };
+  static constexpr int kSlots = 8;
+  Slot slots_[kSlots];
+  int next_ = 0;
+};
+
+cudaError_t upload_async(void *dst, const void *src, size_t bytes, cudaStream_t st) {
+  static thread_local StagingRing *ring = new StagingRing();
+  return ring->upload(dst, src, bytes, st);
+}
+
 // Sequential sub-allocation of the caller's workspace.
 struct Carve {
   size_t off = kStatusBytes;
@@ -239,7 +318,8 @@ struct GatherPlan {
   int32_t tc_rows = 0;
   int32_t nb = 0;
   int64_t cache_rows = 0;  // offs[nb]
-  std::vector<int32_t> row_item, item_row0;
+  // packed_items[k]: the item owning packed rows [k R, (k + 1) R), R = g n_new
+  std::vector<int32_t> packed_items, item_row0;
   std::vector<dbsa_tile_item> tc_tiles;
 };
 
@@ -365,7 +445,7 @@ dbsa_status gather_plan(const dbsa_config *cfg, const int32_t *offs, int32_t nb,
       block_row0[b] = gp.tc_rows;
       for (int32_t it : per_block[b]) {
         gp.item_row0[it] = gp.tc_rows;
-        for (int r = 0; r < R; ++r) gp.row_item.push_back(it);
+        gp.packed_items.push_back(it);
         gp.tc_rows += R;
       }
       block_rows[b] = gp.tc_rows - block_row0[b];
@@ -412,7 +492,7 @@ S1Layout s1_layout(const dbsa_config *cfg, int64_t max_pos, int64_t n_items, int
 }
 
 struct S2Layout {
-  size_t rope, queries, segs, items, run_items, row_item, item_row0,
+  size_t rope, queries, segs, items, run_items, packed_items, item_row0,
       tc_tiles, offs, blob_end, k_hat, v_hat, q_hat, part_acc, part_ml, total;
   int32_t n_hi;
 };
@@ -428,7 +508,7 @@ S2Layout s2_layout(const dbsa_config *cfg, const GatherPlan &gp, int32_t n_new,
   l.segs = cv.take(gp.segs.size() * sizeof(S2Segment));
   l.items = cv.take(gp.items.size() * sizeof(S2Item));
   l.run_items = cv.take(gp.run_items.size() * sizeof(int32_t));
-  l.row_item = cv.take(gp.row_item.size() * sizeof(int32_t));
+  l.packed_items = cv.take(gp.packed_items.size() * sizeof(int32_t));
   l.item_row0 = cv.take(gp.item_row0.size() * sizeof(int32_t));
   l.tc_tiles = cv.take(gp.tc_tiles.size() * sizeof(dbsa_tile_item));
   l.offs = cv.take((size_t)(offs_count(gp)) * sizeof(int32_t));
@@ -587,9 +667,8 @@ dbsa_status dbsa_encode_blocks(const dbsa_config *cfg, const void *q, const void
   if ((e = build_tables(workspace, L.rope, L.n_hi, cfg, st, &rope)) != cudaSuccess)
     return cuda_fail(e, "rope tables");
   count_launches(1);
-  if ((e = cudaMemcpyAsync(at<void>(workspace, L.items), items.data(),
-                           items.size() * sizeof(dbsa_tile_item), cudaMemcpyHostToDevice, st)) !=
-      cudaSuccess)
+  if ((e = upload_async(at<void>(workspace, L.items), items.data(),
+                        items.size() * sizeof(dbsa_tile_item), st)) != cudaSuccess)
     return cuda_fail(e, "tile list upload");
   IngestArgs ia{};
   ia.q = q;
@@ -682,9 +761,8 @@ dbsa_status dbsa_append_block(const dbsa_config *cfg, const void *q, const void 
   if ((e = build_tables(workspace, Ly.rope, Ly.n_hi, cfg, st, &rope)) != cudaSuccess)
     return cuda_fail(e, "rope tables");
   count_launches(1);
-  if ((e = cudaMemcpyAsync(at<void>(workspace, Ly.items), items.data(),
-                           items.size() * sizeof(dbsa_tile_item), cudaMemcpyHostToDevice, st)) !=
-      cudaSuccess)
+  if ((e = upload_async(at<void>(workspace, Ly.items), items.data(),
+                        items.size() * sizeof(dbsa_tile_item), st)) != cudaSuccess)
     return cuda_fail(e, "tile list upload");
   void *k_rot = at<void>(workspace, Ly.k_rot);
   void *v_bf16 = f32 ? at<void>(workspace, Ly.v_bf16) : nullptr;
@@ -833,15 +911,15 @@ dbsa_status gather_impl(const dbsa_config *cfg, const void *k_cache, const void 
                 gp.items.size() * sizeof(S2Item));
     std::memcpy(blob.data() + (L.run_items - L.queries), gp.run_items.data(),
                 gp.run_items.size() * sizeof(int32_t));
-    std::memcpy(blob.data() + (L.row_item - L.queries), gp.row_item.data(),
-                gp.row_item.size() * sizeof(int32_t));
+    std::memcpy(blob.data() + (L.packed_items - L.queries), gp.packed_items.data(),
+                gp.packed_items.size() * sizeof(int32_t));
     std::memcpy(blob.data() + (L.item_row0 - L.queries), gp.item_row0.data(),
                 gp.item_row0.size() * sizeof(int32_t));
     std::memcpy(blob.data() + (L.tc_tiles - L.queries), gp.tc_tiles.data(),
                 gp.tc_tiles.size() * sizeof(dbsa_tile_item));
     std::memcpy(blob.data() + (L.offs - L.queries), offs_host, (size_t)(nb + 1) * sizeof(int32_t));
-    if ((e = cudaMemcpyAsync(at<void>(workspace, L.queries), blob.data(), blob.size(),
-                             cudaMemcpyHostToDevice, st)) != cudaSuccess)
+    if ((e = upload_async(at<void>(workspace, L.queries), blob.data(), blob.size(), st)) !=
+        cudaSuccess)
       return cuda_fail(e, "gather plan upload");
   }
   Stage2Args a{};
@@ -915,7 +993,6 @@ dbsa_status gather_impl(const dbsa_config *cfg, const void *k_cache, const void 
     qa.queries = a.queries;
     qa.items = a.items;
     qa.n_items = a.n_items;
-    qa.row_item = at<int32_t>(workspace, L.row_item);
     qa.item_row0 = at<int32_t>(workspace, L.item_row0);
     qa.rows = gp.tc_rows;
     qa.q_hat = at<void>(workspace, L.q_hat);
@@ -948,8 +1025,7 @@ dbsa_status gather_impl(const dbsa_config *cfg, const void *k_cache, const void 
     sa.status = at<int>(workspace, 0);
     sa.part.acc = a.part_acc;
     sa.part.ml = a.part_ml;
-    sa.part.row_item = qa.row_item;
-    sa.part.item_row0 = qa.item_row0;
+    sa.part.packed_items = at<int32_t>(workspace, L.packed_items);
     sa.part.group = cfg->n_q_heads / cfg->n_kv_heads;
     sa.part.Hq = cfg->n_q_heads;
     sa.part.n_new = n_new;
@@ -1011,9 +1087,8 @@ dbsa_status dbsa_block_keys(const dbsa_config *cfg, const void *k_cache, const v
   if ((e = build_tables(block_keys, B.rope, B.n_hi, cfg, st, &rope)) != cudaSuccess)
     return cuda_fail(e, "rope tables");
   count_launches(1);
-  if ((e = cudaMemcpyAsync(at<void>(block_keys, B.offs), offs_host,
-                           (size_t)(nb + 1) * sizeof(int32_t), cudaMemcpyHostToDevice, st)) !=
-      cudaSuccess)
+  if ((e = upload_async(at<void>(block_keys, B.offs), offs_host,
+                        (size_t)(nb + 1) * sizeof(int32_t), st)) != cudaSuccess)
     return cuda_fail(e, "offset upload");
   RelRopeArgs ra{};
   ra.k_cache = k_cache;

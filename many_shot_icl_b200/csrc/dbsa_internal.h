@@ -100,15 +100,14 @@ cudaError_t launch_window(const WindowArgs &a, int head_dim, bool f32, cudaStrea
 // O = sum_i 2^(M_i - M) L_i O_i / sum_i 2^(M_i - M) L_i.
 //
 // Partial-output mode of the tensor-core attention kernel (Stage 2, block-
-// major): row r of the packed query buffer belongs to split item row_item[r]
-// (rows of an item start at item_row0[item], token-major: u * group + local
-// head); the kernel writes the partial of each row at index
-// ((item * Hq + head) * n_new + u).
+// major): every split item owns group * n_new consecutive rows of the packed
+// query buffer (token-major: u * group + local head), so row r belongs to item
+// packed_items[r / (group * n_new)]; the kernel writes the partial of each row
+// at index ((item * Hq + head) * n_new + u).
 struct Stage1Partial {
   uint16_t *acc;               // bf16 normalised outputs; null: plain mode
   float2 *ml;
-  const int32_t *row_item;
-  const int32_t *item_row0;
+  const int32_t *packed_items; // item of each group * n_new packed rows
   int32_t group, Hq, n_new;
 };
 
@@ -126,17 +125,16 @@ struct RelRopeArgs {
 };
 cudaError_t launch_rel_rope(const RelRopeArgs &a, int head_dim, bool f32, cudaStream_t st);
 
-// Packed query rows of the block-major pass: row r of kv head c is query
-// token u / local head hl of split item row_item[r] (a (query, block) pair),
-// rotated at (its position - the block's fresh start).  Also writes the
-// gather map when dbg_map is set.
+// Packed query rows of the block-major pass: rows item_row0[i] .. + g*n_new
+// of kv head c are query token u / local head hl (row u * g + hl) of split
+// item i (a (query, block) pair), rotated at (its position - the block's
+// fresh start).
 struct QHatArgs {
   const void *q_new;               // [nq][n_new][Hq][D]
   int32_t n_new, tail_len, Hq, Hkv;
   const S2Query *queries;
   const S2Item *items;             // block items: p_begin = fresh start P
   int32_t n_items;                 // items (tail items have item_row0 = -1)
-  const int32_t *row_item;
   const int32_t *item_row0;
   int32_t rows;                    // packed rows per kv head
   void *q_hat;                     // bf16 [Hkv][rows][D]

@@ -616,8 +616,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&bar[B_ML_B]);
         if (partial && row < it.n_rows) {
           const int grow = it.q_row0 + row;
-          const int item = __ldg(p.part.row_item + grow);
-          const int w = grow - __ldg(p.part.item_row0 + item);
+          const int R = p.part.group * p.part.n_new;
+          const int item = __ldg(p.part.packed_items + grow / R);
+          const int w = grow % R;
           const int h = it.head * p.part.group + w % p.part.group;
           p.part.ml[((int64_t)item * p.part.Hq + h) * p.part.n_new + w / p.part.group] =
               make_float2(M, L);
@@ -656,8 +657,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       int64_t prow = 0;
       if (partial && row < it.n_rows) {
         const int grow = it.q_row0 + row;                 // row of the packed query buffer
-        const int item = __ldg(p.part.row_item + grow);
-        const int w = grow - __ldg(p.part.item_row0 + item);
+        const int R = p.part.group * p.part.n_new;
+        const int item = __ldg(p.part.packed_items + grow / R);
+        const int w = grow % R;
         const int h = it.head * p.part.group + w % p.part.group;
         prow = ((int64_t)item * p.part.Hq + h) * p.part.n_new + w / p.part.group;
       }
