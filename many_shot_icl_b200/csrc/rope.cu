@@ -172,19 +172,20 @@ __global__ void __launch_bounds__(256) rel_rope_kernel(RelRopeArgs a) {
 
 template <int D, typename T>
 __global__ void __launch_bounds__(256) qhat_kernel(QHatArgs a) {
-  // One thread per (block item, query token, 8-pair chunk): every query head
-  // of that token shares its position, so the rotation factors are built once
-  // and applied to all Hq rows (the packed row of head h lives in the plane of
-  // its kv head h / g, at the item's first row + token * g + h % g).
+  // One thread per (block item, query token, kv head, 8-pair chunk): the g
+  // query heads of the kv head share the token's position, so the rotation
+  // factors are built once and applied to all g rows (row token * g + local
+  // head of the item, in the plane of the kv head).
   constexpr int H = D / 2;
   constexpr int CP = H / 8;
   const int g = a.Hq / a.Hkv;
-  const int64_t n_units = (int64_t)a.n_items * a.n_new * CP;
+  const int64_t n_units = (int64_t)a.n_items * a.n_new * a.Hkv * CP;
   for (int64_t u = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; u < n_units;
        u += (int64_t)gridDim.x * blockDim.x) {
     const int cp = (int)(u % CP);
-    const int tok = (int)((u / CP) % a.n_new);
-    const int item = (int)(u / ((int64_t)CP * a.n_new));
+    const int c_ = (int)((u / CP) % a.Hkv);
+    const int tok = (int)((u / ((int64_t)CP * a.Hkv)) % a.n_new);
+    const int item = (int)(u / ((int64_t)CP * a.Hkv * a.n_new));
     const int row0 = __ldg(a.item_row0 + item);
     if (row0 < 0) continue;                      // a tail item: no packed rows
     const S2Item it = a.items[item];
@@ -194,16 +195,16 @@ __global__ void __launch_bounds__(256) qhat_kernel(QHatArgs a) {
     const int i0 = cp * 8;
     float c[8], sn[8];
     rope_cs8(a.rope, pos, i0, H, c, sn);
-    const T *src = static_cast<const T *>(a.q_new) + ((int64_t)q * a.n_new + tok) * a.Hq * D;
-    const int32_t r = row0 + tok * g;
-    for (int h = 0; h < a.Hq; ++h) {
+    const T *src =
+        static_cast<const T *>(a.q_new) + (((int64_t)q * a.n_new + tok) * a.Hq + c_ * g) * D;
+    bf16 *dst = static_cast<bf16 *>(a.q_hat) + ((int64_t)c_ * a.rows + row0 + tok * g) * D;
+    for (int hl = 0; hl < g; ++hl) {
       float xl[8], xh[8];
-      load8(src + (int64_t)h * D + i0, xl);
-      load8(src + (int64_t)h * D + H + i0, xh);
+      load8(src + (int64_t)hl * D + i0, xl);
+      load8(src + (int64_t)hl * D + H + i0, xh);
       rotate8(xl, xh, c, sn);
-      bf16 *dst = static_cast<bf16 *>(a.q_hat) + ((int64_t)(h / g) * a.rows + r + h % g) * D;
-      store8_bf16(dst + i0, xl);
-      store8_bf16(dst + H + i0, xh);
+      store8_bf16(dst + (int64_t)hl * D + i0, xl);
+      store8_bf16(dst + (int64_t)hl * D + H + i0, xh);
     }
   }
 }
@@ -253,7 +254,7 @@ cudaError_t launch_rel_rope(const RelRopeArgs &a, int head_dim, bool f32, cudaSt
 
 cudaError_t launch_qhat(const QHatArgs &a, int head_dim, bool f32, cudaStream_t st) {
   if (a.rows <= 0) return cudaSuccess;
-  const int g = grid_for((int64_t)a.n_items * a.n_new * (head_dim / 16), 256);
+  const int g = grid_for((int64_t)a.n_items * a.n_new * a.Hkv * (head_dim / 16), 256);
   if (head_dim == 128) {
     if (f32) qhat_kernel<128, float><<<g, 256, 0, st>>>(a);
     else qhat_kernel<128, bf16><<<g, 256, 0, st>>>(a);
