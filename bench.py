@@ -249,7 +249,9 @@ def e2e_step_time(wl: Workload, host, steps: int):
     layer's Q/K/V upload, its calls and its output download are inside the
     timed region.  Copies run on their own streams and overlap the kernels of
     neighbouring layers (double-buffered device inputs and outputs, ordered
-    with events), as a serving loop would run them."""
+    with events), as a serving loop would run them.  The events are made once
+    and re-recorded: every wait on an event is queued before its next record,
+    so each wait still sees the record it was meant for."""
     import torch
     from many_shot_icl_b200 import dbsa
     comp = torch.cuda.current_stream()
@@ -262,6 +264,13 @@ def e2e_step_time(wl: Workload, host, steps: int):
     # Stage-2 double buffers for the outputs of consecutive calls
     d2out = {True: [wl.out_p, host["dev_op2"]], False: [wl.out_d, host["dev_od2"]]}
     h2out = {True: [host["op"], host["op2"]], False: [host["od"], host["od2"]]}
+    hq = {True: host["qp"], False: host["qd"]}
+    in_done = [ev(), ev()]
+    comp_ev = [ev(), ev()]
+    out_ev = [ev(), ev()]
+    in2 = [ev() for _ in range(wl.layers)]
+    layer_ev = [ev() for _ in range(wl.layers)]
+    out2_ev = {True: [ev(), ev()], False: [ev(), ev()]}
     t1 = t2 = 0.0
     for _ in range(steps):
         torch.cuda.synchronize()
@@ -269,7 +278,7 @@ def e2e_step_time(wl: Workload, host, steps: int):
         e0.record(comp)
         s_in.wait_stream(comp)
         s_out.wait_stream(comp)
-        in_done, comp_done, out_done = [ev(), ev()], [None, None], [None, None]
+        comp_done, out_done = [None, None], [None, None]
         for l in range(wl.layers):
             b = l & 1
             with torch.cuda.stream(s_in):
@@ -283,12 +292,12 @@ def e2e_step_time(wl: Workload, host, steps: int):
                 comp.wait_event(out_done[b])             # output b has been read back
             dbsa.encode_blocks(wl.cfg, din[b][0], din[b][1], din[b][2], wl.offs, wl.kc[l],
                                wl.vc[l], dout[b], wl.ws)
-            comp_done[b] = ev()
+            comp_done[b] = comp_ev[b]
             comp_done[b].record(comp)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(comp_done[b])
                 hout[b].copy_(dout[b], non_blocking=True)
-                out_done[b] = ev()
+                out_done[b] = out_ev[b]
                 out_done[b].record(s_out)
         comp.wait_stream(s_out)
         e1.record(comp)
@@ -301,35 +310,32 @@ def e2e_step_time(wl: Workload, host, steps: int):
         k = 0
         for n_new, tail_len in wl.passes():
             prompt = n_new > 1
+            kt_src, vt_src = host["kt"][:, :n_new], host["vt"][:, :n_new]
             for l in range(wl.layers):
                 b = k & 1
                 k += 1
                 qn = wl.qp[l] if prompt else wl.qd[l]
-                hq = host["qp"] if prompt else host["qd"]
-                done_in = ev()
                 with torch.cuda.stream(s_in):
                     if layer_done[l] is not None:
                         s_in.wait_event(layer_done[l])  # this layer's last call has read qn
-                    qn.copy_(hq, non_blocking=True)
+                    qn.copy_(hq[prompt], non_blocking=True)
                     # the pass's new tail tokens (K and V) arrive from the host too
-                    wl.kt[l][:, tail_len - n_new:tail_len].copy_(host["kt"][:, :n_new],
-                                                                 non_blocking=True)
-                    wl.vt[l][:, tail_len - n_new:tail_len].copy_(host["vt"][:, :n_new],
-                                                                 non_blocking=True)
-                    done_in.record(s_in)
-                comp.wait_event(done_in)
+                    wl.kt[l][:, tail_len - n_new:tail_len].copy_(kt_src, non_blocking=True)
+                    wl.vt[l][:, tail_len - n_new:tail_len].copy_(vt_src, non_blocking=True)
+                    in2[l].record(s_in)
+                comp.wait_event(in2[l])
                 if out_done2[prompt][b] is not None:
                     comp.wait_event(out_done2[prompt][b])
                 out = d2out[prompt][b]
                 dbsa.gather_rope_attend(wl.cfg, wl.kc[l], wl.vc[l], wl.offs, wl.sel_ptr, wl.sel,
                                         qn, wl.kt[l], wl.vt[l], tail_len, out, wl.ws,
                                         block_keys=wl.bk[l])
-                layer_done[l] = ev()
+                layer_done[l] = layer_ev[l]
                 layer_done[l].record(comp)
                 with torch.cuda.stream(s_out):
                     s_out.wait_event(layer_done[l])
                     h2out[prompt][b].copy_(out, non_blocking=True)
-                    out_done2[prompt][b] = ev()
+                    out_done2[prompt][b] = out2_ev[prompt][b]
                     out_done2[prompt][b].record(s_out)
         comp.wait_stream(s_out)
         e2.record(comp)

@@ -74,13 +74,28 @@ __global__ void __launch_bounds__(256) copy_from_host_kernel(uint8_t *dst, const
 // delaying this call by their whole duration.  Each thread keeps a ring of
 // staging slots; a slot is refilled only once the event recorded behind its
 // previous read has completed, so a read never sees a slot being rewritten.
-// The slots live until the process exits.
+// A thread's slots are released when it exits, after their last reads (errors
+// are ignored there: at process exit the runtime may already be gone).
+// Calls that use the ring cannot be captured into a CUDA graph: the host fills
+// the slot at call time.
 class StagingRing {
  public:
-  cudaError_t upload(void *dst, const void *src, size_t bytes, cudaStream_t st) {
-    if (bytes == 0) return cudaSuccess;
+  StagingRing() = default;
+  StagingRing(const StagingRing &) = delete;
+  StagingRing &operator=(const StagingRing &) = delete;
+  ~StagingRing() {
+    for (Slot &s : slots_) {
+      if (s.ev != nullptr) {
+        cudaEventSynchronize(s.ev);
+        cudaEventDestroy(s.ev);
+      }
+      if (s.p != nullptr) cudaFreeHost(s.p);
+    }
+  }
+  // A page-locked buffer of >= bytes for the next upload (waits for the
+  // slot's previous read); the caller fills it, then calls send().
+  cudaError_t stage(size_t bytes, void **host) {
     Slot &s = slots_[next_];
-    next_ = (next_ + 1) % kSlots;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -92,7 +107,7 @@ class StagingRing {
       }
     }
     if (s.cap < bytes) {
-      if (s.p != nullptr) cudaFreeHost(s.p);  // its last copy has completed
+      if (s.p != nullptr) cudaFreeHost(s.p);  // its last read has completed
       s.p = nullptr;
       const size_t cap = align_up(std::max(bytes, 2 * s.cap), size_t(1) << 16);
       s.cap = 0;
@@ -105,13 +120,30 @@ class StagingRing {
       if ((e = cudaEventCreateWithFlags(&s.ev, cudaEventDisableTiming)) != cudaSuccess) return e;
       s.dev = dev;
     }
-    std::memcpy(s.p, src, bytes);
-    const int grid = (int)std::min<size_t>((bytes + 4095) / 4096, 148);
-    copy_from_host_kernel<<<grid, 256, 0, st>>>(static_cast<uint8_t *>(dst),
-                                               static_cast<const uint8_t *>(s.p), bytes);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    count_launches(1);
+    *host = s.p;
+    return cudaSuccess;
+  }
+  // Copies the first bytes of the buffer stage() returned to dst on stream st.
+  cudaError_t send(void *dst, size_t bytes, cudaStream_t st) {
+    Slot &s = slots_[next_];
+    next_ = (next_ + 1) % kSlots;
+    if (bytes > 0) {
+      const int grid = (int)std::min<size_t>((bytes + 4095) / 4096, 148);
+      copy_from_host_kernel<<<grid, 256, 0, st>>>(static_cast<uint8_t *>(dst),
+                                                 static_cast<const uint8_t *>(s.p), bytes);
+      cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+      count_launches(1);
+    }
     return cudaEventRecord(s.ev, st);
+  }
+  cudaError_t upload(void *dst, const void *src, size_t bytes, cudaStream_t st) {
+    if (bytes == 0) return cudaSuccess;
+    void *h = nullptr;
+    cudaError_t e = stage(bytes, &h);
+    if (e != cudaSuccess) return e;
+    std::memcpy(h, src, bytes);
+    return send(dst, bytes, st);
   }
 
  private:
@@ -126,9 +158,12 @@ class StagingRing {
   int next_ = 0;
 };
 
+StagingRing &staging_ring() {
+  static thread_local StagingRing ring;
+  return ring;
+}
 cudaError_t upload_async(void *dst, const void *src, size_t bytes, cudaStream_t st) {
-  static thread_local StagingRing *ring = new StagingRing();
-  return ring->upload(dst, src, bytes, st);
+  return staging_ring().upload(dst, src, bytes, st);
 }
 
 // Sequential sub-allocation of the caller's workspace.
@@ -341,6 +376,13 @@ dbsa_status gather_plan(const dbsa_config *cfg, const int32_t *offs, int32_t nb,
   std::vector<char> seen(nb, 0);
   gp.max_pos = 0;
   int64_t total_keys = 0;
+  // capacity hints only (the loop below validates the selection); a valid
+  // selection has at most nb blocks per query
+  const size_t n_sel = (size_t)std::max<int64_t>(
+      0, std::min<int64_t>(sel_ptr[nq], (int64_t)nq * nb));
+  gp.queries.reserve(nq);
+  gp.segs.reserve(n_sel);
+  gp.items.reserve(n_sel + nq);
   for (int q = 0; q < nq; ++q) {
     const int32_t a = sel_ptr[q], e = sel_ptr[q + 1];
     if (e <= a) return fail(DBSA_ERR_INVALID_ARG, "query %d selects no block", q);
@@ -416,7 +458,13 @@ dbsa_status gather_plan(const dbsa_config *cfg, const int32_t *offs, int32_t nb,
     // order, token-major rows within an item) and cut into 128-row tiles
     // that all read the same block of rotated keys, so a block selected by
     // many queries is read and rotated once per pass.
-    std::vector<std::vector<int32_t>> per_block(nb);   // item ids selecting block b
+    // items selecting each block, in query order: a counting sort by block
+    std::vector<int32_t> block_begin(nb + 1, 0);
+    for (int32_t i = 0; i < sel_ptr[nq]; ++i) ++block_begin[sel[i] + 1];
+    for (int b = 0; b < nb; ++b) block_begin[b + 1] += block_begin[b];
+    std::vector<int32_t> fill(block_begin.begin(), block_begin.end() - 1);
+    gp.packed_items.resize(sel_ptr[nq]);
+    gp.run_items.reserve(nq);
     for (int q = 0; q < nq; ++q) {
       S2Query &qi = gp.queries[q];
       qi.item_begin = (int32_t)gp.items.size();
@@ -427,7 +475,7 @@ dbsa_status gather_plan(const dbsa_config *cfg, const int32_t *offs, int32_t nb,
         it.p_begin = sg.pos0;  // the block's fresh start P
         it.p_end = sg.pos0 + sg.len;
         it.p_lo = sg.pos0;
-        per_block[sel[sel_ptr[q] + sgi]].push_back((int32_t)gp.items.size());
+        gp.packed_items[fill[sel[sel_ptr[q] + sgi]]++] = (int32_t)gp.items.size();
         gp.items.push_back(it);
       }
       S2Item tail;
@@ -439,17 +487,18 @@ dbsa_status gather_plan(const dbsa_config *cfg, const int32_t *offs, int32_t nb,
       gp.items.push_back(tail);
       qi.n_items = (int32_t)gp.items.size() - qi.item_begin;
     }
+    // rows packed block by block: packed_items[k] owns rows [k R, (k + 1) R)
     gp.item_row0.assign(gp.items.size(), -1);
+    for (size_t k = 0; k < gp.packed_items.size(); ++k) gp.item_row0[gp.packed_items[k]] = (int32_t)(k * R);
+    gp.tc_rows = (int32_t)(gp.packed_items.size() * R);
     std::vector<int32_t> block_row0(nb, 0), block_rows(nb, 0);
+    size_t n_tiles = 0;
     for (int b = 0; b < nb; ++b) {
-      block_row0[b] = gp.tc_rows;
-      for (int32_t it : per_block[b]) {
-        gp.item_row0[it] = gp.tc_rows;
-        gp.packed_items.push_back(it);
-        gp.tc_rows += R;
-      }
-      block_rows[b] = gp.tc_rows - block_row0[b];
+      block_row0[b] = block_begin[b] * R;
+      block_rows[b] = (block_begin[b + 1] - block_begin[b]) * R;
+      n_tiles += (block_rows[b] + kTileRows - 1) / kTileRows;
     }
+    gp.tc_tiles.reserve(n_tiles * cfg->n_kv_heads);
     for (int c = 0; c < cfg->n_kv_heads; ++c)
       for (int b = 0; b < nb; ++b)
         for (int m = 0; m < block_rows[b]; m += kTileRows) {
@@ -903,22 +952,26 @@ dbsa_status gather_impl(const dbsa_config *cfg, const void *k_cache, const void 
   count_launches(1);
   // one upload of the three small plan arrays (they are contiguous in the carve)
   {
-    std::vector<uint8_t> blob(L.blob_end - L.queries, 0);
-    std::memcpy(blob.data(), gp.queries.data(), gp.queries.size() * sizeof(S2Query));
-    std::memcpy(blob.data() + (L.segs - L.queries), gp.segs.data(),
+    // the tables, laid out as in the workspace, written straight into staging
+    const size_t blob_bytes = L.blob_end - L.queries;
+    uint8_t *blob = nullptr;
+    if ((e = staging_ring().stage(blob_bytes, reinterpret_cast<void **>(&blob))) != cudaSuccess)
+      return cuda_fail(e, "gather plan staging");
+    std::memcpy(blob, gp.queries.data(), gp.queries.size() * sizeof(S2Query));
+    std::memcpy(blob + (L.segs - L.queries), gp.segs.data(),
                 gp.segs.size() * sizeof(S2Segment));
-    std::memcpy(blob.data() + (L.items - L.queries), gp.items.data(),
+    std::memcpy(blob + (L.items - L.queries), gp.items.data(),
                 gp.items.size() * sizeof(S2Item));
-    std::memcpy(blob.data() + (L.run_items - L.queries), gp.run_items.data(),
+    std::memcpy(blob + (L.run_items - L.queries), gp.run_items.data(),
                 gp.run_items.size() * sizeof(int32_t));
-    std::memcpy(blob.data() + (L.packed_items - L.queries), gp.packed_items.data(),
+    std::memcpy(blob + (L.packed_items - L.queries), gp.packed_items.data(),
                 gp.packed_items.size() * sizeof(int32_t));
-    std::memcpy(blob.data() + (L.item_row0 - L.queries), gp.item_row0.data(),
+    std::memcpy(blob + (L.item_row0 - L.queries), gp.item_row0.data(),
                 gp.item_row0.size() * sizeof(int32_t));
-    std::memcpy(blob.data() + (L.tc_tiles - L.queries), gp.tc_tiles.data(),
+    std::memcpy(blob + (L.tc_tiles - L.queries), gp.tc_tiles.data(),
                 gp.tc_tiles.size() * sizeof(dbsa_tile_item));
-    std::memcpy(blob.data() + (L.offs - L.queries), offs_host, (size_t)(nb + 1) * sizeof(int32_t));
-    if ((e = upload_async(at<void>(workspace, L.queries), blob.data(), blob.size(), st)) !=
+    std::memcpy(blob + (L.offs - L.queries), offs_host, (size_t)(nb + 1) * sizeof(int32_t));
+    if ((e = staging_ring().send(at<void>(workspace, L.queries), blob_bytes, st)) !=
         cudaSuccess)
       return cuda_fail(e, "gather plan upload");
   }
