@@ -219,7 +219,10 @@ dbsa_status dbsa_gather_rope_attend(
  *   block_keys device, bk_bytes >= dbsa_block_keys_size(cfg, offs, nb),
  *              256-byte aligned, owned by the caller: the keys of every cache
  *              row s of block b rotated at s - offs[b] (bf16, [Hkv][T][D]),
- *              a bf16 copy of V for DBSA_F32 caches, and the tables used.
+ *              a bf16 copy of V for DBSA_F32 caches, and RoPE angle tables
+ *              for positions below T + 8192 (a prepared gather whose
+ *              positions fit, i.e. tail_len <= 8192, uses them instead of
+ *              building its own).
  *
  * dbsa_gather_rope_attend_prepared takes the arguments of
  * dbsa_gather_rope_attend plus block_keys, which must come from

@@ -582,13 +582,16 @@ struct BKLayout {
   size_t rope, offs, k_hat, v_hat, total;
   int32_t n_hi;
 };
+// The block-keys tables also cover every position a gather from the same
+// cache reaches with up to this many tail tokens (a query's gathered length is
+// at most T), so a prepared gather reads them instead of building its own.
+constexpr int64_t kBlockKeysTailPositions = 8192;
+
 BKLayout bk_layout(const dbsa_config *cfg, const int32_t *offs, int32_t nb) {
   BKLayout l;
   Carve cv;
-  int32_t max_len = 1;
-  for (int32_t b = 0; b < nb; ++b) max_len = std::max(max_len, offs[b + 1] - offs[b]);
-  l.n_hi = (max_len - 1) / kRopeLo + 1;
   const int64_t T = offs[nb];
+  l.n_hi = (int32_t)((T + kBlockKeysTailPositions - 1) / kRopeLo + 1);
   l.rope = cv.take(rope_table_bytes(l.n_hi, cfg->head_dim));
   l.offs = cv.take((size_t)(nb + 1) * sizeof(int32_t));
   l.k_hat = cv.take((size_t)cfg->n_kv_heads * T * cfg->head_dim * 2);
@@ -947,9 +950,15 @@ dbsa_status gather_impl(const dbsa_config *cfg, const void *k_cache, const void 
   if ((e = cudaMemsetAsync(workspace, 0, kStatusBytes, st)) != cudaSuccess)
     return cuda_fail(e, "status clear");
   RopeTables rope;
-  if ((e = build_tables(workspace, L.rope, L.n_hi, cfg, st, &rope)) != cudaSuccess)
-    return cuda_fail(e, "rope tables");
-  count_launches(1);
+  if (prepared && B.n_hi >= L.n_hi) {
+    // the block-keys tables cover this call's positions (same rows, same values)
+    rope = rope_tables_at(at<float>(const_cast<void *>(block_keys), B.rope), B.n_hi,
+                          cfg->head_dim);
+  } else {
+    if ((e = build_tables(workspace, L.rope, L.n_hi, cfg, st, &rope)) != cudaSuccess)
+      return cuda_fail(e, "rope tables");
+    count_launches(1);
+  }
   // one upload of the three small plan arrays (they are contiguous in the carve)
   {
     // the tables, laid out as in the workspace, written straight into staging

@@ -206,9 +206,12 @@ def test_workspace_sizes(lib):
     dsp, dsel = dbsa.selection_csr([np.arange(0, 101, 3)])
     wd = dbsa.gather_workspace_size(cfg, doffs, dsp, dsel, 40, 40)
     assert 0 < wd < 8 * int(doffs[-1]) * 256
-    # prepared block keys: K at block-relative positions, bf16 [Hkv][T][D], plus small tables
+    # prepared block keys: K at block-relative positions, bf16 [Hkv][T][D], plus
+    # RoPE tables (cos and sin, D/2 floats a row) for positions below T + 8192:
+    # (T + 8192) / 16 coarse rows and 16 fine rows
     bk = dbsa.block_keys_size(cfg, offs)
-    assert 8 * T * 256 <= bk < 8 * T * 256 + (1 << 20)
+    tables = ((T + 8192) // 16 + 1 + 16) * 64 * 2 * 4
+    assert 8 * T * 256 + tables <= bk < 8 * T * 256 + tables + (1 << 20)
     assert dbsa.block_keys_size(dbsa.DbsaConfig(2, 1, 64, "f32"), offs) >= 2 * T * 128
 
 
