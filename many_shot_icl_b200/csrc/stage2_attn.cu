@@ -469,7 +469,9 @@ __global__ void __launch_bounds__(32 * RT * KG, 1) stage2_attn_kernel(const Stag
 }
 
 // One warp per output row (query q, token u, head h): combine the row's split
-// partials, O = sum_i 2^(M_i - M) L_i O_i / sum_i 2^(M_i - M) L_i.
+// partials, O = sum_i 2^(M_i - M) L_i O_i / sum_i 2^(M_i - M) L_i.  The lanes
+// read the items' (M_i, L_i) in parallel (lane i % 32 holds item i's weight);
+// the items' rows are then added in item order, four loads in flight.
 template <int D, typename OT>
 __global__ void __launch_bounds__(128) stage2_merge_kernel(const Stage2Args a) {
   const int64_t row = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
@@ -480,31 +482,50 @@ __global__ void __launch_bounds__(128) stage2_merge_kernel(const Stage2Args a) {
   const int tok = (int)((row / a.Hq) % a.n_new);
   const int q = (int)(row / ((int64_t)a.Hq * a.n_new));
   const S2Query qi = a.queries[q];
+  const int n = qi.n_items;
+  auto part = [&](int i) { return ((int64_t)(qi.item_begin + i) * a.Hq + h) * a.n_new + tok; };
   float M = -INFINITY;
-  for (int i = 0; i < qi.n_items; ++i) {
-    const int64_t pi = ((int64_t)(qi.item_begin + i) * a.Hq + h) * a.n_new + tok;
-    M = fmaxf(M, a.part_ml[pi].x);
-  }
+  for (int i = lane; i < n; i += 32) M = fmaxf(M, a.part_ml[part(i)].x);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   constexpr int PER = D / 32;
   float acc[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) acc[e] = 0.f;
   float L = 0.f;
-  for (int i = 0; i < qi.n_items; ++i) {
-    const int64_t pi = ((int64_t)(qi.item_begin + i) * a.Hq + h) * a.n_new + tok;
-    const float2 ml = a.part_ml[pi];
-    const float w = (ml.x == -INFINITY) ? 0.f : ex2(ml.x - M) * ml.y;
-    L += w;
-    const uint16_t *src = a.part_acc + pi * D + lane * PER;
-    uint16_t v[PER];
+  auto load_row = [&](int i, uint16_t (&v)[PER]) {
+    const uint16_t *src = a.part_acc + part(i) * D + lane * PER;
     if constexpr (PER == 4) {
       *reinterpret_cast<uint2 *>(v) = *reinterpret_cast<const uint2 *>(src);
     } else {
       *reinterpret_cast<uint32_t *>(v) = *reinterpret_cast<const uint32_t *>(src);
     }
+  };
+  for (int i0 = 0; i0 < n; i0 += 32) {
+    float w = 0.f;
+    if (i0 + lane < n) {
+      const float2 ml = a.part_ml[part(i0 + lane)];
+      w = (ml.x == -INFINITY) ? 0.f : ex2(ml.x - M) * ml.y;
+    }
+    L += w;
+    const int cnt = min(32, n - i0);
+    for (int j = 0; j < cnt; j += 4) {
+      uint16_t v[4][PER];
 #pragma unroll
-    for (int e = 0; e < PER; ++e) acc[e] += w * __uint_as_float((uint32_t)v[e] << 16);
+      for (int k = 0; k < 4; ++k)
+        if (j + k < cnt) load_row(i0 + j + k, v[k]);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float wk = __shfl_sync(0xffffffffu, w, (j + k) & 31);
+        if (j + k < cnt) {
+#pragma unroll
+          for (int e = 0; e < PER; ++e) acc[e] += wk * __uint_as_float((uint32_t)v[k][e] << 16);
+        }
+      }
+    }
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
   const float inv = 1.f / L;
   OT *dst = static_cast<OT *>(a.out) + (((int64_t)q * a.n_new + tok) * a.Hq + h) * D + lane * PER;
 #pragma unroll
