@@ -180,3 +180,51 @@ def test_demonstration_granular_gather(n_new, tail_len):
     run.run().check("demo-granular")
     peaky = Stage2Run(cfg, offs, sels[:2], n_new, tail_len, seed=6, q_scale=4.0).run()
     peaky.check("demo-granular peaky", atol=ATOL_PEAKY)
+
+
+def test_plan_staging_reuse_and_threads():
+    """A call's host-built plan reaches the device through a per-thread ring of
+    eight page-locked staging slots; a slot is refilled only after the read
+    behind its previous use has completed.  Calls that wrap the ring several
+    times with plans of different sizes, and two threads calling at once on
+    their own streams, give the same bits as the first run of each call."""
+    import threading
+    cfg = dbsa.DbsaConfig(8, 2, 128, "bf16", 1e4, 2)
+    rng = np.random.default_rng(77)
+    lens = rng.integers(40, 400, size=9)
+    offs = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    shapes = [([0, 3, 5], 1, 9), ([0, 1, 2, 7, 8], 40, 40), ([0, 6], 3, 7), ([0, 2, 4, 8], 1, 1)]
+
+    def make(seed0):
+        return [Stage2Run(cfg, offs, [np.array(s), np.array(s[:2])], n_new, tail, seed=seed0 + i)
+                for i, (s, n_new, tail) in enumerate(shapes)]
+
+    runs = make(30)
+    first = [r.run().out.clone() for r in runs]
+    for _ in range(3):                      # 12 more calls: the ring wraps
+        for r, want in zip(runs, first):
+            assert torch.equal(r.run().out, want)
+    per_thread = [make(30), make(30)]
+    torch.cuda.synchronize()                # inputs are made on the default stream
+    errors = []
+
+    def worker(rs):
+        try:
+            s = torch.cuda.Stream()
+            with torch.cuda.stream(s):
+                for _ in range(3):
+                    for r in rs:
+                        r.run()
+            s.synchronize()
+        except Exception as e:              # reported below, in the test's thread
+            errors.append(e)
+
+    th = [threading.Thread(target=worker, args=(rs,)) for rs in per_thread]
+    for t in th:
+        t.start()
+    for t in th:
+        t.join()
+    assert not errors, errors
+    for rs in per_thread:
+        for r, want in zip(rs, first):
+            assert torch.equal(r.out, want)
