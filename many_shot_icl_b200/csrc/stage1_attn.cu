@@ -15,19 +15,20 @@
 //               for the V tiles (2-stage ring)
 //   warp 1      TMEM owner; one thread issues O += P V (tcgen05, A from TMEM)
 //   warp 10     one thread issues S = Q K^T (tcgen05, both operands in SMEM)
-//   warps 2..9  softmax, two warpgroups in ping-pong: warpgroup w takes the
-//               tiles whose CTA-wide index has parity w (all 128 keys of
-//               each), one thread per query row (TMEM lane), with its own
-//               fp32 running max and sum (lazy rescale threshold) and its own
-//               O accumulator O_w.  While one warpgroup exponentiates (one
-//               MUFU op per score), the other loads, reduces and stores.  At
-//               an item's end they publish the merge factors of the two
-//               states and go on to the next item.
+//   warps 2..9  softmax, two warpgroups splitting every tile by keys:
+//               warpgroup w takes keys 64w..64w+63 of each tile, one thread
+//               per query row (TMEM lane), with its own fp32 running max and
+//               sum (lazy rescale threshold) and its own O accumulator O_w
+//               (the PV of its half of the keys).  Both halves of a tile are
+//               exponentiated at once, so a tile's P is ready in half the
+//               time one warpgroup would take.  At an item's end they publish
+//               the merge factors of the two states and go on.
 //   warps 11..14 epilogue: combine O_0 and O_1 of the finished item, store
 //               the output, free O for the next item's first PV.
-// S = Q K^T lives in TMEM in two 128-column buffers (tile parity), P is
-// written back over the first 64 columns of its own S buffer as bf16 pairs,
-// and O_0, O_1 take D columns each: 512 columns in all.  Q and K arrive
+// S = Q K^T lives in TMEM in two 128-column buffers (tile parity); each
+// warpgroup writes its 64 keys' P as bf16 pairs over the first 32 columns of
+// its own half of the S buffer, and O_0, O_1 take D columns each: 512 columns
+// in all.  Q and K arrive
 // already rotated (bf16) from the preparation pass; V is read straight from
 // the pre-RoPE cache.  Every wait is bounded and reports DBSA_ERR_TIMEOUT.
 //
@@ -68,8 +69,8 @@ enum Bar {
   B_K_FULL = B_Q_EMPTY + kStagesQ, B_K_EMPTY = B_K_FULL + kStagesK,
   B_V_FULL = B_K_EMPTY + kStagesK, B_V_EMPTY = B_V_FULL + kStagesV,
   B_S_FULL = B_V_EMPTY + kStagesV,  // [buffer]
-  B_P_FULL = B_S_FULL + 2,     // [buffer]: P written by the buffer's warpgroup
-  B_PV_DONE = B_P_FULL + 2,    // [buffer]: PV of the buffer's tile done
+  B_P_FULL = B_S_FULL + 2,     // [buffer][half]: P of keys 64h.. written by warpgroup h
+  B_PV_DONE = B_P_FULL + 4,    // [buffer]: both PV halves of the buffer's tile done
   B_O_FREE = B_PV_DONE + 2, B_DRAIN = B_O_FREE + 1,
   B_ML_A = B_DRAIN + 1,       // end of item: warpgroup 1 has published (m, l)
   B_ML_B = B_ML_A + 1,        // end of item: warpgroup 0 has published the merge factors
@@ -249,7 +250,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar[B_S_FULL + s], 1);
-      mbar_init(&bar[B_P_FULL + s], 128);
+      mbar_init(&bar[B_P_FULL + 2 * s], 128);
+      mbar_init(&bar[B_P_FULL + 2 * s + 1], 128);
       mbar_init(&bar[B_PV_DONE + s], 1);
     }
     mbar_init(&bar[B_O_FREE], 128);
@@ -420,21 +422,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_commit(&bar[B_K_EMPTY + st]);
           if (t == ntiles - 1) mma_commit(&bar[B_Q_EMPTY + qs]);
         } else {
-          // O_b (+)= P V, b = the tile's warpgroup; both accumulators must have
+          // O_h (+)= P_h V_h for the key halves h = 0, 1 of the tile, each as
+          // soon as its warpgroup has written P_h; both accumulators must have
           // been read by the previous item's epilogue before the first PV.
-          // The first tile of each warpgroup in an item (t = 0, 1) starts O_b.
+          // The item's first tile starts O_0 and O_1.
           if (!(ok = wait(B_V_FULL + st, ph))) break;
           if (t == 0 && item_no > 0 && !(ok = wait(B_O_FREE, (item_no - 1) & 1))) break;
-          if (!(ok = wait(B_P_FULL + b, (s_it >> 1) & 1))) break;
-          tc_fence_after();
           const uint64_t dv = dV + st * kTileDesc;
           const uint32_t ta = tmem + COL_S + b * 128;
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            // P: 128 keys packed two per column in the first 64 columns of
-            // the tile's S buffer; 8 columns per 16 keys
-            mma_bf16_ts(tmem + COL_O + b * D, ta + kk * 8, dv + kk * 128, IDESC_PV,
-                        (kk > 0 || t >= 2) ? 1u : 0u);
+          for (int h = 0; h < 2; ++h) {
+            if (!(ok = wait(B_P_FULL + 2 * b + h, (s_it >> 1) & 1))) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              // P_h: keys 64h..64h+63 packed two per column in the first 32
+              // columns of half h of the S buffer; 8 columns per 16 keys
+              mma_bf16_ts(tmem + COL_O + h * D, ta + h * 64 + kk * 8, dv + (4 * h + kk) * 128,
+                          IDESC_PV, (kk > 0 || t > 0) ? 1u : 0u);
+          }
+          if (!ok) break;
           mma_commit(&bar[B_PV_DONE + b]);
           mma_commit(&bar[B_V_EMPTY + st]);
         }
@@ -450,17 +457,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     drain_wait(&bar[drain], 0);
   } else if (warp >= 2 && warp < 2 + kSoftmaxThreads / 32) {
     // ------------------------------------------------------------ softmax
-    // Two warpgroups in ping-pong: warpgroup w takes the tiles whose CTA-wide
-    // index has parity w (all 128 keys of each), with its own running max /
-    // sum and its own O accumulator O_w; the two states are combined once, in
-    // the epilogue.  While one warpgroup exponentiates, the other loads,
-    // reduces and stores, so neither the exponential unit nor the tensor core
-    // waits on a lock-step phase.
+    // Two warpgroups split every tile by keys: warpgroup w takes keys
+    // 64w..64w+63 (its half of the S buffer), with its own running max / sum
+    // and its own O accumulator O_w; the two states are combined once, in
+    // the epilogue.  The two warps that share a row quarter sit on the same SM
+    // sub-partition and exponentiate their halves at once.
     const int wg = (warp - 2) >> 2;
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    const uint32_t col_s = COL_S + wg * 128;
     const uint32_t col_o = COL_O + wg * D;
     const float sl2 = p.scale_log2;
     uint32_t s_it = 0, item_no = 0;
@@ -469,38 +474,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Item it = load_item(p.items, idx);
       const int qpos = it.q_pos0 + row;
       float m_ref = -INFINITY, l = 0.f;
-      uint32_t prev = 0;          // CTA-wide index of this warpgroup's previous tile
-      bool mine_any = false;
+      uint32_t prev = 0;          // CTA-wide index of the previous tile
       for (int t = 0; t < it.ntiles; ++t, ++s_it) {
-        if ((int)(s_it & 1) != wg) continue;
         int r, kt;
         tile_of(it, t, r, kt);
-        ok = __all_sync(kFull, mbar_wait(&bar[B_S_FULL + wg], (s_it >> 1) & 1, abort_flag,
+        const uint32_t col_s = COL_S + (s_it & 1) * 128 + wg * 64;   // this half of S
+        ok = __all_sync(kFull, mbar_wait(&bar[B_S_FULL + (s_it & 1)], (s_it >> 1) & 1, abort_flag,
                                          p.status, kWaitLimitNs, DBSA_ERR_TIMEOUT));
         if (!ok) break;
         tc_fence_after();
         const int klim = (r ? it.len[1] : it.len[0]) - kt;   // valid keys of this tile
         const int kpos0 = (r ? it.pos0[1] : it.pos0[0]) + kt;
         const bool need_mask = klim < 128 || kpos0 + 127 > it.q_pos0;
-        const int klast = min(klim - 1, qpos - kpos0);       // last allowed key of this row
-        // -- pass 1: row maximum over the tile's 128 scores, 64 columns per load
+        // last allowed key of this row, counted from this half's first key
+        const int klast = min(klim - 1, qpos - kpos0) - wg * 64;
+        // -- pass 1: row maximum over this half's 64 scores
         float mt[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll 1
-        for (int c = 0; c < 4; c += 2) {
+        {
           uint32_t va[32], vb[32];
-          tmem_ld32(tmem + lane_off + col_s + c * 32, va);
-          tmem_ld32(tmem + lane_off + col_s + c * 32 + 32, vb);
+          tmem_ld32(tmem + lane_off + col_s, va);
+          tmem_ld32(tmem + lane_off + col_s + 32, vb);
           tmem_wait_ld(va);
           tmem_wait_ld(vb);
           if (need_mask) {
             // masked scores are written back as -inf, so pass 2 needs no mask
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
-              if (c * 32 + e > klast) va[e] = __float_as_uint(-INFINITY);
-              if (c * 32 + 32 + e > klast) vb[e] = __float_as_uint(-INFINITY);
+              if (e > klast) va[e] = __float_as_uint(-INFINITY);
+              if (32 + e > klast) vb[e] = __float_as_uint(-INFINITY);
             }
-            tmem_st32(tmem + lane_off + col_s + c * 32, va);
-            tmem_st32(tmem + lane_off + col_s + c * 32 + 32, vb);
+            tmem_st32(tmem + lane_off + col_s, va);
+            tmem_st32(tmem + lane_off + col_s + 32, vb);
           }
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
@@ -511,14 +515,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (need_mask) tmem_wait_st();
         const float mt_x = max3(mt[0], mt[1], fmaxf(mt[2], mt[3])) * sl2;
-        if (!mine_any) {
+        if (t == 0) {
           m_ref = mt_x;
         } else {
           const bool need = mt_x > m_ref + 8.0f;
           if (__any_sync(kFull, need)) {
-            // O_w must hold this warpgroup's earlier tiles before it is rescaled
-            ok = __all_sync(kFull, mbar_wait(&bar[B_PV_DONE + wg], (prev >> 1) & 1, abort_flag,
-                                             p.status, kWaitLimitNs, DBSA_ERR_TIMEOUT));
+            // O_w must hold the item's earlier tiles before it is rescaled
+            ok = __all_sync(kFull, mbar_wait(&bar[B_PV_DONE + (prev & 1)], (prev >> 1) & 1,
+                                             abort_flag, p.status, kWaitLimitNs,
+                                             DBSA_ERR_TIMEOUT));
             if (!ok) break;
             tc_fence_after();
             const float m_new = fmaxf(m_ref, mt_x);
@@ -537,11 +542,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_wait_st();
           }
         }
-        mine_any = true;
         prev = s_it;
-        // -- pass 2: P = 2^(s * scale - m) as bf16 pairs over S columns 0..63.
-        // Chunk c reads S columns 32c..32c+31 and writes P columns 16c..16c+15,
-        // whose scores were already read.
+        // -- pass 2: P = 2^(s * scale - m) as bf16 pairs over this half's
+        // columns 0..31.  Chunk c reads its columns 32c..32c+31 and writes P
+        // columns 16c..16c+15, whose scores were already read.
         const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
         const f32x2 sc2 = f2_pack(sl2, sl2), nmu2 = f2_pack(-mu, -mu);
         f32x2 sum2[2] = {0ull, 0ull};
@@ -568,25 +572,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tmem_st16(tmem + lane_off + col_s + c * 16, pw);
         };
-#pragma unroll 1
-        for (int c = 0; c < 4; c += 2) {
+        {
           uint32_t va[32], vb[32];
-          tmem_ld32(tmem + lane_off + col_s + c * 32, va);
+          tmem_ld32(tmem + lane_off + col_s, va);
           tmem_wait_ld(va);
-          tmem_ld32(tmem + lane_off + col_s + c * 32 + 32, vb);
-          exp_chunk(va, c);
+          tmem_ld32(tmem + lane_off + col_s + 32, vb);
+          exp_chunk(va, 0);
           tmem_wait_ld(vb);
-          exp_chunk(vb, c + 1);
+          exp_chunk(vb, 1);
         }
         tmem_wait_st();
         float sa, sb2, sc, sd;
         f2_unpack(sum2[0], sa, sb2);
         f2_unpack(sum2[1], sc, sd);
         l += (sa + sb2) + (sc + sd);
-        // The S(t + 2) that next writes this buffer is issued after PV(t), and
-        // the tensor core runs one thread's MMAs in order.
+        // The S(t + 2) that next writes this buffer waits for both PV halves
+        // of this tile.
         tc_fence_before();
-        mbar_arrive(&bar[B_P_FULL + wg]);
+        mbar_arrive(&bar[B_P_FULL + 2 * (s_it & 1) + wg]);
       }
       if (!ok) break;
       // ---- end of item: merge factors for O = (O_0 e^{m_0 - M} + O_1 e^{m_1 - M}) /
@@ -630,8 +633,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // One thread per row (TMEM lane).  Per item: the merge factors, then, once
     // the item's last PV is done (in-order tensor core: so are all of its
     // PVs), O_0 and O_1 are read, combined and stored; O is then free for the
-    // next item's first PV.  A warpgroup without a tile in the item
-    // (single-tile items) left a stale O, which the selects discard.
+    // next item's first PV.
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
@@ -640,11 +642,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x, ++item_no) {
       const Item it = load_item(p.items, idx);
-      const uint32_t s_first = s_it;
       s_it += it.ntiles;
       const uint32_t last = s_it - 1;
-      const bool has0 = it.ntiles >= 2 || (s_first & 1) == 0;
-      const bool has1 = it.ntiles >= 2 || (s_first & 1) == 1;
       ok = __all_sync(kFull, mbar_wait(&bar[B_ML_B], item_no & 1, abort_flag, p.status,
                                        kWaitLimitNs, DBSA_ERR_TIMEOUT));
       if (!ok) break;
@@ -675,8 +674,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (row < it.n_rows) {
 #pragma unroll
           for (int e = 0; e < 32; ++e)
-            o0[e] = __float_as_uint((has0 ? __uint_as_float(o0[e]) * fw.x : 0.f) +
-                                    (has1 ? __uint_as_float(o1[e]) * fw.y : 0.f));
+            o0[e] = __float_as_uint(__uint_as_float(o0[e]) * fw.x + __uint_as_float(o1[e]) * fw.y);
           if (OUT_F32 && !partial) {
             float *dst = static_cast<float *>(p.out) + orow + col;
 #pragma unroll
