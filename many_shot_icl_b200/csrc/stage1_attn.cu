@@ -488,32 +488,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool need_mask = klim < 128 || kpos0 + 127 > it.q_pos0;
         // last allowed key of this row, counted from this half's first key
         const int klast = min(klim - 1, qpos - kpos0) - wg * 64;
-        // -- pass 1: row maximum over this half's 64 scores
-        float mt[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-        {
-          uint32_t va[32], vb[32];
-          tmem_ld32(tmem + lane_off + col_s, va);
-          tmem_ld32(tmem + lane_off + col_s + 32, vb);
-          tmem_wait_ld(va);
-          tmem_wait_ld(vb);
-          if (need_mask) {
-            // masked scores are written back as -inf, so pass 2 needs no mask
+        // -- one pass over this half's 64 scores, held in registers: masked
+        // scores become -inf, the row maximum, the lazy rescale, then
+        // P = 2^(s * scale - m) as bf16 pairs over the half's columns 0..31
+        // (every score is in registers before the first P column is written).
+        uint32_t va[32], vb[32];
+        tmem_ld32(tmem + lane_off + col_s, va);
+        tmem_ld32(tmem + lane_off + col_s + 32, vb);
+        tmem_wait_ld(va);
+        tmem_wait_ld(vb);
+        if (need_mask) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              if (e > klast) va[e] = __float_as_uint(-INFINITY);
-              if (32 + e > klast) vb[e] = __float_as_uint(-INFINITY);
-            }
-            tmem_st32(tmem + lane_off + col_s, va);
-            tmem_st32(tmem + lane_off + col_s + 32, vb);
-          }
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            mt[(e >> 1) & 1] = max3(mt[(e >> 1) & 1], __uint_as_float(va[e]), __uint_as_float(va[e + 1]));
-            mt[2 + ((e >> 1) & 1)] =
-                max3(mt[2 + ((e >> 1) & 1)], __uint_as_float(vb[e]), __uint_as_float(vb[e + 1]));
+          for (int e = 0; e < 32; ++e) {
+            if (e > klast) va[e] = __float_as_uint(-INFINITY);
+            if (32 + e > klast) vb[e] = __float_as_uint(-INFINITY);
           }
         }
-        if (need_mask) tmem_wait_st();
+        float mt[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          mt[(e >> 1) & 1] = max3(mt[(e >> 1) & 1], __uint_as_float(va[e]), __uint_as_float(va[e + 1]));
+          mt[2 + ((e >> 1) & 1)] =
+              max3(mt[2 + ((e >> 1) & 1)], __uint_as_float(vb[e]), __uint_as_float(vb[e + 1]));
+        }
         const float mt_x = max3(mt[0], mt[1], fmaxf(mt[2], mt[3])) * sl2;
         if (t == 0) {
           m_ref = mt_x;
@@ -530,7 +527,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float alpha = (m_new == -INFINITY) ? 1.f : ex2(m_ref - m_new);
             l *= alpha;
             m_ref = m_new;
-#pragma unroll
+#pragma unroll 1
             for (int c = 0; c < D / 32; ++c) {
               uint32_t o[32];
               tmem_ld32(tmem + lane_off + col_o + c * 32, o);
@@ -543,14 +540,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         prev = s_it;
-        // -- pass 2: P = 2^(s * scale - m) as bf16 pairs over this half's
-        // columns 0..31.  Chunk c reads its columns 32c..32c+31 and writes P
-        // columns 16c..16c+15, whose scores were already read.
         const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
         const f32x2 sc2 = f2_pack(sl2, sl2), nmu2 = f2_pack(-mu, -mu);
         f32x2 sum2[2] = {0ull, 0ull};
-        // chunk c of 32 scores -> 16 packed P columns; the next chunk's load is
-        // in flight while this one is exponentiated
+        // chunk c of 32 scores -> 16 packed P columns
         auto exp_chunk = [&](const uint32_t (&v)[32], int c) {
           uint32_t pw[16];
 #pragma unroll
@@ -572,15 +565,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tmem_st16(tmem + lane_off + col_s + c * 16, pw);
         };
-        {
-          uint32_t va[32], vb[32];
-          tmem_ld32(tmem + lane_off + col_s, va);
-          tmem_wait_ld(va);
-          tmem_ld32(tmem + lane_off + col_s + 32, vb);
-          exp_chunk(va, 0);
-          tmem_wait_ld(vb);
-          exp_chunk(vb, 1);
-        }
+        exp_chunk(va, 0);
+        exp_chunk(vb, 1);
         tmem_wait_st();
         float sa, sb2, sc, sd;
         f2_unpack(sum2[0], sa, sb2);
