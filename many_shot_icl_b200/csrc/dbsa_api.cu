@@ -902,6 +902,36 @@ namespace {
 // Stage 2 behind both entry points; block_keys = null rotates the cache keys
 // at block-relative positions into the workspace, else takes them from a
 // dbsa_block_keys() buffer.
+// The last gather plan built on this thread, with the inputs it came from.
+// The layers of one prompt pass or decode step share the cache layout, the
+// selection and the pass shape, so every layer after the first reuses it.
+struct PlanCache {
+  std::vector<int32_t> key;
+  GatherPlan gp;
+  bool valid = false;
+};
+
+// The plan inputs as one array (configuration fields, sizes, offsets and the
+// selection); false if sel_ptr is not a well-formed CSR pointer array, in which
+// case the caller plans afresh (and reports the error).
+bool plan_key(const dbsa_config *cfg, const int32_t *offs, int32_t nb, int32_t nq,
+              const int32_t *sel_ptr, const int32_t *sel, int32_t n_new, int32_t tail_len,
+              std::vector<int32_t> &key) {
+  if (nq < 1 || sel_ptr == nullptr || sel == nullptr || sel_ptr[0] != 0) return false;
+  for (int32_t q = 0; q < nq; ++q)
+    if (sel_ptr[q + 1] <= sel_ptr[q]) return false;
+  if ((int64_t)sel_ptr[nq] > (int64_t)nq * nb) return false;
+  const int32_t head[] = {cfg->n_q_heads, cfg->n_kv_heads, cfg->head_dim, (int32_t)cfg->dtype,
+                          cfg->window_j, cfg->pattern, num_sms(), nb, nq, n_new, tail_len};
+  key.clear();
+  key.reserve(sizeof head / sizeof head[0] + (size_t)nb + 1 + (size_t)nq + 1 + sel_ptr[nq]);
+  key.insert(key.end(), head, head + sizeof head / sizeof head[0]);
+  key.insert(key.end(), offs, offs + nb + 1);
+  key.insert(key.end(), sel_ptr, sel_ptr + nq + 1);
+  key.insert(key.end(), sel, sel + sel_ptr[nq]);
+  return true;
+}
+
 dbsa_status gather_impl(const dbsa_config *cfg, const void *k_cache, const void *v_cache,
                         int64_t cap, const int32_t *offs_host, int32_t nb, int32_t nq,
                         const int32_t *sel_ptr_host, const int32_t *sel_blocks_host,
@@ -922,10 +952,22 @@ dbsa_status gather_impl(const dbsa_config *cfg, const void *k_cache, const void 
   if (offs_host[nb] > cap)
     return fail(DBSA_ERR_CAPACITY, "offsets reach %d rows but cap is %lld", offs_host[nb],
                 (long long)cap);
-  GatherPlan gp;
-  if ((s = gather_plan(cfg, offs_host, nb, nq, sel_ptr_host, sel_blocks_host, n_new, tail_len,
-                       gp)) != DBSA_OK)
-    return s;
+  static thread_local PlanCache cache;
+  static thread_local std::vector<int32_t> key;
+  const bool keyed = plan_key(cfg, offs_host, nb, nq, sel_ptr_host, sel_blocks_host, n_new,
+                              tail_len, key);
+  if (!(keyed && cache.valid && key == cache.key)) {
+    cache.valid = false;
+    cache.gp = GatherPlan();
+    if ((s = gather_plan(cfg, offs_host, nb, nq, sel_ptr_host, sel_blocks_host, n_new, tail_len,
+                         cache.gp)) != DBSA_OK)
+      return s;
+    if (keyed) {
+      cache.key.swap(key);
+      cache.valid = true;
+    }
+  }
+  const GatherPlan &gp = cache.gp;
   if (dbg_map != nullptr) {
     if ((reinterpret_cast<uintptr_t>(dbg_map) & 7u) != 0)
       return fail(DBSA_ERR_INVALID_ARG, "dbg_map must be 8-byte aligned");

@@ -185,9 +185,11 @@ def test_demonstration_granular_gather(n_new, tail_len):
 def test_plan_staging_reuse_and_threads():
     """A call's host-built plan reaches the device through a per-thread ring of
     eight page-locked staging slots; a slot is refilled only after the read
-    behind its previous use has completed.  Calls that wrap the ring several
-    times with plans of different sizes, and two threads calling at once on
-    their own streams, give the same bits as the first run of each call."""
+    behind its previous use has completed, and a thread keeps its last plan
+    for calls with the same inputs.  Calls that wrap the ring several times
+    with plans of different sizes, repeated calls that reuse the kept plan,
+    and two threads calling at once on their own streams give the same bits
+    as the first run of each call."""
     import threading
     cfg = dbsa.DbsaConfig(8, 2, 128, "bf16", 1e4, 2)
     rng = np.random.default_rng(77)
@@ -201,8 +203,10 @@ def test_plan_staging_reuse_and_threads():
 
     runs = make(30)
     first = [r.run().out.clone() for r in runs]
-    for _ in range(3):                      # 12 more calls: the ring wraps
+    for _ in range(3):                      # 24 more calls: the ring wraps
         for r, want in zip(runs, first):
+            # a new plan, then the same plan again (the thread's plan cache)
+            assert torch.equal(r.run().out, want)
             assert torch.equal(r.run().out, want)
     per_thread = [make(30), make(30)]
     torch.cuda.synchronize()                # inputs are made on the default stream
