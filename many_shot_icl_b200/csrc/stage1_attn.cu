@@ -13,7 +13,8 @@
 //   warp 0      TMA producer: two independent cursors, one for each item's Q
 //               tile (double-buffered) and its K tiles (3-stage ring), one
 //               for the V tiles (2-stage ring)
-//   warp 1      TMEM owner; one thread issues O += P V (tcgen05, A from TMEM)
+//   warp 1      TMEM owner; one thread issues O_h += P_h V_h for the two key
+//               halves of each tile (tcgen05, A from TMEM)
 //   warp 10     one thread issues S = Q K^T (tcgen05, both operands in SMEM)
 //   warps 2..9  softmax, two warpgroups splitting every tile by keys:
 //               warpgroup w takes keys 64w..64w+63 of each tile, one thread
@@ -21,16 +22,18 @@
 //               sum (lazy rescale threshold) and its own O accumulator O_w
 //               (the PV of its half of the keys).  Both halves of a tile are
 //               exponentiated at once, so a tile's P is ready in half the
-//               time one warpgroup would take.  At an item's end they publish
-//               the merge factors of the two states and go on.
+//               time one warpgroup would take; each thread makes one pass
+//               over its 64 scores held in registers (mask, max, rescale,
+//               exp2).  At an item's end they publish the merge factors of
+//               the two states and go on.
 //   warps 11..14 epilogue: combine O_0 and O_1 of the finished item, store
 //               the output, free O for the next item's first PV.
 // S = Q K^T lives in TMEM in two 128-column buffers (tile parity); each
 // warpgroup writes its 64 keys' P as bf16 pairs over the first 32 columns of
 // its own half of the S buffer, and O_0, O_1 take D columns each: 512 columns
-// in all.  Q and K arrive
-// already rotated (bf16) from the preparation pass; V is read straight from
-// the pre-RoPE cache.  Every wait is bounded and reports DBSA_ERR_TIMEOUT.
+// in all.  Q and K arrive already rotated (bf16) from the preparation pass; V
+// is read straight from the pre-RoPE cache.  Every wait is bounded and
+// reports DBSA_ERR_TIMEOUT.
 //
 // Measured on B200: the tensor core runs a 128x128x16
 // MMA in 64 cycles but keeps only about one MMA queued, so the issuing
