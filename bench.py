@@ -277,7 +277,7 @@ def e2e_step_time(wl: Workload, host, steps: int):
     gc.collect()
     gc_on = gc.isenabled()
     gc.disable()
-    for _ in range(steps):
+    for i in range(steps + 1):                  # step 0 warms up, untimed
         torch.cuda.synchronize()
         e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
         e0.record(comp)
@@ -345,8 +345,9 @@ def e2e_step_time(wl: Workload, host, steps: int):
         comp.wait_stream(s_out)
         e2.record(comp)
         torch.cuda.synchronize()
-        t1 += e0.elapsed_time(e1) / 1e3
-        t2 += e1.elapsed_time(e2) / 1e3
+        if i > 0:
+            t1 += e0.elapsed_time(e1) / 1e3
+            t2 += e1.elapsed_time(e2) / 1e3
     if gc_on:
         gc.enable()
     return t1 / steps, t2 / steps
@@ -682,7 +683,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=inputs.L31_8B_90K.name)
     ap.add_argument("--layers", type=int, default=None, help="override the layer count")
-    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--appends", type=int, default=None)
     ap.add_argument("--cpu-budget", type=float, default=16.0)
     ap.add_argument("--ref-budget", type=float, default=60.0)
