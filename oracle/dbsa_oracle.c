@@ -21,7 +21,7 @@
  * No blocking, no fusion, no reordering: every output row is computed on
  * its own from its explicit boolean mask row.
  *
- * Readings of points the page leaves open (each is listed in the design doc):
+ * Readings of points the page leaves open:
  *   - positions are token positions (not demo indices), 0..T-1 in Stage 1
  *     and 0..T'-1 over the gathered tokens in Stage 2;
  *   - query / tail tokens continue after the gathered cache: T' + u;
