@@ -386,6 +386,10 @@ dbsa_status gather_plan(const dbsa_config *cfg, const int32_t *offs, int32_t nb,
   for (int q = 0; q < nq; ++q) {
     const int32_t a = sel_ptr[q], e = sel_ptr[q + 1];
     if (e <= a) return fail(DBSA_ERR_INVALID_ARG, "query %d selects no block", q);
+    // distinct blocks only, so at most nb: checked before sel is read
+    if ((int64_t)e - a > nb)
+      return fail(DBSA_ERR_INVALID_ARG, "query %d selects %lld blocks of %d", q,
+                  (long long)e - a, nb);
     if (sel[a] != 0) return fail(DBSA_ERR_INVALID_ARG, "query %d: first block must be the sink (0)", q);
     S2Query qi;
     std::memset(&qi, 0, sizeof qi);

@@ -133,6 +133,10 @@ def test_invalid_arguments_are_rejected_before_device_work(lib):
     assert gather(ok_cfg, [0, 3], [0, 2, 2]) == dbsa.ERR_INVALID_ARG    # duplicate
     assert gather(ok_cfg, [0, 2], [0, 3]) == dbsa.ERR_INVALID_ARG       # out of range
     assert gather(ok_cfg, [0, 0], []) == dbsa.ERR_INVALID_ARG           # empty selection
+    assert gather(ok_cfg, [0, 2, 1], [0, 1]) == dbsa.ERR_INVALID_ARG    # sel_ptr decreases
+    # more blocks than exist: rejected before sel (one entry here) is read past its end
+    assert gather(ok_cfg, [0, 1 << 30], [0]) == dbsa.ERR_INVALID_ARG
+    assert "blocks of 3" in dbsa.last_error()
     assert gather(ok_cfg, [0, 1], [0], n_new=3, tail_len=2) == dbsa.ERR_INVALID_ARG
     assert gather(ok_cfg, [0, 1], [0], tail_len=5, tail_cap=4) == dbsa.ERR_INVALID_ARG
     assert gather(ok_cfg, [0, 1], [0], cap=10) == dbsa.ERR_CAPACITY
