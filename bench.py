@@ -133,6 +133,12 @@ def inputs_offsets(w):
     return dbsa.group_blocks(inputs.demo_lengths(w), w.demos_per_block)
 
 
+def oracle_offsets(w):
+    """The block table as the oracle builds it (the CPU legs load no library)."""
+    import oracle
+    return oracle.group_blocks(inputs.demo_lengths(w), w.demos_per_block)
+
+
 def stage1_exact_pairs(offs, j):
     """sum over rows of allowed keys: (t - offs[b] + 1) + lengths of the distinct
     blocks {0} U {max(0, b-j) .. b-1} (bench accounting only)."""
@@ -142,6 +148,55 @@ def stage1_exact_pairs(offs, j):
         others = set(range(max(0, b - j), b)) | ({0} if b > 0 else set())
         total += L * (L + 1) // 2 + L * int(sum(lens[x] for x in others))
     return total
+
+
+# ------------------------------------------------------------------ accounting
+class Stage2Work:
+    """Stage-2 algorithmic work of one layer call (bench bookkeeping only):
+      flop  = 4 D per (row, visible key): row (q, h, u) sees T'_q gathered
+              keys and its own tail tokens up to itself;
+      unique bytes = K/V of the union of selected blocks (what must cross HBM
+              at least once) + tail K/V + Q + O;
+      per-query bytes = K/V of every query's own gathered cache (what a
+              per-query streaming kernel reads; shared blocks count again)."""
+
+    def __init__(self, wl):
+        w = wl.w
+        # plain numbers only: no reference to the workload's device tensors
+        self.T, self.nq, self.passes = wl.T, wl.nq, wl.passes()
+        self.D, self.Hq, self.Hkv = w.head_dim, w.n_q_heads, w.n_kv_heads
+        self.bpe = 2 if w.dtype == "bf16" else 4
+        self.gath = wl.gathered()
+        self.union_tokens = float(sum(int(wl.offs[b + 1] - wl.offs[b])
+                                      for b in sorted(set(int(x) for s_ in wl.sels for x in s_))))
+
+    def flop(self, n_new, tail_len):
+        per_q = n_new * (self.gath + tail_len - n_new + 1) + n_new * (n_new - 1) / 2.0
+        return 4.0 * self.D * self.Hq * float(per_q.sum())
+
+    def small_bytes(self, n_new, tail_len):
+        nq = float(self.nq)
+        return (nq * tail_len * self.Hkv * self.D * self.bpe * 2 +
+                nq * n_new * self.Hq * self.D * self.bpe * 2)
+
+    def unique_bytes(self, n_new, tail_len):
+        return self.union_tokens * self.Hkv * self.D * self.bpe * 2 + self.small_bytes(n_new, tail_len)
+
+    def perquery_bytes(self, n_new, tail_len):
+        return float(self.gath.sum()) * self.Hkv * self.D * self.bpe * 2 + \
+            self.small_bytes(n_new, tail_len)
+
+    def block_keys_bytes(self):
+        """dbsa_block_keys: every cache key read once, its rotated bf16 copy written."""
+        return float(self.T) * self.Hkv * self.D * (self.bpe + 2)
+
+    def bound_s(self, peak_tf, peak_bw):
+        """Roofline time of one layer's Stage 2: per pass the slower of its
+        tensor-core time and its unique-byte HBM time, plus the block-key pass."""
+        t = self.block_keys_bytes() / (peak_bw * 1e9)
+        for n, tl in self.passes:
+            t += max(self.flop(n, tl) / (peak_tf * 1e12), self.unique_bytes(n, tl) / (peak_bw * 1e9))
+        return t
 
 
 # ------------------------------------------------------------------ clocks
@@ -195,10 +250,14 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ our arm
-def run_step(wl: Workload, prof=None):
-    """One step; if prof is given, per-call kernel events are appended to it."""
+def run_step(wl: Workload, prof=None, stage_ev=None):
+    """One step; if prof is given, per-call kernel events are appended to it,
+    and if stage_ev is given (three timing events) they are recorded before
+    Stage 1, between the stages and after Stage 2."""
     import torch
     from many_shot_icl_b200 import dbsa
+    if stage_ev is not None:
+        stage_ev[0].record()
     for l in range(wl.layers):
         if prof is not None:
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -206,6 +265,8 @@ def run_step(wl: Workload, prof=None):
             prof["s1"].append((e0, e1))
         dbsa.encode_blocks(wl.cfg, wl.q[l], wl.k[l], wl.v[l], wl.offs, wl.kc[l], wl.vc[l],
                            wl.out[l], wl.ws)
+    if stage_ev is not None:
+        stage_ev[1].record()
     for l in range(wl.layers):
         dbsa.block_keys(wl.cfg, wl.kc[l], wl.vc[l], wl.offs, wl.bk[l])
     for n_new, tail_len in wl.passes():
@@ -219,29 +280,8 @@ def run_step(wl: Workload, prof=None):
             dbsa.gather_rope_attend(wl.cfg, wl.kc[l], wl.vc[l], wl.offs, wl.sel_ptr, wl.sel, qn,
                                     wl.kt[l], wl.vt[l], tail_len, out, wl.ws,
                                     block_keys=wl.bk[l])
-
-
-def stage_times(wl: Workload):
-    """Device time of Stage 1 and Stage 2 of one step, measured separately."""
-    import torch
-    from many_shot_icl_b200 import dbsa
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
-    ev[0].record()
-    for l in range(wl.layers):
-        dbsa.encode_blocks(wl.cfg, wl.q[l], wl.k[l], wl.v[l], wl.offs, wl.kc[l], wl.vc[l],
-                           wl.out[l], wl.ws)
-    ev[1].record()
-    for l in range(wl.layers):
-        dbsa.block_keys(wl.cfg, wl.kc[l], wl.vc[l], wl.offs, wl.bk[l])
-    for n_new, tail_len in wl.passes():
-        for l in range(wl.layers):
-            qn, out = (wl.qp[l], wl.out_p) if n_new > 1 else (wl.qd[l], wl.out_d)
-            dbsa.gather_rope_attend(wl.cfg, wl.kc[l], wl.vc[l], wl.offs, wl.sel_ptr, wl.sel, qn,
-                                    wl.kt[l], wl.vt[l], tail_len, out, wl.ws,
-                                    block_keys=wl.bk[l])
-    ev[2].record()
-    torch.cuda.synchronize()
-    return ev[0].elapsed_time(ev[1]) / 1e3, ev[1].elapsed_time(ev[2]) / 1e3
+    if stage_ev is not None:
+        stage_ev[2].record()
 
 
 def e2e_step_time(wl: Workload, host, steps: int):
@@ -554,6 +594,66 @@ def comparators(wl: Workload, n_ret_queries: int = 4):
                                    "path": "per-query split (segments shorter than a key tile)"}}
 
 
+# ------------------------------------------------------------------ other workloads
+PER_CONFIG = (
+    ("llama2-7b-30k", {}),
+    ("llama3.1-8b-128k", {}),
+    ("llama3.1-8b-128k", {"window_j": 4}),
+    ("llama3.1-8b-128k", {"order": "ascending"}),
+)
+
+
+def per_config(peaks, peak_src, layers_timed=2, warmup=3, reps=3):
+    """The whole step (Stage 1, then Stage 2) on the other shaped workloads,
+    device-timed with CUDA events.  Layers are identical in shape and
+    independent, so `layers_timed` distinct seeded layers are timed and the
+    throughput is T (or the batch's query tokens) per (time per layer x the
+    workload's layer count)."""
+    import torch
+    from many_shot_icl_b200 import dbsa
+    peak_tf = peaks.get("bf16_tflops_sustained", PEAKS_FALLBACK["bf16_tflops_sustained"])
+    peak_bw = peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
+    res = {}
+    for name, over in PER_CONFIG:
+        w = inputs.WORKLOADS[name].with_(**over)
+        L = min(layers_timed, w.n_layers)
+        wl = Workload(w, L, "cuda")
+        for _ in range(warmup):
+            run_step(wl)
+        torch.cuda.synchronize()
+        prof = {"s1": [], "s2p": [], "s2d": []}
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(reps)]
+        for i in range(reps):
+            run_step(wl, prof, evs[i])
+        torch.cuda.synchronize()
+        t1 = sum(e[0].elapsed_time(e[1]) for e in evs) / 1e3 / reps / L   # per layer
+        t2 = sum(e[1].elapsed_time(e[2]) for e in evs) / 1e3 / reps / L
+        s1_ms = float(np.mean([a.elapsed_time(b) for a, b in prof["s1"]]))
+        exact = 4.0 * w.head_dim * w.n_q_heads * stage1_exact_pairs(wl.offs, w.window_j)
+        s2w = Stage2Work(wl)
+        bound = s2w.bound_s(peak_tf, peak_bw)
+        q_tokens = wl.nq * (w.query_tokens + w.decode_steps)
+        key = "%s j%d %s" % (name, w.window_j, w.order)
+        res[key] = {
+            "layers": w.n_layers, "layers_timed": L, "context_tokens": wl.T, "blocks": wl.nb,
+            "window_j": w.window_j, "order": w.order, "queries": wl.nq,
+            "query_tokens": w.query_tokens, "decode_steps": w.decode_steps,
+            "mean_gathered_tokens": float(s2w.gath.mean()),
+            "stage1_tok_s": round(wl.T / (t1 * w.n_layers), 1),
+            "stage1_kernel_ms_per_layer": round(s1_ms, 4),
+            "stage1_exact_pair_tflops": round(exact / (s1_ms * 1e-3) / 1e12, 1),
+            "stage1_frac": round(exact / (s1_ms * 1e-3) / 1e12 / peak_tf, 4),
+            "stage2_query_tok_s": round(q_tokens / (t2 * w.n_layers), 1),
+            "stage2_ms_per_layer": round(t2 * 1e3, 4),
+            "stage2_bound_ms_per_layer": round(bound * 1e3, 4),
+            "stage2_frac_of_bound": round(bound / t2, 4),
+            "peak": {"bf16_tflops_sustained": peak_tf, "hbm_gbs": peak_bw, "source": peak_src},
+        }
+        del wl
+        torch.cuda.empty_cache()
+    return res
+
+
 # ------------------------------------------------------------------ oracle timing
 def oracle_sample(w: inputs.Workload, budget_s: float, threads: int | None = None):
     """Time the oracle on a bounded sample of the workload (layer 0 inputs):
@@ -561,7 +661,7 @@ def oracle_sample(w: inputs.Workload, budget_s: float, threads: int | None = Non
     Returns (stage-1 tok/s, stage-2 query tok/s, cores, sample description)."""
     import torch
     import oracle
-    offs = inputs_offsets(w)
+    offs = oracle_offsets(w)
     T = int(offs[-1])
     Hq, Hkv, D = w.n_q_heads, w.n_kv_heads, w.head_dim
     q = inputs.randn((T, Hq, D), inputs.tensor_seed(w, 0, 0), w.dtype).float().numpy()
@@ -666,7 +766,7 @@ def run_reference(args, world, rank):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": wall / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": {"workload": w.name, "layers": w.n_layers,
-                                            "context_tokens": int(inputs_offsets(w)[-1])},
+                                            "context_tokens": int(oracle_offsets(w)[-1])},
             "stage2_query_tok_s": s2,
             "cpu_baseline": {"value": s1, "unit": "tok/s", "cores": cores, "kind": "oracle",
                              "sample": desc},
@@ -690,6 +790,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-compare", action="store_true",
                     help="skip the retrieval-ICL / fixed-ICL attention comparators")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the 30k and 128k workload measurements")
     ap.add_argument("--profile-only", choices=["stage1", "stage2"], default=None,
                     help="run W + K steps of one stage only and exit (for ncu captures)")
     args = ap.parse_args()
@@ -730,9 +832,11 @@ def main():
         barrier(world)
         torch.cuda.synchronize()
         e_start, e_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        step_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)]
+                   for _ in range(args.steps)]
         e_start.record()
-        for _ in range(args.steps):
-            run_step(wl, prof)
+        for i in range(args.steps):
+            run_step(wl, prof, step_ev[i])
         e_stop.record()
         torch.cuda.synchronize()
         barrier(world)
@@ -741,8 +845,9 @@ def main():
     step_s_max = max_over_ranks(step_s, world)
     clocks = clk.summary()
 
-    # split of one step into its two stages (separate timed pass)
-    t_s1, t_s2 = stage_times(wl)
+    # each timed step's two stages, from the events recorded inside it
+    t_s1 = sum(ev[0].elapsed_time(ev[1]) for ev in step_ev) / 1e3 / args.steps
+    t_s2 = sum(ev[1].elapsed_time(ev[2]) for ev in step_ev) / 1e3 / args.steps
     t_s1 = max_over_ranks(t_s1, world)
     t_s2 = max_over_ranks(t_s2, world)
 
@@ -752,32 +857,8 @@ def main():
     tile_flop = 4.0 * 128 * 128 * D * tiles                      # per layer, unmasked tiles
     exact_flop = 4.0 * D * Hq * stage1_exact_pairs(wl.offs, w.window_j)  # per layer
     gath = wl.gathered()
-    bpe = 2 if w.dtype == "bf16" else 4
-
-    # Stage-2 accounting per layer call (bench bookkeeping only):
-    #  flop  = 4 D per (row, visible key): row (q, h, u) sees T'_q gathered
-    #          keys and its own tail tokens up to itself;
-    #  unique bytes = K/V of the union of selected blocks (what must cross HBM
-    #          at least once) + tail K/V + Q + O;
-    #  per-query bytes = K/V of every query's own gathered cache (what a
-    #          per-query streaming kernel reads; shared blocks count again).
-    union_tokens = float(sum(int(wl.offs[b + 1] - wl.offs[b])
-                             for b in sorted(set(int(x) for s_ in wl.sels for x in s_))))
-
-    def s2_flop(n_new, tail_len):
-        per_q = n_new * (gath + tail_len - n_new + 1) + n_new * (n_new - 1) / 2.0
-        return 4.0 * D * Hq * float(per_q.sum())
-
-    def s2_small_bytes(n_new, tail_len):
-        tail = float(wl.nq) * tail_len * Hkv * D * bpe * 2
-        qo = float(wl.nq) * n_new * Hq * D * bpe * 2
-        return tail + qo
-
-    def s2_unique_bytes(n_new, tail_len):
-        return union_tokens * Hkv * D * bpe * 2 + s2_small_bytes(n_new, tail_len)
-
-    def s2_perquery_bytes(n_new, tail_len):
-        return float(gath.sum()) * Hkv * D * bpe * 2 + s2_small_bytes(n_new, tail_len)
+    s2w = Stage2Work(wl)
+    s2_flop, s2_unique_bytes, s2_perquery_bytes = s2w.flop, s2w.unique_bytes, s2w.perquery_bytes
 
     def mean_ms(pairs):
         return float(np.mean([a.elapsed_time(b) for a, b in pairs])) if pairs else float("nan")
@@ -812,13 +893,18 @@ def main():
                       "peak_kind": "copy (unique bytes), " + peak_src})
         return r
 
+    # achieved = the method's own work (4 D flop per allowed (query, key) pair,
+    # every head) per launch / launch time; the flops of every evaluated
+    # 128 x 128 tile (masked padding included) are reported beside it
     roof_s1 = {"kernel": "stage1_attn_kernel (tcgen05)", "bound": "tensor",
-               "achieved": round(s1_tflops, 1), "peak": peak_tf, "unit": "TFLOP/s",
-               "frac": round(s1_tflops / peak_tf, 4), "traffic": None,
+               "achieved": round(s1_exact_tflops, 1), "peak": peak_tf, "unit": "TFLOP/s",
+               "frac": round(s1_exact_tflops / peak_tf, 4), "traffic": None,
                "peak_kind": "sustained bf16, " + peak_src,
-               "frac_of_burst_peak": round(s1_tflops / peak_tf_burst, 4),
-               "exact_pair_tflops": round(s1_exact_tflops, 1),
-               "flop_per_launch": tile_flop, "launch_ms": round(s1_ms, 4)}
+               "frac_of_burst_peak": round(s1_exact_tflops / peak_tf_burst, 4),
+               "flop_per_launch": exact_flop, "launch_ms": round(s1_ms, 4),
+               "evaluated_tile_tflops": round(s1_tflops, 1),
+               "evaluated_tile_frac": round(s1_tflops / peak_tf, 4),
+               "evaluated_tile_flop_per_launch": tile_flop}
     roof_s2p = pass_roofline("stage1_attn_kernel, partial mode (block-major tcgen05, prompt pass)",
                              p_pass[:1], s2p_ms)
     roof_s2d = (pass_roofline("stage1_attn_kernel, partial mode (block-major tcgen05, decode step)",
@@ -840,6 +926,7 @@ def main():
     s2_tok_s = weak_scaling_value(q_tokens, world, t_s2)
 
     # end to end from pinned host memory (rank-local)
+    host = None
     if args.e2e_steps > 0:
         host = pinned_host_buffers(wl)
         e2e_t1, e2e_t2 = e2e_step_time(wl, host, args.e2e_steps)
@@ -870,6 +957,26 @@ def main():
             comp["fixed_icl"]["inference_s_per_query"] / comp["retrieval_icl"]["inference_s_per_query"]
         comp["setup_ratio_dbsa_over_fixed_icl"] = t_s1 / comp["fixed_icl"]["setup_s"]
 
+    config = {"workload": w.name, "layers": layers, "context_tokens": T,
+              "blocks": wl.nb, "window_j": w.window_j, "q_heads": Hq, "kv_heads": Hkv,
+              "head_dim": D, "queries": wl.nq, "query_tokens": w.query_tokens,
+              "decode_steps": w.decode_steps,
+              "retrieved_blocks_per_query": int(len(wl.sels[0]) - 1),
+              "mean_gathered_tokens": float(gath.mean()),
+              "parallelism": "dp%d (independent batch per GPU)" % world,
+              "l2": "inputs larger than L2 (per-layer Q/K/V/O ~%.1f GB)" %
+                    ((wl.q[0].numel() * 2 + wl.k[0].numel() * 2 + wl.v[0].numel() * 2) * elt / 1e9)}
+
+    # the other shaped workloads (N = 1 only; the main workload's tensors are
+    # released first)
+    s2_bound = s2w.bound_s(peak_tf, peak_bw) * layers
+    pc = None
+    if rank == 0 and world == 1 and not args.no_per_config:
+        del wl
+        host = None
+        torch.cuda.empty_cache()
+        pc = per_config(peaks, peak_src)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         c1, c2, cores, desc, _ = oracle_sample(w, args.cpu_budget)
@@ -882,19 +989,15 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_s_max * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
             "data": "synthetic",
-            "config": {"workload": w.name, "layers": layers, "context_tokens": T,
-                       "blocks": wl.nb, "window_j": w.window_j, "q_heads": Hq, "kv_heads": Hkv,
-                       "head_dim": D, "queries": wl.nq, "query_tokens": w.query_tokens,
-                       "decode_steps": w.decode_steps,
-                       "retrieved_blocks_per_query": int(len(wl.sels[0]) - 1),
-                       "mean_gathered_tokens": float(gath.mean()),
-                       "parallelism": "dp%d (independent batch per GPU)" % world,
-                       "l2": "inputs larger than L2 (per-layer Q/K/V/O ~%.1f GB)" %
-                             ((wl.q[0].numel() * 2 + wl.k[0].numel() * 2 + wl.v[0].numel() * 2) * elt / 1e9)},
+            "config": config,
             "value_definition": "context tokens encoded through all layers per second of Stage-1 time",
             "stage1": {"tok_s": round(s1_tok_s, 1), "s_per_step": round(t_s1, 4)},
             "stage2": {"query_tok_s": round(s2_tok_s, 1), "s_per_step": round(t_s2, 4),
-                       "query_tokens_per_step": q_tokens},
+                       "query_tokens_per_step": q_tokens,
+                       "bound_s_per_step": round(s2_bound, 4),
+                       "frac_of_bound": round(s2_bound / t_s2, 4),
+                       "bound_definition": "per layer: block-key pass bytes / HBM peak + per pass "
+                                           "max(flop / sustained bf16 peak, unique bytes / HBM peak)"},
             "roofline": roof,
             "rooflines": {k: v for k, v in by_name.items() if v is not None},
             "kernel_ms_per_step": {k: round(v, 2) for k, v in shares.items()},
@@ -907,6 +1010,7 @@ def main():
             "cpu_baseline": cpu,
             "append": app,
             "comparators": comp,
+            "per_config": pc,
             "clocks": clocks,
             "gpu_launches": int(launches / args.steps),
             "gpu_launches_timed_region": int(launches),

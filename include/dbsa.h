@@ -79,7 +79,7 @@ typedef enum dbsa_pattern {
 
 typedef struct dbsa_config {
     int32_t n_q_heads;     /* Hq */
-    int32_t n_kv_heads;    /* Hkv; Hq % Hkv == 0 and Hq / Hkv <= 16 */
+    int32_t n_kv_heads;    /* Hkv; Hq % Hkv == 0 and Hq / Hkv <= 64 */
     int32_t head_dim;      /* D: 64 or 128 */
     int32_t dtype;         /* dbsa_dtype */
     double rope_theta;     /* RoPE base, e.g. 1e4 (Llama-2) or 5e5 (Llama-3.1) */
@@ -178,10 +178,21 @@ dbsa_status dbsa_append_block(const dbsa_config *cfg, const void *q,
  *                               of the tail_len tokens are q_new's tokens
  *                               (the caller writes them before the call)
  *   out      device, [nq][n_new][Hq][D]
- *   dbg_map  device or NULL, [nq][dbg_cap][2] int32: when given, receives
- *                               for every gathered token p of query q the
- *                               pair (cache row, fresh position p), as read
- *                               by the kernel (rows p >= T'_q untouched)
+ *   dbg_map  device or NULL, [nq][dbg_cap][2] int32, 8-byte aligned: when
+ *                               given, entry [q][p] receives, for every
+ *                               gathered token p of query q, the pair (cache
+ *                               row, position) written by the attention
+ *                               kernel that consumes that key: the cache row
+ *                               its K and V were loaded from (-2 if the two
+ *                               differ) and the fresh position its rotation
+ *                               used.  On the block-by-block tensor-core path
+ *                               that position is the query's token-0
+ *                               position minus the position the query rows
+ *                               were rotated at, plus the key's offset
+ *                               inside its block; on the per-query path it is
+ *                               the position of the rotation table entries
+ *                               applied.  Correct results have position p.
+ *                               Entries p >= T'_q are untouched.
  *
  * Query q's gathered cache is the concatenation of its selected blocks'
  * tokens; gathered token p gets position p (0 .. T'_q-1).  Query token u
@@ -256,8 +267,9 @@ dbsa_status dbsa_gather_rope_attend_prepared(
  * code that runs inside another framework's fixed memory budget or a host
  * thread that must not call cudaMalloc (it may synchronise the device).
  * Same arguments, results and errors as dbsa_gather_rope_attend, minus the
- * workspace.  The scratch is one array of 16 MiB in the library's device
- * memory, held by every GPU that loads the library until the process exits.
+ * workspace; the outputs are bit-identical to that call's.  The scratch is
+ * one array of 16 MiB in the library's device memory, held by every GPU that
+ * loads the library until the process exits.
  *  - A batch whose dbsa_gather_workspace_size() exceeds 16 MiB is rejected
  *    with DBSA_ERR_WORKSPACE and a message naming both sizes; nothing runs.
  *  - The first call on a device looks up the array's device address (with
@@ -267,8 +279,12 @@ dbsa_status dbsa_gather_rope_attend_prepared(
  *    behind; the call clears the status word it needs at zero.  Calls whose
  *    work overlaps on the GPU (other streams, other host threads) race on the
  *    array: serialise them.
- *  - dbsa_read_status() does not apply (there is no caller workspace).
- * It allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ *  - Its device status word is read with dbsa_noalloc_read_status(), not
+ *    dbsa_read_status() (there is no caller workspace).
+ * It allocates nothing: no cudaMalloc, cudaFree, page-locked host memory,
+ * event or other allocating library call.  Its plan tables reach the device
+ * with one cudaMemcpyAsync from pageable host memory, which returns once the
+ * driver has taken the bytes (it may wait for the stream's earlier copies).
  * ------------------------------------------------------------------------ */
 dbsa_status dbsa_gather_rope_attend_noalloc(
     const dbsa_config *cfg, const void *k_cache, const void *v_cache,
@@ -290,6 +306,28 @@ const char *dbsa_last_error(void);
  * DBSA_ERR_CUDA if the copy failed.  The word is cleared by each call that
  * uses the workspace. */
 dbsa_status dbsa_read_status(const void *workspace, void *stream);
+
+/* The same for the scratch of dbsa_gather_rope_attend_noalloc on the current
+ * device: synchronises `stream` and returns the status word its last call
+ * left (DBSA_OK or DBSA_ERR_TIMEOUT), or DBSA_ERR_CUDA. */
+dbsa_status dbsa_noalloc_read_status(void *stream);
+
+/* Test hook of the failure detection, for the NEXT call on this thread only
+ * (0 = no hook).  Every device wait of the tensor-core kernel is bounded (4 s
+ * by default); when one runs out, the kernel writes DBSA_ERR_TIMEOUT to the
+ * status word, finishes its copies and tensor-core work in flight, releases
+ * its tensor memory and returns, leaving the context usable.  With the hook,
+ * that call's kernel loads no tile, so each of its waits is for a barrier
+ * that nothing completes, and they give up after `limit_ns` nanoseconds: the
+ * call's status reads DBSA_ERR_TIMEOUT and its outputs are incomplete.
+ * Cleared by the call.  For tests only. */
+void dbsa_test_wait_expiry(uint64_t limit_ns);
+
+/* Calls this library has made (all threads) that allocate or free
+ * page-locked host memory or create or destroy CUDA events: the plan staging
+ * of the workspace-taking calls, on a thread's first calls and when a plan
+ * outgrows its slot.  dbsa_gather_rope_attend_noalloc makes none. */
+int64_t dbsa_host_allocation_calls(void);
 
 /* One Stage-1 tile-list entry: a 128-row query tile of one head, and at most
  * two key ranges (the sink block, then the window up to the diagonal). */

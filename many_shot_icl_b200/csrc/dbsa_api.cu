@@ -17,7 +17,21 @@ using namespace dbsa;
 namespace {
 
 thread_local std::string g_err;
+// Calls this library made that allocate or free page-locked host memory or
+// create or destroy events (each can synchronise the device).
+std::atomic<int64_t> g_host_alloc_calls{0};
+void count_host_alloc() { g_host_alloc_calls.fetch_add(1, std::memory_order_relaxed); }
 thread_local cudaEvent_t g_prof_start = nullptr, g_prof_stop = nullptr;
+// Test hook for the next call on this thread (dbsa_test_wait_expiry): its
+// tensor-core kernel loads no tile and its waits give up after this many
+// nanoseconds (0: no hook).
+thread_local uint64_t g_wait_expiry_ns = 0;
+
+uint64_t take_wait_expiry() {
+  const uint64_t w = g_wait_expiry_ns;
+  g_wait_expiry_ns = 0;
+  return w;
+}
 std::atomic<int64_t> g_launches{0};
 
 void count_launches(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
@@ -88,8 +102,12 @@ class StagingRing {
       if (s.ev != nullptr) {
         cudaEventSynchronize(s.ev);
         cudaEventDestroy(s.ev);
+        count_host_alloc();
       }
-      if (s.p != nullptr) cudaFreeHost(s.p);
+      if (s.p != nullptr) {
+        cudaFreeHost(s.p);
+        count_host_alloc();
+      }
     }
   }
   // A page-locked buffer of >= bytes for the next upload (waits for the
@@ -103,20 +121,26 @@ class StagingRing {
       if ((e = cudaEventSynchronize(s.ev)) != cudaSuccess) return e;
       if (s.dev != dev) {
         cudaEventDestroy(s.ev);
+        count_host_alloc();
         s.ev = nullptr;
       }
     }
     if (s.cap < bytes) {
-      if (s.p != nullptr) cudaFreeHost(s.p);  // its last read has completed
+      if (s.p != nullptr) {
+        cudaFreeHost(s.p);  // its last read has completed
+        count_host_alloc();
+      }
       s.p = nullptr;
       const size_t cap = align_up(std::max(bytes, 2 * s.cap), size_t(1) << 16);
       s.cap = 0;
+      count_host_alloc();
       if ((e = cudaHostAlloc(&s.p, cap, cudaHostAllocPortable | cudaHostAllocMapped)) !=
           cudaSuccess)
         return e;
       s.cap = cap;
     }
     if (s.ev == nullptr) {
+      count_host_alloc();
       if ((e = cudaEventCreateWithFlags(&s.ev, cudaEventDisableTiming)) != cudaSuccess) return e;
       s.dev = dev;
     }
@@ -546,7 +570,7 @@ S1Layout s1_layout(const dbsa_config *cfg, int64_t max_pos, int64_t n_items, int
 
 struct S2Layout {
   size_t rope, queries, segs, items, run_items, packed_items, item_row0,
-      tc_tiles, offs, blob_end, k_hat, v_hat, q_hat, part_acc, part_ml, total;
+      tc_tiles, offs, blob_end, q_rot_pos, k_hat, v_hat, q_hat, part_acc, part_ml, total;
   int32_t n_hi;
 };
 // prepared: the block-relative keys (and bf16 V of fp32 caches) come from a
@@ -566,6 +590,7 @@ S2Layout s2_layout(const dbsa_config *cfg, const GatherPlan &gp, int32_t n_new,
   l.tc_tiles = cv.take(gp.tc_tiles.size() * sizeof(dbsa_tile_item));
   l.offs = cv.take((size_t)(offs_count(gp)) * sizeof(int32_t));
   l.blob_end = cv.take(0);
+  l.q_rot_pos = cv.take(gp.items.size() * sizeof(int32_t));
   const int64_t T = gp.cache_rows;
   const bool own_keys = !prepared && !gp.per_query;
   l.k_hat = cv.take(own_keys ? (size_t)cfg->n_kv_heads * T * cfg->head_dim * 2 : 0);
@@ -643,6 +668,8 @@ const char *dbsa_last_error(void) { return g_err.c_str(); }
 
 int64_t dbsa_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 
+void dbsa_test_wait_expiry(uint64_t limit_ns) { g_wait_expiry_ns = limit_ns; }
+
 void dbsa_set_profile_events(void *start, void *stop) {
   g_prof_start = static_cast<cudaEvent_t>(start);
   g_prof_stop = static_cast<cudaEvent_t>(stop);
@@ -699,6 +726,7 @@ dbsa_status dbsa_encode_blocks(const dbsa_config *cfg, const void *q, const void
                                const void *v, const int32_t *offs_host, int32_t nb,
                                void *k_cache, void *v_cache, int64_t cap, void *out,
                                void *workspace, size_t ws_bytes, void *stream) {
+  const uint64_t wait_expiry = take_wait_expiry();
   dbsa_status s = check_cfg(cfg);
   if (s != DBSA_OK) return s;
   if ((s = check_offs(offs_host, nb)) != DBSA_OK) return s;
@@ -762,6 +790,8 @@ dbsa_status dbsa_encode_blocks(const dbsa_config *cfg, const void *q, const void
   sa.n_items = (int32_t)items.size();
   sa.scale_log2 = scale_log2(cfg);
   sa.status = at<int>(workspace, 0);
+  sa.wait_limit_ns = wait_expiry;
+  sa.withhold_tiles = wait_expiry != 0;
   {
     ProfileScope prof(st);
     e = launch_stage1(sa, cfg->head_dim, f32, num_sms(), st);
@@ -783,6 +813,7 @@ dbsa_status dbsa_append_block(const dbsa_config *cfg, const void *q, const void 
                               int32_t L, const int32_t *offs_host, int32_t nb, void *k_cache,
                               void *v_cache, int64_t cap, void *out, void *workspace,
                               size_t ws_bytes, void *stream) {
+  const uint64_t wait_expiry = take_wait_expiry();
   dbsa_status s = check_cfg(cfg);
   if (s != DBSA_OK) return s;
   if ((s = check_offs(offs_host, nb)) != DBSA_OK) return s;
@@ -878,6 +909,8 @@ dbsa_status dbsa_append_block(const dbsa_config *cfg, const void *q, const void 
   sa.n_items = (int32_t)items.size();
   sa.scale_log2 = scale_log2(cfg);
   sa.status = at<int>(workspace, 0);
+  sa.wait_limit_ns = wait_expiry;
+  sa.withhold_tiles = wait_expiry != 0;
   {
     ProfileScope prof(st);
     e = launch_stage1(sa, cfg->head_dim, f32, num_sms(), st);
@@ -942,7 +975,8 @@ dbsa_status gather_impl(const dbsa_config *cfg, const void *k_cache, const void 
                         const void *q_new, int32_t n_new, const void *k_tail, const void *v_tail,
                         int32_t tail_len, int32_t tail_cap, void *out, int32_t *dbg_map,
                         int64_t dbg_cap, const void *block_keys, size_t bk_bytes, void *workspace,
-                        size_t ws_bytes, void *stream) {
+                        size_t ws_bytes, void *stream, const FixedScratch *fixed = nullptr) {
+  const uint64_t wait_expiry = take_wait_expiry();
   dbsa_status s = check_cfg(cfg);
   if (s != DBSA_OK) return s;
   if ((s = check_offs(offs_host, nb)) != DBSA_OK) return s;
@@ -982,6 +1016,19 @@ dbsa_status gather_impl(const dbsa_config *cfg, const void *k_cache, const void 
   }
   const bool prepared = block_keys != nullptr;
   const S2Layout L = s2_layout(cfg, gp, n_new, prepared);
+  if (fixed != nullptr) {
+    // the no-allocation entry point: its fixed scratch, resolved only now
+    // that the call has been validated and planned
+    if (L.total > fixed->bytes)
+      return fail(DBSA_ERR_WORKSPACE,
+                  "dbsa_gather_rope_attend_noalloc: this batch needs %zu bytes of scratch but the "
+                  "entry point holds %zu; use dbsa_gather_rope_attend with a workspace or split "
+                  "the batch",
+                  L.total, fixed->bytes);
+    cudaError_t re = fixed->resolve(&workspace);
+    if (re != cudaSuccess) return cuda_fail(re, "dbsa_gather_rope_attend_noalloc: scratch address");
+    ws_bytes = fixed->bytes;
+  }
   if ((s = check_ws(workspace, ws_bytes, L.total)) != DBSA_OK) return s;
   BKLayout B{};
   if (prepared) {
@@ -1008,10 +1055,19 @@ dbsa_status gather_impl(const dbsa_config *cfg, const void *k_cache, const void 
   // one upload of the three small plan arrays (they are contiguous in the carve)
   {
     // the tables, laid out as in the workspace, written straight into staging
+    // (the no-allocation entry point: into a host vector, then one
+    // cudaMemcpyAsync from that pageable memory, which returns once the
+    // driver has taken the bytes)
     const size_t blob_bytes = L.blob_end - L.queries;
+    static thread_local std::vector<uint8_t> plain;
     uint8_t *blob = nullptr;
-    if ((e = staging_ring().stage(blob_bytes, reinterpret_cast<void **>(&blob))) != cudaSuccess)
+    if (fixed != nullptr) {
+      if (plain.size() < blob_bytes) plain.resize(blob_bytes);
+      blob = plain.data();
+    } else if ((e = staging_ring().stage(blob_bytes, reinterpret_cast<void **>(&blob))) !=
+               cudaSuccess) {
       return cuda_fail(e, "gather plan staging");
+    }
     std::memcpy(blob, gp.queries.data(), gp.queries.size() * sizeof(S2Query));
     std::memcpy(blob + (L.segs - L.queries), gp.segs.data(),
                 gp.segs.size() * sizeof(S2Segment));
@@ -1026,9 +1082,12 @@ dbsa_status gather_impl(const dbsa_config *cfg, const void *k_cache, const void 
     std::memcpy(blob + (L.tc_tiles - L.queries), gp.tc_tiles.data(),
                 gp.tc_tiles.size() * sizeof(dbsa_tile_item));
     std::memcpy(blob + (L.offs - L.queries), offs_host, (size_t)(nb + 1) * sizeof(int32_t));
-    if ((e = staging_ring().send(at<void>(workspace, L.queries), blob_bytes, st)) !=
-        cudaSuccess)
-      return cuda_fail(e, "gather plan upload");
+    if (fixed != nullptr)
+      e = cudaMemcpyAsync(at<void>(workspace, L.queries), blob, blob_bytes,
+                          cudaMemcpyHostToDevice, st);
+    else
+      e = staging_ring().send(at<void>(workspace, L.queries), blob_bytes, st);
+    if (e != cudaSuccess) return cuda_fail(e, "gather plan upload");
   }
   Stage2Args a{};
   a.k_cache = k_cache;
@@ -1058,14 +1117,8 @@ dbsa_status gather_impl(const dbsa_config *cfg, const void *k_cache, const void 
   a.rope = rope;
   const bool f32 = cfg->dtype == DBSA_F32;
   if (gp.per_query) {
-    // gather map, then the per-query kernel over every split item
-    if (dbg_map != nullptr) {
-      int32_t mx = 0;
-      for (const auto &qi : gp.queries) mx = std::max(mx, qi.n_gathered);
-      if ((e = launch_gather_map(a.queries, a.segs, nq, mx, dbg_map, dbg_cap, st)) != cudaSuccess)
-        return cuda_fail(e, "gather map");
-      count_launches(1);
-    }
+    // the per-query kernel over every split item (it writes the gather map
+    // from its own segment walk)
     {
       ProfileScope prof(st);
       e = launch_stage2_main(a, cfg->head_dim, f32, st);
@@ -1104,18 +1157,12 @@ dbsa_status gather_impl(const dbsa_config *cfg, const void *k_cache, const void 
     qa.item_row0 = at<int32_t>(workspace, L.item_row0);
     qa.rows = gp.tc_rows;
     qa.q_hat = at<void>(workspace, L.q_hat);
+    qa.q_rot_pos = dbg_map != nullptr ? at<int32_t>(workspace, L.q_rot_pos) : nullptr;
     qa.rope = rope;
     if ((e = launch_qhat(qa, cfg->head_dim, f32, st)) != cudaSuccess)
       return cuda_fail(e, "query rotation");
     count_launches(1);
-    if (dbg_map != nullptr) {
-      int32_t mx = 0;
-      for (const auto &qi : gp.queries) mx = std::max(mx, qi.n_gathered);
-      if ((e = launch_gather_map(a.queries, a.segs, nq, mx, dbg_map, dbg_cap, st)) != cudaSuccess)
-        return cuda_fail(e, "gather map");
-      count_launches(1);
-      a.dbg_map = nullptr;  // the per-query kernel below only sees tail keys
-    }
+    a.dbg_map = nullptr;  // the per-query kernel below only sees tail keys
     Stage1Args sa{};
     sa.q_rot = qa.q_hat;
     sa.q_rows = gp.tc_rows;
@@ -1137,6 +1184,14 @@ dbsa_status gather_impl(const dbsa_config *cfg, const void *k_cache, const void 
     sa.part.group = cfg->n_q_heads / cfg->n_kv_heads;
     sa.part.Hq = cfg->n_q_heads;
     sa.part.n_new = n_new;
+    sa.part.dbg = dbg_map;   // written by the kernel's epilogue when given
+    sa.part.dbg_cap = dbg_cap;
+    sa.part.items = a.items;
+    sa.part.queries = a.queries;
+    sa.part.q_rot_pos = qa.q_rot_pos;
+    sa.part.tail_len = tail_len;
+    sa.wait_limit_ns = wait_expiry;
+  sa.withhold_tiles = wait_expiry != 0;
     {
       ProfileScope prof(st);
       e = launch_stage1(sa, cfg->head_dim, false, num_sms(), st);
@@ -1154,6 +1209,17 @@ dbsa_status gather_impl(const dbsa_config *cfg, const void *k_cache, const void 
 }
 
 }  // namespace
+
+dbsa_status dbsa::gather_fixed_scratch(
+    const dbsa_config *cfg, const void *k_cache, const void *v_cache, int64_t cap,
+    const int32_t *offs_host, int32_t nb, int32_t nq, const int32_t *sel_ptr_host,
+    const int32_t *sel_blocks_host, const void *q_new, int32_t n_new, const void *k_tail,
+    const void *v_tail, int32_t tail_len, int32_t tail_cap, void *out, int32_t *dbg_map,
+    int64_t dbg_cap, const FixedScratch &fixed, void *stream) {
+  return gather_impl(cfg, k_cache, v_cache, cap, offs_host, nb, nq, sel_ptr_host,
+                     sel_blocks_host, q_new, n_new, k_tail, v_tail, tail_len, tail_cap, out,
+                     dbg_map, dbg_cap, nullptr, 0, nullptr, 0, stream, &fixed);
+}
 
 extern "C" {
 
@@ -1226,6 +1292,10 @@ dbsa_status dbsa_gather_rope_attend_prepared(
   return gather_impl(cfg, k_cache, v_cache, cap, offs_host, nb, nq, sel_ptr_host,
                      sel_blocks_host, q_new, n_new, k_tail, v_tail, tail_len, tail_cap, out,
                      dbg_map, dbg_cap, block_keys, bk_bytes, workspace, ws_bytes, stream);
+}
+
+int64_t dbsa_host_allocation_calls(void) {
+  return g_host_alloc_calls.load(std::memory_order_relaxed);
 }
 
 dbsa_status dbsa_read_status(const void *workspace, void *stream) {

@@ -109,6 +109,18 @@ struct Stage1Partial {
   float2 *ml;
   const int32_t *packed_items; // item of each group * n_new packed rows
   int32_t group, Hq, n_new;
+  // Gather map (null: not requested), [nq][dbg_cap][2].  For every item whose
+  // first packed row falls in a tile of KV head 0, the epilogue writes, for
+  // each key r of the tile's range, entry [query][p_begin + r] = (the cache
+  // row its K and V tiles were loaded from, the fresh position the pair of
+  // rotations gives it: the query's token-0 position minus the position the
+  // query rotation used (q_rot_pos) plus the key's block-relative position).
+  int32_t *dbg;
+  int64_t dbg_cap;
+  const S2Item *items;
+  const S2Query *queries;
+  const int32_t *q_rot_pos;    // per item: position qhat_kernel rotated token 0 at
+  int32_t tail_len;
 };
 
 // Stage 2, block-major tensor-core passes: keys of every cache row rotated
@@ -138,14 +150,10 @@ struct QHatArgs {
   const int32_t *item_row0;
   int32_t rows;                    // packed rows per kv head
   void *q_hat;                     // bf16 [Hkv][rows][D]
+  int32_t *q_rot_pos;              // per item: rotation position of token 0, or null
   RopeTables rope;
 };
 cudaError_t launch_qhat(const QHatArgs &a, int head_dim, bool f32, cudaStream_t st);
-
-// dbg_map[q][p] = (cache row, p) for every gathered token p of every query.
-cudaError_t launch_gather_map(const S2Query *queries, const S2Segment *segs, int32_t nq,
-                              int32_t max_tokens, int32_t *dbg_map, int64_t dbg_cap,
-                              cudaStream_t st);
 
 // Stage-1 tcgen05 attention over a tile list.
 struct Stage1Args {
@@ -161,6 +169,8 @@ struct Stage1Args {
   int32_t n_items;
   float scale_log2;       // softmax scale * log2(e)
   int *status;
+  uint64_t wait_limit_ns; // limit of every bounded wait (0: the 4 s default)
+  int32_t withhold_tiles; // test hook: load no tile, so every wait runs out
   Stage1Partial part;     // part.acc == null for Stage 1 itself
 };
 cudaError_t launch_stage1(const Stage1Args &a, int head_dim, bool out_f32, int num_sms,
@@ -183,13 +193,35 @@ struct Stage2Args {
   uint16_t *part_acc;              // bf16 [n_items][Hq][n_new][D], normalised (see above)
   float2 *part_ml;                 // [n_items][Hq][n_new] (m in log2 units, l)
   void *out;                       // [nq][n_new][Hq][D]
-  int32_t *dbg_map;                // [nq][dbg_cap][2] or null
+  // [nq][dbg_cap][2] or null: the per-query kernel writes (cache row, the
+  // position its rotation used) for every gathered key it loads (KV head 0,
+  // first row group)
+  int32_t *dbg_map;
   int64_t dbg_cap;
   float scale_log2;
   RopeTables rope;
 };
 // Sets the message dbsa_last_error() returns on this thread.
 void set_last_error(const char *msg);
+
+// Scratch owned by the library rather than the caller: `bytes` of device
+// memory whose address (on the current device) resolve() returns.
+struct FixedScratch {
+  size_t bytes;
+  cudaError_t (*resolve)(void **ptr);
+};
+// Stage 2 out of a FixedScratch (dbsa_gather_rope_attend_noalloc): the call is
+// validated and planned before the scratch is resolved, a batch that does
+// not fit is rejected with DBSA_ERR_WORKSPACE, and the plan goes to the
+// device with one cudaMemcpyAsync from pageable host memory (no page-locked
+// staging, no events).  Otherwise as dbsa_gather_rope_attend.
+dbsa_status gather_fixed_scratch(const dbsa_config *cfg, const void *k_cache, const void *v_cache,
+                                 int64_t cap, const int32_t *offs_host, int32_t nb, int32_t nq,
+                                 const int32_t *sel_ptr_host, const int32_t *sel_blocks_host,
+                                 const void *q_new, int32_t n_new, const void *k_tail,
+                                 const void *v_tail, int32_t tail_len, int32_t tail_cap,
+                                 void *out, int32_t *dbg_map, int64_t dbg_cap,
+                                 const FixedScratch &fixed, void *stream);
 
 cudaError_t launch_stage2_main(const Stage2Args &a, int head_dim, bool f32, cudaStream_t st);
 cudaError_t launch_stage2_merge(const Stage2Args &a, int head_dim, bool f32, cudaStream_t st);

@@ -8,7 +8,9 @@
 // streams).  This entry point takes no workspace.  Its scratch (status word,
 // RoPE tables, gather plan and split partials) lives in one fixed array in
 // the library's own device memory, which every GPU that loads the library
-// holds until the process exits.
+// holds until the process exits.  The call makes no allocating CUDA call:
+// the plan goes up with one cudaMemcpyAsync from pageable host memory rather
+// than through the page-locked staging ring of the other entry points.
 #include <cstdio>
 #include <mutex>
 
@@ -51,38 +53,30 @@ extern "C" dbsa_status dbsa_gather_rope_attend_noalloc(
     const int32_t *sel_blocks_host, const void *q_new, int32_t n_new, const void *k_tail,
     const void *v_tail, int32_t tail_len, int32_t tail_cap, void *out, int32_t *dbg_map,
     int64_t dbg_cap, void *stream) {
-  const size_t need = dbsa_gather_workspace_size(cfg, offs_host, nb, nq, sel_ptr_host,
-                                                 sel_blocks_host, n_new, tail_len);
-  if (need == 0) {
-    // Invalid arguments: the workspace-taking call reports the precise reason
-    // during validation, before it would look at the (absent) workspace.
-    return dbsa_gather_rope_attend(cfg, k_cache, v_cache, cap, offs_host, nb, nq, sel_ptr_host,
-                                   sel_blocks_host, q_new, n_new, k_tail, v_tail, tail_len,
-                                   tail_cap, out, dbg_map, dbg_cap, nullptr, 0, stream);
-  }
-  if (need > kNoAllocScratchBytes) {
-    char buf[256];
-    snprintf(buf, sizeof buf,
-             "dbsa_gather_rope_attend_noalloc: this batch needs %zu bytes of scratch but the "
-             "entry point holds %zu; use dbsa_gather_rope_attend with a workspace or split the "
-             "batch",
-             need, kNoAllocScratchBytes);
-    dbsa::set_last_error(buf);
-    return DBSA_ERR_WORKSPACE;
-  }
+  // Validation and planning come first (a batch that needs more than the
+  // array is rejected there, naming both sizes); the array's address is
+  // looked up after that.  The call clears the status word at the head of the
+  // scratch on `stream` before its kernels run and rewrites every other byte
+  // it reads; the array keeps whatever the previous call left.
+  const dbsa::FixedScratch fixed{kNoAllocScratchBytes, scratch_for_current_device};
+  return dbsa::gather_fixed_scratch(cfg, k_cache, v_cache, cap, offs_host, nb, nq, sel_ptr_host,
+                                    sel_blocks_host, q_new, n_new, k_tail, v_tail, tail_len,
+                                    tail_cap, out, dbg_map, dbg_cap, fixed, stream);
+}
+
+extern "C" dbsa_status dbsa_noalloc_read_status(void *stream) {
   void *ws = nullptr;
-  const cudaError_t e = scratch_for_current_device(&ws);
+  cudaError_t e = scratch_for_current_device(&ws);
+  int word = 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&word, ws, sizeof word, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) {
     char buf[256];
-    snprintf(buf, sizeof buf, "dbsa_gather_rope_attend_noalloc: scratch address lookup: %s",
-             cudaGetErrorString(e));
+    snprintf(buf, sizeof buf, "dbsa_noalloc_read_status: %s", cudaGetErrorString(e));
     dbsa::set_last_error(buf);
     return DBSA_ERR_CUDA;
   }
-  // The workspace-taking entry point clears the status word at the head of
-  // the scratch on `stream` before its kernels run, and rewrites every other
-  // byte it reads; the array keeps whatever the previous call left.
-  return dbsa_gather_rope_attend(cfg, k_cache, v_cache, cap, offs_host, nb, nq, sel_ptr_host,
-                                 sel_blocks_host, q_new, n_new, k_tail, v_tail, tail_len, tail_cap,
-                                 out, dbg_map, dbg_cap, ws, kNoAllocScratchBytes, stream);
+  if (word == DBSA_ERR_TIMEOUT) dbsa::set_last_error("a device-side wait expired");
+  return word == 0 ? DBSA_OK : static_cast<dbsa_status>(word);
 }

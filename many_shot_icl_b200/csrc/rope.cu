@@ -192,6 +192,8 @@ __global__ void __launch_bounds__(256) qhat_kernel(QHatArgs a) {
     const int q = it.query;
     const int64_t pos =
         (int64_t)a.queries[q].n_gathered + a.tail_len - a.n_new + tok - it.p_begin;
+    // the position used for token 0 of the item, for the gather map
+    if (a.q_rot_pos != nullptr && tok == 0 && c_ == 0 && cp == 0) a.q_rot_pos[item] = (int32_t)pos;
     const int i0 = cp * 8;
     float c[8], sn[8];
     rope_cs8(a.rope, pos, i0, H, c, sn);
@@ -206,27 +208,6 @@ __global__ void __launch_bounds__(256) qhat_kernel(QHatArgs a) {
       store8_bf16(dst + (int64_t)hl * D + i0, xl);
       store8_bf16(dst + (int64_t)hl * D + H + i0, xh);
     }
-  }
-}
-
-__global__ void gather_map_kernel(const S2Query *queries, const S2Segment *segs, int32_t nq,
-                                  int32_t max_tokens, int32_t *dbg, int64_t dbg_cap) {
-  const int64_t n = (int64_t)nq * max_tokens;
-  for (int64_t u = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; u < n;
-       u += (int64_t)gridDim.x * blockDim.x) {
-    const int q = (int)(u / max_tokens);
-    const int32_t p = (int32_t)(u % max_tokens);
-    const S2Query qi = queries[q];
-    if (p >= qi.n_gathered) continue;
-    int lo = 0, hi = qi.n_seg;  // segment holding fresh position p
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (segs[qi.seg_begin + mid].pos0 <= p) lo = mid; else hi = mid;
-    }
-    const S2Segment sg = segs[qi.seg_begin + lo];
-    int32_t *m = dbg + ((int64_t)q * dbg_cap + p) * 2;
-    m[0] = sg.cache_row0 + (p - sg.pos0);
-    m[1] = p;
   }
 }
 
@@ -262,15 +243,6 @@ cudaError_t launch_qhat(const QHatArgs &a, int head_dim, bool f32, cudaStream_t 
     if (f32) qhat_kernel<64, float><<<g, 256, 0, st>>>(a);
     else qhat_kernel<64, bf16><<<g, 256, 0, st>>>(a);
   }
-  return cudaGetLastError();
-}
-
-cudaError_t launch_gather_map(const S2Query *queries, const S2Segment *segs, int32_t nq,
-                              int32_t max_tokens, int32_t *dbg_map, int64_t dbg_cap,
-                              cudaStream_t st) {
-  if (nq <= 0 || max_tokens <= 0) return cudaSuccess;
-  gather_map_kernel<<<grid_for((int64_t)nq * max_tokens, 256), 256, 0, st>>>(
-      queries, segs, nq, max_tokens, dbg_map, dbg_cap);
   return cudaGetLastError();
 }
 

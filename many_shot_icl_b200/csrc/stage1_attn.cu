@@ -55,7 +55,7 @@ namespace {
 
 using namespace sm100;
 
-constexpr uint64_t kWaitLimitNs = 4000000000ull;   // 4 s: far above any legitimate wait
+constexpr uint64_t kWaitLimitNs = 4000000000ull;   // default: 4 s, far above any legitimate wait
 constexpr uint64_t kDrainLimitNs = 200000000ull;   // 0.2 s for the exit drain
 constexpr uint32_t kFull = 0xFFFFFFFFu;
 
@@ -204,6 +204,8 @@ struct Params {
   void *out;
   float scale_log2;
   int *status;
+  uint64_t wait_limit_ns;  // limit of every bounded wait
+  int withhold_tiles;      // test hook: the producer loads nothing (every wait runs out)
   Stage1Partial part;  // partial-output mode (part.acc != null)
 };
 
@@ -285,7 +287,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
-    int kidx = blockIdx.x, vidx = blockIdx.x, kt = 0, vt = 0;
+    // Test hook: no tile is loaded, so every wait of the consumers is for a
+    // barrier that nothing completes and can only run out at the wait limit.
+    // This thread waits for the abort they raise (bounded by twice the limit,
+    // then it raises it itself) and issues nothing.
+    const bool withhold = p.withhold_tiles != 0;
+    if (withhold) {
+      const uint64_t t0 = globaltimer_ns();
+      while (!*abort_flag) {
+        if (globaltimer_ns() - t0 > 2 * p.wait_limit_ns) {
+          *abort_flag = 1;
+          atomicExch(p.status, DBSA_ERR_TIMEOUT);
+          break;
+        }
+        __nanosleep(256);
+      }
+    }
+    int kidx = withhold ? p.n_items : blockIdx.x, vidx = kidx, kt = 0, vt = 0;
     Item kit, vit;
     if (kidx < p.n_items) kit = vit = load_item(p.items, kidx);
     bool need_q = kidx < p.n_items;
@@ -366,7 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         t_prog = globaltimer_ns();
       } else if ((++idle & 63u) == 0u) {
         if (*abort_flag) break;
-        if (globaltimer_ns() - t_prog > kWaitLimitNs) {
+        if (globaltimer_ns() - t_prog > p.wait_limit_ns) {
           *abort_flag = 1;
           atomicExch(p.status, DBSA_ERR_TIMEOUT);
           break;
@@ -401,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     auto wait = [&](int b, uint32_t parity) -> bool {
       return mbar_try_wait(&bar[b], parity) ||
-             mbar_wait(&bar[b], parity, abort_flag, p.status, kWaitLimitNs, DBSA_ERR_TIMEOUT);
+             mbar_wait(&bar[b], parity, abort_flag, p.status, p.wait_limit_ns, DBSA_ERR_TIMEOUT);
     };
     for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x, ++item_no) {
       const int ntiles = load_item(p.items, idx).ntiles;
@@ -483,7 +501,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tile_of(it, t, r, kt);
         const uint32_t col_s = COL_S + (s_it & 1) * 128 + wg * 64;   // this half of S
         ok = __all_sync(kFull, mbar_wait(&bar[B_S_FULL + (s_it & 1)], (s_it >> 1) & 1, abort_flag,
-                                         p.status, kWaitLimitNs, DBSA_ERR_TIMEOUT));
+                                         p.status, p.wait_limit_ns, DBSA_ERR_TIMEOUT));
         if (!ok) break;
         tc_fence_after();
         const int klim = (r ? it.len[1] : it.len[0]) - kt;   // valid keys of this tile
@@ -522,7 +540,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (__any_sync(kFull, need)) {
             // O_w must hold the item's earlier tiles before it is rescaled
             ok = __all_sync(kFull, mbar_wait(&bar[B_PV_DONE + (prev & 1)], (prev >> 1) & 1,
-                                             abort_flag, p.status, kWaitLimitNs,
+                                             abort_flag, p.status, p.wait_limit_ns,
                                              DBSA_ERR_TIMEOUT));
             if (!ok) break;
             tc_fence_after();
@@ -590,13 +608,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (wg == 1) {
         if (item_no > 0)
           ok = __all_sync(kFull, mbar_wait(&bar[B_ML_FREE], (item_no - 1) & 1, abort_flag,
-                                           p.status, kWaitLimitNs, DBSA_ERR_TIMEOUT));
+                                           p.status, p.wait_limit_ns, DBSA_ERR_TIMEOUT));
         if (!ok) break;
         sML[row] = make_float2(m_ref, l);
         mbar_arrive(&bar[B_ML_A]);
       } else {
         ok = __all_sync(kFull, mbar_wait(&bar[B_ML_A], item_no & 1, abort_flag, p.status,
-                                         kWaitLimitNs, DBSA_ERR_TIMEOUT));
+                                         p.wait_limit_ns, DBSA_ERR_TIMEOUT));
         if (!ok) break;
         const float2 ml1 = sML[row];
         const float M = fmaxf(m_ref, ml1.x);
@@ -634,12 +652,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       s_it += it.ntiles;
       const uint32_t last = s_it - 1;
       ok = __all_sync(kFull, mbar_wait(&bar[B_ML_B], item_no & 1, abort_flag, p.status,
-                                       kWaitLimitNs, DBSA_ERR_TIMEOUT));
+                                       p.wait_limit_ns, DBSA_ERR_TIMEOUT));
       if (!ok) break;
       const float2 fw = sML[row];
       mbar_arrive(&bar[B_ML_FREE]);
       ok = __all_sync(kFull, mbar_wait(&bar[B_PV_DONE + (last & 1)], (last >> 1) & 1, abort_flag,
-                                       p.status, kWaitLimitNs, DBSA_ERR_TIMEOUT));
+                                       p.status, p.wait_limit_ns, DBSA_ERR_TIMEOUT));
       if (!ok) break;
       tc_fence_after();
       int64_t prow = 0;
@@ -688,6 +706,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       mbar_arrive(&bar[B_O_FREE]);
+      if (partial && p.part.dbg != nullptr && it.head == 0 && row < it.n_rows) {
+        // Gather map: the thread of an item's first packed row records, for
+        // every key of the tile's range, the cache row its K and V tiles came
+        // from and the fresh position that the two rotations combine to (the
+        // query's token-0 position - the query rotation's position + the
+        // key's block-relative position).
+        const int grow = it.q_row0 + row;
+        const int R = p.part.group * p.part.n_new;
+        if (grow % R == 0) {
+          const int item = __ldg(p.part.packed_items + grow / R);
+          const S2Item si = p.part.items[item];
+          const int qabs0 = p.part.queries[si.query].n_gathered + p.part.tail_len - p.part.n_new;
+          const int shift = qabs0 - p.part.q_rot_pos[item];
+          const int64_t room = p.part.dbg_cap - si.p_begin;
+          const int n = si.p_begin < 0 ? 0 : (int)min((int64_t)it.len[0], room);
+          int32_t *m = p.part.dbg + ((int64_t)si.query * p.part.dbg_cap + si.p_begin) * 2;
+          const bool same_rows = it.k_row0[0] == it.v_row0[0];
+          for (int r = 0; r < n; ++r)
+            *reinterpret_cast<int2 *>(m + 2 * r) =
+                make_int2(same_rows ? it.k_row0[0] + r : -2, shift + it.pos0[0] + r);
+        }
+      }
     }
   }
   __syncwarp();
@@ -771,6 +811,8 @@ cudaError_t launch_stage1(const Stage1Args &a, int head_dim, bool out_f32, int n
   p.out = a.out;
   p.scale_log2 = a.scale_log2;
   p.status = a.status;
+  p.wait_limit_ns = a.wait_limit_ns != 0 ? a.wait_limit_ns : kWaitLimitNs;
+  p.withhold_tiles = a.withhold_tiles;
   p.part = a.part;
   const int grid = a.n_items < num_sms ? a.n_items : num_sms;
   if (head_dim == 128)

@@ -182,8 +182,16 @@ __global__ void __launch_bounds__(32 * RT * KG, 1) stage2_attn_kernel(const Stag
   auto stage_ptr = [&](int jl, int kv) -> uint8_t * {
     return sRing + ((size_t)(kg * NST + jl % NST) * 2 + kv) * STAGEB;
   };
+  // Position at which the rotation step turns row r0 + k of the sub-tile that
+  // starts at key position t0 (r0 = a warp's first row): the "hi" factor of
+  // the 16-position group holding t0 + r0 times the "lo" factor (r0 & 15) + k.
+  auto rot_pos = [](int t0, int r0, int k) {
+    return (((t0 + r0) >> kRopeShift) << kRopeShift) + (r0 & (kRopeLo - 1)) + k;
+  };
+  const bool write_map = a.dbg_map != nullptr && c == 0 && blockIdx.z == 0;
   auto issue = [&](int jl) {
-    const int p0 = k_begin + (kg + jl * KG) * KT + wr * RPW;
+    const int t0 = k_begin + (kg + jl * KG) * KT;   // first key position of the sub-tile
+    const int p0 = t0 + wr * RPW;
     // this lane's row pointer (lanes hl < RPW); null past the split end
     const CT *my = nullptr;
     if (hl < RPW) {
@@ -194,6 +202,9 @@ __global__ void __launch_bounds__(32 * RT * KG, 1) stage2_attn_kernel(const Stag
           const int64_t crow = (int64_t)__ldg(&a.segs[qi.seg_begin + seg].cache_row0) +
                                (p - __ldg(&a.segs[qi.seg_begin + seg].pos0));
           my = (half_id ? vc : kc) + ((int64_t)c * a.cap + crow) * D;
+          if (write_map && half_id == 0)   // the row this lane loads, and its rotation position
+            *reinterpret_cast<int2 *>(a.dbg_map + ((int64_t)q * a.dbg_cap + p) * 2) =
+                make_int2((int)crow, rot_pos(t0, wr * RPW, hl));
         } else {        // the query's own tail token p - T'_q
           const int64_t w = p - Tq;
           my = (half_id ? vt : kt) + (((int64_t)q * a.tail_cap + w) * a.Hkv + c) * D;
@@ -298,7 +309,7 @@ __global__ void __launch_bounds__(32 * RT * KG, 1) stage2_attn_kernel(const Stag
         const float hcos = a.rope.hc[hoff + i], hsin = a.rope.hs[hoff + i];
 #pragma unroll 4
         for (int r = r0; r < r0 + RPW; ++r) {
-          const int lr = (p0 + r) & (kRopeLo - 1);
+          const int lr = (r0 & (kRopeLo - 1)) + (r - r0);   // as rot_pos(p0, r0, r - r0)
           const float lcos = sLc[lr * H + i], lsin = sLs[lr * H + i];
           const float cs = __fmaf_rn(hcos, lcos, __fmul_rn(-hsin, lsin));
           const float sn = __fmaf_rn(hcos, lsin, __fmul_rn(hsin, lcos));

@@ -27,7 +27,8 @@ SYMBOLS = (
     "dbsa_gather_rope_attend", "dbsa_last_error", "dbsa_read_status", "dbsa_stage1_plan",
     "dbsa_stage1_tile_count", "dbsa_version", "dbsa_kernel_launches", "dbsa_set_profile_events",
     "dbsa_gather_rope_attend_noalloc", "dbsa_block_keys_size", "dbsa_block_keys",
-    "dbsa_gather_rope_attend_prepared",
+    "dbsa_gather_rope_attend_prepared", "dbsa_noalloc_read_status", "dbsa_test_wait_expiry",
+    "dbsa_host_allocation_calls",
 )
 
 
@@ -123,6 +124,12 @@ def load(path: str = LIB_PATH):
     lib.dbsa_kernel_launches.restype = i64
     lib.dbsa_set_profile_events.argtypes = [vp, vp]
     lib.dbsa_set_profile_events.restype = None
+    lib.dbsa_noalloc_read_status.argtypes = [vp]
+    lib.dbsa_noalloc_read_status.restype = ctypes.c_int
+    lib.dbsa_test_wait_expiry.argtypes = [ctypes.c_uint64]
+    lib.dbsa_test_wait_expiry.restype = None
+    lib.dbsa_host_allocation_calls.argtypes = []
+    lib.dbsa_host_allocation_calls.restype = i64
     _lib = lib
     return lib
 
@@ -291,6 +298,20 @@ def gather_rope_attend_noalloc(cfg: DbsaConfig, k_cache, v_cache, offs, sel_ptr,
 
 def read_status(workspace, stream=None) -> int:
     return int(load().dbsa_read_status(_dp(workspace), _stream(stream)))
+
+
+def noalloc_read_status(stream=None) -> int:
+    return int(load().dbsa_noalloc_read_status(_stream(stream)))
+
+
+def test_wait_expiry(limit_ns: int):
+    """Test hook: the next call on this thread loads no tile, so its device
+    waits run out after limit_ns nanoseconds (see dbsa_test_wait_expiry)."""
+    load().dbsa_test_wait_expiry(int(limit_ns))
+
+
+def host_allocation_calls() -> int:
+    return int(load().dbsa_host_allocation_calls())
 
 
 def selection_csr(selections) -> tuple[np.ndarray, np.ndarray]:

@@ -38,6 +38,11 @@ def host_f32(t) -> np.ndarray:
     return t.detach().float().cpu().numpy()
 
 
+# Every comparison's measured errors, reported at the end of the session
+# (tests/conftest.py prints them; DBSA_PARITY_LOG names a JSON file to write).
+MEASURED: list[dict] = []
+
+
 def compare(got: np.ndarray, want: np.ndarray, head_axis: int, what: str, atol: float = ATOL,
             rtol: float | None = None):
     """max-abs <= atol and, per head, relative Frobenius error <= rtol (RTOL_FRO,
@@ -47,12 +52,22 @@ def compare(got: np.ndarray, want: np.ndarray, head_axis: int, what: str, atol: 
     got = np.asarray(got, dtype=np.float64)
     err = np.abs(got - want)
     assert np.isfinite(got).all(), what + ": non-finite output"
-    assert err.max() <= atol, "%s: max-abs %.3e > %.1e" % (what, err.max(), atol)
     g = np.moveaxis(got, head_axis, 0).reshape(got.shape[head_axis], -1)
     w = np.moveaxis(want, head_axis, 0).reshape(want.shape[head_axis], -1)
     rel = np.linalg.norm(g - w, axis=1) / np.maximum(np.linalg.norm(w, axis=1), 1e-30)
+    MEASURED.append({"what": what, "max_abs": float(err.max()), "rel_fro": float(rel.max()),
+                     "atol": atol, "rtol": rtol, "max_abs_ref": float(np.abs(want).max())})
+    assert err.max() <= atol, "%s: max-abs %.3e > %.1e" % (what, err.max(), atol)
     assert rel.max() <= rtol, "%s: relative Frobenius %.3e > %.1e" % (what, rel.max(), rtol)
     return float(err.max()), float(rel.max())
+
+
+def check_gather_map(dbg_q: np.ndarray, want: np.ndarray, what: str):
+    """The kernel-written gather map of one query equals the oracle's exactly,
+    and the entries past its gathered tokens are untouched (-1)."""
+    n = len(want)
+    np.testing.assert_array_equal(dbg_q[:n], want, err_msg=what + ": gather map")
+    assert (dbg_q[n:] == -1).all(), what + ": gather map written past T'"
 
 
 def offsets(lens) -> np.ndarray:

@@ -38,7 +38,8 @@ def test_tiny_workload_fp32():
     assert torch.equal(run.vc[:, :run.T], run.v.permute(1, 0, 2))
 
 
-@pytest.mark.parametrize("Hq,Hkv,D,theta", [(4, 2, 128, 5e5), (8, 2, 128, 1e4), (2, 2, 64, 1e4)])
+@pytest.mark.parametrize("Hq,Hkv,D,theta", [(4, 2, 128, 5e5), (8, 2, 128, 1e4), (2, 2, 64, 1e4),
+                                            (64, 1, 64, 1e4)])
 def test_multi_tile_bf16(Hq, Hkv, D, theta):
     lens = [300, 129, 128, 1, 257, 400, 77]
     cfg = dbsa.DbsaConfig(Hq, Hkv, D, "bf16", theta, 2)

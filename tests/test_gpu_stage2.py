@@ -1,13 +1,18 @@
 """Stage-2 parity on a B200: dbsa_gather_rope_attend against the CPU oracle
 on the same seeded inputs.  Gathered cache rows and fresh positions are
-compared exactly (dbg_map); attention outputs within the stated tolerance."""
+compared exactly: dbg_map is written by the attention kernels themselves
+(the block-by-block tensor-core kernel's epilogue from the tile it loaded and
+the rotation the query rows got; the per-query kernel from its own segment
+walk and rotation table indices).  Attention outputs within the stated
+tolerance."""
 import numpy as np
 import pytest
 import torch
 
 import oracle
 from many_shot_icl_b200 import dbsa, inputs
-from tests.gpu_helpers import ATOL, ATOL_PEAKY, compare, host_f32, offsets, rand, tdtype
+from tests.gpu_helpers import (ATOL, ATOL_PEAKY, check_gather_map, compare, host_f32, offsets,
+                               rand, tdtype)
 
 pytestmark = pytest.mark.gpu
 
@@ -58,7 +63,7 @@ class Stage2Run:
         dbg = self.dbg.cpu().numpy()
         for q in (range(self.nq) if queries is None else queries):
             m = oracle.stage2_gather_map(self.offs, self.sels[q])
-            np.testing.assert_array_equal(dbg[q, :len(m)], m, err_msg="%s: gather map q%d" % (what, q))
+            check_gather_map(dbg[q], m, "%s q%d" % (what, q))
             want = oracle.stage2_all(kc, vc, self.offs, self.sels[q], qn[q],
                                      kt[q, :self.tail_len], vt[q, :self.tail_len],
                                      self.cfg.rope_theta, scale=self.cfg.softmax_scale)
@@ -83,6 +88,32 @@ def test_bf16_prefill_and_decode(Hq, Hkv, D, n_new, tail_len):
     cfg = dbsa.DbsaConfig(Hq, Hkv, D, "bf16", 5e5, 2)
     Stage2Run(cfg, offs, sels, n_new, tail_len, seed=2).run().check(
         "Hq%d Hkv%d D%d n%d t%d" % (Hq, Hkv, D, n_new, tail_len))
+
+
+@pytest.mark.parametrize("Hq,Hkv,D", [(8, 2, 128), (2, 1, 64)])
+@pytest.mark.parametrize("n_new,tail_len", [(16, 16), (1, 9)])
+def test_fp32_cache_block_major(Hq, Hkv, D, n_new, tail_len):
+    """fp32 caches whose selected blocks average well over one 128-key tile:
+    the block-by-block tensor-core path, which reads a bf16 copy of V made
+    next to the block-relative keys."""
+    rng = np.random.default_rng(Hq * 7 + n_new)
+    offs = offsets(rng.integers(150, 420, size=8))
+    sels = [np.array([0, 2, 5, 7]), np.array([0, 6, 1]), np.array([0]), np.array([0, 3, 4, 1, 7])]
+    cfg = dbsa.DbsaConfig(Hq, Hkv, D, "f32", 5e5, 2)
+    gath = [int(sum(offs[b + 1] - offs[b] for b in s_)) for s_ in sels]
+    assert sum(gath) >= 128 * sum(len(s_) for s_ in sels)   # the block-major mode
+    Stage2Run(cfg, offs, sels, n_new, tail_len, seed=11).run().check(
+        "fp32 block-major Hq%d D%d n%d" % (Hq, D, n_new))
+
+
+@pytest.mark.parametrize("n_new,tail_len", [(3, 5), (1, 4)])
+def test_largest_head_ratio(n_new, tail_len):
+    """64 query heads on one KV head, the largest ratio the ABI accepts: the
+    packed rows of one (query, block) pair span two 128-row tiles."""
+    offs = offsets([180, 260, 140, 300])
+    sels = [np.array([0, 3, 1]), np.array([0, 2])]
+    cfg = dbsa.DbsaConfig(64, 1, 64, "bf16", 1e4, 2)
+    Stage2Run(cfg, offs, sels, n_new, tail_len, seed=12).run().check("Hq/Hkv=64 n%d" % n_new)
 
 
 def test_long_gather_many_splits_peaky():
