@@ -15,12 +15,15 @@ RTOL_FRO = 2e-2  # relative Frobenius error bound per head
 # moves a score by about sqrt(2d) * s_q * s_k * 2^-9 / sqrt(d) ~= 0.011 for
 # s_q = 4, s_k = 1; with |v| up to ~3.5 a sharp softmax turns that into up to
 # ~0.04 on an output element, plus half a bf16 ulp of the output (<= 0.008).
-ATOL_PEAKY = 6e-2
+# Measured over the 17 peaky comparisons of the GPU suite (90k and 128k
+# batches, long gathers, demonstration-granular, Stage 1): at most 0.031
+# max-abs and 0.023 relative Frobenius; the bounds keep about 1.4x over that.
+ATOL_PEAKY = 4.5e-2
 # The same argument bounds the relative Frobenius error of a peaky row: its
 # output is close to one V row (elements ~N(0,1), norm ~sqrt(d)) and each
-# element may move by ~0.04, so up to ~4 % on a row; with few rows per head
+# element may move by up to ~0.04, a few % of the row; with few rows per head
 # (a decode step has one) nothing averages this out.
-RTOL_FRO_PEAKY = 4e-2
+RTOL_FRO_PEAKY = 3e-2
 
 
 def tdtype(dtype: str):
