@@ -64,6 +64,11 @@ dbsa_status cuda_fail(cudaError_t e, const char *where) {
 }
 
 constexpr size_t kAlign = 1024;
+// Block-major passes with at most this many query rows per (query, KV head)
+// (g * n_new) run the tail attention and the merge as one warp-per-row
+// kernel; longer passes (prompt passes) keep the tail on the per-query
+// mma.sync kernel, which shares each tail key among all the rows.
+constexpr int kTailMergeMaxRows = 32;
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Copies bytes from page-locked host memory (read over the bus by the SMs)
@@ -1162,7 +1167,7 @@ dbsa_status gather_impl(const dbsa_config *cfg, const void *k_cache, const void 
     if ((e = launch_qhat(qa, cfg->head_dim, f32, st)) != cudaSuccess)
       return cuda_fail(e, "query rotation");
     count_launches(1);
-    a.dbg_map = nullptr;  // the per-query kernel below only sees tail keys
+    a.dbg_map = nullptr;  // written by the tensor-core kernel's epilogue (sa.part.dbg)
     Stage1Args sa{};
     sa.q_rot = qa.q_hat;
     sa.q_rows = gp.tc_rows;
@@ -1198,6 +1203,17 @@ dbsa_status gather_impl(const dbsa_config *cfg, const void *k_cache, const void 
     }
     if (e != cudaSuccess) return cuda_fail(e, "stage-2 tensor-core attention");
     count_launches(1);
+    const int rows = (cfg->n_q_heads / cfg->n_kv_heads) * n_new;
+    if (rows <= kTailMergeMaxRows) {
+      // few rows per (query, KV head), e.g. a decode step: each query's own
+      // tail tokens and the merge of its block partials in one kernel
+      if ((e = launch_stage2_tail_merge(a, cfg->head_dim, f32, st)) != cudaSuccess)
+        return cuda_fail(e, "stage-2 tail attention and merge");
+      count_launches(1);
+      return DBSA_OK;
+    }
+    // many rows (a prompt pass): the tail keys on the per-query tensor-core
+    // (mma.sync) kernel, then the merge below
     if ((e = launch_stage2_main(a, cfg->head_dim, f32, st)) != cudaSuccess)  // tail items
       return cuda_fail(e, "stage-2 tail attention");
     count_launches(1);

@@ -224,6 +224,11 @@ dbsa_status gather_fixed_scratch(const dbsa_config *cfg, const void *k_cache, co
                                  const FixedScratch &fixed, void *stream);
 
 cudaError_t launch_stage2_main(const Stage2Args &a, int head_dim, bool f32, cudaStream_t st);
+// Block-major mode: every query's tail tokens and the merge of all its
+// partials, writing the output (replaces the per-query kernel's tail items
+// and the merge).
+cudaError_t launch_stage2_tail_merge(const Stage2Args &a, int head_dim, bool f32,
+                                     cudaStream_t st);
 cudaError_t launch_stage2_merge(const Stage2Args &a, int head_dim, bool f32, cudaStream_t st);
 
 }  // namespace dbsa

@@ -564,9 +564,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
         const f32x2 sc2 = f2_pack(sl2, sl2), nmu2 = f2_pack(-mu, -mu);
         f32x2 sum2[2] = {0ull, 0ull};
-        // chunk c of 32 scores -> 16 packed P columns
-        auto exp_chunk = [&](const uint32_t (&v)[32], int c) {
+        // chunk c of 32 scores -> 16 packed P columns.  A chunk whose keys
+        // are all masked for every row of the warp (the ragged end of a key
+        // range, the far side of the causal diagonal) gets P = 0 without
+        // exponentials: the exponential unit bounds this pass.
+        auto exp_chunk = [&](const uint32_t (&v)[32], int c, bool masked) {
           uint32_t pw[16];
+          if (masked) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) pw[e] = 0u;
+            tmem_st16(tmem + lane_off + col_s + c * 16, pw);
+            return;
+          }
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
             const f32x2 x2 =
@@ -586,8 +595,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tmem_st16(tmem + lane_off + col_s + c * 16, pw);
         };
-        exp_chunk(va, 0);
-        exp_chunk(vb, 1);
+        exp_chunk(va, 0, need_mask && __all_sync(kFull, klast < 0));
+        exp_chunk(vb, 1, need_mask && __all_sync(kFull, klast < 32));
         tmem_wait_st();
         float sa, sb2, sc, sd;
         f2_unpack(sum2[0], sa, sb2);

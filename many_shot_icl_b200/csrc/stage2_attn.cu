@@ -1,5 +1,5 @@
-// Stage 2, per-query part: the per-query split kernel, then the log-sum-exp
-// merge of all split partials.
+// Stage 2, per-query parts: the per-query split kernel and the log-sum-exp
+// merge of split partials, and the block-major mode's tail-and-merge kernel.
 //
 // [DBSA notes] §Stage 2, items 2-4: the selected blocks (sink first) are
 // concatenated, their cached pre-RoPE keys are rotated again at fresh
@@ -7,11 +7,12 @@
 // cache and, causally, to the query's own tokens.  Query q's key sequence is
 // [gathered tokens 0..T'_q) ++ [its own tail tokens], positions
 // 0..T'_q + tail_len - 1.  Normally the gathered blocks are handled block by
-// block by the tensor-core kernel (one partial per (query, block)) and this
-// kernel runs each query's tail keys [T'_q, T'_q + tail_len); for selections
-// of short segments (a demonstration-granular gather) it runs whole split
-// items [p_begin, p_end) of a query's key sequence, fetching the gathered
-// keys segment by segment.  The merge combines every partial of a row.
+// block by the tensor-core kernel (one partial per (query, block)) and
+// stage2_tail_merge_kernel runs each query's tail keys [T'_q, T'_q + tail_len)
+// and merges all partials of a row into the output.  For selections of short
+// segments (a demonstration-granular gather) stage2_attn_kernel runs whole
+// split items [p_begin, p_end) of a query's key sequence, fetching the
+// gathered keys segment by segment, and stage2_merge_kernel combines them.
 //
 // Grid: (item, KV head, row group).  A CTA reads each key of its item once
 // and scores it against all g * n_new query rows that share the KV head
@@ -548,6 +549,161 @@ __global__ void __launch_bounds__(128) stage2_merge_kernel(const Stage2Args a) {
   }
 }
 
+// Block-major mode, after the tensor-core pass: each query's own tail tokens
+// and the merge of every partial of a row, in one kernel.  CTA = (query q,
+// KV head c, group of up to 8 rows of the query's g * n_new rows); one warp
+// per output row (query token u, head h).  Lane l holds the elements
+// i = l + 32 j (j < D / 32), so the rotate-half pairs (i, i + D/2) sit in the
+// same lane.  The CTA rotates the query's tail keys, 32 at a time, into
+// shared memory at their positions T'_q + u' (fp32, no rounding), with their
+// values; every warp scores its rotated query row against the keys u' <= its
+// own tail index (the causal rule), in log2 units, with an online softmax.
+// The row's block partials (M_i, L_i, O_i), written by the tensor-core pass,
+// are then merged with the tail state (m, l, acc):
+//   O = (sum_i 2^(M_i - M) L_i O_i + 2^(m - M) acc) / (sum_i 2^(M_i - M) L_i + 2^(m - M) l).
+template <int D, typename CT>
+__global__ void __launch_bounds__(256) stage2_tail_merge_kernel(const Stage2Args a) {
+  constexpr int H = D / 2;
+  constexpr int E = D / 32;           // elements per lane
+  constexpr int CH = 32;              // tail keys per shared-memory chunk
+  __shared__ float sK[CH][D], sV[CH][D];
+  const int q = blockIdx.x, c = blockIdx.y;
+  const int g = a.Hq / a.Hkv;
+  const int R = g * a.n_new;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = blockIdx.z * 8 + warp;          // this warp's row (token-major: u * g + hl)
+  const bool live = r < R;
+  const S2Query qi = a.queries[q];
+  const int Tq = qi.n_gathered;
+  const int tok = live ? r / g : 0;
+  const int h = c * g + (live ? r % g : 0);
+  const int tu = a.tail_len - a.n_new + tok;    // this row's tail index
+  const float sl2 = a.scale_log2;
+  // the query row, rotated at T'_q + tu
+  float qr[E];
+  {
+    const CT *src = static_cast<const CT *>(a.q_new) + (((int64_t)q * a.n_new + tok) * a.Hq + h) * D;
+#pragma unroll
+    for (int j = 0; j < E; ++j) qr[j] = to_f32(src[lane + 32 * j]);
+    const int64_t pq = (int64_t)Tq + tu;
+#pragma unroll
+    for (int j = 0; j < E / 2; ++j) {
+      float cs, sn;
+      rope_cs1(a.rope, pq, lane + 32 * j, H, cs, sn);
+      const float lo = qr[j], hi = qr[j + E / 2];
+      qr[j] = __fmaf_rn(lo, cs, __fmul_rn(-hi, sn));
+      qr[j + E / 2] = __fmaf_rn(hi, cs, __fmul_rn(lo, sn));
+    }
+  }
+  float m = -INFINITY, l = 0.f, acc[E];
+#pragma unroll
+  for (int j = 0; j < E; ++j) acc[j] = 0.f;
+  for (int k0 = 0; k0 < a.tail_len; k0 += CH) {
+    const int nk = min(CH, a.tail_len - k0);
+    __syncthreads();   // the previous chunk has been read by every warp
+#pragma unroll 4
+    for (int u = threadIdx.x; u < nk * H; u += blockDim.x) {
+      const int j = u / H, i = u % H;
+      const int64_t row = ((int64_t)q * a.tail_cap + k0 + j) * a.Hkv + c;
+      const CT *ks = static_cast<const CT *>(a.k_tail) + row * D;
+      const CT *vs = static_cast<const CT *>(a.v_tail) + row * D;
+      float cs, sn;
+      rope_cs1(a.rope, (int64_t)Tq + k0 + j, i, H, cs, sn);
+      const float lo = to_f32(ks[i]), hi = to_f32(ks[i + H]);
+      sK[j][i] = __fmaf_rn(lo, cs, __fmul_rn(-hi, sn));
+      sK[j][i + H] = __fmaf_rn(hi, cs, __fmul_rn(lo, sn));
+      sV[j][i] = to_f32(vs[i]);
+      sV[j][i + H] = to_f32(vs[i + H]);
+    }
+    __syncthreads();
+    // keys k0 .. k0 + n - 1 of this chunk are visible to the row (u' <= tu)
+    const int n = live ? max(0, min(nk, tu - k0 + 1)) : 0;
+    for (int j0 = 0; j0 < n; j0 += 4) {
+      float sc[4];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        float d = 0.f;
+        if (j0 + t < n) {
+#pragma unroll
+          for (int j = 0; j < E; ++j) d = __fmaf_rn(qr[j], sK[j0 + t][lane + 32 * j], d);
+        }
+        sc[t] = d;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int t = 0; t < 4; ++t) sc[t] += __shfl_xor_sync(0xffffffffu, sc[t], o);
+      float mx = m;
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        sc[t] = (j0 + t < n) ? sc[t] * sl2 : -INFINITY;
+        mx = fmaxf(mx, sc[t]);
+      }
+      const float alpha = (m == -INFINITY) ? 0.f : ex2(m - mx);
+      l *= alpha;
+#pragma unroll
+      for (int j = 0; j < E; ++j) acc[j] *= alpha;
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const float pt = ex2(sc[t] - mx);
+        l += pt;
+        if (j0 + t < n) {
+#pragma unroll
+          for (int j = 0; j < E; ++j) acc[j] = __fmaf_rn(pt, sV[j0 + t][lane + 32 * j], acc[j]);
+        }
+      }
+      m = mx;
+    }
+  }
+  if (!live) return;
+  // merge with the row's block partials (every item of the query but the
+  // last, its tail item)
+  const int nb = qi.n_items - 1;
+  auto part = [&](int i) { return ((int64_t)(qi.item_begin + i) * a.Hq + h) * a.n_new + tok; };
+  float M = m;
+  for (int i = lane; i < nb; i += 32) M = fmaxf(M, a.part_ml[part(i)].x);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  const float wt = ex2(m - M);                 // m is finite: key tu is always visible
+  float L = 0.f, out[E];
+#pragma unroll
+  for (int j = 0; j < E; ++j) out[j] = wt * acc[j];
+  for (int i0 = 0; i0 < nb; i0 += 32) {
+    float w = 0.f;
+    if (i0 + lane < nb) {
+      const float2 ml = a.part_ml[part(i0 + lane)];
+      w = (ml.x == -INFINITY) ? 0.f : ex2(ml.x - M) * ml.y;
+    }
+    L += w;
+    const int cnt = min(32, nb - i0);
+    for (int k0 = 0; k0 < cnt; k0 += 4) {   // four partial rows in flight
+      uint16_t v[4][E];
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (k0 + k < cnt) {
+          const uint16_t *src = a.part_acc + part(i0 + k0 + k) * D;
+#pragma unroll
+          for (int j = 0; j < E; ++j) v[k][j] = src[lane + 32 * j];
+        }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float wk = __shfl_sync(0xffffffffu, w, (k0 + k) & 31);
+        if (k0 + k < cnt) {
+#pragma unroll
+          for (int j = 0; j < E; ++j)
+            out[j] = __fmaf_rn(wk, __uint_as_float((uint32_t)v[k][j] << 16), out[j]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+  const float inv = 1.f / (L + wt * l);
+  CT *dst = static_cast<CT *>(a.out) + (((int64_t)q * a.n_new + tok) * a.Hq + h) * D;
+#pragma unroll
+  for (int j = 0; j < E; ++j) from_f32(out[j] * inv, dst[lane + 32 * j]);
+}
+
 template <int D, typename CT, int RT, int KG, int KT>
 cudaError_t launch_main(const Stage2Args &a, cudaStream_t st) {
   constexpr int NST = 3;
@@ -583,6 +739,14 @@ cudaError_t launch_d(const Stage2Args &a, cudaStream_t st) {
 }
 
 template <int D, typename CT>
+cudaError_t launch_tail_merge(const Stage2Args &a, cudaStream_t st) {
+  const int R = (a.Hq / a.Hkv) * a.n_new;
+  dim3 grid(a.n_queries, a.Hkv, (R + 7) / 8);
+  stage2_tail_merge_kernel<D, CT><<<grid, 32 * min(8, R), 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+template <int D, typename CT>
 cudaError_t launch_merge(const Stage2Args &a, cudaStream_t st) {
   const int64_t rows = (int64_t)a.n_queries * a.n_new * a.Hq;
   stage2_merge_kernel<D, CT><<<(unsigned)((rows + 3) / 4), 128, 0, st>>>(a);
@@ -595,6 +759,14 @@ cudaError_t launch_stage2_main(const Stage2Args &a, int head_dim, bool f32, cuda
   if (a.n_items <= 0) return cudaSuccess;
   if (head_dim == 128) return f32 ? launch_d<128, float>(a, st) : launch_d<128, bf16>(a, st);
   return f32 ? launch_d<64, float>(a, st) : launch_d<64, bf16>(a, st);
+}
+
+cudaError_t launch_stage2_tail_merge(const Stage2Args &a, int head_dim, bool f32,
+                                     cudaStream_t st) {
+  if (a.n_queries <= 0) return cudaSuccess;
+  if (head_dim == 128)
+    return f32 ? launch_tail_merge<128, float>(a, st) : launch_tail_merge<128, bf16>(a, st);
+  return f32 ? launch_tail_merge<64, float>(a, st) : launch_tail_merge<64, bf16>(a, st);
 }
 
 cudaError_t launch_stage2_merge(const Stage2Args &a, int head_dim, bool f32, cudaStream_t st) {

@@ -32,6 +32,22 @@ __device__ __forceinline__ void rope_cs8(const RopeTables &t, int64_t p, int i0,
   }
 }
 
+// (cos, sin) of p * w_i for one frequency i, with the rounding of rope_cs8.
+__device__ __forceinline__ void rope_cs1(const RopeTables &t, int64_t p, int i, int half, float &c,
+                                         float &s) {
+  const int64_t hoff = (p >> kRopeShift) * half + i, loff = (p & (kRopeLo - 1)) * half + i;
+  const float ac = __ldg(t.hc + hoff), as = __ldg(t.hs + hoff);
+  const float bc = __ldg(t.lc + loff), bs = __ldg(t.ls + loff);
+  c = __fmaf_rn(ac, bc, __fmul_rn(-as, bs));
+  s = __fmaf_rn(ac, bs, __fmul_rn(as, bc));
+}
+
+// One element between bf16 / fp32 storage and fp32 (output rounding RNE).
+__device__ __forceinline__ float to_f32(bf16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ void from_f32(float x, bf16 &d) { d = __float2bfloat16_rn(x); }
+__device__ __forceinline__ void from_f32(float x, float &d) { d = x; }
+
 // 8 consecutive elements as fp32, from bf16 (16 B) or fp32 (32 B) storage.
 __device__ __forceinline__ void load8(const bf16 *p, float (&f)[8]) {
   const uint4 r = *reinterpret_cast<const uint4 *>(p);
