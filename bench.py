@@ -591,7 +591,10 @@ def comparators(wl: Workload, n_ret_queries: int = 4):
             "dbsa_demo_granular": {"inference_s_per_query": demo_inf,
                                    "demonstrations_per_query": n_pick,
                                    "mean_gathered_tokens": d_tokens,
-                                   "path": "per-query split (segments shorter than a key tile)"}}
+                                   "path": "prompt pass: per-query split (mma.sync); decode "
+                                           "steps: block-major tensor-core pass at "
+                                           "demonstration granularity (keys shared by the "
+                                           "queries that selected them)"}}
 
 
 # ------------------------------------------------------------------ other workloads

@@ -446,11 +446,25 @@ dbsa_status gather_plan(const dbsa_config *cfg, const int32_t *offs, int32_t nb,
     gp.queries.push_back(qi);
   }
   // Selections of short segments (a demonstration-granular gather: blocks of
-  // one demonstration each) go per query: the block-major path keeps one
-  // partial per (query, segment) row, which would then outweigh the K/V.
+  // one demonstration each) go per query when the block-major path's extra
+  // traffic would outweigh the K/V it saves: it keeps one partial per (query,
+  // segment) row and one packed query row per (query, segment, token, head),
+  // each written and read once, and rotates every key of the cache, while
+  // the per-query path streams every query's own gathered keys.  Passes with
+  // few query tokens (decode steps) still share the keys across queries.
   int64_t gathered = 0;
   for (const auto &qi : gp.queries) gathered += qi.n_gathered;
-  if (gathered < (int64_t)kTileKeys * (int64_t)gp.segs.size()) {
+  bool per_query = gathered < (int64_t)kTileKeys * (int64_t)gp.segs.size();
+  if (per_query) {
+    const double elt = cfg->dtype == DBSA_F32 ? 4.0 : 2.0;
+    const double D = cfg->head_dim, Hkv = cfg->n_kv_heads;
+    const double per_query_bytes = (double)(gathered + (int64_t)nq * tail_len) * Hkv * D * elt * 2;
+    const double per_pair = (double)cfg->n_q_heads * n_new * ((2.0 * D + 8.0) * 2 + 2.0 * D * 2);
+    const double block_bytes =
+        (double)offs[nb] * Hkv * D * (2.0 * elt + 4.0) + (double)gp.segs.size() * per_pair;
+    per_query = !(block_bytes < per_query_bytes);
+  }
+  if (per_query) {
     gp.per_query = true;
     // Split size: >= 33 keys per query row of a CTA (bounds the partial
     // traffic to ~3 % of the K/V bytes) and enough CTAs for ~4 waves.  Rows

@@ -26,6 +26,7 @@
 
 #include <cfloat>
 #include <climits>
+#include <type_traits>
 
 #include "dbsa_internal.h"
 #include "vec8.cuh"
@@ -567,6 +568,7 @@ __global__ void __launch_bounds__(256) stage2_tail_merge_kernel(const Stage2Args
   constexpr int E = D / 32;           // elements per lane
   constexpr int CH = 32;              // tail keys per shared-memory chunk
   __shared__ float sK[CH][D], sV[CH][D];
+  __shared__ float sO[8][D];          // a row's tail accumulator, regrouped for the merge
   const int q = blockIdx.x, c = blockIdx.y;
   const int g = a.Hq / a.Hkv;
   const int R = g * a.n_new;
@@ -657,7 +659,15 @@ __global__ void __launch_bounds__(256) stage2_tail_merge_kernel(const Stage2Args
   }
   if (!live) return;
   // merge with the row's block partials (every item of the query but the
-  // last, its tail item)
+  // last, its tail item).  For the merge each lane takes E consecutive
+  // elements (8- or 4-byte loads of every partial row), so the tail
+  // accumulator is regrouped through shared memory first.
+#pragma unroll
+  for (int j = 0; j < E; ++j) sO[warp][lane + 32 * j] = acc[j];
+  __syncwarp();
+  float acc_c[E];
+#pragma unroll
+  for (int j = 0; j < E; ++j) acc_c[j] = sO[warp][E * lane + j];
   const int nb = qi.n_items - 1;
   auto part = [&](int i) { return ((int64_t)(qi.item_begin + i) * a.Hq + h) * a.n_new + tok; };
   float M = m;
@@ -667,7 +677,9 @@ __global__ void __launch_bounds__(256) stage2_tail_merge_kernel(const Stage2Args
   const float wt = ex2(m - M);                 // m is finite: key tu is always visible
   float L = 0.f, out[E];
 #pragma unroll
-  for (int j = 0; j < E; ++j) out[j] = wt * acc[j];
+  for (int j = 0; j < E; ++j) out[j] = wt * acc_c[j];
+  using Vec = typename std::conditional<E == 4, uint2, uint32_t>::type;   // E bf16 values
+  constexpr int U = 8;                         // partial rows in flight
   for (int i0 = 0; i0 < nb; i0 += 32) {
     float w = 0.f;
     if (i0 + lane < nb) {
@@ -676,22 +688,22 @@ __global__ void __launch_bounds__(256) stage2_tail_merge_kernel(const Stage2Args
     }
     L += w;
     const int cnt = min(32, nb - i0);
-    for (int k0 = 0; k0 < cnt; k0 += 4) {   // four partial rows in flight
-      uint16_t v[4][E];
+    for (int k0 = 0; k0 < cnt; k0 += U) {
+      Vec v[U];
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
-        if (k0 + k < cnt) {
-          const uint16_t *src = a.part_acc + part(i0 + k0 + k) * D;
+      for (int k = 0; k < U; ++k)
+        if (k0 + k < cnt)
+          v[k] = *reinterpret_cast<const Vec *>(a.part_acc + part(i0 + k0 + k) * D + E * lane);
 #pragma unroll
-          for (int j = 0; j < E; ++j) v[k][j] = src[lane + 32 * j];
-        }
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
+      for (int k = 0; k < U; ++k) {
         const float wk = __shfl_sync(0xffffffffu, w, (k0 + k) & 31);
         if (k0 + k < cnt) {
+          const uint32_t *wv = reinterpret_cast<const uint32_t *>(&v[k]);
 #pragma unroll
-          for (int j = 0; j < E; ++j)
-            out[j] = __fmaf_rn(wk, __uint_as_float((uint32_t)v[k][j] << 16), out[j]);
+          for (int j = 0; j < E / 2; ++j) {
+            out[2 * j] = __fmaf_rn(wk, __uint_as_float(wv[j] << 16), out[2 * j]);
+            out[2 * j + 1] = __fmaf_rn(wk, __uint_as_float(wv[j] & 0xFFFF0000u), out[2 * j + 1]);
+          }
         }
       }
     }
@@ -699,9 +711,9 @@ __global__ void __launch_bounds__(256) stage2_tail_merge_kernel(const Stage2Args
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
   const float inv = 1.f / (L + wt * l);
-  CT *dst = static_cast<CT *>(a.out) + (((int64_t)q * a.n_new + tok) * a.Hq + h) * D;
+  CT *dst = static_cast<CT *>(a.out) + (((int64_t)q * a.n_new + tok) * a.Hq + h) * D + E * lane;
 #pragma unroll
-  for (int j = 0; j < E; ++j) from_f32(out[j] * inv, dst[lane + 32 * j]);
+  for (int j = 0; j < E; ++j) from_f32(out[j] * inv, dst[j]);
 }
 
 template <int D, typename CT, int RT, int KG, int KT>

@@ -175,16 +175,19 @@ def demo_granular(w, offs, seed):
     return d_offs, sels
 
 
-def test_stage2_demo_granular_full_size():
+@pytest.mark.parametrize("n_new,tail_len", [(40, 40), (1, 41)])
+def test_stage2_demo_granular_full_size(n_new, tail_len):
     """90k cache, 64 queries selecting single demonstrations (~885 segments
-    each): the per-query split path, checked like the block-granular batches."""
+    each), checked like the block-granular batches.  The 40-token prompt pass
+    takes the per-query split path; a decode step takes the block-major path
+    at demonstration granularity (each demonstration's keys shared by the
+    ~19 queries that selected it)."""
     w = inputs.L31_8B_90K
     cfg, offs, q, k, v, kc, vc, _ = run_stage1(w)
     del q, k, v
     d_offs, sels = demo_granular(w, offs, seed=9)
-    n_new = tail_len = w.query_tokens
     qn, kt, vt, out, dbg = run_stage2(w, cfg, kc, vc, d_offs, sels, n_new, tail_len,
-                                      seed=inputs.tensor_seed(w, 0, 3, 77))
+                                      seed=inputs.tensor_seed(w, 0, 3, 77 + n_new))
     dbg = dbg.cpu().numpy()
     for qi, s in enumerate(sels):
         check_gather_map(dbg[qi], oracle.stage2_gather_map(d_offs, s), "demo-granular q%d" % qi)
@@ -193,7 +196,7 @@ def test_stage2_demo_granular_full_size():
         want = oracle.stage2_all(kch, vch, d_offs, sels[qi], host_f32(qn[qi]),
                                  host_f32(kt[qi, :tail_len]), host_f32(vt[qi, :tail_len]),
                                  w.rope_theta)
-        compare(host_f32(out[qi]), want, head_axis=1, what="demo-granular q%d" % qi)
+        compare(host_f32(out[qi]), want, head_axis=1, what="demo-granular n%d q%d" % (n_new, qi))
 
 
 def test_prepared_block_keys_full_size():

@@ -213,6 +213,27 @@ def test_demonstration_granular_gather(n_new, tail_len):
     peaky.check("demo-granular peaky", atol=ATOL_PEAKY)
 
 
+def test_demonstration_granular_decode_shares_blocks():
+    """Decode steps over a demonstration-granular selection (one block per
+    demonstration, many queries selecting overlapping sets): the planner
+    prices the per-(query, demonstration) partials and packed query rows
+    below streaming every query's own keys, so the pass runs block-major on
+    the tensor core, each demonstration's keys read once for all queries.
+    Every query is checked against the oracle, gather maps exact."""
+    cfg = dbsa.DbsaConfig(8, 2, 128, "bf16", 5e5, 2)
+    rng = np.random.default_rng(33)
+    lens = np.concatenate([[200], rng.integers(12, 31, size=200)])
+    offs = offsets(lens)
+    nb, T = len(lens), int(offs[-1])
+    sels = [np.concatenate([[0], np.sort(rng.permutation(np.arange(1, nb))[:60])])
+            for _ in range(32)]
+    run = Stage2Run(cfg, offs, sels, 1, 9, seed=34)
+    assert run.ws.numel() >= cfg.n_kv_heads * T * cfg.head_dim * 2   # the block-major layout
+    run.run().check("demo-granular decode")
+    peaky = Stage2Run(cfg, offs, sels[:8], 1, 9, seed=35, q_scale=4.0).run()
+    peaky.check("demo-granular decode peaky", atol=ATOL_PEAKY)
+
+
 def test_plan_staging_reuse_and_threads():
     """A call's host-built plan reaches the device through a per-thread ring of
     eight page-locked staging slots; a slot is refilled only after the read
