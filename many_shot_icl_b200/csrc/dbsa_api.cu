@@ -69,6 +69,11 @@ constexpr size_t kAlign = 1024;
 // kernel; longer passes (prompt passes) keep the tail on the per-query
 // mma.sync kernel, which shares each tail key among all the rows.
 constexpr int kTailMergeMaxRows = 32;
+// Per-query selections (short segments the block-major path cannot share
+// cheaply) with at least this many query rows per (query, KV head) run in
+// compact mode on the tensor core; fewer rows stay on the per-query mma.sync
+// kernel.
+constexpr int kCompactMinRows = 64;
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Copies bytes from page-locked host memory (read over the bus by the SMs)
@@ -377,6 +382,14 @@ struct GatherPlan {
   // each query's key sequence is split into a few items that the per-query
   // kernel gathers segment by segment; no packed rows, no tensor-core tiles
   bool per_query = false;
+  // compact mode (a per-query selection of short segments with many query
+  // rows, e.g. a demonstration-granular prompt pass): every query's gathered
+  // keys, rotated at their fresh positions, and its values are written to a
+  // compact buffer (query q's rows start at compact_base[q]); the tensor-core
+  // kernel then attends per (KV head, query, 128-row tile) over them
+  bool compact = false;
+  std::vector<int32_t> compact_base;
+  int64_t compact_rows = 0;
   // the query rows of all (query, block) items packed block by block, and the
   // tile list of the tensor-core kernel over them
   int32_t tc_rows = 0;
@@ -434,7 +447,7 @@ dbsa_status gather_plan(const dbsa_config *cfg, const int32_t *offs, int32_t nb,
       s.cache_row0 = offs[b];
       s.pos0 = (int32_t)p;
       s.len = offs[b + 1] - offs[b];
-      s.pad = 0;
+      s.query = q;
       gp.segs.push_back(s);
       p += s.len;
     }
@@ -463,6 +476,60 @@ dbsa_status gather_plan(const dbsa_config *cfg, const int32_t *offs, int32_t nb,
     const double block_bytes =
         (double)offs[nb] * Hkv * D * (2.0 * elt + 4.0) + (double)gp.segs.size() * per_pair;
     per_query = !(block_bytes < per_query_bytes);
+  }
+  if (per_query && R >= kCompactMinRows) {
+    // Compact mode: one block item per query over its whole gathered sequence
+    // (fresh positions 0 .. T'_q - 1, already applied to the compact keys, so
+    // the query rows are rotated at their own positions) and one tail item.
+    gp.compact = true;
+    gp.compact_base.resize(nq);
+    gp.packed_items.resize(nq);
+    gp.run_items.reserve(nq);
+    for (int q = 0; q < nq; ++q) {
+      S2Query &qi = gp.queries[q];
+      gp.compact_base[q] = (int32_t)gp.compact_rows;
+      gp.compact_rows += qi.n_gathered;
+      qi.item_begin = (int32_t)gp.items.size();
+      S2Item it;
+      it.query = q;
+      it.p_begin = 0;
+      it.p_end = qi.n_gathered;
+      it.p_lo = 0;
+      gp.packed_items[q] = (int32_t)gp.items.size();
+      gp.items.push_back(it);
+      S2Item tail;
+      tail.query = q;
+      tail.p_begin = qi.n_gathered & ~(kRopeLo - 1);
+      tail.p_end = qi.n_gathered + tail_len;
+      tail.p_lo = qi.n_gathered;
+      gp.run_items.push_back((int32_t)gp.items.size());
+      gp.items.push_back(tail);
+      qi.n_items = 2;
+    }
+    if (gp.compact_rows > (1 << 30))
+      return fail(DBSA_ERR_INVALID_ARG, "gathered contexts of the batch too long");
+    gp.item_row0.assign(gp.items.size(), -1);
+    for (int q = 0; q < nq; ++q) gp.item_row0[gp.packed_items[q]] = q * R;
+    gp.tc_rows = nq * R;
+    gp.tc_tiles.reserve((size_t)cfg->n_kv_heads * nq * ((R + kTileRows - 1) / kTileRows));
+    for (int c = 0; c < cfg->n_kv_heads; ++c)
+      for (int q = 0; q < nq; ++q)
+        for (int m = 0; m < R; m += kTileRows) {
+          dbsa_tile_item t;
+          std::memset(&t, 0, sizeof t);
+          t.head = c;
+          t.q_row0 = q * R + m;
+          t.q_pos0 = 1 << 30;  // after every gathered key: no causal limit
+          t.n_rows = std::min(kTileRows, R - m);
+          t.n_ranges = 1;
+          t.block = q;
+          t.k_row0[0] = gp.compact_base[q];
+          t.v_row0[0] = gp.compact_base[q];
+          t.pos0[0] = 0;
+          t.len[0] = gp.queries[q].n_gathered;
+          gp.tc_tiles.push_back(t);
+        }
+    return DBSA_OK;
   }
   if (per_query) {
     gp.per_query = true;
@@ -589,7 +656,8 @@ S1Layout s1_layout(const dbsa_config *cfg, int64_t max_pos, int64_t n_items, int
 
 struct S2Layout {
   size_t rope, queries, segs, items, run_items, packed_items, item_row0,
-      tc_tiles, offs, blob_end, q_rot_pos, k_hat, v_hat, q_hat, part_acc, part_ml, total;
+      tc_tiles, offs, compact_base, blob_end, q_rot_pos, k_hat, v_hat, q_hat, part_acc, part_ml,
+      total;
   int32_t n_hi;
 };
 // prepared: the block-relative keys (and bf16 V of fp32 caches) come from a
@@ -608,14 +676,21 @@ S2Layout s2_layout(const dbsa_config *cfg, const GatherPlan &gp, int32_t n_new,
   l.item_row0 = cv.take(gp.item_row0.size() * sizeof(int32_t));
   l.tc_tiles = cv.take(gp.tc_tiles.size() * sizeof(dbsa_tile_item));
   l.offs = cv.take((size_t)(offs_count(gp)) * sizeof(int32_t));
+  l.compact_base = cv.take(gp.compact_base.size() * sizeof(int32_t));
   l.blob_end = cv.take(0);
   l.q_rot_pos = cv.take(gp.items.size() * sizeof(int32_t));
   const int64_t T = gp.cache_rows;
-  const bool own_keys = !prepared && !gp.per_query;
-  l.k_hat = cv.take(own_keys ? (size_t)cfg->n_kv_heads * T * cfg->head_dim * 2 : 0);
-  l.v_hat = cv.take(own_keys && cfg->dtype == DBSA_F32
-                        ? (size_t)cfg->n_kv_heads * T * cfg->head_dim * 2
-                        : 0);
+  if (gp.compact) {
+    // every query's gathered keys (rotated) and values, bf16 [Hkv][rows][D]
+    l.k_hat = cv.take((size_t)cfg->n_kv_heads * gp.compact_rows * cfg->head_dim * 2);
+    l.v_hat = cv.take((size_t)cfg->n_kv_heads * gp.compact_rows * cfg->head_dim * 2);
+  } else {
+    const bool own_keys = !prepared && !gp.per_query;
+    l.k_hat = cv.take(own_keys ? (size_t)cfg->n_kv_heads * T * cfg->head_dim * 2 : 0);
+    l.v_hat = cv.take(own_keys && cfg->dtype == DBSA_F32
+                          ? (size_t)cfg->n_kv_heads * T * cfg->head_dim * 2
+                          : 0);
+  }
   l.q_hat = cv.take((size_t)cfg->n_kv_heads * gp.tc_rows * cfg->head_dim * 2);
   const size_t rows = gp.items.size() * (size_t)cfg->n_q_heads * n_new;
   l.part_acc = cv.take(rows * cfg->head_dim * sizeof(uint16_t));
@@ -1101,6 +1176,8 @@ dbsa_status gather_impl(const dbsa_config *cfg, const void *k_cache, const void 
     std::memcpy(blob + (L.tc_tiles - L.queries), gp.tc_tiles.data(),
                 gp.tc_tiles.size() * sizeof(dbsa_tile_item));
     std::memcpy(blob + (L.offs - L.queries), offs_host, (size_t)(nb + 1) * sizeof(int32_t));
+    std::memcpy(blob + (L.compact_base - L.queries), gp.compact_base.data(),
+                gp.compact_base.size() * sizeof(int32_t));
     if (fixed != nullptr)
       e = cudaMemcpyAsync(at<void>(workspace, L.queries), blob, blob_bytes,
                           cudaMemcpyHostToDevice, st);
@@ -1135,7 +1212,81 @@ dbsa_status gather_impl(const dbsa_config *cfg, const void *k_cache, const void 
   a.scale_log2 = scale_log2(cfg);
   a.rope = rope;
   const bool f32 = cfg->dtype == DBSA_F32;
-  if (gp.per_query) {
+  if (gp.compact) {
+    // every query's gathered keys (rotated at their fresh positions) and
+    // values into the compact buffers (the gather map comes from this
+    // kernel), the packed query rows at their own positions, the tensor-core
+    // kernel over (kv head, query, 128-row tile) in partial mode, then the
+    // tail keys on the per-query kernel and the merge below
+    CompactArgs ca{};
+    ca.k_cache = k_cache;
+    ca.v_cache = v_cache;
+    ca.cap = cap;
+    ca.Hkv = cfg->n_kv_heads;
+    ca.segs = a.segs;
+    ca.n_segs = (int32_t)gp.segs.size();
+    ca.base = at<int32_t>(workspace, L.compact_base);
+    ca.rows = gp.compact_rows;
+    ca.k_hat = at<void>(workspace, L.k_hat);
+    ca.v_hat = at<void>(workspace, L.v_hat);
+    ca.dbg = dbg_map;
+    ca.dbg_cap = dbg_cap;
+    ca.rope = rope;
+    if ((e = launch_compact(ca, cfg->head_dim, f32, st)) != cudaSuccess)
+      return cuda_fail(e, "compact gather");
+    count_launches(1);
+    QHatArgs qa{};
+    qa.q_new = q_new;
+    qa.n_new = n_new;
+    qa.tail_len = tail_len;
+    qa.Hq = cfg->n_q_heads;
+    qa.Hkv = cfg->n_kv_heads;
+    qa.queries = a.queries;
+    qa.items = a.items;
+    qa.n_items = a.n_items;
+    qa.item_row0 = at<int32_t>(workspace, L.item_row0);
+    qa.rows = gp.tc_rows;
+    qa.q_hat = at<void>(workspace, L.q_hat);
+    qa.q_rot_pos = nullptr;
+    qa.rope = rope;
+    if ((e = launch_qhat(qa, cfg->head_dim, f32, st)) != cudaSuccess)
+      return cuda_fail(e, "query rotation");
+    count_launches(1);
+    a.dbg_map = nullptr;  // written by the compact gather above
+    Stage1Args sa{};
+    sa.q_rot = qa.q_hat;
+    sa.q_rows = gp.tc_rows;
+    sa.k_rot = ca.k_hat;
+    sa.k_rows = gp.compact_rows;
+    sa.v = ca.v_hat;
+    sa.v_rows = gp.compact_rows;
+    sa.v_head_stride = gp.compact_rows;
+    sa.out = nullptr;
+    sa.Hq = cfg->n_kv_heads;  // packed rows are per kv head
+    sa.Hkv = cfg->n_kv_heads;
+    sa.items = at<dbsa_tile_item>(workspace, L.tc_tiles);
+    sa.n_items = (int32_t)gp.tc_tiles.size();
+    sa.scale_log2 = a.scale_log2;
+    sa.status = at<int>(workspace, 0);
+    sa.part.acc = a.part_acc;
+    sa.part.ml = a.part_ml;
+    sa.part.packed_items = at<int32_t>(workspace, L.packed_items);
+    sa.part.group = cfg->n_q_heads / cfg->n_kv_heads;
+    sa.part.Hq = cfg->n_q_heads;
+    sa.part.n_new = n_new;
+    sa.part.dbg = nullptr;
+    sa.wait_limit_ns = wait_expiry;
+    sa.withhold_tiles = wait_expiry != 0;
+    {
+      ProfileScope prof(st);
+      e = launch_stage1(sa, cfg->head_dim, false, num_sms(), st);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "stage-2 tensor-core attention");
+    count_launches(1);
+    if ((e = launch_stage2_main(a, cfg->head_dim, f32, st)) != cudaSuccess)  // tail items
+      return cuda_fail(e, "stage-2 tail attention");
+    count_launches(1);
+  } else if (gp.per_query) {
     // the per-query kernel over every split item (it writes the gather map
     // from its own segment walk)
     {

@@ -34,7 +34,7 @@ struct S2Segment {
   int32_t cache_row0;  // first cache row of the block
   int32_t pos0;        // fresh position of its first token
   int32_t len;         // tokens
-  int32_t pad;
+  int32_t query;       // the query that selected it
 };
 struct S2Query {
   int32_t seg_begin;   // index into the segment array
@@ -154,6 +154,24 @@ struct QHatArgs {
   RopeTables rope;
 };
 cudaError_t launch_qhat(const QHatArgs &a, int head_dim, bool f32, cudaStream_t st);
+
+// Compact mode of Stage 2: every query's gathered keys, rotated at their fresh
+// positions, and its values, bf16 [Hkv][rows][D]; query q's gathered token p
+// goes to row base[q] + p.  With dbg non-null, dbg[q][p] = (cache row, p).
+struct CompactArgs {
+  const void *k_cache, *v_cache;   // [Hkv][cap][D], input dtype
+  int64_t cap;
+  int32_t Hkv;
+  const S2Segment *segs;           // every query's segments
+  int32_t n_segs;
+  const int32_t *base;             // [nq]: compact row of each query's first gathered token
+  int64_t rows;                    // sum of the queries' gathered tokens
+  void *k_hat, *v_hat;             // bf16 [Hkv][rows][D]
+  int32_t *dbg;
+  int64_t dbg_cap;
+  RopeTables rope;
+};
+cudaError_t launch_compact(const CompactArgs &a, int head_dim, bool f32, cudaStream_t st);
 
 // Stage-1 tcgen05 attention over a tile list.
 struct Stage1Args {

@@ -211,6 +211,72 @@ __global__ void __launch_bounds__(256) qhat_kernel(QHatArgs a) {
   }
 }
 
+// Compact mode of Stage 2: compact row r of KV head c holds gathered token p
+// of query q (r = base[q] + p): its key rotated at its fresh position p, and
+// its value, both bf16.  One warp per (segment, KV head) walks the segment's
+// contiguous cache rows, four rows in flight; lane l owns the frequencies
+// 2l and 2l + 1 (lanes 2l >= D/2 have none), so each rotate-half pair
+// (i, i + D/2) stays in one lane.  With a gather map requested, KV head 0's
+// warp records (cache row, p) for every row it reads.
+template <int D, typename T>
+__global__ void __launch_bounds__(256) compact_kernel(CompactArgs a) {
+  constexpr int H = D / 2;
+  const int lane = threadIdx.x & 31;
+  const bool has_pair = 2 * lane < H;
+  const int64_t n_tasks = (int64_t)a.n_segs * a.Hkv;
+  const int64_t warp0 = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+  const int64_t n_warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t task = warp0; task < n_tasks; task += n_warps) {
+    const int c_ = (int)(task % a.Hkv);
+    const S2Segment sg = a.segs[task / a.Hkv];
+    const int64_t rbase = (int64_t)__ldg(a.base + sg.query) + sg.pos0;
+    const T *ksrc = static_cast<const T *>(a.k_cache) + ((int64_t)c_ * a.cap + sg.cache_row0) * D;
+    const T *vsrc = static_cast<const T *>(a.v_cache) + ((int64_t)c_ * a.cap + sg.cache_row0) * D;
+    bf16 *kdst = static_cast<bf16 *>(a.k_hat) + ((int64_t)c_ * a.rows + rbase) * D;
+    bf16 *vdst = static_cast<bf16 *>(a.v_hat) + ((int64_t)c_ * a.rows + rbase) * D;
+    const int i = 2 * lane;   // this lane's frequencies i, i + 1
+    for (int r0 = 0; r0 < sg.len; r0 += 4) {
+      // the four rows' loads first (the stores below could alias them as far
+      // as the compiler knows), then rotation and stores
+      float kl[4][2], kh[4][2], vl[4][2], vh[4][2];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int r = r0 + k;
+        if (has_pair && r < sg.len) {
+          load2(ksrc + (int64_t)r * D + i, kl[k]);
+          load2(ksrc + (int64_t)r * D + H + i, kh[k]);
+          load2(vsrc + (int64_t)r * D + i, vl[k]);
+          load2(vsrc + (int64_t)r * D + H + i, vh[k]);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int r = r0 + k;
+        if (r >= sg.len) break;
+        const int64_t pos = (int64_t)sg.pos0 + r;
+        if (has_pair) {
+          float cs[2], sn[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) rope_cs1(a.rope, pos, i + e, H, cs[e], sn[e]);
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const float x = kl[k][e], y = kh[k][e];
+            kl[k][e] = __fmaf_rn(x, cs[e], __fmul_rn(-y, sn[e]));
+            kh[k][e] = __fmaf_rn(y, cs[e], __fmul_rn(x, sn[e]));
+          }
+          store2_bf16(kdst + (int64_t)r * D + i, kl[k]);
+          store2_bf16(kdst + (int64_t)r * D + H + i, kh[k]);
+          store2_bf16(vdst + (int64_t)r * D + i, vl[k]);
+          store2_bf16(vdst + (int64_t)r * D + H + i, vh[k]);
+        }
+        if (a.dbg != nullptr && c_ == 0 && lane == 0)   // the row read and its rotation position
+          *reinterpret_cast<int2 *>(a.dbg + ((int64_t)sg.query * a.dbg_cap + pos) * 2) =
+              make_int2(sg.cache_row0 + r, (int)pos);
+      }
+    }
+  }
+}
+
 int grid_for(int64_t n_units, int block) {
   int64_t g = (n_units + block - 1) / block;
   if (g > 148 * 16) g = 148 * 16;
@@ -242,6 +308,19 @@ cudaError_t launch_qhat(const QHatArgs &a, int head_dim, bool f32, cudaStream_t 
   } else {
     if (f32) qhat_kernel<64, float><<<g, 256, 0, st>>>(a);
     else qhat_kernel<64, bf16><<<g, 256, 0, st>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_compact(const CompactArgs &a, int head_dim, bool f32, cudaStream_t st) {
+  if (a.rows <= 0 || a.n_segs <= 0) return cudaSuccess;
+  const int g = grid_for((int64_t)a.n_segs * a.Hkv * 32, 256);
+  if (head_dim == 128) {
+    if (f32) compact_kernel<128, float><<<g, 256, 0, st>>>(a);
+    else compact_kernel<128, bf16><<<g, 256, 0, st>>>(a);
+  } else {
+    if (f32) compact_kernel<64, float><<<g, 256, 0, st>>>(a);
+    else compact_kernel<64, bf16><<<g, 256, 0, st>>>(a);
   }
   return cudaGetLastError();
 }

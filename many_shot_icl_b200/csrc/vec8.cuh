@@ -48,6 +48,23 @@ __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ void from_f32(float x, bf16 &d) { d = __float2bfloat16_rn(x); }
 __device__ __forceinline__ void from_f32(float x, float &d) { d = x; }
 
+// 2 consecutive elements as fp32, from bf16 (4 B) or fp32 (8 B) storage, and
+// back to bf16 (RNE).
+__device__ __forceinline__ void load2(const bf16 *p, float (&f)[2]) {
+  const uint32_t w = *reinterpret_cast<const uint32_t *>(p);
+  f[0] = __uint_as_float(w << 16);
+  f[1] = __uint_as_float(w & 0xFFFF0000u);
+}
+__device__ __forceinline__ void load2(const float *p, float (&f)[2]) {
+  const float2 v = *reinterpret_cast<const float2 *>(p);
+  f[0] = v.x;
+  f[1] = v.y;
+}
+__device__ __forceinline__ void store2_bf16(bf16 *p, const float (&f)[2]) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(f[0], f[1]);
+  *reinterpret_cast<__nv_bfloat162 *>(p) = h;
+}
+
 // 8 consecutive elements as fp32, from bf16 (16 B) or fp32 (32 B) storage.
 __device__ __forceinline__ void load8(const bf16 *p, float (&f)[8]) {
   const uint4 r = *reinterpret_cast<const uint4 *>(p);

@@ -196,9 +196,13 @@ def test_prepared_block_keys_bit_identical(dtype, Hq, Hkv, D, n_new, tail_len):
 def test_demonstration_granular_gather(n_new, tail_len):
     """Example-level selection ([DBSA notes] §Ablations, selection granularity):
     the offsets table makes every demonstration after the sink block its own
-    block, and each query selects the sink and single demonstrations.  Such
-    short segments go through the per-query split path (its workspace holds
-    no block-relative keys); checked against the oracle, gather maps exact."""
+    block, and each query selects the sink and single demonstrations.  These
+    few queries share little, so the keys are not shared across queries:
+    with 64 query rows per (query, KV head) (16 tokens x 4 heads) each query's
+    gathered keys are rotated into a compact buffer and attended on the
+    tensor core; a single-token pass takes the per-query split kernel (its
+    workspace holds no rotated keys).  Checked against the oracle, gather
+    maps exact."""
     cfg = dbsa.DbsaConfig(8, 2, 128, "bf16", 5e5, 2)
     rng = np.random.default_rng(21)
     lens = np.concatenate([[200], rng.integers(8, 31, size=60)])
@@ -207,7 +211,11 @@ def test_demonstration_granular_gather(n_new, tail_len):
     sels = [np.concatenate([[0], rng.permutation(np.arange(1, nb))[:k]]) for k in (18, 3, 40, 1)]
     run = Stage2Run(cfg, offs, sels, n_new, tail_len, seed=5)
     T = int(offs[-1])
-    assert run.ws.numel() < cfg.n_kv_heads * T * cfg.head_dim * 2
+    gathered = sum(int(sum(offs[b + 1] - offs[b] for b in s_)) for s_ in sels)
+    if n_new == 1:
+        assert run.ws.numel() < cfg.n_kv_heads * T * cfg.head_dim * 2
+    else:       # the compact buffers: rotated keys and values of every gathered token
+        assert run.ws.numel() >= 2 * cfg.n_kv_heads * gathered * cfg.head_dim * 2
     run.run().check("demo-granular")
     peaky = Stage2Run(cfg, offs, sels[:2], n_new, tail_len, seed=6, q_scale=4.0).run()
     peaky.check("demo-granular peaky", atol=ATOL_PEAKY)
