@@ -203,13 +203,20 @@ def test_workspace_sizes(lib):
     wg = dbsa.gather_workspace_size(cfg, offs, sel_ptr, sel, 40, 40)
     assert wg > 0
     assert dbsa.gather_workspace_size(cfg, offs, sel_ptr, np.array([2, 3, 9, 0, 1]), 40, 40) == 0
-    # a demonstration-granular selection (blocks of ~30 tokens) goes per query:
-    # its workspace holds no block-relative keys
+    # a demonstration-granular selection (blocks of ~30 tokens) of one query
+    # shares nothing across queries, so it goes per query.  A single-token
+    # pass runs on the per-query kernel: its workspace holds no rotated keys.
+    # A 40-token pass (160 query rows per KV head) runs in compact mode: the
+    # query's gathered keys, rotated, and its values, bf16 [Hkv][T'][D] each
     lens = np.concatenate([[1500], np.full(100, 30)])
     doffs = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
     dsp, dsel = dbsa.selection_csr([np.arange(0, 101, 3)])
+    gathered = 1500 + 30 * (len(dsel) - 1)
+    wd1 = dbsa.gather_workspace_size(cfg, doffs, dsp, dsel, 1, 41)
+    assert 0 < wd1 < 8 * int(doffs[-1]) * 256
     wd = dbsa.gather_workspace_size(cfg, doffs, dsp, dsel, 40, 40)
-    assert 0 < wd < 8 * int(doffs[-1]) * 256
+    compact = 2 * 8 * gathered * 128 * 2
+    assert compact <= wd < compact + (8 << 20)
     # prepared block keys: K at block-relative positions, bf16 [Hkv][T][D], plus
     # RoPE tables (cos and sin, D/2 floats a row) for positions below T + 8192:
     # (T + 8192) / 16 coarse rows and 16 fine rows
