@@ -71,11 +71,25 @@ def load_peaks():
 
 
 # ------------------------------------------------------------------ workload
+def head_shard(n_q_heads: int, n_kv_heads: int, rank: int, world: int):
+    """The KV heads [kv0, kv1) and query heads [q0, q1) a rank owns when one
+    context is split across `world` GPUs by KV-head groups: attention is
+    independent per head, so each rank runs every call on its own heads and no
+    collective is needed on the data path."""
+    if n_kv_heads % world:
+        raise ValueError("%d KV heads do not split over %d ranks" % (n_kv_heads, world))
+    per, g = n_kv_heads // world, n_q_heads // n_kv_heads
+    kv0 = rank * per
+    return kv0, kv0 + per, kv0 * g, (kv0 + per) * g
+
+
 class Workload:
-    """Offsets, selections and per-layer tensors of one batch."""
+    """Offsets, selections and per-layer tensors of one batch.  With
+    heads=(rank, world), the batch is the same on every rank (one context)
+    and this rank holds only its KV-head group of it."""
 
     def __init__(self, w: inputs.Workload, layers: int, device, rank: int = 0,
-                 append_room: int = 0):
+                 append_room: int = 0, heads=None):
         import torch
         self.w = w
         self.layers = layers
@@ -83,30 +97,42 @@ class Workload:
         self.nb = len(self.offs) - 1
         self.T = int(self.offs[-1])
         self.cap = self.T + append_room
-        self.sels = inputs.selections(w, seed_offset=rank)
+        batch = 0 if heads is not None else rank   # whose batch: one shared, or one per rank
+        self.sels = inputs.selections(w, seed_offset=batch)
         from many_shot_icl_b200 import dbsa
         self.sel_ptr, self.sel = dbsa.selection_csr(self.sels)
-        self.cfg = dbsa.DbsaConfig(w.n_q_heads, w.n_kv_heads, w.head_dim, w.dtype, w.rope_theta,
+        kv0, kv1, q0, q1 = (head_shard(w.n_q_heads, w.n_kv_heads, *heads) if heads is not None
+                            else (0, w.n_kv_heads, 0, w.n_q_heads))
+        self.heads = (kv0, kv1, q0, q1)
+        self.cfg = dbsa.DbsaConfig(q1 - q0, kv1 - kv0, w.head_dim, w.dtype, w.rope_theta,
                                    w.window_j)
-        Hq, Hkv, D, T = w.n_q_heads, w.n_kv_heads, w.head_dim, self.T
+        Hq, Hkv, D, T = q1 - q0, kv1 - kv0, w.head_dim, self.T
         dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
         self.dt = dt
         self.nq = w.n_queries
         self.tail_cap = w.query_tokens + w.decode_steps
         self.q, self.k, self.v, self.kc, self.vc, self.out = [], [], [], [], [], []
         self.qp, self.qd, self.kt, self.vt = [], [], [], []
+        Hq_all, Hkv_all = w.n_q_heads, w.n_kv_heads
+
+        def gen(shape, seed, lo, hi):
+            # the tensor of the whole batch (all heads, axis -2), then this
+            # rank's heads [lo, hi) of it
+            full = inputs.randn(shape[:-2] + (shape[-2], D), seed, w.dtype, device)
+            return full if (lo, hi) == (0, shape[-2]) else full[..., lo:hi, :].contiguous()
+
         for l in range(layers):
-            s = lambda role, step=0: inputs.tensor_seed(w, l, role, step) + 7919 * rank
-            self.q.append(inputs.randn((T, Hq, D), s(0), w.dtype, device))
-            self.k.append(inputs.randn((T, Hkv, D), s(1), w.dtype, device))
-            self.v.append(inputs.randn((T, Hkv, D), s(2), w.dtype, device))
+            s = lambda role, step=0: inputs.tensor_seed(w, l, role, step) + 7919 * batch
+            self.q.append(gen((T, Hq_all, D), s(0), q0, q1))
+            self.k.append(gen((T, Hkv_all, D), s(1), kv0, kv1))
+            self.v.append(gen((T, Hkv_all, D), s(2), kv0, kv1))
             self.kc.append(torch.empty((Hkv, self.cap, D), dtype=dt, device=device))
             self.vc.append(torch.empty((Hkv, self.cap, D), dtype=dt, device=device))
             self.out.append(torch.empty((T, Hq, D), dtype=dt, device=device))
-            self.qp.append(inputs.randn((self.nq, w.query_tokens, Hq, D), s(3, 0), w.dtype, device))
-            self.qd.append(inputs.randn((self.nq, 1, Hq, D), s(3, 1), w.dtype, device))
-            self.kt.append(inputs.randn((self.nq, self.tail_cap, Hkv, D), s(3, 2), w.dtype, device))
-            self.vt.append(inputs.randn((self.nq, self.tail_cap, Hkv, D), s(3, 3), w.dtype, device))
+            self.qp.append(gen((self.nq, w.query_tokens, Hq_all, D), s(3, 0), q0, q1))
+            self.qd.append(gen((self.nq, 1, Hq_all, D), s(3, 1), q0, q1))
+            self.kt.append(gen((self.nq, self.tail_cap, Hkv_all, D), s(3, 2), kv0, kv1))
+            self.vt.append(gen((self.nq, self.tail_cap, Hkv_all, D), s(3, 3), kv0, kv1))
         self.out_p = torch.empty((self.nq, w.query_tokens, Hq, D), dtype=dt, device=device)
         self.out_d = torch.empty((self.nq, 1, Hq, D), dtype=dt, device=device)
         # keys at block-relative positions: refreshed once per layer after each
@@ -164,7 +190,8 @@ class Stage2Work:
         w = wl.w
         # plain numbers only: no reference to the workload's device tensors
         self.T, self.nq, self.passes = wl.T, wl.nq, wl.passes()
-        self.D, self.Hq, self.Hkv = w.head_dim, w.n_q_heads, w.n_kv_heads
+        # this rank's heads (all of them unless the batch is split by heads)
+        self.D, self.Hq, self.Hkv = w.head_dim, wl.cfg.n_q_heads, wl.cfg.n_kv_heads
         self.bpe = 2 if w.dtype == "bf16" else 4
         self.gath = wl.gathered()
         self.union_tokens = float(sum(int(wl.offs[b + 1] - wl.offs[b])
@@ -451,7 +478,7 @@ def append_series(wl: Workload, n_appends: int):
     all_offs = dbsa.group_blocks(lens, w.demos_per_block)
     assert np.array_equal(all_offs[:wl.nb + 1], wl.offs)
     Lmax = int(np.diff(all_offs[wl.nb:]).max())
-    Hq, Hkv, D = w.n_q_heads, w.n_kv_heads, w.head_dim
+    Hq, Hkv, D = wl.cfg.n_q_heads, wl.cfg.n_kv_heads, w.head_dim  # this rank's heads
     qa = inputs.randn((Lmax, Hq, D), 4242, w.dtype, "cuda")
     ka = inputs.randn((Lmax, Hkv, D), 4243, w.dtype, "cuda")
     va = inputs.randn((Lmax, Hkv, D), 4244, w.dtype, "cuda")
@@ -489,7 +516,7 @@ def comparators(wl: Workload, n_ret_queries: int = 4):
     import torch
     from many_shot_icl_b200 import dbsa
     w, L = wl.w, wl.layers
-    Hq, Hkv, D = w.n_q_heads, w.n_kv_heads, w.head_dim
+    Hq, Hkv, D = wl.cfg.n_q_heads, wl.cfg.n_kv_heads, w.head_dim  # this rank's heads
     ev = lambda: torch.cuda.Event(enable_timing=True)
 
     def timed(fn, reps=2):
@@ -743,6 +770,12 @@ def weak_scaling_value(units_per_rank: float, world: int, t_max: float) -> float
     return units_per_rank * world / t_max
 
 
+def strong_scaling_value(units: float, t_max: float) -> float:
+    """Whole-job throughput when the ranks split one batch (by heads): its
+    units over the slowest rank's time."""
+    return units / t_max
+
+
 def barrier(world):
     if world > 1:
         import torch.distributed as tdist
@@ -795,6 +828,9 @@ def main():
                     help="skip the retrieval-ICL / fixed-ICL attention comparators")
     ap.add_argument("--no-per-config", action="store_true",
                     help="skip the 30k and 128k workload measurements")
+    ap.add_argument("--shard", choices=["batch", "heads"], default="batch",
+                    help="N > 1: an independent batch per GPU (weak scaling), or one batch "
+                         "split by KV-head groups (strong scaling)")
     ap.add_argument("--profile-only", choices=["stage1", "stage2"], default=None,
                     help="run W + K steps of one stage only and exit (for ncu captures)")
     args = ap.parse_args()
@@ -817,7 +853,9 @@ def main():
     layers = args.layers or w.n_layers
     n_appends = inputs.L31_8B_APPEND.n_appends if args.appends is None else args.appends
     room = (n_appends + 1) * w.demos_per_block * w.demo_len_hi if n_appends else 0
-    wl = Workload(w, layers, "cuda", rank=rank, append_room=room)
+    by_heads = args.shard == "heads"
+    wl = Workload(w, layers, "cuda", rank=rank, append_room=room,
+                  heads=(rank, world) if by_heads else None)
     torch.cuda.synchronize()
     if args.profile_only:
         return profile_only(wl, args)
@@ -855,7 +893,7 @@ def main():
     t_s2 = max_over_ranks(t_s2, world)
 
     # algorithmic work
-    Hq, Hkv, D = w.n_q_heads, w.n_kv_heads, w.head_dim
+    Hq, Hkv, D = wl.cfg.n_q_heads, wl.cfg.n_kv_heads, w.head_dim  # this rank's heads
     tiles = dbsa.stage1_tile_count(wl.cfg, wl.offs)
     tile_flop = 4.0 * 128 * 128 * D * tiles                      # per layer, unmasked tiles
     exact_flop = 4.0 * D * Hq * stage1_exact_pairs(wl.offs, w.window_j)  # per layer
@@ -925,8 +963,13 @@ def main():
 
     T = wl.T
     q_tokens = wl.nq * (w.query_tokens + w.decode_steps)
-    s1_tok_s = weak_scaling_value(T, world, t_s1)
-    s2_tok_s = weak_scaling_value(q_tokens, world, t_s2)
+    ranks_per_batch = 1 if by_heads else world   # batches the job completes per step
+    if by_heads:
+        s1_tok_s = strong_scaling_value(T, t_s1)
+        s2_tok_s = strong_scaling_value(q_tokens, t_s2)
+    else:
+        s1_tok_s = weak_scaling_value(T, world, t_s1)
+        s2_tok_s = weak_scaling_value(q_tokens, world, t_s2)
 
     # end to end from pinned host memory (rank-local)
     host = None
@@ -961,12 +1004,15 @@ def main():
         comp["setup_ratio_dbsa_over_fixed_icl"] = t_s1 / comp["fixed_icl"]["setup_s"]
 
     config = {"workload": w.name, "layers": layers, "context_tokens": T,
-              "blocks": wl.nb, "window_j": w.window_j, "q_heads": Hq, "kv_heads": Hkv,
+              "blocks": wl.nb, "window_j": w.window_j, "q_heads": w.n_q_heads,
+              "kv_heads": w.n_kv_heads,
               "head_dim": D, "queries": wl.nq, "query_tokens": w.query_tokens,
               "decode_steps": w.decode_steps,
               "retrieved_blocks_per_query": int(len(wl.sels[0]) - 1),
               "mean_gathered_tokens": float(gath.mean()),
-              "parallelism": "dp%d (independent batch per GPU)" % world,
+              "parallelism": ("heads/%d (one batch, KV heads [%d, %d) of %d on rank 0)"
+                              % (world, wl.heads[0], wl.heads[1], w.n_kv_heads)) if by_heads
+                             else "dp%d (independent batch per GPU)" % world,
               "l2": "inputs larger than L2 (per-layer Q/K/V/O ~%.1f GB)" %
                     ((wl.q[0].numel() * 2 + wl.k[0].numel() * 2 + wl.v[0].numel() * 2) * elt / 1e9)}
 
@@ -990,8 +1036,8 @@ def main():
         line = {
             "metric": METRIC, "value": round(s1_tok_s, 1), "unit": "tok/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_s_max * 1e3, 3),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
-            "data": "synthetic",
+            "higher_is_better": True, "scaling": "strong" if by_heads else "weak",
+            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
             "config": config,
             "value_definition": "context tokens encoded through all layers per second of Stage-1 time",
             "stage1": {"tok_s": round(s1_tok_s, 1), "s_per_step": round(t_s1, 4)},
@@ -1005,10 +1051,10 @@ def main():
             "rooflines": {k: v for k, v in by_name.items() if v is not None},
             "kernel_ms_per_step": {k: round(v, 2) for k, v in shares.items()},
             # null when the end-to-end pass was skipped (--e2e-steps 0)
-            "e2e": {"value": round(T * world / e2e_t1, 1) if e2e_t1 == e2e_t1 else None,
+            "e2e": {"value": round(T * ranks_per_batch / e2e_t1, 1) if e2e_t1 == e2e_t1 else None,
                     "unit": "tok/s",
                     "stage2_query_tok_s":
-                        round(q_tokens * world / e2e_t2, 1) if e2e_t2 == e2e_t2 else None,
+                        round(q_tokens * ranks_per_batch / e2e_t2, 1) if e2e_t2 == e2e_t2 else None,
                     "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
             "cpu_baseline": cpu,
             "append": app,
