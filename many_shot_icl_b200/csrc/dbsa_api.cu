@@ -79,7 +79,9 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // Copies bytes from page-locked host memory (read over the bus by the SMs)
 // into device memory: 16-byte words while both sides allow, then bytes.
 __global__ void __launch_bounds__(256) copy_from_host_kernel(uint8_t *dst, const uint8_t *src,
-                                                             size_t bytes) {
+                                                             size_t bytes, uint32_t *clear) {
+  // the call's status head, cleared here rather than by a separate memset
+  if (clear != nullptr && blockIdx.x == 0 && threadIdx.x < kStatusBytes / 4) clear[threadIdx.x] = 0;
   const size_t stride = (size_t)gridDim.x * blockDim.x;
   const size_t i0 = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   const bool vec = ((reinterpret_cast<uintptr_t>(dst) | reinterpret_cast<uintptr_t>(src)) & 15u) == 0;
@@ -135,13 +137,18 @@ class StagingRing {
         s.ev = nullptr;
       }
     }
-    if (s.cap < bytes) {
+    // All slots share one capacity, which doubles when a plan outgrows it;
+    // each slot is brought up to it on its next use, so that after one round
+    // of the ring no plan of that size reallocates (freeing a page-locked
+    // buffer synchronizes the device).
+    if (bytes > cap_all_) cap_all_ = align_up(std::max(bytes, 2 * cap_all_), size_t(1) << 16);
+    if (s.cap < cap_all_) {
       if (s.p != nullptr) {
         cudaFreeHost(s.p);  // its last read has completed
         count_host_alloc();
       }
       s.p = nullptr;
-      const size_t cap = align_up(std::max(bytes, 2 * s.cap), size_t(1) << 16);
+      const size_t cap = cap_all_;
       s.cap = 0;
       count_host_alloc();
       if ((e = cudaHostAlloc(&s.p, cap, cudaHostAllocPortable | cudaHostAllocMapped)) !=
@@ -157,27 +164,30 @@ class StagingRing {
     *host = s.p;
     return cudaSuccess;
   }
-  // Copies the first bytes of the buffer stage() returned to dst on stream st.
-  cudaError_t send(void *dst, size_t bytes, cudaStream_t st) {
+  // Copies the first bytes of the buffer stage() returned to dst on stream st
+  // and, when clear is given, zeroes the kStatusBytes status head there.
+  cudaError_t send(void *dst, size_t bytes, cudaStream_t st, void *clear = nullptr) {
     Slot &s = slots_[next_];
     next_ = (next_ + 1) % kSlots;
-    if (bytes > 0) {
-      const int grid = (int)std::min<size_t>((bytes + 4095) / 4096, 148);
+    if (bytes > 0 || clear != nullptr) {
+      const int grid = (int)std::max<size_t>(1, std::min<size_t>((bytes + 4095) / 4096, 148));
       copy_from_host_kernel<<<grid, 256, 0, st>>>(static_cast<uint8_t *>(dst),
-                                                 static_cast<const uint8_t *>(s.p), bytes);
+                                                 static_cast<const uint8_t *>(s.p), bytes,
+                                                 static_cast<uint32_t *>(clear));
       cudaError_t e = cudaGetLastError();
       if (e != cudaSuccess) return e;
       count_launches(1);
     }
     return cudaEventRecord(s.ev, st);
   }
-  cudaError_t upload(void *dst, const void *src, size_t bytes, cudaStream_t st) {
-    if (bytes == 0) return cudaSuccess;
+  cudaError_t upload(void *dst, const void *src, size_t bytes, cudaStream_t st,
+                     void *clear = nullptr) {
+    if (bytes == 0 && clear == nullptr) return cudaSuccess;
     void *h = nullptr;
-    cudaError_t e = stage(bytes, &h);
+    cudaError_t e = stage(std::max<size_t>(bytes, 16), &h);
     if (e != cudaSuccess) return e;
-    std::memcpy(h, src, bytes);
-    return send(dst, bytes, st);
+    if (bytes > 0) std::memcpy(h, src, bytes);
+    return send(dst, bytes, st, clear);
   }
 
  private:
@@ -190,14 +200,18 @@ class StagingRing {
   static constexpr int kSlots = 8;
   Slot slots_[kSlots];
   int next_ = 0;
+  size_t cap_all_ = 0;
 };
 
 StagingRing &staging_ring() {
   static thread_local StagingRing ring;
   return ring;
 }
-cudaError_t upload_async(void *dst, const void *src, size_t bytes, cudaStream_t st) {
-  return staging_ring().upload(dst, src, bytes, st);
+// Uploads a host-built plan through the staging ring; `clear` (a workspace
+// head, or null) gets its status bytes zeroed by the same kernel.
+cudaError_t upload_async(void *dst, const void *src, size_t bytes, cudaStream_t st,
+                         void *clear = nullptr) {
+  return staging_ring().upload(dst, src, bytes, st, clear);
 }
 
 // Sequential sub-allocation of the caller's workspace.
@@ -396,11 +410,27 @@ struct GatherPlan {
   int32_t nb = 0;
   int64_t cache_rows = 0;  // offs[nb]
   // packed_items[k]: the item owning packed rows [k R, (k + 1) R), R = g n_new
-  std::vector<int32_t> packed_items, item_row0;
+  std::vector<int32_t> packed_items;
+  // per item: (first packed row or -1 for a tail item, the position its query
+  // rows are rotated at for token 0, its query, 0), read by the packing kernel
+  std::vector<int4> item_meta;
   std::vector<dbsa_tile_item> tc_tiles;
 };
 
 int32_t offs_count(const GatherPlan &gp) { return gp.nb + 1; }
+
+// Packed rows of the items: packed_items[k] owns rows [k R, (k + 1) R), and
+// its query rows are rotated at (the query's token position - the item's
+// p_begin); the other items (tails) have no packed rows.
+void set_item_meta(GatherPlan &gp, int R, int32_t n_new, int32_t tail_len) {
+  gp.item_meta.assign(gp.items.size(), make_int4(-1, 0, 0, 0));
+  for (size_t k = 0; k < gp.packed_items.size(); ++k) {
+    const int32_t i = gp.packed_items[k];
+    const S2Item &it = gp.items[i];
+    const int32_t pos0 = gp.queries[it.query].n_gathered + tail_len - n_new - it.p_begin;
+    gp.item_meta[i] = make_int4((int32_t)(k * R), pos0, it.query, 0);
+  }
+}
 
 dbsa_status gather_plan(const dbsa_config *cfg, const int32_t *offs, int32_t nb, int32_t nq,
                         const int32_t *sel_ptr, const int32_t *sel, int32_t n_new,
@@ -508,8 +538,7 @@ dbsa_status gather_plan(const dbsa_config *cfg, const int32_t *offs, int32_t nb,
     }
     if (gp.compact_rows > (1 << 30))
       return fail(DBSA_ERR_INVALID_ARG, "gathered contexts of the batch too long");
-    gp.item_row0.assign(gp.items.size(), -1);
-    for (int q = 0; q < nq; ++q) gp.item_row0[gp.packed_items[q]] = q * R;
+    set_item_meta(gp, R, n_new, tail_len);
     gp.tc_rows = nq * R;
     gp.tc_tiles.reserve((size_t)cfg->n_kv_heads * nq * ((R + kTileRows - 1) / kTileRows));
     for (int c = 0; c < cfg->n_kv_heads; ++c)
@@ -602,8 +631,7 @@ dbsa_status gather_plan(const dbsa_config *cfg, const int32_t *offs, int32_t nb,
       qi.n_items = (int32_t)gp.items.size() - qi.item_begin;
     }
     // rows packed block by block: packed_items[k] owns rows [k R, (k + 1) R)
-    gp.item_row0.assign(gp.items.size(), -1);
-    for (size_t k = 0; k < gp.packed_items.size(); ++k) gp.item_row0[gp.packed_items[k]] = (int32_t)(k * R);
+    set_item_meta(gp, R, n_new, tail_len);
     gp.tc_rows = (int32_t)(gp.packed_items.size() * R);
     std::vector<int32_t> block_row0(nb, 0), block_rows(nb, 0);
     size_t n_tiles = 0;
@@ -655,7 +683,7 @@ S1Layout s1_layout(const dbsa_config *cfg, int64_t max_pos, int64_t n_items, int
 }
 
 struct S2Layout {
-  size_t rope, queries, segs, items, run_items, packed_items, item_row0,
+  size_t rope, queries, segs, items, run_items, packed_items, item_meta,
       tc_tiles, offs, compact_base, blob_end, q_rot_pos, k_hat, v_hat, q_hat, part_acc, part_ml,
       total;
   int32_t n_hi;
@@ -673,7 +701,7 @@ S2Layout s2_layout(const dbsa_config *cfg, const GatherPlan &gp, int32_t n_new,
   l.items = cv.take(gp.items.size() * sizeof(S2Item));
   l.run_items = cv.take(gp.run_items.size() * sizeof(int32_t));
   l.packed_items = cv.take(gp.packed_items.size() * sizeof(int32_t));
-  l.item_row0 = cv.take(gp.item_row0.size() * sizeof(int32_t));
+  l.item_meta = cv.take(gp.item_meta.size() * sizeof(int4));
   l.tc_tiles = cv.take(gp.tc_tiles.size() * sizeof(dbsa_tile_item));
   l.offs = cv.take((size_t)(offs_count(gp)) * sizeof(int32_t));
   l.compact_base = cv.take(gp.compact_base.size() * sizeof(int32_t));
@@ -839,14 +867,13 @@ dbsa_status dbsa_encode_blocks(const dbsa_config *cfg, const void *q, const void
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const bool f32 = cfg->dtype == DBSA_F32;
   cudaError_t e;
-  if ((e = cudaMemsetAsync(workspace, 0, kStatusBytes, st)) != cudaSuccess)
-    return cuda_fail(e, "status clear");
   RopeTables rope;
   if ((e = build_tables(workspace, L.rope, L.n_hi, cfg, st, &rope)) != cudaSuccess)
     return cuda_fail(e, "rope tables");
   count_launches(1);
+  // the upload kernel also clears the status word
   if ((e = upload_async(at<void>(workspace, L.items), items.data(),
-                        items.size() * sizeof(dbsa_tile_item), st)) != cudaSuccess)
+                        items.size() * sizeof(dbsa_tile_item), st, workspace)) != cudaSuccess)
     return cuda_fail(e, "tile list upload");
   IngestArgs ia{};
   ia.q = q;
@@ -936,14 +963,13 @@ dbsa_status dbsa_append_block(const dbsa_config *cfg, const void *q, const void 
   if ((s = check_ws(workspace, ws_bytes, Ly.total)) != DBSA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
-  if ((e = cudaMemsetAsync(workspace, 0, kStatusBytes, st)) != cudaSuccess)
-    return cuda_fail(e, "status clear");
   RopeTables rope;
   if ((e = build_tables(workspace, Ly.rope, Ly.n_hi, cfg, st, &rope)) != cudaSuccess)
     return cuda_fail(e, "rope tables");
   count_launches(1);
+  // the upload kernel also clears the status word
   if ((e = upload_async(at<void>(workspace, Ly.items), items.data(),
-                        items.size() * sizeof(dbsa_tile_item), st)) != cudaSuccess)
+                        items.size() * sizeof(dbsa_tile_item), st, workspace)) != cudaSuccess)
     return cuda_fail(e, "tile list upload");
   void *k_rot = at<void>(workspace, Ly.k_rot);
   void *v_bf16 = f32 ? at<void>(workspace, Ly.v_bf16) : nullptr;
@@ -1134,7 +1160,9 @@ dbsa_status gather_impl(const dbsa_config *cfg, const void *k_cache, const void 
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
-  if ((e = cudaMemsetAsync(workspace, 0, kStatusBytes, st)) != cudaSuccess)
+  // the status word: cleared here for the plain-copy upload of a fixed
+  // scratch, else by the staging upload's kernel below
+  if (fixed != nullptr && (e = cudaMemsetAsync(workspace, 0, kStatusBytes, st)) != cudaSuccess)
     return cuda_fail(e, "status clear");
   RopeTables rope;
   if (prepared && B.n_hi >= L.n_hi) {
@@ -1171,8 +1199,8 @@ dbsa_status gather_impl(const dbsa_config *cfg, const void *k_cache, const void 
                 gp.run_items.size() * sizeof(int32_t));
     std::memcpy(blob + (L.packed_items - L.queries), gp.packed_items.data(),
                 gp.packed_items.size() * sizeof(int32_t));
-    std::memcpy(blob + (L.item_row0 - L.queries), gp.item_row0.data(),
-                gp.item_row0.size() * sizeof(int32_t));
+    std::memcpy(blob + (L.item_meta - L.queries), gp.item_meta.data(),
+                gp.item_meta.size() * sizeof(int4));
     std::memcpy(blob + (L.tc_tiles - L.queries), gp.tc_tiles.data(),
                 gp.tc_tiles.size() * sizeof(dbsa_tile_item));
     std::memcpy(blob + (L.offs - L.queries), offs_host, (size_t)(nb + 1) * sizeof(int32_t));
@@ -1182,7 +1210,7 @@ dbsa_status gather_impl(const dbsa_config *cfg, const void *k_cache, const void 
       e = cudaMemcpyAsync(at<void>(workspace, L.queries), blob, blob_bytes,
                           cudaMemcpyHostToDevice, st);
     else
-      e = staging_ring().send(at<void>(workspace, L.queries), blob_bytes, st);
+      e = staging_ring().send(at<void>(workspace, L.queries), blob_bytes, st, workspace);
     if (e != cudaSuccess) return cuda_fail(e, "gather plan upload");
   }
   Stage2Args a{};
@@ -1241,10 +1269,8 @@ dbsa_status gather_impl(const dbsa_config *cfg, const void *k_cache, const void 
     qa.tail_len = tail_len;
     qa.Hq = cfg->n_q_heads;
     qa.Hkv = cfg->n_kv_heads;
-    qa.queries = a.queries;
-    qa.items = a.items;
     qa.n_items = a.n_items;
-    qa.item_row0 = at<int32_t>(workspace, L.item_row0);
+    qa.item_meta = at<int4>(workspace, L.item_meta);
     qa.rows = gp.tc_rows;
     qa.q_hat = at<void>(workspace, L.q_hat);
     qa.q_rot_pos = nullptr;
@@ -1321,10 +1347,8 @@ dbsa_status gather_impl(const dbsa_config *cfg, const void *k_cache, const void 
     qa.tail_len = tail_len;
     qa.Hq = cfg->n_q_heads;
     qa.Hkv = cfg->n_kv_heads;
-    qa.queries = a.queries;
-    qa.items = a.items;
     qa.n_items = a.n_items;
-    qa.item_row0 = at<int32_t>(workspace, L.item_row0);
+    qa.item_meta = at<int4>(workspace, L.item_meta);
     qa.rows = gp.tc_rows;
     qa.q_hat = at<void>(workspace, L.q_hat);
     qa.q_rot_pos = dbg_map != nullptr ? at<int32_t>(workspace, L.q_rot_pos) : nullptr;
@@ -1361,7 +1385,7 @@ dbsa_status gather_impl(const dbsa_config *cfg, const void *k_cache, const void 
     sa.part.q_rot_pos = qa.q_rot_pos;
     sa.part.tail_len = tail_len;
     sa.wait_limit_ns = wait_expiry;
-  sa.withhold_tiles = wait_expiry != 0;
+    sa.withhold_tiles = wait_expiry != 0;
     {
       ProfileScope prof(st);
       e = launch_stage1(sa, cfg->head_dim, false, num_sms(), st);

@@ -137,17 +137,16 @@ struct RelRopeArgs {
 };
 cudaError_t launch_rel_rope(const RelRopeArgs &a, int head_dim, bool f32, cudaStream_t st);
 
-// Packed query rows of the block-major pass: rows item_row0[i] .. + g*n_new
+// Packed query rows of the block-major pass: rows item_meta[i].x .. + g*n_new
 // of kv head c are query token u / local head hl (row u * g + hl) of split
 // item i (a (query, block) pair), rotated at (its position - the block's
-// fresh start).
+// fresh start), i.e. at item_meta[i].y + u.
 struct QHatArgs {
   const void *q_new;               // [nq][n_new][Hq][D]
   int32_t n_new, tail_len, Hq, Hkv;
-  const S2Query *queries;
-  const S2Item *items;             // block items: p_begin = fresh start P
-  int32_t n_items;                 // items (tail items have item_row0 = -1)
-  const int32_t *item_row0;
+  int32_t n_items;                 // items (tail items have item_meta.x = -1)
+  // per item: (first packed row, position of token 0's rotation, query, 0)
+  const int4 *item_meta;
   int32_t rows;                    // packed rows per kv head
   void *q_hat;                     // bf16 [Hkv][rows][D]
   int32_t *q_rot_pos;              // per item: rotation position of token 0, or null

@@ -186,12 +186,11 @@ __global__ void __launch_bounds__(256) qhat_kernel(QHatArgs a) {
     const int c_ = (int)((u / CP) % a.Hkv);
     const int tok = (int)((u / ((int64_t)CP * a.Hkv)) % a.n_new);
     const int item = (int)(u / ((int64_t)CP * a.Hkv * a.n_new));
-    const int row0 = __ldg(a.item_row0 + item);
+    const int4 meta = __ldg(a.item_meta + item);
+    const int row0 = meta.x;
     if (row0 < 0) continue;                      // a tail item: no packed rows
-    const S2Item it = a.items[item];
-    const int q = it.query;
-    const int64_t pos =
-        (int64_t)a.queries[q].n_gathered + a.tail_len - a.n_new + tok - it.p_begin;
+    const int q = meta.z;
+    const int64_t pos = (int64_t)meta.y + tok;   // (its position - the block's fresh start)
     // the position used for token 0 of the item, for the gather map
     if (a.q_rot_pos != nullptr && tok == 0 && c_ == 0 && cp == 0) a.q_rot_pos[item] = (int32_t)pos;
     const int i0 = cp * 8;

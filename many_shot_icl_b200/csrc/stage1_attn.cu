@@ -10,9 +10,9 @@
 // holds only the tiles that contain an allowed pair).
 //
 // One persistent CTA per SM walks items round-robin.  Warp roles:
-//   warp 0      TMA producer: two independent cursors, one for each item's Q
-//               tile (double-buffered) and its K tiles (3-stage ring), one
-//               for the V tiles (2-stage ring)
+//   warp 0      TMA producer: three independent cursors, for the items' Q
+//               tiles (double-buffered), K tiles (3-stage ring) and V tiles
+//               (2-stage ring)
 //   warp 1      TMEM owner; one thread issues O_h += P_h V_h for the two key
 //               halves of each tile (tcgen05, A from TMEM)
 //   warp 10     one thread issues S = Q K^T (tcgen05, both operands in SMEM)
@@ -26,8 +26,9 @@
 //               over its 64 scores held in registers (mask, max, rescale,
 //               exp2).  At an item's end they publish the merge factors of
 //               the two states and go on.
-//   warps 11..14 epilogue: combine O_0 and O_1 of the finished item, store
-//               the output, free O for the next item's first PV.
+//   warps 11..14 epilogue: combine O_0 and O_1 of the finished item, free O
+//               for the next item's first PV, and write the rows out (bf16:
+//               staged in the item's Q tile, then one bulk copy per row).
 // S = Q K^T lives in TMEM in two 128-column buffers (tile parity); each
 // warpgroup writes its 64 keys' P as bf16 pairs over the first 32 columns of
 // its own half of the S buffer, and O_0, O_1 take D columns each: 512 columns
@@ -62,7 +63,9 @@ constexpr uint32_t kFull = 0xFFFFFFFFu;
 // Ring depths (tiles in flight).  A K slot frees when its QK^T has run and is
 // needed again kStagesK tiles later; a V slot frees only after its PV, about
 // two tiles after the QK, and is needed kStagesV tiles later.  Q is double
-// buffered so that the next item's Q tile loads during the current item.
+// buffered so that the next item's Q tile loads during the current item; a Q
+// slot frees once the item's epilogue has staged and copied its rows out
+// through it.
 constexpr int kStagesK = 3;
 constexpr int kStagesV = 2;
 constexpr int kStagesQ = 2;
@@ -243,7 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStagesQ; ++s) {
       mbar_init(&bar[B_Q_FULL + s], 1);
-      mbar_init(&bar[B_Q_EMPTY + s], 1);
+      mbar_init(&bar[B_Q_EMPTY + s], 128);   // the epilogue warpgroup, after its staging
     }
     for (int s = 0; s < kStagesK; ++s) {
       mbar_init(&bar[B_K_FULL + s], 1);
@@ -279,11 +282,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ producer
-    // Two independent cursors over the CTA's tile sequence: K tiles (each
-    // item's Q tile first) and V tiles.  A K slot frees when its QK^T has
-    // run, a V slot only when its PV has run, which happens about two tiles
-    // later; separate cursors keep the K loads from queueing behind V slots.
-    // Neither cursor blocks: the thread polls whichever slot it needs next.
+    // Three independent cursors over the CTA's items: Q tiles (one per item),
+    // K tiles and V tiles.  A K slot frees when its QK^T has run, a V slot
+    // only when its PV has run, which happens about two tiles later, and a Q
+    // slot when the item's epilogue has copied out the rows it staged there;
+    // separate cursors keep each kind of load from queueing behind another's
+    // slots.  No cursor blocks: the thread polls whichever slots it needs next.
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
@@ -303,10 +307,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         __nanosleep(256);
       }
     }
-    int kidx = withhold ? p.n_items : blockIdx.x, vidx = kidx, kt = 0, vt = 0;
+    int qidx = withhold ? p.n_items : blockIdx.x, kidx = qidx, vidx = qidx, kt = 0, vt = 0;
     Item kit, vit;
     if (kidx < p.n_items) kit = vit = load_item(p.items, kidx);
-    bool need_q = kidx < p.n_items;
     uint32_t qn = 0, kn = 0, vn = 0;          // Q, K, V tiles issued
     int armed_q[kStagesQ], armed_k[kStagesK], armed_v[kStagesV];
 #pragma unroll
@@ -317,44 +320,43 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kStagesV; ++s) armed_v[s] = -1;
     uint64_t t_prog = globaltimer_ns();
     uint32_t idle = 0;
-    while (kidx < p.n_items || vidx < p.n_items) {
+    while (qidx < p.n_items || kidx < p.n_items || vidx < p.n_items) {
       bool prog = false;
+      if (qidx < p.n_items) {
+        // Q tiles run ahead by up to kStagesQ items: a slot frees when the
+        // epilogue has copied out the rows it staged there
+        const uint32_t qs = qn % kStagesQ, nq = qn / kStagesQ;
+        if (nq == 0 || mbar_try_wait(&bar[B_Q_EMPTY + qs], (nq - 1) & 1)) {
+          const Item qit = load_item(p.items, qidx);
+          mbar_arrive_expect_tx(&bar[B_Q_FULL + qs], TILE);
+#pragma unroll
+          for (int h = 0; h < NH; ++h)
+            tma_load_3d(sQ + qs * TILE + h * HALF, &tmQ, &bar[B_Q_FULL + qs], h * 64, qit.q_row0,
+                        qit.head);
+          armed_q[qs] = nq & 1;
+          ++qn;
+          qidx += gridDim.x;
+          prog = true;
+        }
+      }
       if (kidx < p.n_items) {
         const int kvh = kit.head / p.group;
-        if (need_q) {
-          const uint32_t qs = qn % kStagesQ, nq = qn / kStagesQ;
-          if (nq == 0 || mbar_try_wait(&bar[B_Q_EMPTY + qs], (nq - 1) & 1)) {
-            mbar_arrive_expect_tx(&bar[B_Q_FULL + qs], TILE);
+        const uint32_t st = kn % kStagesK, n = kn / kStagesK;
+        if (n == 0 || mbar_try_wait(&bar[B_K_EMPTY + st], (n - 1) & 1)) {
+          int r, k0;
+          tile_of(kit, kt, r, k0);
+          mbar_arrive_expect_tx(&bar[B_K_FULL + st], TILE);
 #pragma unroll
-            for (int h = 0; h < NH; ++h)
-              tma_load_3d(sQ + qs * TILE + h * HALF, &tmQ, &bar[B_Q_FULL + qs], h * 64, kit.q_row0,
-                          kit.head);
-            armed_q[qs] = nq & 1;
-            ++qn;
-            need_q = false;
-            prog = true;
-          }
-        } else {
-          const uint32_t st = kn % kStagesK, n = kn / kStagesK;
-          if (n == 0 || mbar_try_wait(&bar[B_K_EMPTY + st], (n - 1) & 1)) {
-            int r, k0;
-            tile_of(kit, kt, r, k0);
-            mbar_arrive_expect_tx(&bar[B_K_FULL + st], TILE);
-#pragma unroll
-            for (int h = 0; h < NH; ++h)
-              tma_load_3d(sK + st * TILE + h * HALF, &tmK, &bar[B_K_FULL + st], h * 64,
-                          (r ? kit.k_row0[1] : kit.k_row0[0]) + k0, kvh);
-            armed_k[st] = n & 1;
-            ++kn;
-            prog = true;
-            if (++kt == kit.ntiles) {
-              kt = 0;
-              kidx += gridDim.x;
-              if (kidx < p.n_items) {
-                kit = load_item(p.items, kidx);
-                need_q = true;
-              }
-            }
+          for (int h = 0; h < NH; ++h)
+            tma_load_3d(sK + st * TILE + h * HALF, &tmK, &bar[B_K_FULL + st], h * 64,
+                        (r ? kit.k_row0[1] : kit.k_row0[0]) + k0, kvh);
+          armed_k[st] = n & 1;
+          ++kn;
+          prog = true;
+          if (++kt == kit.ntiles) {
+            kt = 0;
+            kidx += gridDim.x;
+            if (kidx < p.n_items) kit = load_item(p.items, kidx);
           }
         }
       }
@@ -441,7 +443,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           mma_commit(&bar[B_S_FULL + b]);
           mma_commit(&bar[B_K_EMPTY + st]);
-          if (t == ntiles - 1) mma_commit(&bar[B_Q_EMPTY + qs]);
         } else {
           // O_h (+)= P_h V_h for the key halves h = 0, 1 of the tile, each as
           // soon as its warpgroup has written P_h; both accumulators must have
@@ -648,8 +649,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ epilogue
     // One thread per row (TMEM lane).  Per item: the merge factors, then, once
     // the item's last PV is done (in-order tensor core: so are all of its
-    // PVs), O_0 and O_1 are read, combined and stored; O is then free for the
-    // next item's first PV.
+    // PVs), O_0 and O_1 are read and combined, O is released for the next
+    // item's first PV, and the rows are written out; the item's Q tile, used
+    // to stage them, is then released to the producer.
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
@@ -680,41 +682,80 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const int64_t orow = ((int64_t)(it.q_row0 + row) * p.Hq + it.head) * D;
       uint16_t *pacc = partial ? p.part.acc + prow * D : nullptr;
+      const uint32_t qs = item_no % kStagesQ;
+      if (OUT_F32 && !partial) {
+        // fp32 output: read, combine and store O 32 columns at a time
 #pragma unroll 1
-      for (int col = 0; col < D; col += 32) {
-        uint32_t o0[32], o1[32];
-        tmem_ld32(tmem + lane_off + COL_O + col, o0);
-        tmem_ld32(tmem + lane_off + COL_O + D + col, o1);
-        tmem_wait_ld(o0);
-        tmem_wait_ld(o1);
-        if (row < it.n_rows) {
-#pragma unroll
-          for (int e = 0; e < 32; ++e)
-            o0[e] = __float_as_uint(__uint_as_float(o0[e]) * fw.x + __uint_as_float(o1[e]) * fw.y);
-          if (OUT_F32 && !partial) {
+        for (int col = 0; col < D; col += 32) {
+          uint32_t o0[32], o1[32];
+          tmem_ld32(tmem + lane_off + COL_O + col, o0);
+          tmem_ld32(tmem + lane_off + COL_O + D + col, o1);
+          tmem_wait_ld(o0);
+          tmem_wait_ld(o1);
+          if (row < it.n_rows) {
             float *dst = static_cast<float *>(p.out) + orow + col;
 #pragma unroll
             for (int e = 0; e < 32; e += 4)
-              *reinterpret_cast<uint4 *>(dst + e) = make_uint4(o0[e], o0[e + 1], o0[e + 2], o0[e + 3]);
-          } else {
-            // bf16 output, or the bf16 normalised partial of the row
-            uint16_t *dst = partial ? pacc + col : static_cast<uint16_t *>(p.out) + orow + col;
-#pragma unroll
-            for (int e = 0; e < 32; e += 8) {
-              uint32_t w[4];
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                __nv_bfloat162 hh = __floats2bfloat162_rn(__uint_as_float(o0[e + 2 * q]),
-                                                          __uint_as_float(o0[e + 2 * q + 1]));
-                w[q] = *reinterpret_cast<uint32_t *>(&hh);
-              }
-              *reinterpret_cast<uint4 *>(dst + e) = make_uint4(w[0], w[1], w[2], w[3]);
-            }
+              *reinterpret_cast<uint4 *>(dst + e) = make_uint4(
+                  __float_as_uint(__uint_as_float(o0[e]) * fw.x + __uint_as_float(o1[e]) * fw.y),
+                  __float_as_uint(__uint_as_float(o0[e + 1]) * fw.x + __uint_as_float(o1[e + 1]) * fw.y),
+                  __float_as_uint(__uint_as_float(o0[e + 2]) * fw.x + __uint_as_float(o1[e + 2]) * fw.y),
+                  __float_as_uint(__uint_as_float(o0[e + 3]) * fw.x + __uint_as_float(o1[e + 3]) * fw.y));
           }
         }
+        tc_fence_before();
+        mbar_arrive(&bar[B_O_FREE]);
+      } else {
+        // bf16 output, or the bf16 normalised partial of the row: O is read,
+        // combined, packed and staged in this item's Q tile (its last QK^T
+        // completed before its last PV), then released for the next item's
+        // first PV, and the row goes out by the bulk-copy engine as one
+        // contiguous piece.  Per-thread 16-byte global stores of 128 rows
+        // would put 32 rows in flight per warp instruction on the load/store
+        // pipe, which the softmax and issuing warps share.
+        // Row r of the staging tile holds its NC 16-byte chunks rotated by
+        // r mod NC (chunk j in slot (j + r) mod NC), so that the 32 rows of a
+        // warp's store fall in distinct bank groups; the copy then takes the
+        // row in two contiguous pieces.
+        constexpr int NC = D / 8;
+        uint8_t *srow = sQ + qs * TILE + row * (D * 2);
+        const int rot = row % NC;
+#pragma unroll
+        for (int col = 0; col < D; col += 16) {
+          uint32_t o0[16], o1[16];
+          tmem_ld16(tmem + lane_off + COL_O + col, o0);
+          tmem_ld16(tmem + lane_off + COL_O + D + col, o1);
+          tmem_wait_ld16(o0);
+          tmem_wait_ld16(o1);
+          uint32_t pk[8];
+#pragma unroll
+          for (int e = 0; e < 16; e += 2) {
+            __nv_bfloat162 hh = __floats2bfloat162_rn(
+                __uint_as_float(o0[e]) * fw.x + __uint_as_float(o1[e]) * fw.y,
+                __uint_as_float(o0[e + 1]) * fw.x + __uint_as_float(o1[e + 1]) * fw.y);
+            pk[e / 2] = *reinterpret_cast<uint32_t *>(&hh);
+          }
+          const int j = col / 8;   // chunks j, j + 1 of the row
+          *reinterpret_cast<uint4 *>(srow + ((j + rot) % NC) * 16) =
+              make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          *reinterpret_cast<uint4 *>(srow + ((j + 1 + rot) % NC) * 16) =
+              make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        }
+        tc_fence_before();
+        mbar_arrive(&bar[B_O_FREE]);
+        fence_proxy_async_smem();
+        if (row < it.n_rows) {
+          uint8_t *dst = reinterpret_cast<uint8_t *>(
+              partial ? pacc : static_cast<uint16_t *>(p.out) + orow);
+          const uint32_t s0 = smem_u32(srow);
+          bulk_store(dst, s0 + rot * 16, (NC - rot) * 16);   // chunks 0 .. NC - rot - 1
+          if (rot > 0) bulk_store(dst + (NC - rot) * 16, s0, rot * 16);
+          bulk_commit();
+        }
+        bulk_wait_read();
       }
-      tc_fence_before();
-      mbar_arrive(&bar[B_O_FREE]);
+      // the Q tile is free for the producer's next load into its stage
+      mbar_arrive(&bar[B_Q_EMPTY + qs]);
       if (partial && p.part.dbg != nullptr && it.head == 0 && row < it.n_rows) {
         // Gather map: the thread of an item's first packed row records, for
         // every key of the tile's range, the cache row its K and V tiles came
@@ -738,6 +779,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
+    bulk_wait_all();   // this thread's row copies have landed
   }
   __syncwarp();
   __syncthreads();
