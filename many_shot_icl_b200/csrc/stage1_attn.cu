@@ -10,9 +10,9 @@
 // holds only the tiles that contain an allowed pair).
 //
 // One persistent CTA per SM walks items round-robin.  Warp roles:
-//   warp 0      TMA producer: three independent cursors, for the items' Q
-//               tiles (double-buffered), K tiles (3-stage ring) and V tiles
-//               (2-stage ring)
+//   warp 0      TMA producer: two independent cursors, one for each item's Q
+//               tile (double-buffered) and its K tiles (3-stage ring), one
+//               for the V tiles (2-stage ring)
 //   warp 1      TMEM owner; one thread issues O_h += P_h V_h for the two key
 //               halves of each tile (tcgen05, A from TMEM)
 //   warp 10     one thread issues S = Q K^T (tcgen05, both operands in SMEM)
@@ -68,6 +68,12 @@ constexpr uint32_t kFull = 0xFFFFFFFFu;
 // through it.
 constexpr int kStagesK = 3;
 constexpr int kStagesV = 2;
+// The epilogue stages an item's bf16 rows in its Q tile only when the item
+// has at least this many key tiles: the Q slot then frees once the rows are
+// copied out, which for shorter items would hold up the next-but-one item's
+// Q load.  Shorter items store their rows directly and free the slot at
+// their last QK^T.
+constexpr int kStageMinTiles = 3;
 constexpr int kStagesQ = 2;
 
 enum Bar {
@@ -82,7 +88,8 @@ enum Bar {
   B_ML_B = B_ML_A + 1,        // end of item: warpgroup 0 has published the merge factors
   B_ML_FREE = B_ML_B + 1,     // the epilogue warpgroup has read the merge factors
   B_DRAIN_QK = B_ML_FREE + 1,
-  B_COUNT = B_DRAIN_QK + 1
+  B_Q_COPIED = B_DRAIN_QK + 1,  // [Q stage]: the epilogue has copied out the rows it staged there
+  B_COUNT = B_Q_COPIED + kStagesQ
 };
 
 constexpr int kSoftmaxThreads = 256;              // warps 2..9: two warpgroups
@@ -209,6 +216,7 @@ struct Params {
   int *status;
   uint64_t wait_limit_ns;  // limit of every bounded wait
   int withhold_tiles;      // test hook: the producer loads nothing (every wait runs out)
+  int stage_min_tiles;     // items with at least this many key tiles stage their rows
   Stage1Partial part;  // partial-output mode (part.acc != null)
 };
 
@@ -242,11 +250,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // whether the epilogue stages an item's rows in its Q tile (bf16 rows of
+  // items with at least kStageMinTiles key tiles), which decides who frees
+  // the item's Q slot
+  auto stages_rows = [&](int ntiles) {
+    return !(OUT_F32 && p.part.acc == nullptr) && ntiles >= p.stage_min_tiles;
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStagesQ; ++s) {
       mbar_init(&bar[B_Q_FULL + s], 1);
-      mbar_init(&bar[B_Q_EMPTY + s], 128);   // the epilogue warpgroup, after its staging
+      mbar_init(&bar[B_Q_EMPTY + s], 1);     // an unstaged item's last QK^T
+      mbar_init(&bar[B_Q_COPIED + s], 128);  // a staged item's epilogue warpgroup
     }
     for (int s = 0; s < kStagesK; ++s) {
       mbar_init(&bar[B_K_FULL + s], 1);
@@ -282,12 +297,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ producer
-    // Three independent cursors over the CTA's items: Q tiles (one per item),
-    // K tiles and V tiles.  A K slot frees when its QK^T has run, a V slot
-    // only when its PV has run, which happens about two tiles later, and a Q
-    // slot when the item's epilogue has copied out the rows it staged there;
-    // separate cursors keep each kind of load from queueing behind another's
-    // slots.  No cursor blocks: the thread polls whichever slots it needs next.
+    // Two independent cursors over the CTA's tile sequence: K tiles (each
+    // item's Q tile first) and V tiles.  A K slot frees when its QK^T has
+    // run, a V slot only when its PV has run, which happens about two tiles
+    // later; separate cursors keep the K loads from queueing behind V slots.
+    // A Q slot frees at its item's last QK^T, or, when the epilogue staged
+    // the item's rows there, once it has copied them out.  Neither cursor
+    // blocks: the thread polls whichever slot it needs next.
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
@@ -307,56 +323,73 @@ __global__ void __launch_bounds__(kThreads, 1)
         __nanosleep(256);
       }
     }
-    int qidx = withhold ? p.n_items : blockIdx.x, kidx = qidx, vidx = qidx, kt = 0, vt = 0;
+    int kidx = withhold ? p.n_items : blockIdx.x, vidx = kidx, kt = 0, vt = 0;
     Item kit, vit;
     if (kidx < p.n_items) kit = vit = load_item(p.items, kidx);
+    bool need_q = kidx < p.n_items;
     uint32_t qn = 0, kn = 0, vn = 0;          // Q, K, V tiles issued
     int armed_q[kStagesQ], armed_k[kStagesK], armed_v[kStagesV];
+    // per Q slot: how its last item frees it (-1 unused, 0 at its last QK^T,
+    // 1 after the epilogue's copies of the rows it staged there) and the
+    // uses of each kind so far; each kind has its own barrier
+    int q_prev[kStagesQ];
+    uint32_t q_staged[kStagesQ], q_direct[kStagesQ];
 #pragma unroll
-    for (int s = 0; s < kStagesQ; ++s) armed_q[s] = -1;
+    for (int s = 0; s < kStagesQ; ++s) {
+      armed_q[s] = -1;
+      q_prev[s] = -1;
+      q_staged[s] = q_direct[s] = 0;
+    }
 #pragma unroll
     for (int s = 0; s < kStagesK; ++s) armed_k[s] = -1;
 #pragma unroll
     for (int s = 0; s < kStagesV; ++s) armed_v[s] = -1;
     uint64_t t_prog = globaltimer_ns();
     uint32_t idle = 0;
-    while (qidx < p.n_items || kidx < p.n_items || vidx < p.n_items) {
+    while (kidx < p.n_items || vidx < p.n_items) {
       bool prog = false;
-      if (qidx < p.n_items) {
-        // Q tiles run ahead by up to kStagesQ items: a slot frees when the
-        // epilogue has copied out the rows it staged there
-        const uint32_t qs = qn % kStagesQ, nq = qn / kStagesQ;
-        if (nq == 0 || mbar_try_wait(&bar[B_Q_EMPTY + qs], (nq - 1) & 1)) {
-          const Item qit = load_item(p.items, qidx);
-          mbar_arrive_expect_tx(&bar[B_Q_FULL + qs], TILE);
-#pragma unroll
-          for (int h = 0; h < NH; ++h)
-            tma_load_3d(sQ + qs * TILE + h * HALF, &tmQ, &bar[B_Q_FULL + qs], h * 64, qit.q_row0,
-                        qit.head);
-          armed_q[qs] = nq & 1;
-          ++qn;
-          qidx += gridDim.x;
-          prog = true;
-        }
-      }
       if (kidx < p.n_items) {
         const int kvh = kit.head / p.group;
-        const uint32_t st = kn % kStagesK, n = kn / kStagesK;
-        if (n == 0 || mbar_try_wait(&bar[B_K_EMPTY + st], (n - 1) & 1)) {
-          int r, k0;
-          tile_of(kit, kt, r, k0);
-          mbar_arrive_expect_tx(&bar[B_K_FULL + st], TILE);
+        if (need_q) {
+          const uint32_t qs = qn % kStagesQ, nq = qn / kStagesQ;
+          const bool free_slot =
+              q_prev[qs] < 0 ||
+              (q_prev[qs] == 1 ? mbar_try_wait(&bar[B_Q_COPIED + qs], (q_staged[qs] - 1) & 1)
+                               : mbar_try_wait(&bar[B_Q_EMPTY + qs], (q_direct[qs] - 1) & 1));
+          if (free_slot) {
+            mbar_arrive_expect_tx(&bar[B_Q_FULL + qs], TILE);
 #pragma unroll
-          for (int h = 0; h < NH; ++h)
-            tma_load_3d(sK + st * TILE + h * HALF, &tmK, &bar[B_K_FULL + st], h * 64,
-                        (r ? kit.k_row0[1] : kit.k_row0[0]) + k0, kvh);
-          armed_k[st] = n & 1;
-          ++kn;
-          prog = true;
-          if (++kt == kit.ntiles) {
-            kt = 0;
-            kidx += gridDim.x;
-            if (kidx < p.n_items) kit = load_item(p.items, kidx);
+            for (int h = 0; h < NH; ++h)
+              tma_load_3d(sQ + qs * TILE + h * HALF, &tmQ, &bar[B_Q_FULL + qs], h * 64, kit.q_row0,
+                          kit.head);
+            armed_q[qs] = nq & 1;
+            q_prev[qs] = stages_rows(kit.ntiles) ? 1 : 0;
+            ++(q_prev[qs] ? q_staged[qs] : q_direct[qs]);
+            ++qn;
+            need_q = false;
+            prog = true;
+          }
+        } else {
+          const uint32_t st = kn % kStagesK, n = kn / kStagesK;
+          if (n == 0 || mbar_try_wait(&bar[B_K_EMPTY + st], (n - 1) & 1)) {
+            int r, k0;
+            tile_of(kit, kt, r, k0);
+            mbar_arrive_expect_tx(&bar[B_K_FULL + st], TILE);
+#pragma unroll
+            for (int h = 0; h < NH; ++h)
+              tma_load_3d(sK + st * TILE + h * HALF, &tmK, &bar[B_K_FULL + st], h * 64,
+                          (r ? kit.k_row0[1] : kit.k_row0[0]) + k0, kvh);
+            armed_k[st] = n & 1;
+            ++kn;
+            prog = true;
+            if (++kt == kit.ntiles) {
+              kt = 0;
+              kidx += gridDim.x;
+              if (kidx < p.n_items) {
+                kit = load_item(p.items, kidx);
+                need_q = true;
+              }
+            }
           }
         }
       }
@@ -443,6 +476,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           mma_commit(&bar[B_S_FULL + b]);
           mma_commit(&bar[B_K_EMPTY + st]);
+          if (t == ntiles - 1 && !stages_rows(ntiles)) mma_commit(&bar[B_Q_EMPTY + qs]);
         } else {
           // O_h (+)= P_h V_h for the key halves h = 0, 1 of the tile, each as
           // soon as its warpgroup has written P_h; both accumulators must have
@@ -683,8 +717,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t orow = ((int64_t)(it.q_row0 + row) * p.Hq + it.head) * D;
       uint16_t *pacc = partial ? p.part.acc + prow * D : nullptr;
       const uint32_t qs = item_no % kStagesQ;
-      if (OUT_F32 && !partial) {
-        // fp32 output: read, combine and store O 32 columns at a time
+      if (!stages_rows(it.ntiles)) {
+        // fp32 output, or a short item: read, combine and store O 32 columns
+        // at a time (the item's last QK^T freed its Q slot)
 #pragma unroll 1
         for (int col = 0; col < D; col += 32) {
           uint32_t o0[32], o1[32];
@@ -693,26 +728,40 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait_ld(o0);
           tmem_wait_ld(o1);
           if (row < it.n_rows) {
-            float *dst = static_cast<float *>(p.out) + orow + col;
 #pragma unroll
-            for (int e = 0; e < 32; e += 4)
-              *reinterpret_cast<uint4 *>(dst + e) = make_uint4(
-                  __float_as_uint(__uint_as_float(o0[e]) * fw.x + __uint_as_float(o1[e]) * fw.y),
-                  __float_as_uint(__uint_as_float(o0[e + 1]) * fw.x + __uint_as_float(o1[e + 1]) * fw.y),
-                  __float_as_uint(__uint_as_float(o0[e + 2]) * fw.x + __uint_as_float(o1[e + 2]) * fw.y),
-                  __float_as_uint(__uint_as_float(o0[e + 3]) * fw.x + __uint_as_float(o1[e + 3]) * fw.y));
+            for (int e = 0; e < 32; ++e)
+              o0[e] = __float_as_uint(__uint_as_float(o0[e]) * fw.x + __uint_as_float(o1[e]) * fw.y);
+            if (OUT_F32 && !partial) {
+              float *dst = static_cast<float *>(p.out) + orow + col;
+#pragma unroll
+              for (int e = 0; e < 32; e += 4)
+                *reinterpret_cast<uint4 *>(dst + e) = make_uint4(o0[e], o0[e + 1], o0[e + 2], o0[e + 3]);
+            } else {
+              uint16_t *dst = partial ? pacc + col : static_cast<uint16_t *>(p.out) + orow + col;
+#pragma unroll
+              for (int e = 0; e < 32; e += 8) {
+                uint32_t w[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                  __nv_bfloat162 hh = __floats2bfloat162_rn(__uint_as_float(o0[e + 2 * q]),
+                                                            __uint_as_float(o0[e + 2 * q + 1]));
+                  w[q] = *reinterpret_cast<uint32_t *>(&hh);
+                }
+                *reinterpret_cast<uint4 *>(dst + e) = make_uint4(w[0], w[1], w[2], w[3]);
+              }
+            }
           }
         }
         tc_fence_before();
         mbar_arrive(&bar[B_O_FREE]);
       } else {
-        // bf16 output, or the bf16 normalised partial of the row: O is read,
-        // combined, packed and staged in this item's Q tile (its last QK^T
-        // completed before its last PV), then released for the next item's
-        // first PV, and the row goes out by the bulk-copy engine as one
-        // contiguous piece.  Per-thread 16-byte global stores of 128 rows
-        // would put 32 rows in flight per warp instruction on the load/store
-        // pipe, which the softmax and issuing warps share.
+        // bf16 rows of a long item: O is read, combined, packed and staged in
+        // the item's Q tile (its last QK^T completed before its last PV),
+        // then released for the next item's first PV, and the rows go out by
+        // the bulk-copy engine as one contiguous piece each.  Per-thread
+        // 16-byte global stores of 128 rows put 32 rows in flight per warp
+        // instruction on the load/store pipe, which the softmax and issuing
+        // warps share.
         // Row r of the staging tile holds its NC 16-byte chunks rotated by
         // r mod NC (chunk j in slot (j + r) mod NC), so that the 32 rows of a
         // warp's store fall in distinct bank groups; the copy then takes the
@@ -753,9 +802,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           bulk_commit();
         }
         bulk_wait_read();
+        // once every row's copy has read the tile, its Q slot is free for the
+        // producer's next load there
+        mbar_arrive(&bar[B_Q_COPIED + qs]);
       }
-      // the Q tile is free for the producer's next load into its stage
-      mbar_arrive(&bar[B_Q_EMPTY + qs]);
       if (partial && p.part.dbg != nullptr && it.head == 0 && row < it.n_rows) {
         // Gather map: the thread of an item's first packed row records, for
         // every key of the tile's range, the cache row its K and V tiles came
@@ -864,6 +914,11 @@ cudaError_t launch_stage1(const Stage1Args &a, int head_dim, bool out_f32, int n
   p.status = a.status;
   p.wait_limit_ns = a.wait_limit_ns != 0 ? a.wait_limit_ns : kWaitLimitNs;
   p.withhold_tiles = a.withhold_tiles;
+  // Passes with few query rows per (query, KV head) (decode steps) stream
+  // their K/V from HBM and keep the TMA unit busy with loads: their rows are
+  // stored directly rather than queued on it as bulk copies.
+  p.stage_min_tiles =
+      a.part.acc != nullptr && a.part.group * a.part.n_new < 32 ? (1 << 30) : kStageMinTiles;
   p.part = a.part;
   const int grid = a.n_items < num_sms ? a.n_items : num_sms;
   if (head_dim == 128)

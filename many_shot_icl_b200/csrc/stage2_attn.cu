@@ -552,28 +552,34 @@ __global__ void __launch_bounds__(128) stage2_merge_kernel(const Stage2Args a) {
 
 // Block-major mode, after the tensor-core pass: each query's own tail tokens
 // and the merge of every partial of a row, in one kernel.  CTA = (query q,
-// KV head c, group of up to 8 rows of the query's g * n_new rows); one warp
-// per output row (query token u, head h).  Lane l holds the elements
-// i = l + 32 j (j < D / 32), so the rotate-half pairs (i, i + D/2) sit in the
-// same lane.  The CTA rotates the query's tail keys, 32 at a time, into
-// shared memory at their positions T'_q + u' (fp32, no rounding), with their
-// values; every warp scores its rotated query row against the keys u' <= its
-// own tail index (the causal rule), in log2 units, with an online softmax.
-// The row's block partials (M_i, L_i, O_i), written by the tensor-core pass,
-// are then merged with the tail state (m, l, acc):
-//   O = (sum_i 2^(M_i - M) L_i O_i + 2^(m - M) acc) / (sum_i 2^(M_i - M) L_i + 2^(m - M) l).
+// KV head c, group of up to 8 rows of the query's g * n_new rows); two warps
+// per output row (query token u, head h), each taking half of the row's
+// sources: alternate groups of 4 tail keys, and one half of its partials.
+// Lane l holds the elements i = l + 32 j (j < D / 32), so the rotate-half
+// pairs (i, i + D/2) sit in the same lane.  The CTA rotates the query's tail
+// keys, 32 at a time, into shared memory at their positions T'_q + u' (fp32,
+// no rounding), with their values; a warp scores its rotated query row
+// against its keys u' <= the row's tail index (the causal rule), in log2
+// units, with an online softmax.  It then merges its half of the row's block
+// partials (M_i, L_i, O_i), written by the tensor-core pass, into that state
+// (m, l, acc):  with M = max(m, max_i M_i),
+//   o = 2^(m - M) acc + sum_i 2^(M_i - M) L_i O_i,   n = 2^(m - M) l + sum_i 2^(M_i - M) L_i,
+// and the two warps' (M, n, o) are combined into O = o / n.
 template <int D, typename CT>
-__global__ void __launch_bounds__(256) stage2_tail_merge_kernel(const Stage2Args a) {
+__global__ void __launch_bounds__(512, 2) stage2_tail_merge_kernel(const Stage2Args a) {
   constexpr int H = D / 2;
   constexpr int E = D / 32;           // elements per lane
   constexpr int CH = 32;              // tail keys per shared-memory chunk
   __shared__ float sK[CH][D], sV[CH][D];
-  __shared__ float sO[8][D];          // a row's tail accumulator, regrouped for the merge
+  __shared__ float sO[16][D];         // a warp's tail accumulator, regrouped for the merge
+  __shared__ float sC[8][D + 2];      // the second warp of each row: (M, n, o)
   const int q = blockIdx.x, c = blockIdx.y;
   const int g = a.Hq / a.Hkv;
   const int R = g * a.n_new;
+  const int RW = min(8, R);                     // rows per CTA
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r = blockIdx.z * 8 + warp;          // this warp's row (token-major: u * g + hl)
+  const int rw = warp % RW, hf = warp / RW;     // row slot, half of the row's sources
+  const int r = blockIdx.z * 8 + rw;            // this warp's row (token-major: u * g + hl)
   const bool live = r < R;
   const S2Query qi = a.queries[q];
   const int Tq = qi.n_gathered;
@@ -618,9 +624,10 @@ __global__ void __launch_bounds__(256) stage2_tail_merge_kernel(const Stage2Args
       sV[j][i + H] = to_f32(vs[i + H]);
     }
     __syncthreads();
-    // keys k0 .. k0 + n - 1 of this chunk are visible to the row (u' <= tu)
+    // keys k0 .. k0 + n - 1 of this chunk are visible to the row (u' <= tu);
+    // this warp takes the groups of 4 starting at 4 hf, 4 hf + 8, ...
     const int n = live ? max(0, min(nk, tu - k0 + 1)) : 0;
-    for (int j0 = 0; j0 < n; j0 += 4) {
+    for (int j0 = 4 * hf; j0 < n; j0 += 8) {
       float sc[4];
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
@@ -657,9 +664,8 @@ __global__ void __launch_bounds__(256) stage2_tail_merge_kernel(const Stage2Args
       m = mx;
     }
   }
-  if (!live) return;
-  // merge with the row's block partials (every item of the query but the
-  // last, its tail item).  For the merge each lane takes E consecutive
+  // this warp's half of the row's block partials (every item of the query but
+  // the last, its tail item).  For the merge each lane takes E consecutive
   // elements (8- or 4-byte loads of every partial row), so the tail
   // accumulator is regrouped through shared memory first.
 #pragma unroll
@@ -669,25 +675,27 @@ __global__ void __launch_bounds__(256) stage2_tail_merge_kernel(const Stage2Args
 #pragma unroll
   for (int j = 0; j < E; ++j) acc_c[j] = sO[warp][E * lane + j];
   const int nb = qi.n_items - 1;
+  const int nb0 = (nb + 1) / 2;
+  const int i_lo = hf == 0 ? 0 : nb0, i_hi = live ? (hf == 0 ? nb0 : nb) : i_lo;
   auto part = [&](int i) { return ((int64_t)(qi.item_begin + i) * a.Hq + h) * a.n_new + tok; };
   float M = m;
-  for (int i = lane; i < nb; i += 32) M = fmaxf(M, a.part_ml[part(i)].x);
+  for (int i = i_lo + lane; i < i_hi; i += 32) M = fmaxf(M, a.part_ml[part(i)].x);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  const float wt = ex2(m - M);                 // m is finite: key tu is always visible
+  const float wt = (m == -INFINITY) ? 0.f : ex2(m - M);   // this warp may have no tail key
   float L = 0.f, out[E];
 #pragma unroll
   for (int j = 0; j < E; ++j) out[j] = wt * acc_c[j];
   using Vec = typename std::conditional<E == 4, uint2, uint32_t>::type;   // E bf16 values
-  constexpr int U = 8;                         // partial rows in flight
-  for (int i0 = 0; i0 < nb; i0 += 32) {
+  constexpr int U = 6;                         // partial rows in flight (64 registers)
+  for (int i0 = i_lo; i0 < i_hi; i0 += 32) {
     float w = 0.f;
-    if (i0 + lane < nb) {
+    if (i0 + lane < i_hi) {
       const float2 ml = a.part_ml[part(i0 + lane)];
       w = (ml.x == -INFINITY) ? 0.f : ex2(ml.x - M) * ml.y;
     }
     L += w;
-    const int cnt = min(32, nb - i0);
+    const int cnt = min(32, i_hi - i0);
     for (int k0 = 0; k0 < cnt; k0 += U) {
       Vec v[U];
 #pragma unroll
@@ -710,10 +718,26 @@ __global__ void __launch_bounds__(256) stage2_tail_merge_kernel(const Stage2Args
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-  const float inv = 1.f / (L + wt * l);
+  const float nrm = L + wt * l;                // this warp's normaliser at scale M
+  // the second warp of the row hands (M, n, o) to the first, which combines
+  if (hf == 1) {
+    if (lane == 0) {
+      sC[rw][0] = M;
+      sC[rw][1] = nrm;
+    }
+#pragma unroll
+    for (int j = 0; j < E; ++j) sC[rw][2 + E * lane + j] = out[j];
+  }
+  __syncthreads();
+  if (hf == 1 || !live) return;
+  const float M1 = sC[rw][0], n1 = sC[rw][1];
+  const float Mx = fmaxf(M, M1);
+  const float f0 = (M == -INFINITY) ? 0.f : ex2(M - Mx);
+  const float f1 = (M1 == -INFINITY) ? 0.f : ex2(M1 - Mx);
+  const float inv = 1.f / (f0 * nrm + f1 * n1);
   CT *dst = static_cast<CT *>(a.out) + (((int64_t)q * a.n_new + tok) * a.Hq + h) * D + E * lane;
 #pragma unroll
-  for (int j = 0; j < E; ++j) from_f32(out[j] * inv, dst[j]);
+  for (int j = 0; j < E; ++j) from_f32((f0 * out[j] + f1 * sC[rw][2 + E * lane + j]) * inv, dst[j]);
 }
 
 template <int D, typename CT, int RT, int KG, int KT>
@@ -754,7 +778,7 @@ template <int D, typename CT>
 cudaError_t launch_tail_merge(const Stage2Args &a, cudaStream_t st) {
   const int R = (a.Hq / a.Hkv) * a.n_new;
   dim3 grid(a.n_queries, a.Hkv, (R + 7) / 8);
-  stage2_tail_merge_kernel<D, CT><<<grid, 32 * min(8, R), 0, st>>>(a);
+  stage2_tail_merge_kernel<D, CT><<<grid, 64 * min(8, R), 0, st>>>(a);   // two warps per row
   return cudaGetLastError();
 }
 
