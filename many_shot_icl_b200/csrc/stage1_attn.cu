@@ -216,11 +216,13 @@ struct Params {
   int *status;
   uint64_t wait_limit_ns;  // limit of every bounded wait
   int withhold_tiles;      // test hook: the producer loads nothing (every wait runs out)
-  int stage_min_tiles;     // items with at least this many key tiles stage their rows
   Stage1Partial part;  // partial-output mode (part.acc != null)
 };
 
-template <int D, bool OUT_F32>
+// STAGE: the launch stages the bf16 rows of its items of at least
+// kStageMinTiles key tiles in their Q tiles (Stage 1 and prompt passes); a
+// launch without it (decode steps, fp32 outputs) has none of that code.
+template <int D, bool OUT_F32, bool STAGE>
 __global__ void __launch_bounds__(kThreads, 1)
     stage1_attn_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
@@ -253,9 +255,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // whether the epilogue stages an item's rows in its Q tile (bf16 rows of
   // items with at least kStageMinTiles key tiles), which decides who frees
   // the item's Q slot
-  auto stages_rows = [&](int ntiles) {
-    return !(OUT_F32 && p.part.acc == nullptr) && ntiles >= p.stage_min_tiles;
-  };
+  auto stages_rows = [&](int ntiles) { return STAGE && ntiles >= kStageMinTiles; };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStagesQ; ++s) {
@@ -329,17 +329,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool need_q = kidx < p.n_items;
     uint32_t qn = 0, kn = 0, vn = 0;          // Q, K, V tiles issued
     int armed_q[kStagesQ], armed_k[kStagesK], armed_v[kStagesV];
-    // per Q slot: how its last item frees it (-1 unused, 0 at its last QK^T,
+    // Per Q slot: how its last item frees it (-1 unused, 0 at its last QK^T,
     // 1 after the epilogue's copies of the rows it staged there) and the
-    // uses of each kind so far; each kind has its own barrier
-    int q_prev[kStagesQ];
-    uint32_t q_staged[kStagesQ], q_direct[kStagesQ];
+    // uses of each kind so far; each kind has its own barrier.  The slots are
+    // used in turn, so the state is kept in registers as (slot used next,
+    // the other slot) and swapped after each Q load.
+    static_assert(kStagesQ == 2, "the Q slot state rotates between two slots");
+    int qa_prev = -1, qb_prev = -1;
+    uint32_t qa_staged = 0, qa_direct = 0, qb_staged = 0, qb_direct = 0;
 #pragma unroll
-    for (int s = 0; s < kStagesQ; ++s) {
-      armed_q[s] = -1;
-      q_prev[s] = -1;
-      q_staged[s] = q_direct[s] = 0;
-    }
+    for (int s = 0; s < kStagesQ; ++s) armed_q[s] = -1;
 #pragma unroll
     for (int s = 0; s < kStagesK; ++s) armed_k[s] = -1;
 #pragma unroll
@@ -353,9 +352,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (need_q) {
           const uint32_t qs = qn % kStagesQ, nq = qn / kStagesQ;
           const bool free_slot =
-              q_prev[qs] < 0 ||
-              (q_prev[qs] == 1 ? mbar_try_wait(&bar[B_Q_COPIED + qs], (q_staged[qs] - 1) & 1)
-                               : mbar_try_wait(&bar[B_Q_EMPTY + qs], (q_direct[qs] - 1) & 1));
+              qa_prev < 0 ||
+              (qa_prev == 1 ? mbar_try_wait(&bar[B_Q_COPIED + qs], (qa_staged - 1) & 1)
+                            : mbar_try_wait(&bar[B_Q_EMPTY + qs], (qa_direct - 1) & 1));
           if (free_slot) {
             mbar_arrive_expect_tx(&bar[B_Q_FULL + qs], TILE);
 #pragma unroll
@@ -363,8 +362,18 @@ __global__ void __launch_bounds__(kThreads, 1)
               tma_load_3d(sQ + qs * TILE + h * HALF, &tmQ, &bar[B_Q_FULL + qs], h * 64, kit.q_row0,
                           kit.head);
             armed_q[qs] = nq & 1;
-            q_prev[qs] = stages_rows(kit.ntiles) ? 1 : 0;
-            ++(q_prev[qs] ? q_staged[qs] : q_direct[qs]);
+            qa_prev = stages_rows(kit.ntiles) ? 1 : 0;
+            qa_staged += qa_prev;
+            qa_direct += 1 - qa_prev;
+            // the next Q load goes to the other slot
+            const int tp = qa_prev;
+            const uint32_t ts = qa_staged, td = qa_direct;
+            qa_prev = qb_prev;
+            qa_staged = qb_staged;
+            qa_direct = qb_direct;
+            qb_prev = tp;
+            qb_staged = ts;
+            qb_direct = td;
             ++qn;
             need_q = false;
             prog = true;
@@ -881,16 +890,16 @@ constexpr size_t smem_bytes() {
   return need > one_per_sm ? need : one_per_sm;
 }
 
-template <int D, bool F32>
+template <int D, bool F32, bool STAGE>
 cudaError_t launch_t(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
                      const Params &p, int grid, cudaStream_t st) {
   constexpr size_t smem = smem_bytes<D>();
   static_assert(smem <= 232448, "shared memory budget");
   static_assert(smem > 232448 / 2, "one CTA per SM (the kernel owns all 512 TMEM columns)");
-  cudaError_t e = cudaFuncSetAttribute(stage1_attn_kernel<D, F32>,
+  cudaError_t e = cudaFuncSetAttribute(stage1_attn_kernel<D, F32, STAGE>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  stage1_attn_kernel<D, F32><<<grid, kThreads, smem, st>>>(mq, mk, mv, p);
+  stage1_attn_kernel<D, F32, STAGE><<<grid, kThreads, smem, st>>>(mq, mk, mv, p);
   return cudaGetLastError();
 }
 
@@ -914,18 +923,21 @@ cudaError_t launch_stage1(const Stage1Args &a, int head_dim, bool out_f32, int n
   p.status = a.status;
   p.wait_limit_ns = a.wait_limit_ns != 0 ? a.wait_limit_ns : kWaitLimitNs;
   p.withhold_tiles = a.withhold_tiles;
-  // Passes with few query rows per (query, KV head) (decode steps) stream
-  // their K/V from HBM and keep the TMA unit busy with loads: their rows are
-  // stored directly rather than queued on it as bulk copies.
-  p.stage_min_tiles =
-      a.part.acc != nullptr && a.part.group * a.part.n_new < 32 ? (1 << 30) : kStageMinTiles;
   p.part = a.part;
   const int grid = a.n_items < num_sms ? a.n_items : num_sms;
+  // Rows are staged (bf16 outputs) except in passes with few query rows per
+  // (query, KV head) (decode steps): those stream their K/V from HBM and keep
+  // the TMA unit busy with loads, so their rows are stored directly rather
+  // than queued on it as bulk copies.
+  const bool stage =
+      !out_f32 && (a.part.acc == nullptr || a.part.group * a.part.n_new >= 32);
   if (head_dim == 128)
-    return out_f32 ? launch_t<128, true>(mq, mk, mv, p, grid, st)
-                   : launch_t<128, false>(mq, mk, mv, p, grid, st);
-  return out_f32 ? launch_t<64, true>(mq, mk, mv, p, grid, st)
-                 : launch_t<64, false>(mq, mk, mv, p, grid, st);
+    return out_f32 ? launch_t<128, true, false>(mq, mk, mv, p, grid, st)
+           : stage ? launch_t<128, false, true>(mq, mk, mv, p, grid, st)
+                   : launch_t<128, false, false>(mq, mk, mv, p, grid, st);
+  return out_f32 ? launch_t<64, true, false>(mq, mk, mv, p, grid, st)
+         : stage ? launch_t<64, false, true>(mq, mk, mv, p, grid, st)
+                 : launch_t<64, false, false>(mq, mk, mv, p, grid, st);
 }
 
 }  // namespace dbsa
