@@ -80,6 +80,7 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // into device memory: 16-byte words while both sides allow, then bytes.
 __global__ void __launch_bounds__(256) copy_from_host_kernel(uint8_t *dst, const uint8_t *src,
                                                              size_t bytes, uint32_t *clear) {
+  pdl_enter();
   // the call's status head, cleared here rather than by a separate memset
   if (clear != nullptr && blockIdx.x == 0 && threadIdx.x < kStatusBytes / 4) clear[threadIdx.x] = 0;
   const size_t stride = (size_t)gridDim.x * blockDim.x;
@@ -171,7 +172,7 @@ class StagingRing {
     next_ = (next_ + 1) % kSlots;
     if (bytes > 0 || clear != nullptr) {
       const int grid = (int)std::max<size_t>(1, std::min<size_t>((bytes + 4095) / 4096, 148));
-      copy_from_host_kernel<<<grid, 256, 0, st>>>(static_cast<uint8_t *>(dst),
+      pdl_launch(copy_from_host_kernel, dim3(grid), dim3(256), 0, st, static_cast<uint8_t *>(dst),
                                                  static_cast<const uint8_t *>(s.p), bytes,
                                                  static_cast<uint32_t *>(clear));
       cudaError_t e = cudaGetLastError();

@@ -11,6 +11,34 @@
 
 namespace dbsa {
 
+// Programmatic dependent launch.  Every kernel of the library is launched
+// with programmatic stream serialisation and starts with pdl_enter(): it
+// waits there until the previous kernel in the stream has completed and its
+// memory is visible (griddepcontrol.wait), then lets the next kernel be
+// scheduled (griddepcontrol.launch_dependents; the next grid is scheduled
+// once every CTA of this one has started, and waits in its own pdl_enter).
+// Nothing before pdl_enter() touches global memory, so the overlap is the
+// launch latency and the next kernel's block scheduling, not data.
+__device__ __forceinline__ void pdl_enter() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+template <typename... KArgs, typename... Args>
+cudaError_t pdl_launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args &&>(args)...);
+}
+
 constexpr int kTileRows = 128;   // Stage-1 query rows per tile (tcgen05 M)
 constexpr int kTileKeys = 128;   // Stage-1 keys per score tile (tcgen05 N)
 constexpr int kRopeLo = 16;      // positions per RoPE "hi" table step

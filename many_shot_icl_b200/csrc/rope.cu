@@ -16,6 +16,7 @@ namespace dbsa {
 namespace {
 
 __global__ void rope_tables_kernel(float *base, int32_t n_hi, int32_t half, double theta) {
+  pdl_enter();
   const int64_t n = (int64_t)(n_hi + kRopeLo) * half;
   float *hc = base, *hs = hc + (int64_t)n_hi * half;
   float *lc = hs + (int64_t)n_hi * half, *ls = lc + (int64_t)kRopeLo * half;
@@ -42,6 +43,7 @@ __global__ void rope_tables_kernel(float *base, int32_t n_hi, int32_t half, doub
 // the first half and the matching 8 of the second half.
 template <int D, typename T>
 __global__ void __launch_bounds__(256) ingest_kernel(IngestArgs a) {
+  pdl_enter();
   constexpr int H = D / 2;
   constexpr int CP = H / 8;
   const int slots = a.Hq + 2 * a.Hkv;
@@ -102,6 +104,7 @@ __global__ void __launch_bounds__(256) ingest_kernel(IngestArgs a) {
 // Cache rows [row0, row0+n) of every KV head, at positions equal to the row.
 template <int D, typename T>
 __global__ void __launch_bounds__(256) window_kernel(WindowArgs a) {
+  pdl_enter();
   constexpr int H = D / 2;
   constexpr int CP = H / 8;
   const int64_t n_units = (int64_t)a.n * a.Hkv * CP;
@@ -135,6 +138,7 @@ __global__ void __launch_bounds__(256) window_kernel(WindowArgs a) {
 // Key rows at block-relative positions (row s of block b at s - offs[b]).
 template <int D, typename T>
 __global__ void __launch_bounds__(256) rel_rope_kernel(RelRopeArgs a) {
+  pdl_enter();
   constexpr int H = D / 2;
   constexpr int CP = H / 8;
   const int64_t n_units = (int64_t)a.T * a.Hkv * CP;
@@ -172,6 +176,7 @@ __global__ void __launch_bounds__(256) rel_rope_kernel(RelRopeArgs a) {
 
 template <int D, typename T>
 __global__ void __launch_bounds__(256) qhat_kernel(QHatArgs a) {
+  pdl_enter();
   // One thread per (block item, query token, kv head, 8-pair chunk): the g
   // query heads of the kv head share the token's position, so the rotation
   // factors are built once and applied to all g rows (row token * g + local
@@ -219,6 +224,7 @@ __global__ void __launch_bounds__(256) qhat_kernel(QHatArgs a) {
 // warp records (cache row, p) for every row it reads.
 template <int D, typename T>
 __global__ void __launch_bounds__(256) compact_kernel(CompactArgs a) {
+  pdl_enter();
   constexpr int H = D / 2;
   const int lane = threadIdx.x & 31;
   const bool has_pair = 2 * lane < H;
@@ -289,11 +295,11 @@ cudaError_t launch_rel_rope(const RelRopeArgs &a, int head_dim, bool f32, cudaSt
   if (a.T <= 0) return cudaSuccess;
   const int g = grid_for((int64_t)a.T * a.Hkv * (head_dim / 16), 256);
   if (head_dim == 128) {
-    if (f32) rel_rope_kernel<128, float><<<g, 256, 0, st>>>(a);
-    else rel_rope_kernel<128, bf16><<<g, 256, 0, st>>>(a);
+    if (f32) pdl_launch(rel_rope_kernel<128, float>, dim3(g), dim3(256), 0, st, a);
+    else pdl_launch(rel_rope_kernel<128, bf16>, dim3(g), dim3(256), 0, st, a);
   } else {
-    if (f32) rel_rope_kernel<64, float><<<g, 256, 0, st>>>(a);
-    else rel_rope_kernel<64, bf16><<<g, 256, 0, st>>>(a);
+    if (f32) pdl_launch(rel_rope_kernel<64, float>, dim3(g), dim3(256), 0, st, a);
+    else pdl_launch(rel_rope_kernel<64, bf16>, dim3(g), dim3(256), 0, st, a);
   }
   return cudaGetLastError();
 }
@@ -302,11 +308,11 @@ cudaError_t launch_qhat(const QHatArgs &a, int head_dim, bool f32, cudaStream_t 
   if (a.rows <= 0) return cudaSuccess;
   const int g = grid_for((int64_t)a.n_items * a.n_new * a.Hkv * (head_dim / 16), 256);
   if (head_dim == 128) {
-    if (f32) qhat_kernel<128, float><<<g, 256, 0, st>>>(a);
-    else qhat_kernel<128, bf16><<<g, 256, 0, st>>>(a);
+    if (f32) pdl_launch(qhat_kernel<128, float>, dim3(g), dim3(256), 0, st, a);
+    else pdl_launch(qhat_kernel<128, bf16>, dim3(g), dim3(256), 0, st, a);
   } else {
-    if (f32) qhat_kernel<64, float><<<g, 256, 0, st>>>(a);
-    else qhat_kernel<64, bf16><<<g, 256, 0, st>>>(a);
+    if (f32) pdl_launch(qhat_kernel<64, float>, dim3(g), dim3(256), 0, st, a);
+    else pdl_launch(qhat_kernel<64, bf16>, dim3(g), dim3(256), 0, st, a);
   }
   return cudaGetLastError();
 }
@@ -315,11 +321,11 @@ cudaError_t launch_compact(const CompactArgs &a, int head_dim, bool f32, cudaStr
   if (a.rows <= 0 || a.n_segs <= 0) return cudaSuccess;
   const int g = grid_for((int64_t)a.n_segs * a.Hkv * 32, 256);
   if (head_dim == 128) {
-    if (f32) compact_kernel<128, float><<<g, 256, 0, st>>>(a);
-    else compact_kernel<128, bf16><<<g, 256, 0, st>>>(a);
+    if (f32) pdl_launch(compact_kernel<128, float>, dim3(g), dim3(256), 0, st, a);
+    else pdl_launch(compact_kernel<128, bf16>, dim3(g), dim3(256), 0, st, a);
   } else {
-    if (f32) compact_kernel<64, float><<<g, 256, 0, st>>>(a);
-    else compact_kernel<64, bf16><<<g, 256, 0, st>>>(a);
+    if (f32) pdl_launch(compact_kernel<64, float>, dim3(g), dim3(256), 0, st, a);
+    else pdl_launch(compact_kernel<64, bf16>, dim3(g), dim3(256), 0, st, a);
   }
   return cudaGetLastError();
 }
@@ -343,7 +349,7 @@ cudaError_t launch_rope_tables(float *base, int32_t n_hi, int32_t head_dim, doub
                                cudaStream_t st) {
   const int half = head_dim / 2;
   const int64_t n = (int64_t)(n_hi + kRopeLo) * half;
-  rope_tables_kernel<<<grid_for(n, 256), 256, 0, st>>>(base, n_hi, half, theta);
+  pdl_launch(rope_tables_kernel, dim3(grid_for(n, 256)), dim3(256), 0, st, base, n_hi, half, theta);
   return cudaGetLastError();
 }
 
@@ -351,11 +357,11 @@ cudaError_t launch_ingest(const IngestArgs &a, int head_dim, bool f32, cudaStrea
   const int64_t n = (int64_t)a.n_tok * (a.Hq + 2 * a.Hkv) * (head_dim / 16);
   const int g = grid_for(n, 256);
   if (head_dim == 128) {
-    if (f32) ingest_kernel<128, float><<<g, 256, 0, st>>>(a);
-    else ingest_kernel<128, bf16><<<g, 256, 0, st>>>(a);
+    if (f32) pdl_launch(ingest_kernel<128, float>, dim3(g), dim3(256), 0, st, a);
+    else pdl_launch(ingest_kernel<128, bf16>, dim3(g), dim3(256), 0, st, a);
   } else {
-    if (f32) ingest_kernel<64, float><<<g, 256, 0, st>>>(a);
-    else ingest_kernel<64, bf16><<<g, 256, 0, st>>>(a);
+    if (f32) pdl_launch(ingest_kernel<64, float>, dim3(g), dim3(256), 0, st, a);
+    else pdl_launch(ingest_kernel<64, bf16>, dim3(g), dim3(256), 0, st, a);
   }
   return cudaGetLastError();
 }
@@ -365,11 +371,11 @@ cudaError_t launch_window(const WindowArgs &a, int head_dim, bool f32, cudaStrea
   const int64_t n = (int64_t)a.n * a.Hkv * (head_dim / 16);
   const int g = grid_for(n, 256);
   if (head_dim == 128) {
-    if (f32) window_kernel<128, float><<<g, 256, 0, st>>>(a);
-    else window_kernel<128, bf16><<<g, 256, 0, st>>>(a);
+    if (f32) pdl_launch(window_kernel<128, float>, dim3(g), dim3(256), 0, st, a);
+    else pdl_launch(window_kernel<128, bf16>, dim3(g), dim3(256), 0, st, a);
   } else {
-    if (f32) window_kernel<64, float><<<g, 256, 0, st>>>(a);
-    else window_kernel<64, bf16><<<g, 256, 0, st>>>(a);
+    if (f32) pdl_launch(window_kernel<64, float>, dim3(g), dim3(256), 0, st, a);
+    else pdl_launch(window_kernel<64, bf16>, dim3(g), dim3(256), 0, st, a);
   }
   return cudaGetLastError();
 }

@@ -294,6 +294,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // the set-up above touches shared memory and TMEM only
+  pdl_enter();
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ producer
@@ -899,7 +901,7 @@ cudaError_t launch_t(const CUtensorMap &mq, const CUtensorMap &mk, const CUtenso
   cudaError_t e = cudaFuncSetAttribute(stage1_attn_kernel<D, F32, STAGE>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  stage1_attn_kernel<D, F32, STAGE><<<grid, kThreads, smem, st>>>(mq, mk, mv, p);
+  pdl_launch(stage1_attn_kernel<D, F32, STAGE>, dim3(grid), dim3(kThreads), smem, st, mq, mk, mv, p);
   return cudaGetLastError();
 }
 

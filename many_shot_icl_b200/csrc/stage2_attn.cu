@@ -98,6 +98,7 @@ __device__ __forceinline__ uint32_t soff(int row, int chunk) {
 //
 template <int D, typename CT, int RT, int KG, int KT, int NST>
 __global__ void __launch_bounds__(32 * RT * KG, 1) stage2_attn_kernel(const Stage2Args a) {
+  pdl_enter();
   constexpr int H = D / 2;
   constexpr int CH = D / 8;                 // 16-byte chunks per row
   constexpr int ROWB = D * 2;
@@ -487,6 +488,7 @@ __global__ void __launch_bounds__(32 * RT * KG, 1) stage2_attn_kernel(const Stag
 // the items' rows are then added in item order, four loads in flight.
 template <int D, typename OT>
 __global__ void __launch_bounds__(128) stage2_merge_kernel(const Stage2Args a) {
+  pdl_enter();
   const int64_t row = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   const int64_t n_rows = (int64_t)a.n_queries * a.n_new * a.Hq;
@@ -567,6 +569,7 @@ __global__ void __launch_bounds__(128) stage2_merge_kernel(const Stage2Args a) {
 // and the two warps' (M, n, o) are combined into O = o / n.
 template <int D, typename CT>
 __global__ void __launch_bounds__(512, 2) stage2_tail_merge_kernel(const Stage2Args a) {
+  pdl_enter();
   constexpr int H = D / 2;
   constexpr int E = D / 32;           // elements per lane
   constexpr int CH = 32;              // tail keys per shared-memory chunk
@@ -755,7 +758,7 @@ cudaError_t launch_main(const Stage2Args &a, cudaStream_t st) {
   const int R = (a.Hq / a.Hkv) * a.n_new;
   if (a.n_run <= 0) return cudaSuccess;
   dim3 grid(a.n_run, a.Hkv, (R + MROWS - 1) / MROWS);
-  stage2_attn_kernel<D, CT, RT, KG, KT, NST><<<grid, 32 * RT * KG, smem, st>>>(a);
+  pdl_launch(stage2_attn_kernel<D, CT, RT, KG, KT, NST>, dim3(grid), dim3(32 * RT * KG), smem, st, a);
   return cudaGetLastError();
 }
 
@@ -778,14 +781,14 @@ template <int D, typename CT>
 cudaError_t launch_tail_merge(const Stage2Args &a, cudaStream_t st) {
   const int R = (a.Hq / a.Hkv) * a.n_new;
   dim3 grid(a.n_queries, a.Hkv, (R + 7) / 8);
-  stage2_tail_merge_kernel<D, CT><<<grid, 64 * min(8, R), 0, st>>>(a);   // two warps per row
+  pdl_launch(stage2_tail_merge_kernel<D, CT>, dim3(grid), dim3(64 * min(8, R)), 0, st, a);   // two warps per row
   return cudaGetLastError();
 }
 
 template <int D, typename CT>
 cudaError_t launch_merge(const Stage2Args &a, cudaStream_t st) {
   const int64_t rows = (int64_t)a.n_queries * a.n_new * a.Hq;
-  stage2_merge_kernel<D, CT><<<(unsigned)((rows + 3) / 4), 128, 0, st>>>(a);
+  pdl_launch(stage2_merge_kernel<D, CT>, dim3((unsigned)((rows + 3) / 4)), dim3(128), 0, st, a);
   return cudaGetLastError();
 }
 
