@@ -684,9 +684,8 @@ S1Layout s1_layout(const dbsa_config *cfg, int64_t max_pos, int64_t n_items, int
 }
 
 struct S2Layout {
-  size_t rope, queries, segs, items, run_items, packed_items, item_meta,
-      tc_tiles, offs, compact_base, blob_end, q_rot_pos, k_hat, v_hat, q_hat, part_acc, part_ml,
-      total;
+  size_t rope, queries, packed_items, item_meta, tc_tiles, offs, compact_base, core_end, segs,
+      items, run_items, blob_end, q_rot_pos, k_hat, v_hat, q_hat, part_acc, part_ml, total;
   int32_t n_hi;
 };
 // prepared: the block-relative keys (and bf16 V of fp32 caches) come from a
@@ -697,15 +696,19 @@ S2Layout s2_layout(const dbsa_config *cfg, const GatherPlan &gp, int32_t n_new,
   Carve cv;
   l.n_hi = (int32_t)(std::max<int64_t>(gp.max_pos - 1, 0) / kRopeLo + 1);
   l.rope = cv.take(rope_table_bytes(l.n_hi, cfg->head_dim));
+  // the plan tables, uploaded as one blob: first those every mode reads,
+  // then those only the per-query kernel, the compact gather and the gather
+  // map read (a decode step's block-major pass needs none of them)
   l.queries = cv.take(gp.queries.size() * sizeof(S2Query));
-  l.segs = cv.take(gp.segs.size() * sizeof(S2Segment));
-  l.items = cv.take(gp.items.size() * sizeof(S2Item));
-  l.run_items = cv.take(gp.run_items.size() * sizeof(int32_t));
   l.packed_items = cv.take(gp.packed_items.size() * sizeof(int32_t));
   l.item_meta = cv.take(gp.item_meta.size() * sizeof(int4));
   l.tc_tiles = cv.take(gp.tc_tiles.size() * sizeof(dbsa_tile_item));
   l.offs = cv.take((size_t)(offs_count(gp)) * sizeof(int32_t));
   l.compact_base = cv.take(gp.compact_base.size() * sizeof(int32_t));
+  l.core_end = cv.take(0);
+  l.segs = cv.take(gp.segs.size() * sizeof(S2Segment));
+  l.items = cv.take(gp.items.size() * sizeof(S2Item));
+  l.run_items = cv.take(gp.run_items.size() * sizeof(int32_t));
   l.blob_end = cv.take(0);
   l.q_rot_pos = cv.take(gp.items.size() * sizeof(int32_t));
   const int64_t T = gp.cache_rows;
@@ -1181,7 +1184,13 @@ dbsa_status gather_impl(const dbsa_config *cfg, const void *k_cache, const void 
     // (the no-allocation entry point: into a host vector, then one
     // cudaMemcpyAsync from that pageable memory, which returns once the
     // driver has taken the bytes)
-    const size_t blob_bytes = L.blob_end - L.queries;
+    // a block-major pass whose tails run in the tail-and-merge kernel, with
+    // no gather map requested, reads none of the segment, item and run-item
+    // tables: they stay on the host
+    const bool block_major = !gp.per_query && !gp.compact;
+    const bool tail_merge = (cfg->n_q_heads / cfg->n_kv_heads) * n_new <= kTailMergeMaxRows;
+    const bool core_only = block_major && tail_merge && dbg_map == nullptr;
+    const size_t blob_bytes = (core_only ? L.core_end : L.blob_end) - L.queries;
     static thread_local std::vector<uint8_t> plain;
     uint8_t *blob = nullptr;
     if (fixed != nullptr) {
@@ -1192,12 +1201,14 @@ dbsa_status gather_impl(const dbsa_config *cfg, const void *k_cache, const void 
       return cuda_fail(e, "gather plan staging");
     }
     std::memcpy(blob, gp.queries.data(), gp.queries.size() * sizeof(S2Query));
-    std::memcpy(blob + (L.segs - L.queries), gp.segs.data(),
-                gp.segs.size() * sizeof(S2Segment));
-    std::memcpy(blob + (L.items - L.queries), gp.items.data(),
-                gp.items.size() * sizeof(S2Item));
-    std::memcpy(blob + (L.run_items - L.queries), gp.run_items.data(),
-                gp.run_items.size() * sizeof(int32_t));
+    if (!core_only) {
+      std::memcpy(blob + (L.segs - L.queries), gp.segs.data(),
+                  gp.segs.size() * sizeof(S2Segment));
+      std::memcpy(blob + (L.items - L.queries), gp.items.data(),
+                  gp.items.size() * sizeof(S2Item));
+      std::memcpy(blob + (L.run_items - L.queries), gp.run_items.data(),
+                  gp.run_items.size() * sizeof(int32_t));
+    }
     std::memcpy(blob + (L.packed_items - L.queries), gp.packed_items.data(),
                 gp.packed_items.size() * sizeof(int32_t));
     std::memcpy(blob + (L.item_meta - L.queries), gp.item_meta.data(),
