@@ -420,6 +420,31 @@ struct GatherPlan {
 
 int32_t offs_count(const GatherPlan &gp) { return gp.nb + 1; }
 
+// Orders a tile list for the persistent kernel, whose CTA j (of G = min(n,
+// sms)) takes entries j, j + G, j + 2G, ...: largest items (by key tiles)
+// first, dealt to the CTAs in rows of G that alternate in direction (a
+// snake), so that a CTA that drew a large item in one row draws a small one
+// in the next.  The last, partial row runs in ascending CTA order (CTAs
+// 0 .. of it take an extra item), so the rows are oriented from there back.
+constexpr int kBalanceItemsPerSm = 8;
+void balance_tiles(std::vector<dbsa_tile_item> &tiles, int sms) {
+  const int64_t n = (int64_t)tiles.size();
+  const int64_t G = std::min<int64_t>(n, std::max(1, sms));
+  if (G <= 1) return;
+  auto key_tiles = [&](int64_t i) { return (tiles[i].len[0] + kTileKeys - 1) / kTileKeys; };
+  std::vector<int64_t> order(n);
+  for (int64_t i = 0; i < n; ++i) order[i] = i;
+  std::stable_sort(order.begin(), order.end(),
+                   [&](int64_t a, int64_t b) { return key_tiles(a) > key_tiles(b); });
+  const int64_t last_row = (n - 1) / G;
+  std::vector<dbsa_tile_item> sorted(n);
+  for (int64_t k = 0; k < n; ++k) {
+    const int64_t r = k / G, j = k % G;
+    sorted[r * G + (((last_row - r) & 1) == 0 ? j : G - 1 - j)] = tiles[order[k]];
+  }
+  tiles.swap(sorted);
+}
+
 // Packed rows of the items: packed_items[k] owns rows [k R, (k + 1) R), and
 // its query rows are rotated at (the query's token position - the item's
 // p_begin); the other items (tails) have no packed rows.
@@ -659,6 +684,12 @@ dbsa_status gather_plan(const dbsa_config *cfg, const int32_t *offs, int32_t nb,
           t.len[0] = offs[b + 1] - offs[b];
           gp.tc_tiles.push_back(t);
         }
+    // A pass with a few items per SM (a decode step: one 128-row tile per (KV
+    // head, block)) is ordered for the persistent kernel's balance; longer
+    // lists keep the order in which the row tiles of one block run together
+    // (their K/V tiles are then read from L2).
+    if ((int64_t)gp.tc_tiles.size() < (int64_t)kBalanceItemsPerSm * num_sms())
+      balance_tiles(gp.tc_tiles, num_sms());
   }
   return DBSA_OK;
 }
