@@ -131,6 +131,28 @@ def test_long_gather_many_splits_peaky():
         Stage2Run(cfg, offs, sels, n_new, tail_len, seed=13).run().check("long n%d" % n_new)
 
 
+def test_staged_and_direct_items_share_q_slots():
+    """A prompt pass whose blocks alternate between short ones (at most two
+    128-key tiles: the kernel stores those items' rows directly and frees
+    their Q slot at the last QK) and long ones (three or more tiles: rows
+    staged in the Q tile, slot freed after the copies), with several items
+    per CTA, so that each Q slot is reused by both kinds in turn; then a
+    decode step on the same cache (a launch without staging)."""
+    rng = np.random.default_rng(21)
+    lens = [int(rng.integers(60, 250)) if b % 2 else int(rng.integers(390, 600))
+            for b in range(16)]
+    offs = offsets(lens)
+    sels = [np.concatenate([[0], np.sort(rng.choice(np.arange(1, 16), 8, replace=False))])
+            for _ in range(24)]
+    cfg = dbsa.DbsaConfig(8, 2, 128, "bf16", 5e5, 2)
+    run = Stage2Run(cfg, offs, sels, 40, 40, seed=21).run()
+    rows = 4 * 40 * np.bincount(np.concatenate(sels), minlength=16)
+    items = 2 * int(np.sum((rows + 127) // 128))
+    assert items > 3 * 148   # several items per CTA of the persistent kernel
+    run.check("staged/direct prompt", queries=[0, 5, 11, 23])
+    Stage2Run(cfg, offs, sels, 1, 41, seed=22).run().check("decode", queries=[0, 23])
+
+
 def test_all_blocks_in_order_equals_stage1_positions():
     # selecting every block in encoding order reproduces the original positions
     lens = [100, 130, 90]
