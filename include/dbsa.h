@@ -326,7 +326,9 @@ void dbsa_test_wait_expiry(uint64_t limit_ns);
 /* Calls this library has made (all threads) that allocate or free
  * page-locked host memory or create or destroy CUDA events: the plan staging
  * of the workspace-taking calls, on a thread's first calls and when a plan
- * outgrows its slot.  dbsa_gather_rope_attend_noalloc makes none. */
+ * outgrows the staging capacity (which then doubles, and each of the eight
+ * staging slots is brought up to it on its next use).
+ * dbsa_gather_rope_attend_noalloc makes none. */
 int64_t dbsa_host_allocation_calls(void);
 
 /* One Stage-1 tile-list entry: a 128-row query tile of one head, and at most
