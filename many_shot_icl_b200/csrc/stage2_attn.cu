@@ -485,7 +485,9 @@ __global__ void __launch_bounds__(32 * RT * KG, 1) stage2_attn_kernel(const Stag
 // One warp per output row (query q, token u, head h): combine the row's split
 // partials, O = sum_i 2^(M_i - M) L_i O_i / sum_i 2^(M_i - M) L_i.  The lanes
 // read the items' (M_i, L_i) in parallel (lane i % 32 holds item i's weight);
-// the items' rows are then added in item order, four loads in flight.
+// the items' rows are then added in item order, four loads in flight.  Rows
+// run token-fastest, the order of an item's partial rows, so the warps of a
+// CTA read adjacent rows of each item.
 template <int D, typename OT>
 __global__ void __launch_bounds__(128) stage2_merge_kernel(const Stage2Args a) {
   pdl_enter();
@@ -493,8 +495,8 @@ __global__ void __launch_bounds__(128) stage2_merge_kernel(const Stage2Args a) {
   const int lane = threadIdx.x & 31;
   const int64_t n_rows = (int64_t)a.n_queries * a.n_new * a.Hq;
   if (row >= n_rows) return;
-  const int h = (int)(row % a.Hq);
-  const int tok = (int)((row / a.Hq) % a.n_new);
+  const int tok = (int)(row % a.n_new);
+  const int h = (int)((row / a.n_new) % a.Hq);
   const int q = (int)(row / ((int64_t)a.Hq * a.n_new));
   const S2Query qi = a.queries[q];
   const int n = qi.n_items;
@@ -558,9 +560,9 @@ __global__ void __launch_bounds__(128) stage2_merge_kernel(const Stage2Args a) {
 // per output row (query token u, head h), each taking half of the row's
 // sources: alternate groups of 4 tail keys, and one half of its partials.
 // Lane l holds the elements i = l + 32 j (j < D / 32), so the rotate-half
-// pairs (i, i + D/2) sit in the same lane.  The CTA rotates the query's tail
-// keys, 32 at a time, into shared memory at their positions T'_q + u' (fp32,
-// no rounding), with their values; a warp scores its rotated query row
+// pairs (i, i + D/2) sit in the same lane.  The CTA rotates the tail keys its
+// rows can see, 32 at a time, into shared memory at their positions T'_q + u'
+// (fp32, no rounding), with their values; a warp scores its rotated query row
 // against its keys u' <= the row's tail index (the causal rule), in log2
 // units, with an online softmax.  It then merges its half of the row's block
 // partials (M_i, L_i, O_i), written by the tensor-core pass, into that state
@@ -609,8 +611,11 @@ __global__ void __launch_bounds__(512, 2) stage2_tail_merge_kernel(const Stage2A
   float m = -INFINITY, l = 0.f, acc[E];
 #pragma unroll
   for (int j = 0; j < E; ++j) acc[j] = 0.f;
-  for (int k0 = 0; k0 < a.tail_len; k0 += CH) {
-    const int nk = min(CH, a.tail_len - k0);
+  // the CTA's rows see the tail keys up to its last row's tail index
+  const int r_last = min(R, blockIdx.z * 8 + RW) - 1;
+  const int k_end = a.tail_len - a.n_new + r_last / g + 1;
+  for (int k0 = 0; k0 < k_end; k0 += CH) {
+    const int nk = min(CH, k_end - k0);
     __syncthreads();   // the previous chunk has been read by every warp
 #pragma unroll 4
     for (int u = threadIdx.x; u < nk * H; u += blockDim.x) {
