@@ -74,6 +74,13 @@ constexpr int kTailMergeMaxRows = 32;
 // compact mode on the tensor core; fewer rows stay on the per-query mma.sync
 // kernel.
 constexpr int kCompactMinRows = 64;
+// Tensor-core passes whose items average at least this many key tiles rotate
+// the packed query rows inside the kernel (the epilogue warpgroup fills the
+// Q tile of the item two ahead while the next one runs); with shorter items
+// (demonstration-granular decode steps, one key tile each) every item would
+// wait for its rotation, so qhat_kernel packs the rows beforehand and the
+// kernel loads them by TMA.
+constexpr int kRotateQMinTiles = 4;
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Copies bytes from page-locked host memory (read over the bus by the SMs)
@@ -420,6 +427,13 @@ struct GatherPlan {
 
 int32_t offs_count(const GatherPlan &gp) { return gp.nb + 1; }
 
+// Whether the pass's tensor-core kernel rotates its packed query rows itself.
+bool rotates_q(const GatherPlan &gp) {
+  int64_t tiles = 0;
+  for (const dbsa_tile_item &t : gp.tc_tiles) tiles += (t.len[0] + kTileKeys - 1) / kTileKeys;
+  return tiles >= (int64_t)kRotateQMinTiles * (int64_t)gp.tc_tiles.size();
+}
+
 // Orders a tile list for the persistent kernel, whose CTA j (of G = min(n,
 // sms)) takes entries j, j + G, j + 2G, ...: largest items (by key tiles)
 // first, dealt to the CTAs in rows of G that alternate in direction (a
@@ -696,17 +710,15 @@ dbsa_status gather_plan(const dbsa_config *cfg, const int32_t *offs, int32_t nb,
 
 // -------------------------------------------------------------- workspace layouts
 struct S1Layout {
-  size_t rope, items, q_rot, k_rot, v_bf16, total;
+  size_t rope, items, k_rot, v_bf16, total;
   int32_t n_hi;
 };
-S1Layout s1_layout(const dbsa_config *cfg, int64_t max_pos, int64_t n_items, int64_t q_rows,
-                   int64_t k_rows) {
+S1Layout s1_layout(const dbsa_config *cfg, int64_t max_pos, int64_t n_items, int64_t k_rows) {
   S1Layout l;
   Carve cv;
   l.n_hi = (int32_t)(std::max<int64_t>(max_pos - 1, 0) / kRopeLo + 1);
   l.rope = cv.take(rope_table_bytes(l.n_hi, cfg->head_dim));
   l.items = cv.take((size_t)n_items * sizeof(dbsa_tile_item));
-  l.q_rot = cv.take((size_t)cfg->n_q_heads * q_rows * cfg->head_dim * 2);
   l.k_rot = cv.take((size_t)cfg->n_kv_heads * k_rows * cfg->head_dim * 2);
   l.v_bf16 = cfg->dtype == DBSA_F32 ? cv.take((size_t)cfg->n_kv_heads * k_rows * cfg->head_dim * 2)
                                     : 0;
@@ -741,7 +753,9 @@ S2Layout s2_layout(const dbsa_config *cfg, const GatherPlan &gp, int32_t n_new,
   l.items = cv.take(gp.items.size() * sizeof(S2Item));
   l.run_items = cv.take(gp.run_items.size() * sizeof(int32_t));
   l.blob_end = cv.take(0);
-  l.q_rot_pos = cv.take(gp.items.size() * sizeof(int32_t));
+  // rows packed by qhat_kernel (passes of short items only)
+  const bool packs_q = !gp.per_query && !rotates_q(gp);
+  l.q_rot_pos = cv.take(packs_q ? gp.items.size() * sizeof(int32_t) : 0);
   const int64_t T = gp.cache_rows;
   if (gp.compact) {
     // every query's gathered keys (rotated) and values, bf16 [Hkv][rows][D]
@@ -754,7 +768,7 @@ S2Layout s2_layout(const dbsa_config *cfg, const GatherPlan &gp, int32_t n_new,
                           ? (size_t)cfg->n_kv_heads * T * cfg->head_dim * 2
                           : 0);
   }
-  l.q_hat = cv.take((size_t)cfg->n_kv_heads * gp.tc_rows * cfg->head_dim * 2);
+  l.q_hat = cv.take(packs_q ? (size_t)cfg->n_kv_heads * gp.tc_rows * cfg->head_dim * 2 : 0);
   const size_t rows = gp.items.size() * (size_t)cfg->n_q_heads * n_new;
   l.part_acc = cv.take(rows * cfg->head_dim * sizeof(uint16_t));
   l.part_ml = cv.take(rows * sizeof(float2));
@@ -876,7 +890,7 @@ int64_t dbsa_stage1_tile_count(const dbsa_config *cfg, const int32_t *offs_host,
 
 size_t dbsa_encode_workspace_size(const dbsa_config *cfg, int64_t n_tokens, int32_t nb) {
   if (check_cfg(cfg) != DBSA_OK || n_tokens <= 0 || nb <= 0) return 0;
-  return s1_layout(cfg, n_tokens, encode_item_bound(cfg, n_tokens, nb), n_tokens, n_tokens).total;
+  return s1_layout(cfg, n_tokens, encode_item_bound(cfg, n_tokens, nb), n_tokens).total;
 }
 
 dbsa_status dbsa_encode_blocks(const dbsa_config *cfg, const void *q, const void *k,
@@ -897,7 +911,7 @@ dbsa_status dbsa_encode_blocks(const dbsa_config *cfg, const void *q, const void
                            (long long)T);
   std::vector<dbsa_tile_item> items;
   encode_items(cfg, offs_host, nb, items);
-  const S1Layout L = s1_layout(cfg, T, encode_item_bound(cfg, T, nb), T, T);
+  const S1Layout L = s1_layout(cfg, T, encode_item_bound(cfg, T, nb), T);
   if ((s = check_ws(workspace, ws_bytes, L.total)) != DBSA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const bool f32 = cfg->dtype == DBSA_F32;
@@ -911,16 +925,11 @@ dbsa_status dbsa_encode_blocks(const dbsa_config *cfg, const void *q, const void
                         items.size() * sizeof(dbsa_tile_item), st, workspace)) != cudaSuccess)
     return cuda_fail(e, "tile list upload");
   IngestArgs ia{};
-  ia.q = q;
   ia.k = k;
   ia.v = v;
   ia.n_tok = (int32_t)T;
   ia.pos0 = 0;
-  ia.Hq = cfg->n_q_heads;
   ia.Hkv = cfg->n_kv_heads;
-  ia.q_rot = at<void>(workspace, L.q_rot);
-  ia.q_rows = T;
-  ia.q_row_base = 0;
   ia.k_rot = at<void>(workspace, L.k_rot);
   ia.k_rows = T;
   ia.k_row_base = 0;
@@ -932,8 +941,10 @@ dbsa_status dbsa_encode_blocks(const dbsa_config *cfg, const void *q, const void
   if ((e = launch_ingest(ia, cfg->head_dim, f32, st)) != cudaSuccess) return cuda_fail(e, "ingest");
   count_launches(1);
   Stage1Args sa{};
-  sa.q_rot = ia.q_rot;
-  sa.q_rows = T;
+  sa.q_src = q;
+  sa.q_f32 = f32;
+  sa.q_heads = cfg->n_q_heads;
+  sa.rope = rope;
   sa.k_rot = ia.k_rot;
   sa.k_rows = T;
   sa.v = f32 ? ia.v_bf16 : v_cache;
@@ -962,7 +973,7 @@ size_t dbsa_append_workspace_size(const dbsa_config *cfg, const int32_t *offs_ho
   if (check_cfg(cfg) != DBSA_OK || check_offs(offs_host, nb) != DBSA_OK || L < 1) return 0;
   const AppendPlan ap = append_plan(cfg, offs_host, nb, L);
   const int64_t n_items = (int64_t)cfg->n_q_heads * ((L + kTileRows - 1) / kTileRows);
-  return s1_layout(cfg, (int64_t)offs_host[nb] + L, n_items, L, ap.k_rows).total;
+  return s1_layout(cfg, (int64_t)offs_host[nb] + L, n_items, ap.k_rows).total;
 }
 
 dbsa_status dbsa_append_block(const dbsa_config *cfg, const void *q, const void *k, const void *v,
@@ -994,7 +1005,7 @@ dbsa_status dbsa_append_block(const dbsa_config *cfg, const void *q, const void 
     block_items(cfg, ap.offs.data(), nb, (int32_t)T0, krow, vrow, ap.nr, ap.rs, ap.re, items);
   }
   const int64_t n_items_bound = (int64_t)cfg->n_q_heads * ((L + kTileRows - 1) / kTileRows);
-  const S1Layout Ly = s1_layout(cfg, T0 + L, n_items_bound, L, ap.k_rows);
+  const S1Layout Ly = s1_layout(cfg, T0 + L, n_items_bound, ap.k_rows);
   if ((s = check_ws(workspace, ws_bytes, Ly.total)) != DBSA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
@@ -1029,16 +1040,11 @@ dbsa_status dbsa_append_block(const dbsa_config *cfg, const void *q, const void 
     count_launches(1);
   }
   IngestArgs ia{};
-  ia.q = q;
   ia.k = k;
   ia.v = v;
   ia.n_tok = L;
   ia.pos0 = (int32_t)T0;
-  ia.Hq = cfg->n_q_heads;
   ia.Hkv = cfg->n_kv_heads;
-  ia.q_rot = at<void>(workspace, Ly.q_rot);
-  ia.q_rows = L;
-  ia.q_row_base = 0;
   ia.k_rot = k_rot;
   ia.k_rows = ap.k_rows;
   ia.k_row_base = ap.new_row;
@@ -1050,8 +1056,10 @@ dbsa_status dbsa_append_block(const dbsa_config *cfg, const void *q, const void 
   if ((e = launch_ingest(ia, cfg->head_dim, f32, st)) != cudaSuccess) return cuda_fail(e, "ingest");
   count_launches(1);
   Stage1Args sa{};
-  sa.q_rot = ia.q_rot;
-  sa.q_rows = L;
+  sa.q_src = q;
+  sa.q_f32 = f32;
+  sa.q_heads = cfg->n_q_heads;
+  sa.rope = rope;
   sa.k_rot = k_rot;
   sa.k_rows = ap.k_rows;
   sa.v = f32 ? v_bf16 : v_cache;
@@ -1122,6 +1130,45 @@ bool plan_key(const dbsa_config *cfg, const int32_t *offs, int32_t nb, int32_t n
   key.insert(key.end(), sel_ptr, sel_ptr + nq + 1);
   key.insert(key.end(), sel, sel + sel_ptr[nq]);
   return true;
+}
+
+// The query rows of a partial-mode tensor-core pass.  Passes of long items
+// hand the kernel the unrotated q_new (it rotates the packed rows itself);
+// passes of short items run qhat_kernel first (recording, when a gather map
+// is requested, the position each item's token 0 was rotated at) and the
+// kernel loads the packed rows by TMA.
+cudaError_t set_query_rows(Stage1Args &sa, const dbsa_config *cfg, const GatherPlan &gp,
+                           const S2Layout &L, const void *q_new, int32_t n_new, int32_t tail_len,
+                           int32_t n_items, const RopeTables &rope, void *workspace,
+                           const int32_t *dbg_map, cudaStream_t st) {
+  const bool f32 = cfg->dtype == DBSA_F32;
+  sa.part.item_meta = at<int4>(workspace, L.item_meta);
+  if (rotates_q(gp)) {
+    sa.q_src = q_new;
+    sa.q_f32 = f32;
+    sa.q_heads = cfg->n_q_heads;
+    sa.rope = rope;
+    return cudaSuccess;
+  }
+  QHatArgs qa{};
+  qa.q_new = q_new;
+  qa.n_new = n_new;
+  qa.tail_len = tail_len;
+  qa.Hq = cfg->n_q_heads;
+  qa.Hkv = cfg->n_kv_heads;
+  qa.n_items = n_items;
+  qa.item_meta = sa.part.item_meta;
+  qa.rows = gp.tc_rows;
+  qa.q_hat = at<void>(workspace, L.q_hat);
+  qa.q_rot_pos = dbg_map != nullptr ? at<int32_t>(workspace, L.q_rot_pos) : nullptr;
+  qa.rope = rope;
+  cudaError_t e = launch_qhat(qa, cfg->head_dim, f32, st);
+  if (e != cudaSuccess) return e;
+  count_launches(1);
+  sa.q_rot = qa.q_hat;
+  sa.q_rows = gp.tc_rows;
+  sa.part.q_rot_pos = qa.q_rot_pos;
+  return cudaSuccess;
 }
 
 dbsa_status gather_impl(const dbsa_config *cfg, const void *k_cache, const void *v_cache,
@@ -1306,25 +1353,11 @@ dbsa_status gather_impl(const dbsa_config *cfg, const void *k_cache, const void 
     if ((e = launch_compact(ca, cfg->head_dim, f32, st)) != cudaSuccess)
       return cuda_fail(e, "compact gather");
     count_launches(1);
-    QHatArgs qa{};
-    qa.q_new = q_new;
-    qa.n_new = n_new;
-    qa.tail_len = tail_len;
-    qa.Hq = cfg->n_q_heads;
-    qa.Hkv = cfg->n_kv_heads;
-    qa.n_items = a.n_items;
-    qa.item_meta = at<int4>(workspace, L.item_meta);
-    qa.rows = gp.tc_rows;
-    qa.q_hat = at<void>(workspace, L.q_hat);
-    qa.q_rot_pos = nullptr;
-    qa.rope = rope;
-    if ((e = launch_qhat(qa, cfg->head_dim, f32, st)) != cudaSuccess)
-      return cuda_fail(e, "query rotation");
-    count_launches(1);
     a.dbg_map = nullptr;  // written by the compact gather above
     Stage1Args sa{};
-    sa.q_rot = qa.q_hat;
-    sa.q_rows = gp.tc_rows;
+    if ((e = set_query_rows(sa, cfg, gp, L, q_new, n_new, tail_len, a.n_items, rope, workspace,
+                            nullptr, st)) != cudaSuccess)
+      return cuda_fail(e, "query rotation");
     sa.k_rot = ca.k_hat;
     sa.k_rows = gp.compact_rows;
     sa.v = ca.v_hat;
@@ -1384,25 +1417,11 @@ dbsa_status gather_impl(const dbsa_config *cfg, const void *k_cache, const void 
         return cuda_fail(e, "block-relative rotation");
       count_launches(1);
     }
-    QHatArgs qa{};
-    qa.q_new = q_new;
-    qa.n_new = n_new;
-    qa.tail_len = tail_len;
-    qa.Hq = cfg->n_q_heads;
-    qa.Hkv = cfg->n_kv_heads;
-    qa.n_items = a.n_items;
-    qa.item_meta = at<int4>(workspace, L.item_meta);
-    qa.rows = gp.tc_rows;
-    qa.q_hat = at<void>(workspace, L.q_hat);
-    qa.q_rot_pos = dbg_map != nullptr ? at<int32_t>(workspace, L.q_rot_pos) : nullptr;
-    qa.rope = rope;
-    if ((e = launch_qhat(qa, cfg->head_dim, f32, st)) != cudaSuccess)
-      return cuda_fail(e, "query rotation");
-    count_launches(1);
     a.dbg_map = nullptr;  // written by the tensor-core kernel's epilogue (sa.part.dbg)
     Stage1Args sa{};
-    sa.q_rot = qa.q_hat;
-    sa.q_rows = gp.tc_rows;
+    if ((e = set_query_rows(sa, cfg, gp, L, q_new, n_new, tail_len, a.n_items, rope, workspace,
+                            dbg_map, st)) != cudaSuccess)
+      return cuda_fail(e, "query rotation");
     sa.k_rot = ra.k_hat;
     sa.k_rows = gp.cache_rows;
     sa.v = f32 ? ra.v_bf16 : v_cache;
@@ -1425,7 +1444,6 @@ dbsa_status gather_impl(const dbsa_config *cfg, const void *k_cache, const void 
     sa.part.dbg_cap = dbg_cap;
     sa.part.items = a.items;
     sa.part.queries = a.queries;
-    sa.part.q_rot_pos = qa.q_rot_pos;
     sa.part.tail_len = tail_len;
     sa.wait_limit_ns = wait_expiry;
     sa.withhold_tiles = wait_expiry != 0;

@@ -87,15 +87,13 @@ cudaError_t launch_rope_tables(float *base, int32_t n_hi, int32_t head_dim, doub
 RopeTables rope_tables_at(const float *base, int32_t n_hi, int32_t head_dim);
 size_t rope_table_bytes(int32_t n_hi, int32_t head_dim);
 
-// Rotate Q and K of n_tok token-major input rows (positions pos0..), copy the
-// raw K/V into the cache rows pos0.., and (f32 inputs) write bf16 V.
+// Rotate K of n_tok token-major input rows (positions pos0..), copy the raw
+// K/V into the cache rows pos0.., and (f32 inputs) write bf16 V.  (The
+// queries are rotated by the tensor-core kernel as it reads them.)
 struct IngestArgs {
-  const void *q, *k, *v;           // [n_tok][H][D] input dtype
+  const void *k, *v;               // [n_tok][Hkv][D] input dtype
   int32_t n_tok, pos0;
-  int32_t Hq, Hkv;
-  void *q_rot;                     // bf16 [Hq][q_rows][D], row q_row_base + t
-  int64_t q_rows;
-  int32_t q_row_base;
+  int32_t Hkv;
   void *k_rot;                     // bf16 [Hkv][k_rows][D], row k_row_base + t
   int64_t k_rows;
   int32_t k_row_base;
@@ -142,12 +140,19 @@ struct Stage1Partial {
   // each key r of the tile's range, entry [query][p_begin + r] = (the cache
   // row its K and V tiles were loaded from, the fresh position the pair of
   // rotations gives it: the query's token-0 position minus the position the
-  // query rotation used (q_rot_pos) plus the key's block-relative position).
+  // kernel rotated the item's token-0 query rows at plus the key's
+  // block-relative position).
   int32_t *dbg;
   int64_t dbg_cap;
   const S2Item *items;
   const S2Query *queries;
-  const int32_t *q_rot_pos;    // per item: position qhat_kernel rotated token 0 at
+  // per item (first packed row or -1, the position its query rows are
+  // rotated at for token 0, its query, 0): read where the kernel rotates the
+  // packed query rows (q_src set)
+  const int4 *item_meta;
+  // passes whose packed rows qhat_kernel rotated (q_rot set): per item, the
+  // position it rotated token 0 at
+  const int32_t *q_rot_pos;
   int32_t tail_len;
 };
 
@@ -202,7 +207,16 @@ cudaError_t launch_compact(const CompactArgs &a, int head_dim, bool f32, cudaStr
 
 // Stage-1 tcgen05 attention over a tile list.
 struct Stage1Args {
-  const void *q_rot;      // bf16 [Hq][q_rows][D]
+  // The queries, in one of two forms.  q_src (non-null): unrotated, bf16 or
+  // fp32 (q_f32), rotated by the kernel itself as it fills each Q tile.
+  // Stage 1: [rows][q_heads][D], row q_row0 + r of an item at position
+  // q_pos0 + r.  Partial mode: [queries][n_new][q_heads][D], packed rows
+  // found through part.packed_items and part.item_meta.  Otherwise q_rot:
+  // already rotated bf16 [Hq][q_rows][D] rows, loaded by TMA.
+  const void *q_src;
+  int32_t q_f32, q_heads;
+  RopeTables rope;
+  const void *q_rot;
   int64_t q_rows;
   const void *k_rot;      // bf16 [Hkv][k_rows][D]
   int64_t k_rows;

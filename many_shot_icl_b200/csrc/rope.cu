@@ -3,10 +3,10 @@
 // [DBSA notes] §Stage 1, item 3: queries and keys are rotated at sequential
 // positions, while the cache keeps K/V BEFORE the rotary transform.  The
 // preparation pass therefore (a) copies the raw K/V into the head-major cache,
-// (b) writes a rotated bf16 copy of Q and K into the workspace for the
-// tensor-core kernel, and for fp32 inputs (c) a bf16 copy of V.  It is pure
-// streaming work (HBM-bound); the angle factors come from two small tables
-// built once per call in fp64.
+// (b) writes a rotated bf16 copy of K into the workspace for the tensor-core
+// kernel (which rotates the queries itself as it reads them), and for fp32
+// inputs (c) a bf16 copy of V.  It is pure streaming work (HBM-bound); the
+// angle factors come from two small tables built once per call in fp64.
 #include <cuda_bf16.h>
 
 #include "dbsa_internal.h"
@@ -40,15 +40,15 @@ __global__ void rope_tables_kernel(float *base, int32_t n_hi, int32_t half, doub
 }
 
 // One work unit = (token t, head slot hh, chunk cp): elements [8cp, 8cp+8) of
-// the first half and the matching 8 of the second half.
+// the first half and the matching 8 of the second half; slots 0..Hkv-1 are
+// the key heads, the rest the value heads.
 template <int D, typename T>
 __global__ void __launch_bounds__(256) ingest_kernel(IngestArgs a) {
   pdl_enter();
   constexpr int H = D / 2;
   constexpr int CP = H / 8;
-  const int slots = a.Hq + 2 * a.Hkv;
+  const int slots = 2 * a.Hkv;
   const int64_t n_units = (int64_t)a.n_tok * slots * CP;
-  const T *q = static_cast<const T *>(a.q);
   const T *k = static_cast<const T *>(a.k);
   const T *v = static_cast<const T *>(a.v);
   for (int64_t u = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; u < n_units;
@@ -59,18 +59,8 @@ __global__ void __launch_bounds__(256) ingest_kernel(IngestArgs a) {
     const int64_t pos = a.pos0 + t;
     const int i0 = cp * 8;
     float lo[8], hi[8];
-    if (hh < a.Hq) {  // query head: rotate into q_rot
-      const T *src = q + (t * a.Hq + hh) * D;
-      load8(src + i0, lo);
-      load8(src + H + i0, hi);
-      float c[8], s[8];
-      rope_cs8(a.rope, pos, i0, H, c, s);
-      rotate8(lo, hi, c, s);
-      bf16 *dst = static_cast<bf16 *>(a.q_rot) + ((int64_t)hh * a.q_rows + a.q_row_base + t) * D;
-      store8_bf16(dst + i0, lo);
-      store8_bf16(dst + H + i0, hi);
-    } else if (hh < a.Hq + a.Hkv) {  // key head: cache the raw key, rotate into k_rot
-      const int c_ = hh - a.Hq;
+    if (hh < a.Hkv) {  // key head: cache the raw key, rotate into k_rot
+      const int c_ = hh;
       const T *src = k + (t * a.Hkv + c_) * D;
       T *cache = static_cast<T *>(a.k_cache) + ((int64_t)c_ * a.cap + pos) * D;
       copy8(src + i0, cache + i0);
@@ -84,7 +74,7 @@ __global__ void __launch_bounds__(256) ingest_kernel(IngestArgs a) {
       store8_bf16(dst + i0, lo);
       store8_bf16(dst + H + i0, hi);
     } else {  // value head: cache the raw value (and a bf16 copy for fp32 inputs)
-      const int c_ = hh - a.Hq - a.Hkv;
+      const int c_ = hh - a.Hkv;
       const T *src = v + (t * a.Hkv + c_) * D;
       T *cache = static_cast<T *>(a.v_cache) + ((int64_t)c_ * a.cap + pos) * D;
       copy8(src + i0, cache + i0);
@@ -354,7 +344,7 @@ cudaError_t launch_rope_tables(float *base, int32_t n_hi, int32_t head_dim, doub
 }
 
 cudaError_t launch_ingest(const IngestArgs &a, int head_dim, bool f32, cudaStream_t st) {
-  const int64_t n = (int64_t)a.n_tok * (a.Hq + 2 * a.Hkv) * (head_dim / 16);
+  const int64_t n = (int64_t)a.n_tok * 2 * a.Hkv * (head_dim / 16);
   const int g = grid_for(n, 256);
   if (head_dim == 128) {
     if (f32) pdl_launch(ingest_kernel<128, float>, dim3(g), dim3(256), 0, st, a);

@@ -10,9 +10,9 @@
 // holds only the tiles that contain an allowed pair).
 //
 // One persistent CTA per SM walks items round-robin.  Warp roles:
-//   warp 0      TMA producer: two independent cursors, one for each item's Q
-//               tile (double-buffered) and its K tiles (3-stage ring), one
-//               for the V tiles (2-stage ring)
+//   warp 0      TMA producer: two independent cursors, one for the K tiles
+//               (3-stage ring, preceded by each item's Q tile when the Q
+//               rows come pre-rotated), one for the V tiles (2-stage ring)
 //   warp 1      TMEM owner; one thread issues O_h += P_h V_h for the two key
 //               halves of each tile (tcgen05, A from TMEM)
 //   warp 10     one thread issues S = Q K^T (tcgen05, both operands in SMEM)
@@ -26,15 +26,20 @@
 //               over its 64 scores held in registers (mask, max, rescale,
 //               exp2).  At an item's end they publish the merge factors of
 //               the two states and go on.
-//   warps 11..14 epilogue: combine O_0 and O_1 of the finished item, free O
+//   warps 11..14 Q tiles and epilogue: rotate each item's query rows into
+//               its Q tile (double-buffered, two items ahead; launches with
+//               ROTQ), then, at the item's end, combine O_0 and O_1, free O
 //               for the next item's first PV, and write the rows out (bf16:
 //               staged in the item's Q tile, then one bulk copy per row).
 // S = Q K^T lives in TMEM in two 128-column buffers (tile parity); each
 // warpgroup writes its 64 keys' P as bf16 pairs over the first 32 columns of
 // its own half of the S buffer, and O_0, O_1 take D columns each: 512 columns
-// in all.  Q and K arrive already rotated (bf16) from the preparation pass; V
-// is read straight from the pre-RoPE cache.  Every wait is bounded and
-// reports DBSA_ERR_TIMEOUT.
+// in all.  With ROTQ the query rows are read unrotated and rotated in the
+// kernel (one thread per row, fp32, rounded once to bf16); without it they
+// arrive rotated (bf16, packed by a preceding kernel) and are loaded by TMA.
+// K arrives already rotated (bf16) from the preparation pass and V is read
+// straight from the pre-RoPE cache.  Every wait is bounded and reports
+// DBSA_ERR_TIMEOUT.
 //
 // Measured on B200: the tensor core runs a 128x128x16
 // MMA in 64 cycles but keeps only about one MMA queued, so the issuing
@@ -50,6 +55,7 @@
 
 #include "dbsa_internal.h"
 #include "sm100.cuh"
+#include "vec8.cuh"
 
 namespace dbsa {
 namespace {
@@ -63,21 +69,22 @@ constexpr uint32_t kFull = 0xFFFFFFFFu;
 // Ring depths (tiles in flight).  A K slot frees when its QK^T has run and is
 // needed again kStagesK tiles later; a V slot frees only after its PV, about
 // two tiles after the QK, and is needed kStagesV tiles later.  Q is double
-// buffered so that the next item's Q tile loads during the current item; a Q
-// slot frees once the item's epilogue has staged and copied its rows out
-// through it.
+// buffered: the epilogue warpgroup writes an item's Q tile once it has
+// finished the item two before it in the same slot (ROTQ), or the producer
+// loads it once that item's last QK^T has run or its staged rows have been
+// copied out.
 constexpr int kStagesK = 3;
 constexpr int kStagesV = 2;
 // The epilogue stages an item's bf16 rows in its Q tile only when the item
 // has at least this many key tiles: the Q slot then frees once the rows are
 // copied out, which for shorter items would hold up the next-but-one item's
-// Q load.  Shorter items store their rows directly and free the slot at
-// their last QK^T.
+// Q tile.  Shorter items store their rows directly.
 constexpr int kStageMinTiles = 3;
 constexpr int kStagesQ = 2;
 
 enum Bar {
-  B_Q_FULL = 0, B_Q_EMPTY = B_Q_FULL + kStagesQ,
+  B_Q_FULL = 0,                // [Q stage]: the Q tile is in place
+  B_Q_EMPTY = B_Q_FULL + kStagesQ,   // [Q stage]: an unstaged item's last QK^T (TMA Q tiles)
   B_K_FULL = B_Q_EMPTY + kStagesQ, B_K_EMPTY = B_K_FULL + kStagesK,
   B_V_FULL = B_K_EMPTY + kStagesK, B_V_EMPTY = B_V_FULL + kStagesV,
   B_S_FULL = B_V_EMPTY + kStagesV,  // [buffer]
@@ -88,7 +95,7 @@ enum Bar {
   B_ML_B = B_ML_A + 1,        // end of item: warpgroup 0 has published the merge factors
   B_ML_FREE = B_ML_B + 1,     // the epilogue warpgroup has read the merge factors
   B_DRAIN_QK = B_ML_FREE + 1,
-  B_Q_COPIED = B_DRAIN_QK + 1,  // [Q stage]: the epilogue has copied out the rows it staged there
+  B_Q_COPIED = B_DRAIN_QK + 1,  // [Q stage]: every row staged there has been copied out
   B_COUNT = B_Q_COPIED + kStagesQ
 };
 
@@ -217,12 +224,87 @@ struct Params {
   uint64_t wait_limit_ns;  // limit of every bounded wait
   int withhold_tiles;      // test hook: the producer loads nothing (every wait runs out)
   Stage1Partial part;  // partial-output mode (part.acc != null)
+  // Unrotated query rows.  Stage 1: row q_row0 + r of an item is q_src row
+  // (q_row0 + r) x q_heads + head, rotated at q_pos0 + r.  Partial mode:
+  // packed row w of an item's query (token w / g, local head w % g) comes
+  // from q_src [query][n_new][q_heads], rotated at item_meta.y + token.
+  const void *q_src;
+  int q_f32;               // q_src is fp32 (else bf16)
+  int q_heads;
+  RopeTables rope;
 };
+
+// One row of a Q tile in the layout a 128-byte-swizzled TMA tile load writes
+// and the QK^T descriptor reads: columns 64a..64a+63 in atom column a (HALF
+// bytes apart), row r at byte 128 r inside it, and the row's 16-byte chunk c
+// at chunk position c ^ (r mod 8).  Chunk j of the row holds columns
+// 8j..8j+7, rounded to bf16 here.
+__device__ __forceinline__ void put_q_chunk(uint8_t *tile, int row, int j, const float (&f)[8]) {
+  constexpr uint32_t HALF = 128 * 64 * 2;
+  uint32_t w[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * e], f[2 * e + 1]);
+    w[e] = *reinterpret_cast<uint32_t *>(&h);
+  }
+  *reinterpret_cast<uint4 *>(tile + (j >> 3) * HALF + row * 128 + (((j & 7) ^ (row & 7)) << 4)) =
+      make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// This thread's row of an item's Q tile: the unrotated query vector, rotated
+// at its position (rotate-half RoPE with the angle tables, the rounding of
+// every other rotation in the library) and stored as bf16; rows past the
+// item's n_rows are zero.  Returns the position the row was rotated at.
+template <int D, typename T>
+__device__ __forceinline__ int rotate_q_row(const Params &p, const Item &it, int row,
+                                            uint8_t *tile) {
+  constexpr int H = D / 2;
+  const bool valid = row < it.n_rows;
+  int pos = 0;
+  int64_t off = 0;
+  if (valid) {
+    if (p.part.acc != nullptr) {
+      const int grow = it.q_row0 + row;                 // row of the kv head's packed rows
+      const int R = p.part.group * p.part.n_new;
+      const int item = __ldg(p.part.packed_items + grow / R);
+      const int w = grow % R;
+      const int4 meta = __ldg(p.part.item_meta + item);
+      const int tok = w / p.part.group;
+      pos = meta.y + tok;
+      off = (((int64_t)meta.z * p.part.n_new + tok) * p.q_heads + it.head * p.part.group +
+             w % p.part.group) * D;
+    } else {
+      pos = it.q_pos0 + row;
+      off = ((int64_t)(it.q_row0 + row) * p.q_heads + it.head) * D;
+    }
+  }
+  const T *src = static_cast<const T *>(p.q_src) + off;
+#pragma unroll 4
+  for (int i0 = 0; i0 < H; i0 += 8) {
+    float lo[8], hi[8];
+    if (valid) {
+      float c[8], sn[8];
+      load8(src + i0, lo);
+      load8(src + H + i0, hi);
+      rope_cs8(p.rope, pos, i0, H, c, sn);
+      rotate8(lo, hi, c, sn);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) lo[e] = hi[e] = 0.f;
+    }
+    put_q_chunk(tile, row, i0 / 8, lo);
+    put_q_chunk(tile, row, (H + i0) / 8, hi);
+  }
+  return pos;
+}
 
 // STAGE: the launch stages the bf16 rows of its items of at least
 // kStageMinTiles key tiles in their Q tiles (Stage 1 and prompt passes); a
 // launch without it (decode steps, fp32 outputs) has none of that code.
-template <int D, bool OUT_F32, bool STAGE>
+// ROTQ: the epilogue warpgroup rotates the query rows into the Q tiles (the
+// tensor map tmQ is unused); without it the producer loads pre-rotated Q
+// tiles through tmQ.
+template <int D, bool OUT_F32, bool STAGE, bool ROTQ>
 __global__ void __launch_bounds__(kThreads, 1)
     stage1_attn_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
@@ -259,9 +341,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStagesQ; ++s) {
-      mbar_init(&bar[B_Q_FULL + s], 1);
+      mbar_init(&bar[B_Q_FULL + s], ROTQ ? 128 : 1);   // the epilogue's rows / one TMA load
       mbar_init(&bar[B_Q_EMPTY + s], 1);     // an unstaged item's last QK^T
-      mbar_init(&bar[B_Q_COPIED + s], 128);  // a staged item's epilogue warpgroup
+      mbar_init(&bar[B_Q_COPIED + s], 128);  // a staged item's row copies
     }
     for (int s = 0; s < kStagesK; ++s) {
       mbar_init(&bar[B_K_FULL + s], 1);
@@ -299,14 +381,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ producer
-    // Two independent cursors over the CTA's tile sequence: K tiles (each
-    // item's Q tile first) and V tiles.  A K slot frees when its QK^T has
-    // run, a V slot only when its PV has run, which happens about two tiles
-    // later; separate cursors keep the K loads from queueing behind V slots.
-    // A Q slot frees at its item's last QK^T, or, when the epilogue staged
-    // the item's rows there, once it has copied them out.  Neither cursor
-    // blocks: the thread polls whichever slot it needs next.
-    tma_prefetch_desc(&tmQ);
+    // Two independent cursors over the CTA's tile sequence: K tiles (without
+    // ROTQ, each item's Q tile first) and V tiles.  A K slot frees when its
+    // QK^T has run, a V slot only when its PV has run, which happens about two
+    // tiles later; separate cursors keep the K loads from queueing behind V
+    // slots.  A Q slot frees at its item's last QK^T, or, when the epilogue
+    // staged the item's rows there, once it has copied them out.  Neither
+    // cursor blocks: the thread polls whichever slot it needs next.
+    if (!ROTQ) tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
     // Test hook: no tile is loaded, so every wait of the consumers is for a
@@ -328,14 +410,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     int kidx = withhold ? p.n_items : blockIdx.x, vidx = kidx, kt = 0, vt = 0;
     Item kit, vit;
     if (kidx < p.n_items) kit = vit = load_item(p.items, kidx);
-    bool need_q = kidx < p.n_items;
+    bool need_q = !ROTQ && kidx < p.n_items;
     uint32_t qn = 0, kn = 0, vn = 0;          // Q, K, V tiles issued
     int armed_q[kStagesQ], armed_k[kStagesK], armed_v[kStagesV];
-    // Per Q slot: how its last item frees it (-1 unused, 0 at its last QK^T,
-    // 1 after the epilogue's copies of the rows it staged there) and the
-    // uses of each kind so far; each kind has its own barrier.  The slots are
-    // used in turn, so the state is kept in registers as (slot used next,
-    // the other slot) and swapped after each Q load.
+    // Per Q slot (TMA Q tiles): how its last item frees it (-1 unused, 0 at
+    // its last QK^T, 1 after the epilogue's copies of the rows it staged
+    // there) and the uses of each kind so far; each kind has its own barrier.
+    // The slots are used in turn, so the state is kept in registers as (slot
+    // used next, the other slot) and swapped after each Q load.
     static_assert(kStagesQ == 2, "the Q slot state rotates between two slots");
     int qa_prev = -1, qb_prev = -1;
     uint32_t qa_staged = 0, qa_direct = 0, qb_staged = 0, qb_direct = 0;
@@ -398,7 +480,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               kidx += gridDim.x;
               if (kidx < p.n_items) {
                 kit = load_item(p.items, kidx);
-                need_q = true;
+                need_q = !ROTQ;
               }
             }
           }
@@ -487,7 +569,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           mma_commit(&bar[B_S_FULL + b]);
           mma_commit(&bar[B_K_EMPTY + st]);
-          if (t == ntiles - 1 && !stages_rows(ntiles)) mma_commit(&bar[B_Q_EMPTY + qs]);
+          if (!ROTQ && t == ntiles - 1 && !stages_rows(ntiles)) mma_commit(&bar[B_Q_EMPTY + qs]);
         } else {
           // O_h (+)= P_h V_h for the key halves h = 0, 1 of the tile, each as
           // soon as its warpgroup has written P_h; both accumulators must have
@@ -691,16 +773,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
-    // ------------------------------------------------------------ epilogue
-    // One thread per row (TMEM lane).  Per item: the merge factors, then, once
-    // the item's last PV is done (in-order tensor core: so are all of its
-    // PVs), O_0 and O_1 are read and combined, O is released for the next
-    // item's first PV, and the rows are written out; the item's Q tile, used
-    // to stage them, is then released to the producer.
+    // ------------------------------------------------------------ Q tiles and epilogue
+    // One thread per row (TMEM lane).  The Q tiles of the CTA's first two
+    // items are written first.  Per item: the merge factors, then, once the
+    // item's last PV is done (in-order tensor core: so are all of its PVs,
+    // and the QK^T that read its Q tile), O_0 and O_1 are read and combined,
+    // O is released for the next item's first PV, and the rows are written
+    // out; the item's Q slot, which may have staged them, then takes the Q
+    // tile of the item two ahead.
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const bool partial = p.part.acc != nullptr;
+    // The Q tile of item idx into slot qs; returns the position this
+    // thread's row was rotated at.
+    auto put_q = [&](int idx, uint32_t qs) -> int {
+      const Item it = load_item(p.items, idx);
+      uint8_t *tile = sQ + qs * TILE;
+      const int pos = p.q_f32 ? rotate_q_row<D, float>(p, it, row, tile)
+                              : rotate_q_row<D, bf16>(p, it, row, tile);
+      fence_proxy_async_smem();   // visible to the tensor core's reads
+      mbar_arrive(&bar[B_Q_FULL + qs]);
+      return pos;
+    };
+    static_assert(kStagesQ == 2, "Q slots alternate between two items");
+    int qpos0 = 0, qpos1 = 0;        // positions the rows in Q slots 0 and 1 were rotated at
+    uint32_t n_staged0 = 0, n_staged1 = 0;   // staged items per Q slot so far
+    if (ROTQ && blockIdx.x < p.n_items) qpos0 = put_q(blockIdx.x, 0);
+    if (ROTQ && blockIdx.x + gridDim.x < p.n_items) qpos1 = put_q(blockIdx.x + gridDim.x, 1);
     uint32_t s_it = 0, item_no = 0;
     bool ok = true;
     for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x, ++item_no) {
@@ -730,7 +830,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t qs = item_no % kStagesQ;
       if (!stages_rows(it.ntiles)) {
         // fp32 output, or a short item: read, combine and store O 32 columns
-        // at a time (the item's last QK^T freed its Q slot)
+        // at a time
 #pragma unroll 1
         for (int col = 0; col < D; col += 32) {
           uint32_t o0[32], o1[32];
@@ -813,23 +913,28 @@ __global__ void __launch_bounds__(kThreads, 1)
           bulk_commit();
         }
         bulk_wait_read();
-        // once every row's copy has read the tile, its Q slot is free for the
-        // producer's next load there
+        // once every row's copy has read the tile, the slot may take the Q
+        // tile of the item two ahead (written below, or by the producer)
         mbar_arrive(&bar[B_Q_COPIED + qs]);
+        if (ROTQ) {
+          const uint32_t n_st = qs ? n_staged1++ : n_staged0++;
+          ok = __all_sync(kFull, mbar_wait(&bar[B_Q_COPIED + qs], n_st & 1, abort_flag, p.status,
+                                           p.wait_limit_ns, DBSA_ERR_TIMEOUT));
+        }
       }
       if (partial && p.part.dbg != nullptr && it.head == 0 && row < it.n_rows) {
         // Gather map: the thread of an item's first packed row records, for
         // every key of the tile's range, the cache row its K and V tiles came
         // from and the fresh position that the two rotations combine to (the
-        // query's token-0 position - the query rotation's position + the
-        // key's block-relative position).
+        // query's token-0 position - the position this kernel rotated the
+        // item's token-0 rows at + the key's block-relative position).
         const int grow = it.q_row0 + row;
         const int R = p.part.group * p.part.n_new;
         if (grow % R == 0) {
           const int item = __ldg(p.part.packed_items + grow / R);
           const S2Item si = p.part.items[item];
           const int qabs0 = p.part.queries[si.query].n_gathered + p.part.tail_len - p.part.n_new;
-          const int shift = qabs0 - p.part.q_rot_pos[item];
+          const int shift = qabs0 - (ROTQ ? (qs ? qpos1 : qpos0) : p.part.q_rot_pos[item]);
           const int64_t room = p.part.dbg_cap - si.p_begin;
           const int n = si.p_begin < 0 ? 0 : (int)min((int64_t)it.len[0], room);
           int32_t *m = p.part.dbg + ((int64_t)si.query * p.part.dbg_cap + si.p_begin) * 2;
@@ -838,6 +943,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             *reinterpret_cast<int2 *>(m + 2 * r) =
                 make_int2(same_rows ? it.k_row0[0] + r : -2, shift + it.pos0[0] + r);
         }
+      }
+      const int nidx = idx + 2 * gridDim.x;
+      if (ROTQ && ok && nidx < p.n_items) {
+        const int pos = put_q(nidx, qs);
+        if (qs) qpos1 = pos; else qpos0 = pos;
       }
     }
     bulk_wait_all();   // this thread's row copies have landed
@@ -892,17 +1002,33 @@ constexpr size_t smem_bytes() {
   return need > one_per_sm ? need : one_per_sm;
 }
 
-template <int D, bool F32, bool STAGE>
+template <int D, bool F32, bool STAGE, bool ROTQ>
 cudaError_t launch_t(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
                      const Params &p, int grid, cudaStream_t st) {
   constexpr size_t smem = smem_bytes<D>();
   static_assert(smem <= 232448, "shared memory budget");
   static_assert(smem > 232448 / 2, "one CTA per SM (the kernel owns all 512 TMEM columns)");
-  cudaError_t e = cudaFuncSetAttribute(stage1_attn_kernel<D, F32, STAGE>,
+  cudaError_t e = cudaFuncSetAttribute(stage1_attn_kernel<D, F32, STAGE, ROTQ>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  pdl_launch(stage1_attn_kernel<D, F32, STAGE>, dim3(grid), dim3(kThreads), smem, st, mq, mk, mv, p);
+  pdl_launch(stage1_attn_kernel<D, F32, STAGE, ROTQ>, dim3(grid), dim3(kThreads), smem, st, mq, mk,
+             mv, p);
   return cudaGetLastError();
+}
+
+// The launch shapes in use: Stage 1 always rotates its queries in the kernel
+// (fp32 or bf16 outputs); partial-mode passes (bf16 partials) either way.
+template <int D>
+cudaError_t launch_shape(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                         const Params &p, int grid, bool f32, bool stage, bool rotq,
+                         cudaStream_t st) {
+  if (f32)
+    return rotq ? launch_t<D, true, false, true>(mq, mk, mv, p, grid, st) : cudaErrorInvalidValue;
+  if (stage)
+    return rotq ? launch_t<D, false, true, true>(mq, mk, mv, p, grid, st)
+                : launch_t<D, false, true, false>(mq, mk, mv, p, grid, st);
+  return rotq ? launch_t<D, false, false, true>(mq, mk, mv, p, grid, st)
+              : launch_t<D, false, false, false>(mq, mk, mv, p, grid, st);
 }
 
 }  // namespace
@@ -910,10 +1036,17 @@ cudaError_t launch_t(const CUtensorMap &mq, const CUtensorMap &mk, const CUtenso
 cudaError_t launch_stage1(const Stage1Args &a, int head_dim, bool out_f32, int num_sms,
                           cudaStream_t st) {
   if (a.n_items <= 0) return cudaSuccess;
+  // queries rotated here (q_src) or pre-rotated rows loaded by TMA (q_rot)
+  const bool rotq = a.q_src != nullptr;
+  if (rotq ? (a.part.acc != nullptr && a.part.item_meta == nullptr) : a.q_rot == nullptr)
+    return cudaErrorInvalidValue;
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, a.q_rot, head_dim, a.q_rows, a.Hq, a.q_rows) ||
-      !make_map(&mk, a.k_rot, head_dim, a.k_rows, a.Hkv, a.k_rows) ||
+  if (!make_map(&mk, a.k_rot, head_dim, a.k_rows, a.Hkv, a.k_rows) ||
       !make_map(&mv, a.v, head_dim, a.v_rows, a.Hkv, a.v_head_stride))
+    return cudaErrorInvalidValue;
+  if (rotq)
+    mq = mk;   // a placeholder: the kernel reads no Q tile through it
+  else if (!make_map(&mq, a.q_rot, head_dim, a.q_rows, a.Hq, a.q_rows))
     return cudaErrorInvalidValue;
   Params p;
   p.items = a.items;
@@ -926,6 +1059,10 @@ cudaError_t launch_stage1(const Stage1Args &a, int head_dim, bool out_f32, int n
   p.wait_limit_ns = a.wait_limit_ns != 0 ? a.wait_limit_ns : kWaitLimitNs;
   p.withhold_tiles = a.withhold_tiles;
   p.part = a.part;
+  p.q_src = a.q_src;
+  p.q_f32 = a.q_f32;
+  p.q_heads = a.q_heads;
+  p.rope = a.rope;
   const int grid = a.n_items < num_sms ? a.n_items : num_sms;
   // Rows are staged (bf16 outputs) except in passes with few query rows per
   // (query, KV head) (decode steps): those stream their K/V from HBM and keep
@@ -933,13 +1070,8 @@ cudaError_t launch_stage1(const Stage1Args &a, int head_dim, bool out_f32, int n
   // than queued on it as bulk copies.
   const bool stage =
       !out_f32 && (a.part.acc == nullptr || a.part.group * a.part.n_new >= 32);
-  if (head_dim == 128)
-    return out_f32 ? launch_t<128, true, false>(mq, mk, mv, p, grid, st)
-           : stage ? launch_t<128, false, true>(mq, mk, mv, p, grid, st)
-                   : launch_t<128, false, false>(mq, mk, mv, p, grid, st);
-  return out_f32 ? launch_t<64, true, false>(mq, mk, mv, p, grid, st)
-         : stage ? launch_t<64, false, true>(mq, mk, mv, p, grid, st)
-                 : launch_t<64, false, false>(mq, mk, mv, p, grid, st);
+  if (head_dim == 128) return launch_shape<128>(mq, mk, mv, p, grid, out_f32, stage, rotq, st);
+  return launch_shape<64>(mq, mk, mv, p, grid, out_f32, stage, rotq, st);
 }
 
 }  // namespace dbsa
