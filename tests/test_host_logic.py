@@ -203,6 +203,14 @@ def test_workspace_sizes(lib):
     sel_ptr, sel = dbsa.selection_csr([np.array([0, 3, 9]), np.array([0, 1])])
     wg = dbsa.gather_workspace_size(cfg, offs, sel_ptr, sel, 40, 40)
     assert wg > 0
+    # a block-major pass over 1 500-token blocks (~12 key tiles per item): the
+    # tensor-core kernel rotates the packed query rows itself, so the workspace
+    # holds K at block-relative positions [Hkv][T][D] and the partials of the
+    # 5 (query, block) items + 2 tail items, plus small tables, and no packed
+    # query rows (they would add 8 x 5 x 160 rows x 256 B = 1.6 MB)
+    k_hat = 8 * T * 256
+    partials = 7 * 32 * 40 * (128 * 2 + 8)
+    assert k_hat + partials <= wg < k_hat + partials + (1 << 20)
     assert dbsa.gather_workspace_size(cfg, offs, sel_ptr, np.array([2, 3, 9, 0, 1]), 40, 40) == 0
     # a demonstration-granular selection (blocks of ~30 tokens) of one query
     # shares nothing across queries, so it goes per query.  A single-token
@@ -218,6 +226,19 @@ def test_workspace_sizes(lib):
     wd = dbsa.gather_workspace_size(cfg, doffs, dsp, dsel, 40, 40)
     compact = 2 * 8 * gathered * 128 * 2
     assert compact <= wd < compact + (8 << 20)
+    # a decode step over 30-token demonstrations, shared by 64 queries, runs
+    # block-major with items of one key tile: its packed query rows are written
+    # before the tensor-core pass (bf16 [Hkv][pairs x g][D]), on top of the keys
+    # and the partials
+    rng = np.random.default_rng(5)
+    dl = np.concatenate([[1500], np.full(2950, 30)])
+    do = np.concatenate([[0], np.cumsum(dl)]).astype(np.int32)
+    sels = [np.concatenate([[0], np.sort(rng.permutation(np.arange(1, len(dl)))[:885])])
+            for _ in range(64)]
+    dp, db = dbsa.selection_csr(sels)
+    pairs = sum(len(x) for x in sels)
+    need = 8 * int(do[-1]) * 256 + (pairs + 64) * 32 * (128 * 2 + 8) + 8 * pairs * 4 * 256
+    assert need <= dbsa.gather_workspace_size(cfg, do, dp, db, 1, 41) < need + (16 << 20)
     # prepared block keys: K at block-relative positions, bf16 [Hkv][T][D], plus
     # RoPE tables (cos and sin, D/2 floats a row) for positions below T + 8192:
     # (T + 8192) / 16 coarse rows and 16 fine rows
